@@ -1,0 +1,381 @@
+"""Benchmark of the fused Gaussian-mixture EM step on B200.
+
+A step is one EM iteration (log-sum-exp sweep, statistics sweep, M-step) over the
+whole resident X.  Default workload: N = 100,000,000, D = 128, K = 1024, diagonal
+model, fp32 X (51.2 GB resident in HBM, far larger than L2), the Table-1 generator
+of synth/ with seed = rank.  Prints one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload table1-1e8|table1-1e6|c1] [--prec auto|fp32|fp16x3]
+
+Multi-GPU (torchrun, one process per GPU): each rank fits its own independent
+mixture problem of the full per-rank size (weak scaling, no data-path
+collective); only the timing is reduced (max over ranks).
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only) and scales it to the metric.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    "table1-1e8": dict(gen="table1", N=100_000_000, D=128, K=1024),
+    "table1-1e6": dict(gen="table1", N=1_000_000, D=128, K=1024),
+    "table1-1e5": dict(gen="table1", N=100_000, D=128, K=1024),
+    "c1": dict(gen="c1", N=10_000, D=16, K=16),
+}
+METRIC = "EM iters/s at N=100M,K=1024,D=128 fp32"
+
+
+def workload_name(w):
+    return f"{w['gen']} N={w['N']} D={w['D']} K={w['K']} diag fp32"
+
+
+# ------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 7:
+                continue
+            try:
+                sm.append(float(p[0]))
+                mx.append(float(p[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, p[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id_for(dev: int) -> str:
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev)
+
+
+# ------------------------------------------------------------------------------- peaks
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "ivf_quantizer_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".h", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, prec: str):
+    """Per-launch DRAM bytes of `kernel` from a committed ncu summary, or None when
+    the summary was taken on other kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    e = rec.get(f"{prec}/{kernel}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------- CPU oracle
+def oracle_sample_time(w, sample_n: int, seed: int = 0):
+    """One oracle EM step on the first sample_n points of the same workload; returns
+    (seconds, sample_n).  BLAS limited to one thread."""
+    import torch
+
+    import synth
+    from oracle import gmm_oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        limiter = None
+    X = synth.generate(w["gen"], sample_n, seed=seed)
+    wt, mu, var = synth.init_params(X, w["K"], seed=seed)
+    Xn = X.double().numpy()
+    t0 = time.perf_counter()
+    O.em_step(Xn, wt.double().numpy(), mu.double().numpy(), var.double().numpy())
+    dt = time.perf_counter() - t0
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    del torch
+    return dt, sample_n
+
+
+def oracle_sample_size(w, target_s=15.0):
+    # the oracle's cost is ~ N*K*D fp64 element operations; ~6 ns each on one core
+    per_point = w["K"] * w["D"] * 6e-9
+    n = int(max(64, min(w["N"], target_s / per_point)))
+    return max(w["K"], n)
+
+
+# ------------------------------------------------------------------------------- main
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="table1-1e8", choices=sorted(WORKLOADS))
+    ap.add_argument("--prec", default="auto", choices=["auto", "fp32", "fp16x3"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    return ap.parse_args()
+
+
+def run_reference(args, w):  # noqa: C901
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    n_s = oracle_sample_size(w, target_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample_time(w, min(n_s, 2048))
+    times = []
+    for _ in range(args.steps):
+        dt, _ = oracle_sample_time(w, n_s)
+        times.append(dt * w["N"] / n_s)
+    t_step = sum(times) / len(times)
+    value = 1.0 / t_step
+    sample = f"one oracle EM step on {n_s} of {w['N']} points, scaled by N"
+    metric = METRIC if args.workload == "table1-1e8" else f"EM iters/s ({args.workload})"
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": "iters/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_name(w)},
+            "cpu_baseline": {"value": value, "unit": "iters/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "iters/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+
+    import ivf_quantizer_b200 as q
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    N, D, K = w["N"], w["D"], w["K"]
+    prec = {"auto": q.PREC_AUTO, "fp32": q.PREC_FP32, "fp16x3": q.PREC_FP16X3}[args.prec]
+    X = torch.empty(N, D, device=dev, dtype=torch.float32)
+    synth.generate(w["gen"], N, seed=rank, device=dev, out=X)
+    wt, mu, var = synth.init_params(X, K, seed=rank)
+    g = q.GMM(K, D)
+    try:
+        g.set_precision(prec)
+    except q.FgmmError:
+        g.set_precision(q.PREC_FP32)
+    prec_used = {q.PREC_FP32: "fp32", q.PREC_FP16X3: "fp16x3", q.PREC_AUTO: "auto"}[g.precision]
+    wd, md, vd = g.new_params(wt, mu, var)
+    ll = torch.zeros(1, dtype=torch.float64, device=dev)
+
+    for _ in range(args.warmup):
+        g.step(X, wd, md, vd, loglik=ll)
+    torch.cuda.synchronize()
+    g.check_status()
+    barrier()
+
+    sampler = ClockSampler(gpu_id_for(local))
+    sampler.start()
+    time.sleep(0.3)
+    g.profile(True)
+    g.profile_read(reset=True)
+    stream = torch.cuda.current_stream()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier()
+    t0.record(stream)
+    for _ in range(args.steps):
+        g.step(X, wd, md, vd, loglik=ll)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    prof = g.profile_read(reset=True)
+    g.profile(False)
+    g.check_status()
+    ms = t0.elapsed_time(t1)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    iters_per_s = world * args.steps / (ms_max / 1e3)
+
+    # ---- roofline of the dominant kernel (per launch, live CUDA-event durations)
+    peaks, peak_src = measured_peaks()
+    s1, s2 = prof["sweep1_ms"], prof["sweep2_ms"]
+    dom = "sweep2" if s2 >= s1 else "sweep1"
+    launches = prof[f"{dom}_launches"]
+    avg_ms = prof[f"{dom}_ms"] / max(1, launches)
+    pts_per_launch = N * args.steps / max(1, launches)
+    flops_per_launch = 4.0 * D * K * pts_per_launch     # each sweep: 4*D flops per (point, comp)
+    achieved = flops_per_launch / (avg_ms / 1e3) / 1e12
+    if prec_used == "fp32":
+        clk = float(peaks.get("sm_max_mhz", 1965.0))
+        peak = 148 * 128 * 2 * clk * 1e6 / 1e12
+        roof = {"bound": "alu", "unit": "TFLOP/s", "peak_note":
+                f"fp32 FMA: 148 SMs x 128 lanes x 2 x {clk:.0f} MHz"}
+    else:
+        peak = float(peaks["bf16_tflops_sustained"])
+        roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_note":
+                f"fp16 dense = bf16 {peak_src} sustained"}
+    traffic = recorded_traffic(dom, prec_used)
+    roof.update({"kernel": dom, "achieved": achieved, "peak": peak, "frac": achieved / peak,
+                 "traffic": traffic, "peak_source": peak_src,
+                 "launches": launches, "avg_launch_ms": avg_ms,
+                 "share_of_step": prof[f"{dom}_ms"] / max(1e-9, ms)})
+
+    # ---- end to end through the public API from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        try:
+            Xh = torch.empty(N, D, dtype=torch.float32, pin_memory=True)
+            Xh.copy_(X)
+            wd2, md2, vd2 = g.new_params(wt, mu, var)
+            llh = torch.zeros(1, dtype=torch.float64, pin_memory=True)
+
+            def e2e_step():
+                X.copy_(Xh, non_blocking=True)
+                g.step(X, wd2, md2, vd2, loglik=ll)
+                llh.copy_(ll, non_blocking=True)
+                torch.cuda.current_stream().synchronize()
+                return float(llh.item())
+
+            e2e_step()
+            barrier()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(args.e2e_steps):
+                e2e_step()
+            b.record()
+            torch.cuda.synchronize()
+            e_ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+            if world > 1:
+                dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+            e2e = {"value": world * args.e2e_steps / (float(e_ms.item()) / 1e3), "unit": "iters/s",
+                   "h2d_bytes_per_step": N * D * 4, "d2h_bytes_per_step": 8,
+                   "steps": args.e2e_steps}
+            del Xh
+        except Exception as ex:  # pinned allocation of X may fail on small hosts
+            e2e = {"value": None, "unit": "iters/s", "error": str(ex)[:200]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        n_s = oracle_sample_size(w)
+        dt, _ = oracle_sample_time(w, n_s)
+        cpu = {"value": 1.0 / (dt * N / n_s), "unit": "iters/s", "cores": 1, "kind": "oracle",
+               "sample": f"one fp64 oracle EM step on {n_s} of {N} points (K={K}, D={D}), "
+                         f"{dt:.1f} s, scaled by N/{n_s}"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC if args.workload == "table1-1e8" else f"EM iters/s ({args.workload})",
+            "value": iters_per_s, "unit": "iters/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": workload_name(w), "precision": prec_used,
+                       "l2": f"inputs larger than L2 (X = {N * D * 4 / 1e9:.1f} GB per GPU)"
+                       if N * D * 4 > 126e6 else "inputs smaller than L2",
+                       "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
+            "evals_per_s": iters_per_s * N * K,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(prof["launches"]),
+            "workspace_bytes": g.workspace_bytes,
+            "clocks": clocks,
+            "loglik_last": float(ll.item()),
+        }
+        print(json.dumps(line), flush=True)
+    g.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,165 @@
+/*
+ * fgmm.h — C-ABI of the fused Gaussian-mixture EM library for NVIDIA B200 (sm_100a).
+ *
+ * The operations are those of "Flash-GMM: A Memory-Efficient Kernel for
+ * Scalable Soft Clustering" (Bloch et al., arXiv 2606.10896):
+ *   - §2: mixture density, log-likelihood, E-step responsibilities computed in
+ *     log space, M-step Eqs. (1)-(3), stopping rule;
+ *   - §3.1, Algorithm 1: one EM iteration as a fused two-sweep pass over point
+ *     tiles that never stores the N x K responsibility matrix;
+ *   - §4.2-4.3: argmax and top-2 thresholded multi-assignment for IVF lists.
+ *
+ * Conventions for every call:
+ *   - Device pointers unless a name ends in _host.  All device work is
+ *     enqueued on the caller's stream and is asynchronous, unless a call says
+ *     it synchronises.
+ *   - X is row-major [N, D] with row stride ldx elements (ldx >= D).  x_dtype is
+ *     FGMM_F32 or FGMM_BF16.  The tensor-core precision modes require
+ *     ldx * sizeof(element) to be a multiple of 16 bytes and X 16-byte aligned.
+ *   - Parameters: weights float[K]; means float[K*D] row-major; vars float[K*D]
+ *     (diagonal model) or float[K] (isotropic model).  They are read at the
+ *     start of a step and overwritten in place with the M-step result.
+ *   - The caller owns X, the parameters and every output buffer.  The handle
+ *     owns only its workspace (allocated by fgmm_create, O(K*D), independent of
+ *     N) and its device status word.
+ *   - Errors are returned as fgmm_status codes; nothing throws across the ABI.
+ *     Errors found on the device (non-finite log-likelihood, invalid
+ *     parameters, every component empty) are latched in the handle's status
+ *     word and read with fgmm_get_status.
+ *   - A handle must not be used from two streams concurrently.
+ */
+#ifndef FGMM_H
+#define FGMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct fgmm_ctx* fgmm_handle;
+/* Same object as cudaStream_t / CUstream; 0 is the legacy default stream. */
+typedef struct CUstream_st* fgmm_stream_t;
+
+/* Covariance model.  SPHERICAL is the paper's isotropic sigma_k^2 I (§2,
+ * footnote 1; Appendix A); DIAG has one variance per component and dimension. */
+enum fgmm_cov { FGMM_COV_DIAG = 0, FGMM_COV_SPHERICAL = 1 };
+
+/* Arithmetic of the log-density evaluation and of the sufficient statistics.
+ *   FP32   : CUDA cores, fp32, log-densities in the direct (x - mu)^2 form and
+ *            statistics centred on each component's current mean.
+ *   FP16X3 : tensor cores (tcgen05), expanded form [x, x^2] . W with every
+ *            operand split into two fp16 halves and three products, fp32
+ *            accumulation (about 22 significant bits per product).
+ *   FP16   : tensor cores, one fp16 product per term (fast, ~11 bits; fails
+ *            the 1e-4 log-likelihood tolerance on the Table-1 generator).
+ *   AUTO   : the default; FP16X3 where every component is well conditioned for
+ *            the expanded form, FP32 otherwise (decided on the device per step). */
+enum fgmm_prec { FGMM_PREC_FP32 = 0, FGMM_PREC_FP16X3 = 1, FGMM_PREC_FP16 = 2, FGMM_PREC_AUTO = 3 };
+
+/* Element type of X. */
+enum fgmm_dtype { FGMM_F32 = 0, FGMM_BF16 = 1 };
+
+enum fgmm_status {
+  FGMM_OK = 0,
+  FGMM_ERR_INVALID_ARG = 1, /* bad size, null pointer, bad enum, or invalid parameters */
+  FGMM_ERR_UNSUPPORTED = 2, /* valid request this build or device cannot run */
+  FGMM_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+  FGMM_ERR_OOM = 4,         /* workspace allocation failed */
+  FGMM_ERR_NUMERIC = 5,     /* non-finite log-likelihood, or every component empty */
+  FGMM_ERR_TIMEOUT = 6      /* a bounded device-side wait expired */
+};
+
+/* Largest top_m accepted by fgmm_soft_assign. */
+#define FGMM_MAX_TOP_M 16
+/* A component with responsibility mass N_k below this is treated as empty:
+ * its mean and variance are kept and its weight becomes 0. */
+#define FGMM_EMPTY_NK 1e-6
+
+/* Create a handle for K components in D dimensions.
+ * reg_covar >= 0 is added to every variance after each M-step (variance floor).
+ * Allocates the workspace on the current CUDA device; the handle is bound to
+ * that device.  Returns FGMM_ERR_INVALID_ARG for K < 1, D < 1, a bad cov_type or
+ * a negative / non-finite reg_covar, FGMM_ERR_OOM if allocation fails. */
+int fgmm_create(int K, int D, int cov_type, double reg_covar, fgmm_handle* out);
+
+/* Free the workspace (synchronises the device first).  NULL is accepted. */
+int fgmm_destroy(fgmm_handle h);
+
+/* Select the precision mode (enum fgmm_prec).  FGMM_ERR_INVALID_ARG for an
+ * unknown value. */
+int fgmm_set_precision(fgmm_handle h, int prec);
+int fgmm_get_precision(fgmm_handle h, int* prec_out);
+
+/* Bytes of device memory the handle holds (independent of N). */
+int fgmm_workspace_bytes(fgmm_handle h, size_t* bytes_out);
+
+/* One EM iteration (§2; §3.1 Algorithm 1) on device data.
+ *   E-step with a log-sum-exp over the K components, responsibilities folded
+ *   straight into the sufficient statistics N_k, sum r (x - c), sum r (x - c)^2
+ *   (never stored as an N x K matrix), then the M-step Eqs. (1)-(3) with the
+ *   updated mean in the variance, pi_k = N_k / sum_k' N_k', the variance floor,
+ *   and the empty-component rule (FGMM_EMPTY_NK).
+ *   weights, means, vars : in/out, the parameters Theta_in are replaced by Theta_out.
+ *   loglik_out           : device double, receives log p(X | Theta_in) (may be NULL).
+ *   logz_out             : optional device float[N], per-point log p(x_i | Theta_in)
+ *                          (NULL to skip; the library itself never stores it).
+ * N must be >= 1.  Asynchronous; device-side errors go to the status word. */
+int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                 float* weights, float* means, float* vars,
+                 double* loglik_out, float* logz_out, fgmm_stream_t stream);
+
+/* Repeat fgmm_em_step up to max_iters times (§2, stopping rule).  With tol > 0
+ * it stops early once |L_t - L_{t-1}| / N < tol, which needs one 8-byte
+ * device-to-host read per iteration; with tol == 0 it only enqueues work.
+ * Synchronises the stream before returning.
+ *   final_loglik_host : log-likelihood of the last step's input parameters (may be NULL)
+ *   iters_done_host   : iterations run (may be NULL)
+ * Returns the first error of any step, including the device status word. */
+int fgmm_fit(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+             float* weights, float* means, float* vars, int max_iters, double tol,
+             double* final_loglik_host, int* iters_done_host, fgmm_stream_t stream);
+
+/* Multi-assignment from responsibilities under the given parameters (§4.2 argmax,
+ * §4.3 top-2 with r_ik > tau).  Per point the components are ranked by their
+ * log joint (ties to the lower index); rank 1 is always kept; ranks 2..top_m are
+ * kept only where r_ik > r_threshold (strict); the rest is padded with id -1 and
+ * responsibility 0.
+ *   ids  : device int32[N * top_m], row-major
+ *   resp : device float[N * top_m], row-major (may be NULL)
+ * 1 <= top_m <= min(K, FGMM_MAX_TOP_M), 0 <= r_threshold < 1. */
+int fgmm_soft_assign(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                     const float* weights, const float* means, const float* vars,
+                     int top_m, float r_threshold, int32_t* ids, float* resp,
+                     fgmm_stream_t stream);
+
+/* Kernel timing, for benchmarks.  When enabled, the library records a CUDA
+ * event pair on the call's stream around every kernel it launches and keeps a
+ * launch counter; fgmm_profile_read synchronises the device, sums the elapsed
+ * times per kernel kind and (if reset != 0) clears the record.  Disabled by
+ * default; costs two event records per launch when enabled. */
+typedef struct fgmm_profile {
+  int64_t launches;          /* kernels launched while enabled (all kinds) */
+  int64_t sweep1_launches;   /* log-sum-exp sweep (first pass over the components) */
+  double sweep1_ms;
+  int64_t sweep2_launches;   /* statistics sweep (recompute + responsibilities + stats) */
+  double sweep2_ms;
+  int64_t other_launches;    /* preparation, reductions, M-step, soft assignment */
+  double other_ms;
+} fgmm_profile;
+int fgmm_profile_enable(fgmm_handle h, int enable);
+int fgmm_profile_read(fgmm_handle h, fgmm_profile* out, int reset);
+
+/* Synchronise the stream and return the device status word (first error
+ * latched since the last call), then clear it. */
+int fgmm_get_status(fgmm_handle h, fgmm_stream_t stream);
+
+/* Static text for a status code. */
+const char* fgmm_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FGMM_H */

@@ -1,0 +1,379 @@
+// Host side of the C-ABI declared in include/fgmm.h: argument checks, workspace
+// ownership, the chunk loop over N and the kernel sequence of one EM step.
+//
+// One EM step ("Flash-GMM: A Memory-Efficient Kernel for Scalable Soft
+// Clustering", §3.1, Algorithm 1) is enqueued as
+//   prep                       parameters -> padded means / precisions / constants
+//   for each chunk of <= kChunk points:
+//     sweep 1 (log-sum-exp)    log Z_i for the chunk, partial log-likelihood
+//     ll_accumulate            adds the chunk's partials in a fixed order
+//     sweep 2 (statistics)     recompute, responsibilities, sufficient statistics
+//   M-step + finalize          Eqs. (1)-(3), weights, log-likelihood, status
+// Every buffer the step touches is O(K D) or O(kChunk): device memory beyond X
+// does not grow with N.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <new>
+
+#include "fgmm_internal.h"
+
+#include <vector>
+
+using namespace fgmm;
+
+struct fgmm_ctx {
+  Ctx c;
+};
+
+// Optional per-launch event timing (fgmm_profile_*).  Events are pooled and
+// reused after each read.
+struct fgmm::Profiler {
+  bool enabled = false;
+  int64_t launches = 0;
+  struct Rec {
+    cudaEvent_t a, b;
+    int kind;
+  };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t pending = nullptr;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  ~Profiler() {
+    for (auto& r : recs) {
+      cudaEventDestroy(r.a);
+      cudaEventDestroy(r.b);
+    }
+    for (auto e : pool) cudaEventDestroy(e);
+    if (pending) cudaEventDestroy(pending);
+  }
+};
+
+namespace fgmm {
+void prof_begin(const Ctx& c, KernelKind, cudaStream_t s) {
+  Profiler* p = c.prof;
+  if (!p) return;
+  ++p->launches;
+  if (!p->enabled) return;
+  p->pending = p->get();
+  cudaEventRecord(p->pending, s);
+}
+void prof_end(const Ctx& c, KernelKind k, cudaStream_t s) {
+  Profiler* p = c.prof;
+  if (!p || !p->enabled || !p->pending) return;
+  cudaEvent_t b = p->get();
+  cudaEventRecord(b, s);
+  p->recs.push_back({p->pending, b, (int)k});
+  p->pending = nullptr;
+}
+}  // namespace fgmm
+
+namespace {
+
+bool valid_dtype(int t) { return t == FGMM_F32 || t == FGMM_BF16; }
+size_t dtype_bytes(int t) { return t == FGMM_BF16 ? 2 : 4; }
+
+int map_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return FGMM_OK;
+  if (e == cudaErrorMemoryAllocation) return FGMM_ERR_OOM;
+  return FGMM_ERR_CUDA;
+}
+
+void free_ws(Workspace& w) {
+  void* ptrs[] = {w.mu, w.prec, w.cconst, w.logz, w.ll_tiles, w.ll_total, w.stats, w.nk, w.status};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  w = Workspace{};
+}
+
+template <typename T>
+cudaError_t alloc(T** p, size_t count, size_t* total) {
+  *total += count * sizeof(T);
+  return cudaMalloc((void**)p, count * sizeof(T));
+}
+
+cudaError_t alloc_ws(Ctx& c) {
+  Workspace& w = c.ws;
+  w.Kp = round_up(c.K, kKB);
+  w.Dp = round_up(c.D, kDC);
+  size_t t = 0;
+  cudaError_t e;
+  const size_t kd = (size_t)w.Kp * w.Dp;
+  if ((e = alloc(&w.mu, kd, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.prec, kd, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.cconst, (size_t)w.Kp, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.logz, (size_t)kChunk, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.ll_tiles, (size_t)(kChunk / kTP), &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.ll_total, (size_t)1, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.stats, (size_t)kSlices * w.Kp * (1 + 2 * (size_t)w.Dp), &t)) != cudaSuccess)
+    return e;
+  if ((e = alloc(&w.nk, (size_t)w.Kp, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.status, (size_t)1, &t)) != cudaSuccess) return e;
+  if ((e = cudaMemset(w.status, 0, sizeof(int))) != cudaSuccess) return e;
+  w.bytes = t;
+  return cudaSuccess;
+}
+
+int check_x(const fgmm_ctx* h, const void* X, int x_dtype, int64_t N, int64_t ldx) {
+  if (!h || !X) return FGMM_ERR_INVALID_ARG;
+  if (!valid_dtype(x_dtype)) return FGMM_ERR_INVALID_ARG;
+  if (N < 1 || ldx < h->c.D) return FGMM_ERR_INVALID_ARG;
+  return FGMM_OK;
+}
+
+int set_device(const Ctx& c) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return FGMM_ERR_CUDA;
+  if (cur != c.device && cudaSetDevice(c.device) != cudaSuccess) return FGMM_ERR_CUDA;
+  return FGMM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fgmm_create(int K, int D, int cov_type, double reg_covar, fgmm_handle* out) {
+  if (!out) return FGMM_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (K < 1 || D < 1 || (cov_type != FGMM_COV_DIAG && cov_type != FGMM_COV_SPHERICAL))
+    return FGMM_ERR_INVALID_ARG;
+  if (!(reg_covar >= 0.0) || !isfinite(reg_covar)) return FGMM_ERR_INVALID_ARG;
+  // 32-bit index arithmetic inside the kernels: bound the parameter block.
+  if ((int64_t)K * D > (int64_t)1 << 28 || K > (1 << 24) || D > (1 << 16))
+    return FGMM_ERR_UNSUPPORTED;
+  fgmm_ctx* h = new (std::nothrow) fgmm_ctx();
+  if (!h) return FGMM_ERR_OOM;
+  h->c.K = K;
+  h->c.D = D;
+  h->c.cov = cov_type;
+  h->c.reg = reg_covar;
+  h->c.prec = FGMM_PREC_FP32;
+  if (cudaGetDevice(&h->c.device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->c.num_sms, cudaDevAttrMultiProcessorCount, h->c.device) !=
+          cudaSuccess) {
+    delete h;
+    return FGMM_ERR_CUDA;
+  }
+  h->c.prof = new (std::nothrow) Profiler();
+  cudaError_t e = alloc_ws(h->c);
+  if (e != cudaSuccess) {
+    free_ws(h->c.ws);
+    delete h->c.prof;
+    delete h;
+    cudaGetLastError();
+    return map_cuda(e);
+  }
+  *out = h;
+  return FGMM_OK;
+}
+
+int fgmm_destroy(fgmm_handle h) {
+  if (!h) return FGMM_OK;
+  int rc = set_device(h->c);
+  cudaDeviceSynchronize();
+  free_ws(h->c.ws);
+  delete h->c.prof;
+  delete h;
+  return rc;
+}
+
+int fgmm_set_precision(fgmm_handle h, int prec) {
+  if (!h) return FGMM_ERR_INVALID_ARG;
+  if (prec != FGMM_PREC_FP32 && prec != FGMM_PREC_FP16X3 && prec != FGMM_PREC_FP16 &&
+      prec != FGMM_PREC_AUTO)
+    return FGMM_ERR_INVALID_ARG;
+  if (prec == FGMM_PREC_FP16X3 || prec == FGMM_PREC_FP16) return FGMM_ERR_UNSUPPORTED;
+  h->c.prec = prec;
+  return FGMM_OK;
+}
+
+int fgmm_get_precision(fgmm_handle h, int* prec_out) {
+  if (!h || !prec_out) return FGMM_ERR_INVALID_ARG;
+  *prec_out = h->c.prec;
+  return FGMM_OK;
+}
+
+int fgmm_workspace_bytes(fgmm_handle h, size_t* bytes_out) {
+  if (!h || !bytes_out) return FGMM_ERR_INVALID_ARG;
+  *bytes_out = h->c.ws.bytes;
+  return FGMM_OK;
+}
+
+int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                 float* weights, float* means, float* vars, double* loglik_out, float* logz_out,
+                 fgmm_stream_t stream) {
+  int rc = check_x(h, X, x_dtype, N, ldx);
+  if (rc) return rc;
+  if (!weights || !means || !vars) return FGMM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if ((rc = set_device(c))) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  const Workspace& w = c.ws;
+  if ((e = cudaMemsetAsync(w.ll_total, 0, sizeof(double), s)) != cudaSuccess) return map_cuda(e);
+  if ((e = cudaMemsetAsync(w.stats, 0, (size_t)kSlices * w.Kp * (1 + 2 * (size_t)w.Dp) * 8, s)) !=
+      cudaSuccess)
+    return map_cuda(e);
+  if ((e = launch_prep_simt(c, weights, means, vars, s)) != cudaSuccess) return map_cuda(e);
+  const size_t eb = dtype_bytes(x_dtype);
+  for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
+    const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
+    const void* Xc = (const char*)X + (size_t)c0 * ldx * eb;
+    if ((e = launch_lse_simt(c, Xc, x_dtype, nc, ldx, logz_out ? logz_out + c0 : nullptr, s)) !=
+        cudaSuccess)
+      return map_cuda(e);
+    if ((e = launch_ll_accumulate(c, nc, s)) != cudaSuccess) return map_cuda(e);
+    if ((e = launch_stats_simt(c, Xc, x_dtype, nc, ldx, s)) != cudaSuccess) return map_cuda(e);
+  }
+  if ((e = launch_mstep(c, weights, means, vars, loglik_out, s)) != cudaSuccess)
+    return map_cuda(e);
+  return FGMM_OK;
+}
+
+int fgmm_fit(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx, float* weights,
+             float* means, float* vars, int max_iters, double tol, double* final_loglik_host,
+             int* iters_done_host, fgmm_stream_t stream) {
+  int rc = check_x(h, X, x_dtype, N, ldx);
+  if (rc) return rc;
+  if (max_iters < 0 || !(tol >= 0.0)) return FGMM_ERR_INVALID_ARG;
+  if (!weights || !means || !vars) return FGMM_ERR_INVALID_ARG;
+  if ((rc = set_device(h->c))) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  double* d_ll = nullptr;
+  cudaError_t e = cudaMalloc(&d_ll, 2 * sizeof(double));
+  if (e != cudaSuccess) return map_cuda(e);
+  double prev = 0.0, cur = NAN;
+  int it = 0;
+  for (it = 0; it < max_iters; ++it) {
+    rc = fgmm_em_step(h, X, x_dtype, N, ldx, weights, means, vars, d_ll, nullptr, stream);
+    if (rc) break;
+    if (tol > 0.0) {
+      if ((e = cudaMemcpyAsync(&cur, d_ll, sizeof(double), cudaMemcpyDeviceToHost, s)) !=
+              cudaSuccess ||
+          (e = cudaStreamSynchronize(s)) != cudaSuccess) {
+        rc = map_cuda(e);
+        break;
+      }
+      if (it > 0 && fabs(cur - prev) / (double)N < tol) {
+        ++it;
+        break;
+      }
+      prev = cur;
+    }
+  }
+  if (!rc) {
+    if ((e = cudaMemcpyAsync(&cur, d_ll, sizeof(double), cudaMemcpyDeviceToHost, s)) !=
+        cudaSuccess)
+      rc = map_cuda(e);
+    else if ((e = cudaStreamSynchronize(s)) != cudaSuccess)
+      rc = map_cuda(e);
+  }
+  cudaFree(d_ll);
+  if (!rc) rc = fgmm_get_status(h, stream);
+  if (final_loglik_host) *final_loglik_host = (max_iters > 0) ? cur : NAN;
+  if (iters_done_host) *iters_done_host = it;
+  return rc;
+}
+
+int fgmm_soft_assign(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                     const float* weights, const float* means, const float* vars, int top_m,
+                     float r_threshold, int32_t* ids, float* resp, fgmm_stream_t stream) {
+  int rc = check_x(h, X, x_dtype, N, ldx);
+  if (rc) return rc;
+  if (!weights || !means || !vars || !ids) return FGMM_ERR_INVALID_ARG;
+  if (top_m < 1 || top_m > FGMM_MAX_TOP_M || top_m > h->c.K) return FGMM_ERR_INVALID_ARG;
+  if (!(r_threshold >= 0.f) || !(r_threshold < 1.f)) return FGMM_ERR_INVALID_ARG;
+  const Ctx& c = h->c;
+  if ((rc = set_device(c))) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  if ((e = launch_prep_simt(c, weights, means, vars, s)) != cudaSuccess) return map_cuda(e);
+  const size_t eb = dtype_bytes(x_dtype);
+  for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
+    const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
+    const void* Xc = (const char*)X + (size_t)c0 * ldx * eb;
+    if ((e = launch_soft_assign_simt(c, Xc, x_dtype, nc, ldx, top_m, r_threshold,
+                                     ids + c0 * top_m, resp ? resp + c0 * top_m : nullptr, s)) !=
+        cudaSuccess)
+      return map_cuda(e);
+  }
+  return FGMM_OK;
+}
+
+int fgmm_get_status(fgmm_handle h, fgmm_stream_t stream) {
+  if (!h) return FGMM_ERR_INVALID_ARG;
+  int rc = set_device(h->c);
+  if (rc) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  int st = 0;
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(&st, h->c.ws.status, sizeof(int), cudaMemcpyDeviceToHost, s)) !=
+      cudaSuccess)
+    return map_cuda(e);
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return map_cuda(e);
+  if (st != FGMM_OK) {
+    if ((e = cudaMemsetAsync(h->c.ws.status, 0, sizeof(int), s)) != cudaSuccess)
+      return map_cuda(e);
+    if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return map_cuda(e);
+  }
+  return st;
+}
+
+int fgmm_profile_enable(fgmm_handle h, int enable) {
+  if (!h || !h->c.prof) return FGMM_ERR_INVALID_ARG;
+  h->c.prof->enabled = enable != 0;
+  return FGMM_OK;
+}
+
+int fgmm_profile_read(fgmm_handle h, fgmm_profile* out, int reset) {
+  if (!h || !h->c.prof || !out) return FGMM_ERR_INVALID_ARG;
+  int rc = set_device(h->c);
+  if (rc) return rc;
+  Profiler* p = h->c.prof;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return map_cuda(e);
+  fgmm_profile r{};
+  r.launches = p->launches;
+  for (auto& rec : p->recs) {
+    float ms = 0.f;
+    if ((e = cudaEventElapsedTime(&ms, rec.a, rec.b)) != cudaSuccess) return map_cuda(e);
+    if (rec.kind == KK_SWEEP1) { r.sweep1_launches++; r.sweep1_ms += ms; }
+    else if (rec.kind == KK_SWEEP2) { r.sweep2_launches++; r.sweep2_ms += ms; }
+    else { r.other_launches++; r.other_ms += ms; }
+  }
+  *out = r;
+  if (reset) {
+    for (auto& rec : p->recs) {
+      p->pool.push_back(rec.a);
+      p->pool.push_back(rec.b);
+    }
+    p->recs.clear();
+    p->launches = 0;
+  }
+  return FGMM_OK;
+}
+
+const char* fgmm_status_string(int status) {
+  switch (status) {
+    case FGMM_OK: return "ok";
+    case FGMM_ERR_INVALID_ARG: return "invalid argument";
+    case FGMM_ERR_UNSUPPORTED: return "unsupported";
+    case FGMM_ERR_CUDA: return "CUDA runtime error";
+    case FGMM_ERR_OOM: return "out of device memory";
+    case FGMM_ERR_NUMERIC: return "non-finite log-likelihood or every component empty";
+    case FGMM_ERR_TIMEOUT: return "bounded device wait expired";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

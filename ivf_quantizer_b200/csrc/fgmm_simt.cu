@@ -1,0 +1,565 @@
+// CUDA-core (fp32) kernels of the fused EM step and of the soft assignment.
+//
+// Paper: "Flash-GMM: A Memory-Efficient Kernel for Scalable Soft Clustering".
+//   §2            log N(x | mu_k, Sigma_k), log-sum-exp over k, Eqs. (1)-(3)
+//   §3.1, Alg. 1  two sweeps over the components per point tile: the first
+//                 builds log Z_i with an online log-sum-exp, the second
+//                 recomputes the log-densities, forms r_ik = exp(log z_ik - log Z_i)
+//                 and folds them into per-component sufficient statistics.
+//   §4.2-4.3      argmax / top-m thresholded assignment.
+//
+// This is the FGMM_PREC_FP32 mode: log-densities in the direct form
+// sum_d -(x_d - mu_kd)^2 / (2 sigma_kd^2), statistics centred on each
+// component's current mean (sum r (x - mu), sum r (x - mu)^2), which keeps the
+// variance update free of cancellation.  The N x K matrix of responsibilities
+// only ever exists as one 64 x 32 tile in shared memory.
+//
+// Data layout: prepared parameters are zero padded to [Kp, Dp] (Kp multiple of
+// 64, Dp multiple of 32); padded / dead components carry cconst = -inf so that
+// they contribute exp(-inf) = 0.  Statistics partials live in [kSlices][Kp][1+2Dp]
+// fp64 slots, each written by exactly one CTA, summed in a fixed order by the
+// M-step kernel: the result is bitwise reproducible.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "fgmm_internal.h"
+
+namespace fgmm {
+
+__device__ __forceinline__ float ld_x(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float ld_x(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+__device__ __forceinline__ void set_status(int* st, int code) { atomicCAS(st, FGMM_OK, code); }
+
+// ------------------------------------------------------------------ parameter preparation
+// One CTA per (padded) component.  cconst_k = log pi_k - 1/2 sum_d log(2 pi sigma_kd^2),
+// the d-independent part of log z_ik (§2); the sum is taken in fp64.
+__global__ void prep_simt_kernel(int K, int D, int Kp, int Dp, int cov, const float* __restrict__ w,
+                                 const float* __restrict__ means, const float* __restrict__ vars,
+                                 float* __restrict__ mu, float* __restrict__ prec,
+                                 float* __restrict__ cconst, int* status) {
+  __shared__ double red[kSimtThreads];
+  const int k = blockIdx.x;
+  double acc = 0.0;
+  bool bad = false;
+  for (int d = threadIdx.x; d < Dp; d += blockDim.x) {
+    float m = 0.f, p = 0.f;
+    if (k < K && d < D) {
+      const float v = (cov == FGMM_COV_DIAG) ? vars[(size_t)k * D + d] : vars[k];
+      m = means[(size_t)k * D + d];
+      if (!(v > 0.f) || !isfinite(v) || !isfinite(m)) bad = true;
+      p = -0.5f / v;
+      acc += log(2.0 * CUDART_PI * (double)v);
+    }
+    mu[(size_t)k * Dp + d] = m;
+    prec[(size_t)k * Dp + d] = p;
+  }
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    float c = -CUDART_INF_F;
+    if (k < K) {
+      const float wk = w[k];
+      if (!(wk >= 0.f) || !isfinite(wk)) bad = true;
+      if (wk > 0.f) c = (float)(log((double)wk) - 0.5 * red[0]);
+    }
+    cconst[k] = c;
+  }
+  if (bad) set_status(status, FGMM_ERR_INVALID_ARG);
+}
+
+// ------------------------------------------------------------------ shared logit tile
+// Computes acc[j][q] = sum_d prec_kd (x_id - mu_kd)^2 for points r = ty + 16 j of the
+// tile and components kb + tx + 16 q, looping over the features in chunks of kDC staged
+// in shared memory.  NJ points x NQ components per thread.
+template <int NQ, typename T>
+__device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, int64_t ldx, int D,
+                                           int Dp, int64_t i0, int kb,
+                                           const float* __restrict__ mu,
+                                           const float* __restrict__ prec,
+                                           float (*xs)[kDC + 4], float (*ms)[kDC + 4],
+                                           float (*ps)[kDC + 4], float (&acc)[4][NQ]) {
+  constexpr int KBLK = 16 * NQ;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) acc[j][q] = 0.f;
+  for (int d0 = 0; d0 < Dp; d0 += kDC) {
+    for (int e = threadIdx.x; e < kTP * kDC; e += kSimtThreads) {
+      const int r = e / kDC, cx = e % kDC;
+      const int64_t i = i0 + r;
+      const int d = d0 + cx;
+      xs[r][cx] = (i < n && d < D) ? ld_x(X + i * ldx + d) : 0.f;
+    }
+    for (int e = threadIdx.x; e < KBLK * kDC; e += kSimtThreads) {
+      const int r = e / kDC, cx = e % kDC;
+      ms[r][cx] = mu[(size_t)(kb + r) * Dp + d0 + cx];
+      ps[r][cx] = prec[(size_t)(kb + r) * Dp + d0 + cx];
+    }
+    __syncthreads();
+#pragma unroll 2
+    for (int d = 0; d < kDC; d += 4) {
+      float4 xv[4], mv[NQ], pv[NQ];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) xv[j] = *reinterpret_cast<const float4*>(&xs[ty + 16 * j][d]);
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        mv[q] = *reinterpret_cast<const float4*>(&ms[tx + 16 * q][d]);
+        pv[q] = *reinterpret_cast<const float4*>(&ps[tx + 16 * q][d]);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          float t;
+          t = xv[j].x - mv[q].x; acc[j][q] = fmaf(pv[q].x * t, t, acc[j][q]);
+          t = xv[j].y - mv[q].y; acc[j][q] = fmaf(pv[q].y * t, t, acc[j][q]);
+          t = xv[j].z - mv[q].z; acc[j][q] = fmaf(pv[q].z * t, t, acc[j][q]);
+          t = xv[j].w - mv[q].w; acc[j][q] = fmaf(pv[q].w * t, t, acc[j][q]);
+        }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ sweep 1: log Z_i
+// One CTA per 64-point tile; online log-sum-exp over blocks of 64 components
+// (Alg. 1, step 1).  Writes log Z_i for the chunk, optionally to the caller's
+// per-point buffer, and one fp64 partial log-likelihood per tile.
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+    lse_simt_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp, int Kp,
+                    const float* __restrict__ mu, const float* __restrict__ prec,
+                    const float* __restrict__ cconst, float* __restrict__ logz,
+                    float* __restrict__ logz_out, double* __restrict__ ll_tiles) {
+  __shared__ __align__(16) float xs[kTP][kDC + 4];
+  __shared__ __align__(16) float ms[kKB][kDC + 4];
+  __shared__ __align__(16) float ps[kKB][kDC + 4];
+  __shared__ double lls[kTP];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int64_t i0 = (int64_t)blockIdx.x * kTP;
+  float run_m[4], run_s[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) { run_m[j] = -CUDART_INF_F; run_s[j] = 0.f; }
+
+  for (int kb = 0; kb < Kp; kb += kKB) {
+    float acc[4][4];
+    logit_tile<4>(X, n, ldx, D, Dp, i0, kb, mu, prec, xs, ms, ps, acc);
+    float cc[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) cc[q] = cconst[kb + tx + 16 * q];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float l[4];
+      float bm = -CUDART_INF_F;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) { l[q] = acc[j][q] + cc[q]; bm = fmaxf(bm, l[q]); }
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+      const float nm = fmaxf(run_m[j], bm);
+      const bool live = nm > -CUDART_INF_F;
+      float s = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) s += live ? expf(l[q] - nm) : 0.f;
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      run_s[j] = live ? run_s[j] * expf(run_m[j] - nm) + s : 0.f;
+      run_m[j] = nm;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int r = ty + 16 * j;
+    const int64_t i = i0 + r;
+    const float lz = run_m[j] + logf(run_s[j]);
+    if (tx == 0) {
+      if (i < n) {
+        logz[i] = lz;
+        if (logz_out) logz_out[i] = lz;
+      }
+      lls[r] = (i < n) ? (double)lz : 0.0;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int r = 0; r < kTP; ++r) s += lls[r];
+    ll_tiles[blockIdx.x] = s;
+  }
+}
+
+// Adds the chunk's per-tile partial log-likelihoods, in tile order, to ll_total.
+__global__ void ll_accumulate_kernel(const double* __restrict__ ll_tiles, int ntiles,
+                                     double* __restrict__ ll_total) {
+  __shared__ double red[kSimtThreads];
+  double s = 0.0;
+  for (int t = threadIdx.x; t < ntiles; t += blockDim.x) s += ll_tiles[t];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *ll_total += red[0];
+}
+
+// ------------------------------------------------------------------ sweep 2: statistics
+// Grid (Kp / 32 component blocks, kSlices point slices, ceil(Dp / 128) feature blocks).
+// Each CTA recomputes the log-densities of its 32 components for every 64-point tile
+// of its slice (Alg. 1, step 2), forms r = exp(l - log Z_i), and accumulates
+//   N_k = sum_i r_ik,  S1_kd = sum_i r_ik (x_id - mu_kd),  S2_kd = sum_i r_ik (x_id - mu_kd)^2
+// for its 128 features in fp32 registers, flushed to its fp64 slot every kFlushTiles tiles.
+struct StatsSmem {
+  float xs[kTP][kDC + 4];
+  float ms[kKBs][kDC + 4];
+  float ps[kKBs][kDC + 4];
+  float rs[kTP][kKBs + 4];
+  float xf[kTP][kFC];
+  float lz[kTP];
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+    stats_simt_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp, int Kp,
+                      const float* __restrict__ mu, const float* __restrict__ prec,
+                      const float* __restrict__ cconst, const float* __restrict__ logz,
+                      double* __restrict__ stats, int64_t slice_len) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  StatsSmem& sm = *reinterpret_cast<StatsSmem*>(smem_raw);
+  const int kb = blockIdx.x * kKBs;
+  const int s = blockIdx.y;
+  const int f0 = blockIdx.z * kFC;
+  const int64_t p_begin = (int64_t)s * slice_len;
+  const int64_t p_end = min(n, p_begin + slice_len);
+  if (p_begin >= p_end) return;  // uniform over the CTA
+
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int fl = threadIdx.x % kFC;            // this thread's feature (local)
+  const int h = threadIdx.x / kFC;             // component half: comps h*16 .. h*16+15
+  const int f = f0 + fl;
+  const bool f_ok = f < D;
+  const size_t row = (size_t)(1 + 2 * Dp);
+  double* slot = stats + (size_t)s * Kp * row;
+
+  float mreg[16];
+#pragma unroll
+  for (int jj = 0; jj < 16; ++jj) mreg[jj] = f_ok ? mu[(size_t)(kb + h * 16 + jj) * Dp + f] : 0.f;
+  float acc1[16], acc2[16], nka[16];
+#pragma unroll
+  for (int jj = 0; jj < 16; ++jj) { acc1[jj] = 0.f; acc2[jj] = 0.f; nka[jj] = 0.f; }
+  const bool nk_owner = (blockIdx.z == 0) && (fl == 0);
+  float cc[2];
+  cc[0] = cconst[kb + tx];
+  cc[1] = cconst[kb + tx + 16];
+
+  auto flush = [&]() {
+    if (f_ok) {
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        double* r = slot + (size_t)(kb + h * 16 + jj) * row;
+        r[1 + f] += (double)acc1[jj];
+        r[1 + Dp + f] += (double)acc2[jj];
+        acc1[jj] = 0.f;
+        acc2[jj] = 0.f;
+      }
+    }
+    if (nk_owner) {
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        slot[(size_t)(kb + h * 16 + jj) * row] += (double)nka[jj];
+        nka[jj] = 0.f;
+      }
+    }
+  };
+
+  int tiles = 0;
+  for (int64_t i0 = p_begin; i0 < p_end; i0 += kTP) {
+    if (threadIdx.x < kTP) {
+      const int64_t i = i0 + threadIdx.x;
+      sm.lz[threadIdx.x] = (i < p_end) ? logz[i] : -CUDART_INF_F;
+    }
+    float acc[4][2];
+    logit_tile<2>(X, p_end, ldx, D, Dp, i0, kb, mu, prec, sm.xs, sm.ms, sm.ps, acc);
+    // responsibilities of this tile for the CTA's 32 components
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = ty + 16 * j;
+      const float lz = sm.lz[r];
+      const bool ok = lz > -CUDART_INF_F && lz < CUDART_INF_F;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) sm.rs[r][tx + 16 * q] = ok ? expf(acc[j][q] + cc[q] - lz) : 0.f;
+    }
+    // the tile's features for the statistics
+    for (int e = threadIdx.x; e < kTP * kFC; e += kSimtThreads) {
+      const int r = e / kFC, cx = e % kFC;
+      const int64_t i = i0 + r;
+      const int d = f0 + cx;
+      sm.xf[r][cx] = (i < p_end && d < D) ? ld_x(X + i * ldx + d) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 2
+    for (int r = 0; r < kTP; ++r) {
+      const float x = sm.xf[r][fl];
+      float rv[16];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const float4 t = *reinterpret_cast<const float4*>(&sm.rs[r][h * 16 + 4 * v]);
+        rv[4 * v] = t.x; rv[4 * v + 1] = t.y; rv[4 * v + 2] = t.z; rv[4 * v + 3] = t.w;
+      }
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const float dv = x - mreg[jj];
+        const float rd = rv[jj] * dv;
+        acc1[jj] += rd;
+        acc2[jj] = fmaf(rd, dv, acc2[jj]);
+        nka[jj] += rv[jj];
+      }
+    }
+    __syncthreads();
+    if (++tiles == kFlushTiles) { flush(); tiles = 0; }
+  }
+  flush();
+}
+
+// ------------------------------------------------------------------ M-step
+// One CTA per component: fixed-order fp64 sum over the slice slots, then Eqs. (1)-(3):
+//   mu_new = mu_old + S1/N_k,  sigma^2 = max(S2/N_k - (S1/N_k)^2, 0) + reg_covar
+// (isotropic: averaged over d).  Empty components keep their parameters.  Nothing is
+// written when the log-likelihood of the step is not finite.
+__global__ void mstep_kernel(int K, int D, int Dp, int Kp, int cov, double reg,
+                             const double* __restrict__ stats, const float* __restrict__ mu_old,
+                             const double* __restrict__ ll_total, float* __restrict__ means,
+                             float* __restrict__ vars, double* __restrict__ nk_out, int* status) {
+  __shared__ double red[kSimtThreads];
+  const int k = blockIdx.x;
+  const size_t row = (size_t)(1 + 2 * Dp);
+  const bool ll_ok = isfinite(*ll_total);
+  double nk = 0.0;
+  for (int s = 0; s < kSlices; ++s) nk += stats[((size_t)s * Kp + k) * row];
+  if (threadIdx.x == 0) nk_out[k] = nk;
+  const bool live = ll_ok && (nk >= FGMM_EMPTY_NK);
+  double vsum = 0.0;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    double s1 = 0.0, s2 = 0.0;
+    for (int s = 0; s < kSlices; ++s) {
+      const double* r = stats + ((size_t)s * Kp + k) * row;
+      s1 += r[1 + d];
+      s2 += r[1 + Dp + d];
+    }
+    if (live) {
+      const double m1 = s1 / nk;
+      const double v = fmax(s2 / nk - m1 * m1, 0.0);
+      means[(size_t)k * D + d] = (float)((double)mu_old[(size_t)k * Dp + d] + m1);
+      if (cov == FGMM_COV_DIAG) vars[(size_t)k * D + d] = (float)(v + reg);
+      vsum += v;
+    }
+  }
+  if (cov == FGMM_COV_SPHERICAL) {
+    red[threadIdx.x] = vsum;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+      if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0 && live) vars[k] = (float)(red[0] / D + reg);
+  }
+  if (threadIdx.x == 0 && !isfinite(nk)) set_status(status, FGMM_ERR_NUMERIC);
+}
+
+// Weights pi_k = N_k / sum_{live k'} N_k' (Alg. 1, final step), log-likelihood output,
+// and the numeric checks.  One CTA, fixed-order sums.
+__global__ void finalize_kernel(int K, const double* __restrict__ nk, const double* __restrict__ ll_total,
+                                float* __restrict__ weights, double* __restrict__ loglik_out,
+                                int* status) {
+  __shared__ double red[kSimtThreads];
+  const double ll = *ll_total;
+  const bool ll_ok = isfinite(ll);
+  double s = 0.0;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) s += (nk[k] >= FGMM_EMPTY_NK) ? nk[k] : 0.0;
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  const double tot = red[0];
+  if (ll_ok && tot > 0.0) {
+    for (int k = threadIdx.x; k < K; k += blockDim.x)
+      weights[k] = (nk[k] >= FGMM_EMPTY_NK) ? (float)(nk[k] / tot) : 0.f;
+  }
+  if (threadIdx.x == 0) {
+    if (loglik_out) *loglik_out = ll;
+    if (!ll_ok || !(tot > 0.0)) set_status(status, FGMM_ERR_NUMERIC);
+  }
+}
+
+// ------------------------------------------------------------------ soft assignment
+// One CTA per 64-point tile, one sweep over the components: log-densities, an online
+// log-sum-exp and a running top-m of log z (ranking by log z equals ranking by r,
+// exp being monotone), ties kept in component order.  Epilogue per §4.3.
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads)
+    soft_assign_simt_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp, int Kp,
+                            int K, const float* __restrict__ mu, const float* __restrict__ prec,
+                            const float* __restrict__ cconst, int top_m, float thr,
+                            int32_t* __restrict__ ids, float* __restrict__ resp) {
+  __shared__ __align__(16) float xs[kTP][kDC + 4];
+  __shared__ __align__(16) float ms[kKB][kDC + 4];
+  __shared__ __align__(16) float ps[kKB][kDC + 4];
+  __shared__ float ls[kTP][kKB + 1];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int64_t i0 = (int64_t)blockIdx.x * kTP;
+  float tv[FGMM_MAX_TOP_M];
+  int ti[FGMM_MAX_TOP_M];
+  int cnt = 0;
+  float m = -CUDART_INF_F, ssum = 0.f;
+  for (int kb = 0; kb < Kp; kb += kKB) {
+    float acc[4][4];
+    logit_tile<4>(X, n, ldx, D, Dp, i0, kb, mu, prec, xs, ms, ps, acc);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float cc = cconst[kb + tx + 16 * q];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) ls[ty + 16 * j][tx + 16 * q] = acc[j][q] + cc;
+    }
+    __syncthreads();
+    if (threadIdx.x < kTP) {
+      const int r = threadIdx.x;
+      const int kend = min(kKB, K - kb);
+      for (int c = 0; c < kend; ++c) {
+        const float l = ls[r][c];
+        const float nm = fmaxf(m, l);
+        if (nm > -CUDART_INF_F) {
+          ssum = ssum * expf(m - nm) + expf(l - nm);
+          m = nm;
+        }
+        if (cnt < top_m || l > tv[top_m - 1]) {
+          int p = (cnt < top_m) ? cnt : top_m - 1;
+          while (p > 0 && tv[p - 1] < l) { tv[p] = tv[p - 1]; ti[p] = ti[p - 1]; --p; }
+          tv[p] = l;
+          ti[p] = kb + c;
+          if (cnt < top_m) ++cnt;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x < kTP) {
+    const int64_t i = i0 + threadIdx.x;
+    if (i < n) {
+      const float lz = m + logf(ssum);
+      for (int rnk = 0; rnk < top_m; ++rnk) {
+        int id = -1;
+        float rv = 0.f;
+        if (rnk < cnt) {
+          const float rr = expf(tv[rnk] - lz);
+          if (rnk == 0 || rr > thr) { id = ti[rnk]; rv = rr; }
+        }
+        ids[i * top_m + rnk] = id;
+        if (resp) resp[i * top_m + rnk] = rv;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ launchers
+cudaError_t launch_prep_simt(const Ctx& c, const float* weights, const float* means,
+                             const float* vars, cudaStream_t s) {
+  prof_begin(c, KK_OTHER, s);
+  prep_simt_kernel<<<c.ws.Kp, kSimtThreads, 0, s>>>(c.K, c.D, c.ws.Kp, c.ws.Dp, c.cov, weights,
+                                                    means, vars, c.ws.mu, c.ws.prec,
+                                                    c.ws.cconst, c.ws.status);
+  prof_end(c, KK_OTHER, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lse_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                            float* logz_out, cudaStream_t s) {
+  const unsigned grid = (unsigned)ceil_div64(n, kTP);
+  prof_begin(c, KK_SWEEP1, s);
+  if (x_dtype == FGMM_BF16)
+    lse_simt_kernel<<<grid, kSimtThreads, 0, s>>>(
+        (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
+        c.ws.logz, logz_out, c.ws.ll_tiles);
+  else
+    lse_simt_kernel<<<grid, kSimtThreads, 0, s>>>((const float*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp,
+                                                  c.ws.mu, c.ws.prec, c.ws.cconst, c.ws.logz,
+                                                  logz_out, c.ws.ll_tiles);
+  prof_end(c, KK_SWEEP1, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ll_accumulate(const Ctx& c, int64_t n, cudaStream_t s) {
+  prof_begin(c, KK_OTHER, s);
+  ll_accumulate_kernel<<<1, kSimtThreads, 0, s>>>(c.ws.ll_tiles, (int)ceil_div64(n, kTP),
+                                                  c.ws.ll_total);
+  prof_end(c, KK_OTHER, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                              cudaStream_t s) {
+  const size_t smem = sizeof(StatsSmem);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(stats_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    cudaFuncSetAttribute(stats_simt_kernel<__nv_bfloat16>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attr_set = true;
+  }
+  int64_t slice = ceil_div64(n, kSlices);
+  slice = ceil_div64(slice, kTP) * kTP;
+  dim3 grid(c.ws.Kp / kKBs, kSlices, (unsigned)ceil_div64(c.ws.Dp, kFC));
+  prof_begin(c, KK_SWEEP2, s);
+  if (x_dtype == FGMM_BF16)
+    stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>(
+        (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
+        c.ws.logz, c.ws.stats, slice);
+  else
+    stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>((const float*)X, n, ldx, c.D, c.ws.Dp,
+                                                       c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
+                                                       c.ws.logz, c.ws.stats, slice);
+  prof_end(c, KK_SWEEP2, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mstep(const Ctx& c, float* weights, float* means, float* vars,
+                         double* loglik_out, cudaStream_t s) {
+  prof_begin(c, KK_OTHER, s);
+  mstep_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, c.ws.Dp, c.ws.Kp, c.cov, c.reg,
+                                            c.ws.stats, c.ws.mu, c.ws.ll_total, means, vars,
+                                            c.ws.nk, c.ws.status);
+  prof_end(c, KK_OTHER, s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  prof_begin(c, KK_OTHER, s);
+  finalize_kernel<<<1, kSimtThreads, 0, s>>>(c.K, c.ws.nk, c.ws.ll_total, weights, loglik_out,
+                                             c.ws.status);
+  prof_end(c, KK_OTHER, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_soft_assign_simt(const Ctx& c, const void* X, int x_dtype, int64_t n,
+                                    int64_t ldx, int top_m, float r_threshold, int32_t* ids,
+                                    float* resp, cudaStream_t s) {
+  const unsigned grid = (unsigned)ceil_div64(n, kTP);
+  prof_begin(c, KK_OTHER, s);
+  if (x_dtype == FGMM_BF16)
+    soft_assign_simt_kernel<<<grid, kSimtThreads, 0, s>>>(
+        (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.K, c.ws.mu, c.ws.prec,
+        c.ws.cconst, top_m, r_threshold, ids, resp);
+  else
+    soft_assign_simt_kernel<<<grid, kSimtThreads, 0, s>>>(
+        (const float*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.K, c.ws.mu, c.ws.prec, c.ws.cconst,
+        top_m, r_threshold, ids, resp);
+  prof_end(c, KK_OTHER, s);
+  return cudaGetLastError();
+}
+
+}  // namespace fgmm

@@ -1,0 +1,158 @@
+"""``GMM``: a thin object over one fgmm handle (include/fgmm.h).
+
+All tensors are CUDA tensors on the handle's device; the current torch stream
+is the stream of every call.  Parameters are float32: weights [K], means [K, D],
+variances [K, D] (diagonal) or [K] (isotropic), updated in place by ``step``
+and ``fit``.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import LIB, check
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _x_args(X: torch.Tensor):
+    if X.dim() != 2 or not X.is_cuda:
+        raise ValueError("X must be a 2-D CUDA tensor")
+    if X.dtype == torch.float32:
+        dt = _lib.F32
+    elif X.dtype == torch.bfloat16:
+        dt = _lib.BF16
+    else:
+        raise TypeError("X must be float32 or bfloat16")
+    if X.stride(1) != 1:
+        raise ValueError("X rows must be contiguous")
+    return _ptr(X), dt, X.shape[0], X.stride(0)
+
+
+class GMM:
+    def __init__(self, K: int, D: int, cov_type: int = _lib.COV_DIAG, reg_covar: float = 1e-6,
+                 precision: int | None = None):
+        self.K, self.D, self.cov_type, self.reg_covar = K, D, cov_type, reg_covar
+        h = ctypes.c_void_p()
+        check(LIB.fgmm_create(K, D, cov_type, reg_covar, ctypes.byref(h)), "fgmm_create")
+        self._h = h
+        if precision is not None:
+            self.set_precision(precision)
+
+    # ---------------------------------------------------------------- lifecycle
+    def close(self):
+        if getattr(self, "_h", None):
+            LIB.fgmm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        self.close()
+
+    # ---------------------------------------------------------------- settings
+    def set_precision(self, prec: int):
+        check(LIB.fgmm_set_precision(self._h, prec), "fgmm_set_precision")
+
+    @property
+    def precision(self) -> int:
+        v = ctypes.c_int()
+        check(LIB.fgmm_get_precision(self._h, ctypes.byref(v)), "fgmm_get_precision")
+        return v.value
+
+    @property
+    def workspace_bytes(self) -> int:
+        v = ctypes.c_size_t()
+        check(LIB.fgmm_workspace_bytes(self._h, ctypes.byref(v)), "fgmm_workspace_bytes")
+        return v.value
+
+    # ---------------------------------------------------------------- parameters
+    def new_params(self, weights, means, variances, device="cuda"):
+        """Copy (weights, means, variances) into contiguous float32 CUDA tensors."""
+        w = torch.as_tensor(weights, dtype=torch.float32).to(device).contiguous()
+        m = torch.as_tensor(means, dtype=torch.float32).to(device).contiguous()
+        v = torch.as_tensor(variances, dtype=torch.float32).to(device).contiguous()
+        self._check_params(w, m, v)
+        return w, m, v
+
+    def _check_params(self, w, m, v):
+        K, D = self.K, self.D
+        want_v = (K,) if self.cov_type == _lib.COV_SPHERICAL else (K, D)
+        for t in (w, m, v):
+            if not (t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()):
+                raise ValueError("parameters must be contiguous float32 CUDA tensors")
+        if tuple(w.shape) != (K,) or tuple(m.shape) != (K, D) or tuple(v.shape) != want_v:
+            raise ValueError("parameter shapes do not match (K, D, cov_type)")
+
+    # ---------------------------------------------------------------- EM
+    def step(self, X, weights, means, variances, loglik=None, logz=None):
+        """One fused EM iteration; updates the parameters in place.
+
+        loglik: optional CUDA float64 tensor [1] receiving log p(X | Θ_in).
+        logz:   optional CUDA float32 tensor [N] receiving per-point log p(x_i | Θ_in).
+        """
+        self._check_params(weights, means, variances)
+        xp, dt, n, ldx = _x_args(X)
+        if loglik is not None and not (loglik.is_cuda and loglik.dtype == torch.float64):
+            raise ValueError("loglik must be a CUDA float64 tensor")
+        if logz is not None and not (logz.is_cuda and logz.dtype == torch.float32
+                                     and logz.numel() >= n):
+            raise ValueError("logz must be a CUDA float32 tensor with N elements")
+        check(LIB.fgmm_em_step(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means),
+                               _ptr(variances), _ptr(loglik), _ptr(logz), _stream()),
+              "fgmm_em_step")
+
+    def fit(self, X, weights, means, variances, max_iters=100, tol=0.0):
+        """Repeat step up to max_iters times; returns (final_loglik, iters_done)."""
+        self._check_params(weights, means, variances)
+        xp, dt, n, ldx = _x_args(X)
+        ll = ctypes.c_double()
+        it = ctypes.c_int()
+        check(LIB.fgmm_fit(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means),
+                           _ptr(variances), max_iters, tol, ctypes.byref(ll),
+                           ctypes.byref(it), _stream()), "fgmm_fit")
+        return ll.value, it.value
+
+    def soft_assign(self, X, weights, means, variances, top_m=2, r_threshold=0.0,
+                    ids=None, resp=None):
+        """§4.3 multi-assignment; returns (ids int32 [N, top_m], resp float32 [N, top_m])."""
+        self._check_params(weights, means, variances)
+        xp, dt, n, ldx = _x_args(X)
+        if ids is None:
+            ids = torch.empty(n, top_m, dtype=torch.int32, device=X.device)
+        if resp is None:
+            resp = torch.empty(n, top_m, dtype=torch.float32, device=X.device)
+        check(LIB.fgmm_soft_assign(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means),
+                                   _ptr(variances), top_m, r_threshold, _ptr(ids), _ptr(resp),
+                                   _stream()), "fgmm_soft_assign")
+        return ids, resp
+
+    def profile(self, enable: bool = True):
+        check(LIB.fgmm_profile_enable(self._h, int(enable)), "fgmm_profile_enable")
+
+    def profile_read(self, reset: bool = True) -> dict:
+        p = _lib.Profile()
+        check(LIB.fgmm_profile_read(self._h, ctypes.byref(p), int(reset)), "fgmm_profile_read")
+        return {f: getattr(p, f) for f, _ in _lib.Profile._fields_}
+
+    def status(self) -> int:
+        """Synchronise and return (then clear) the device status word."""
+        return LIB.fgmm_get_status(self._h, _stream())
+
+    def check_status(self):
+        check(self.status(), "device status")

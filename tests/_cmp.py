@@ -1,0 +1,67 @@
+"""Comparison helpers for GPU-vs-oracle parity tests (tolerances from the spec of
+the fused EM step: per-point log-likelihood relative error <= 1e-4, post-step
+means / variances relative error <= 1e-3 in fp32-class modes)."""
+import numpy as np
+
+LOGZ_RTOL = 1e-4
+PARAM_RTOL = 1e-3
+# components whose responsibility mass is below one effective point are compared
+# only for validity: their M-step rests on far-tail responsibilities
+MIN_NK_COMPARED = 1.0
+
+
+def rel_err(a, b, floor=0.0):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return np.abs(a - b) / np.maximum(np.abs(b), floor)
+
+
+def compare_step(gpu, ref, X, cov_spherical=False, logz_gpu=None, loglik_gpu=None,
+                 param_rtol=PARAM_RTOL, logz_rtol=LOGZ_RTOL):
+    """gpu = (w, mu, var) numpy; ref = oracle StepResult. Returns a dict of max errors
+    and asserts the tolerances."""
+    w, mu, var = (np.asarray(t, np.float64) for t in gpu)
+    out = {}
+    X = np.asarray(X, np.float64)
+    scale = np.maximum(X.std(axis=0), 1e-30)
+    cmp = ref.Nk >= MIN_NK_COMPARED
+    assert np.all(np.isfinite(w)) and np.all(np.isfinite(mu)) and np.all(np.isfinite(var))
+    assert np.all(var > 0)
+    if logz_gpu is not None:
+        e = rel_err(logz_gpu, ref.logZ, floor=1e-30)
+        out["logz"] = float(e.max())
+        assert out["logz"] <= logz_rtol, out
+    if loglik_gpu is not None:
+        out["loglik"] = float(abs(loglik_gpu - ref.loglik) / abs(ref.loglik))
+        assert out["loglik"] <= logz_rtol, out
+    # empty decisions agree wherever N_k is far from the threshold
+    far = (ref.Nk < 1e-2 * 1e-6) | (ref.Nk > 1e2 * 1e-6)
+    assert np.array_equal((w == 0)[far], ref.empty[far]), "empty-component decision differs"
+    if cmp.any():
+        out["weights"] = float(rel_err(w[cmp], ref.weights[cmp]).max())
+        # relative to max(|mu|, per-dim data std): a mean near 0 is judged on the data's scale
+        out["means"] = float((np.abs(mu[cmp] - ref.means[cmp]) /
+                              np.maximum(np.abs(ref.means[cmp]), scale[None, :])).max())
+        vref = ref.variances[cmp]
+        out["vars"] = float(rel_err(var[cmp], vref).max())
+        assert out["weights"] <= param_rtol, out
+        assert out["means"] <= param_rtol, out
+        assert out["vars"] <= param_rtol, out
+    return out
+
+
+def ids_match_where_decisive(ids_gpu, ids_ref, resp_ref, R_full, thr, gap=1e-3):
+    """Soft-assign ids must be bit-exact wherever the decision is not within `gap`:
+    adjacent sorted responsibilities differ by > gap and |r - thr| > gap."""
+    ids_gpu = np.asarray(ids_gpu)
+    ids_ref = np.asarray(ids_ref)
+    m = ids_ref.shape[1]
+    Rs = -np.sort(-R_full, axis=1)
+    N, K = R_full.shape
+    decisive = np.ones(N, dtype=bool)
+    for j in range(min(m, K - 1)):
+        decisive &= (Rs[:, j] - Rs[:, j + 1]) > gap
+    for j in range(1, min(m, K)):
+        decisive &= np.abs(Rs[:, j] - thr) > gap
+    bad = np.nonzero(decisive & np.any(ids_gpu != ids_ref, axis=1))[0]
+    return decisive, bad

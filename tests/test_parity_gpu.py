@@ -1,0 +1,274 @@
+"""GPU parity: the CUDA EM step, fit and soft-assignment against the fp64 oracle
+on the same seeded inputs, through the C-ABI (via the ctypes binding).
+
+Sizes are small enough for the oracle to finish in seconds but span several
+tiles, several component blocks, ragged tails and the chunk boundary.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import gmm_oracle as O
+from tests._cmp import compare_step, ids_match_where_decisive
+
+pytestmark = pytest.mark.gpu
+
+PRECISIONS = ["fp32"]
+
+
+def _gmm(K, D, cov=0, reg=1e-6, prec="fp32"):
+    import ivf_quantizer_b200 as q
+    g = q.GMM(K, D, cov, reg)
+    g.set_precision({"fp32": q.PREC_FP32, "fp16x3": q.PREC_FP16X3, "auto": q.PREC_AUTO}[prec])
+    return g
+
+
+def _run_step(X, w, mu, var, cov=0, reg=1e-6, prec="fp32"):
+    K, D = mu.shape
+    g = _gmm(K, D, cov, reg, prec)
+    Xd = torch.as_tensor(X).cuda().contiguous()
+    wd, md, vd = g.new_params(w, mu, var)
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    lz = torch.empty(Xd.shape[0], dtype=torch.float32, device="cuda")
+    g.step(Xd, wd, md, vd, loglik=ll, logz=lz)
+    torch.cuda.synchronize()
+    assert g.status() == 0
+    out = (wd.cpu().numpy(), md.cpu().numpy(), vd.cpu().numpy(), float(ll.item()), lz.cpu().numpy())
+    g.close()
+    return out
+
+
+def _check(X, w, mu, var, cov=0, reg=1e-6, prec="fp32"):
+    Xf = X.float() if X.dtype != torch.bfloat16 else X
+    gw, gm, gv, gll, glz = _run_step(Xf, w, mu, var, cov, reg, prec)
+    ref = O.em_step(Xf.double().numpy() if Xf.dtype != torch.bfloat16 else Xf.float().double().numpy(),
+                    np.asarray(w, np.float64), np.asarray(mu, np.float64),
+                    np.asarray(var, np.float64), cov, reg)
+    return compare_step((gw, gm, gv), ref, Xf.float().numpy(), logz_gpu=glz, loglik_gpu=gll)
+
+
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_c1_first_step(prec):
+    X = synth.generate("c1", 10_000, seed=0)
+    w, mu, var = synth.init_params(X, 16, seed=0)
+    print(_check(X, w, mu, var, prec=prec))
+
+
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_c1_fit_trajectory(prec):
+    """Free-running 10 iterations on the small D=16, K=16 workload: per-iteration
+    log-likelihood and final parameters against the oracle's own trajectory."""
+    import ivf_quantizer_b200 as q
+    X = synth.generate("c1", 10_000, seed=1)
+    w, mu, var = synth.init_params(X, 16, seed=1)
+    g = _gmm(16, 16, prec=prec)
+    Xd = X.cuda()
+    wd, md, vd = g.new_params(w, mu, var)
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    lls = []
+    for _ in range(10):
+        g.step(Xd, wd, md, vd, loglik=ll)
+        lls.append(ll.item())
+    assert g.status() == 0
+    rw, rm, rv, rlls, _ = O.fit(X.double().numpy(), w.double().numpy(), mu.double().numpy(),
+                                var.double().numpy(), 0, 1e-6, max_iters=10)
+    np.testing.assert_allclose(lls, rlls, rtol=1e-5)
+    np.testing.assert_allclose(md.cpu().numpy(), rm, rtol=1e-3, atol=1e-3)
+    np.testing.assert_allclose(vd.cpu().numpy(), rv, rtol=1e-3)
+    # fit() through the ABI gives the same result as repeated steps
+    wd2, md2, vd2 = g.new_params(w, mu, var)
+    fll, it = g.fit(Xd, wd2, md2, vd2, max_iters=10, tol=0.0)
+    assert it == 10
+    assert torch.equal(md2, md) and torch.equal(vd2, vd) and torch.equal(wd2, wd)
+    assert fll == pytest.approx(lls[-1], rel=1e-12)
+
+
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_table1_shape_first_step(prec):
+    """D=128, K=256 slice of the Table-1 generator, N=3000 (ragged vs 64)."""
+    X = synth.generate("table1", 3000, seed=2)
+    w, mu, var = synth.init_params(X, 256, seed=2)
+    print(_check(X, w, mu, var, prec=prec))
+
+
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_table1_teacher_forced_late_iteration(prec):
+    """Run 8 GPU iterations, then check one step from the GPU's own Θ_8 (teacher
+    forcing: both sides start from the same parameters)."""
+    X = synth.generate("table1", 2500, seed=3)
+    w, mu, var = synth.init_params(X, 192, seed=3)
+    g = _gmm(192, 128, prec=prec)
+    Xd = X.cuda()
+    wd, md, vd = g.new_params(w, mu, var)
+    for _ in range(8):
+        g.step(Xd, wd, md, vd)
+    assert g.status() == 0
+    print(_check(X, wd.cpu().numpy(), md.cpu().numpy(), vd.cpu().numpy(), prec=prec))
+
+
+@pytest.mark.parametrize("N,D,K", [(1, 1, 1), (5, 3, 2), (63, 7, 5), (65, 33, 65), (130, 130, 3),
+                                   (200, 1, 70), (777, 100, 100), (300, 260, 9)])
+@pytest.mark.parametrize("cov", [0, 1])
+def test_edge_shapes(N, D, K, cov):
+    X = synth.uniform_points(N, D, seed=N + D + K, lo=-3, hi=3)
+    g = torch.Generator().manual_seed(N * 31 + K)
+    mu = X[torch.randint(0, N, (K,), generator=g)] + 0.3 * torch.randn(K, D, generator=g)
+    w = torch.rand(K, generator=g) + 0.2
+    w = w / w.sum()
+    var = (torch.rand(K, generator=g) + 0.5) if cov == 1 else (torch.rand(K, D, generator=g) + 0.5)
+    _check(X, w.numpy(), mu.numpy(), var.numpy(), cov=cov, reg=1e-4)
+
+
+def test_k1_closed_form_on_gpu():
+    """K = 1: one step returns the sample mean and the population variance (+ floor)."""
+    X = synth.uniform_points(1000, 20, seed=5, lo=-2, hi=4)
+    gw, gm, gv, gll, _ = _run_step(X, np.ones(1), np.zeros((1, 20)), np.ones((1, 20)), reg=1e-3)
+    Xn = X.double().numpy()
+    np.testing.assert_allclose(gw, [1.0], rtol=1e-7)
+    np.testing.assert_allclose(gm[0], Xn.mean(0), rtol=1e-5, atol=1e-5)
+    np.testing.assert_allclose(gv[0], Xn.var(0) + 1e-3, rtol=1e-5)
+
+
+def test_dead_and_duplicate_components():
+    X = synth.uniform_points(500, 4, seed=6)
+    mu = np.array([[0, 0, 0, 0], [0.5, 0.5, 0.5, 0.5], [0.5, 0.5, 0.5, 0.5], [1e4] * 4], float)
+    var = np.ones((4, 4))
+    w = np.array([0.3, 0.3, 0.3, 0.1])
+    gw, gm, gv, _, _ = _run_step(X, w, mu, var)
+    assert gw[3] == 0.0
+    np.testing.assert_array_equal(gm[3], mu[3].astype(np.float32))
+    np.testing.assert_array_equal(gv[3], var[3].astype(np.float32))
+    # duplicates stay identical and share the mass
+    np.testing.assert_array_equal(gm[1], gm[2])
+    assert gw[1] == gw[2]
+    _check(X, w, mu, var)
+
+
+def test_zero_weight_component_is_excluded():
+    X = synth.uniform_points(300, 3, seed=7)
+    mu = np.array([[0, 0, 0], [0.2, 0.2, 0.2]], float)
+    gw, gm, gv, _, _ = _run_step(X, np.array([1.0, 0.0]), mu, np.ones((2, 3)))
+    assert gw[1] == 0.0 and gw[0] == 1.0
+    np.testing.assert_allclose(gm[0], X.double().numpy().mean(0), rtol=1e-5, atol=1e-6)
+
+
+def test_bf16_input():
+    """bf16 X: the oracle consumes the same rounded values."""
+    X = synth.generate("c1", 4000, seed=8).to(torch.bfloat16)
+    w, mu, var = synth.init_params(X.float(), 16, seed=8)
+    K, D = mu.shape
+    g = _gmm(K, D)
+    Xd = X.cuda()
+    wd, md, vd = g.new_params(w, mu, var)
+    lz = torch.empty(4000, device="cuda")
+    g.step(Xd, wd, md, vd, logz=lz)
+    assert g.status() == 0
+    ref = O.em_step(X.float().double().numpy(), w.double().numpy(), mu.double().numpy(),
+                    var.double().numpy())
+    compare_step((wd.cpu().numpy(), md.cpu().numpy(), vd.cpu().numpy()), ref,
+                 X.float().numpy(), logz_gpu=lz.cpu().numpy())
+
+
+def test_strided_rows():
+    """ldx > D: X is a column slice of a wider matrix."""
+    W = synth.uniform_points(700, 40, seed=9)
+    X = W[:, :24]
+    g = torch.Generator().manual_seed(1)
+    mu = X[torch.randperm(700, generator=g)[:10]]
+    Xd = W.cuda()[:, :24]
+    gg = _gmm(10, 24)
+    wd, md, vd = gg.new_params(torch.full((10,), 0.1), mu, torch.ones(10, 24))
+    lz = torch.empty(700, device="cuda")
+    gg.step(Xd, wd, md, vd, logz=lz)
+    assert gg.status() == 0
+    ref = O.em_step(X.double().numpy(), np.full(10, 0.1), mu.double().numpy(), np.ones((10, 24)))
+    compare_step((wd.cpu().numpy(), md.cpu().numpy(), vd.cpu().numpy()), ref, X.numpy(),
+                 logz_gpu=lz.cpu().numpy())
+
+
+def test_chunk_boundary():
+    """N crosses the 2^20-point chunk of the library: statistics accumulate across chunks."""
+    N = (1 << 20) + 4099
+    X = synth.generate("c1", N, seed=10)
+    w, mu, var = synth.init_params(X, 16, seed=10)
+    print(_check(X, w, mu, var))
+
+
+def test_deterministic_bitwise():
+    X = synth.generate("table1", 3000, seed=11)
+    w, mu, var = synth.init_params(X, 128, seed=11)
+    a = _run_step(X, w, mu, var)
+    b = _run_step(X, w, mu, var)
+    for x, y in zip(a, b):
+        assert np.array_equal(np.asarray(x), np.asarray(y))
+
+
+def test_workspace_independent_of_n():
+    import ivf_quantizer_b200 as q
+    X = synth.generate("c1", 200_000, seed=12).cuda()
+    w, mu, var = synth.init_params(X.cpu(), 16, seed=12)
+    g = q.GMM(16, 16)
+    wd, md, vd = g.new_params(w, mu, var)
+    g.step(X[:1000], wd, md, vd)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    g.step(X, wd, md, vd)
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
+    assert free0 == free1
+    assert g.status() == 0
+
+
+def test_invalid_parameters_latch_status():
+    import ivf_quantizer_b200 as q
+    X = synth.uniform_points(100, 3, seed=13).cuda()
+    g = q.GMM(2, 3)
+    wd, md, vd = g.new_params([0.5, 0.5], [[0, 0, 0], [1, 1, 1]], [[1, 1, 1], [1, -1, 1]])
+    g.step(X, wd, md, vd)
+    assert g.status() == q._lib.ERR_INVALID_ARG
+    assert g.status() == 0  # cleared
+    wd, md, vd = g.new_params([0.0, 0.0], [[0, 0, 0], [1, 1, 1]], [[1, 1, 1], [1, 1, 1]])
+    g.step(X, wd, md, vd)
+    assert g.status() == q._lib.ERR_NUMERIC
+    # parameters are left untouched on a numeric failure
+    assert torch.equal(md.cpu(), torch.tensor([[0., 0, 0], [1, 1, 1]]))
+
+
+@pytest.mark.parametrize("top_m,thr", [(1, 0.0), (2, 1.0 / 64), (2, 0.1), (5, 0.0)])
+def test_soft_assign(top_m, thr):
+    X = synth.generate("table1", 2000, seed=14)
+    w, mu, var = synth.init_params(X, 64, seed=14)
+    var = var * 4.0  # broad components: many points have several responsible clusters
+    import ivf_quantizer_b200 as q
+    g = q.GMM(64, 128)
+    wd, md, vd = g.new_params(w, mu, var)
+    ids, resp = g.soft_assign(X.cuda(), wd, md, vd, top_m=top_m, r_threshold=thr)
+    torch.cuda.synchronize()
+    rid, rresp = O.soft_assign(X.double().numpy(), w.double().numpy(), mu.double().numpy(),
+                               var.double().numpy(), 0, top_m, thr)
+    _, R = O.e_step(X.double().numpy(), w.double().numpy(), mu.double().numpy(),
+                    var.double().numpy())
+    decisive, bad = ids_match_where_decisive(ids.cpu().numpy(), rid, rresp, R, thr)
+    assert decisive.mean() > 0.5
+    assert len(bad) == 0, bad[:10]
+    gr = resp.cpu().numpy()
+    ok = decisive[:, None] & (rid >= 0)
+    np.testing.assert_allclose(gr[ok], rresp[ok], rtol=1e-4, atol=1e-7)
+    assert np.all(ids.cpu().numpy()[:, 0] >= 0)
+
+
+def test_soft_assign_spherical_and_argmax():
+    import ivf_quantizer_b200 as q
+    X = synth.generate("c1", 5000, seed=15)
+    w, mu, var = synth.init_params(X, 16, seed=15)
+    vs = torch.full((16,), 1.5)
+    g = q.GMM(16, 16, q.COV_SPHERICAL)
+    wd, md, vd = g.new_params(w, mu, vs)
+    ids, resp = g.soft_assign(X.cuda(), wd, md, vd, top_m=1)
+    _, R = O.e_step(X.double().numpy(), w.double().numpy(), mu.double().numpy(),
+                    vs.double().numpy(), O.COV_SPHERICAL)
+    arg = np.argmax(R, 1)
+    Rs = -np.sort(-R, 1)
+    dec = (Rs[:, 0] - Rs[:, 1]) > 1e-3
+    assert np.array_equal(ids.cpu().numpy()[dec, 0], arg[dec])
