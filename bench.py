@@ -249,7 +249,7 @@ def main():
         g.set_precision(prec)
     except q.FgmmError:
         g.set_precision(q.PREC_FP32)
-    prec_used = {q.PREC_FP32: "fp32", q.PREC_FP16X3: "fp16x3", q.PREC_AUTO: "auto"}[g.precision]
+    prec_set = {q.PREC_FP32: "fp32", q.PREC_FP16X3: "fp16x3", q.PREC_AUTO: "auto"}[g.precision]
     wd, md, vd = g.new_params(wt, mu, var)
     ll = torch.zeros(1, dtype=torch.float64, device=dev)
 
@@ -258,6 +258,7 @@ def main():
     torch.cuda.synchronize()
     g.check_status()
     barrier()
+    paths = set()
 
     sampler = ClockSampler(gpu_id_for(local))
     sampler.start()
@@ -273,6 +274,8 @@ def main():
     for _ in range(args.steps):
         g.step(X, wd, md, vd, loglik=ll)
     t1.record(stream)
+    torch.cuda.synchronize()
+    paths.add(g.last_step_path())
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
@@ -295,6 +298,9 @@ def main():
     pts_per_launch = N * args.steps / max(1, launches)
     flops_per_launch = 4.0 * D * K * pts_per_launch     # each sweep: 4*D flops per (point, comp)
     achieved = flops_per_launch / (avg_ms / 1e3) / 1e12
+    # the path the timed steps ran (AUTO decides per step on the device; the timed
+    # region's last step is representative once warm-up has passed)
+    prec_used = "fp16x3" if paths == {q.PREC_FP16X3} else "fp32"
     if prec_used == "fp32":
         clk = float(peaks.get("sm_max_mhz", 1965.0))
         peak = 148 * 128 * 2 * clk * 1e6 / 1e12
@@ -303,7 +309,9 @@ def main():
     else:
         peak = float(peaks["bf16_tflops_sustained"])
         roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_note":
-                f"fp16 dense = bf16 {peak_src} sustained"}
+                f"fp16 dense peak = bf16 dense, {peak_src}, sustained; algorithmic flops "
+                f"(4*D per point-component per sweep), the three-product split and the "
+                f"recompute are not counted"}
     traffic = recorded_traffic(dom, prec_used)
     roof.update({"kernel": dom, "achieved": achieved, "peak": peak, "frac": achieved / peak,
                  "traffic": traffic, "peak_source": peak_src,
@@ -360,6 +368,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": workload_name(w), "precision": prec_used,
+                       "precision_setting": prec_set,
                        "l2": f"inputs larger than L2 (X = {N * D * 4 / 1e9:.1f} GB per GPU)"
                        if N * D * 4 > 126e6 else "inputs smaller than L2",
                        "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},

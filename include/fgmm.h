@@ -92,6 +92,11 @@ int fgmm_destroy(fgmm_handle h);
 int fgmm_set_precision(fgmm_handle h, int prec);
 int fgmm_get_precision(fgmm_handle h, int* prec_out);
 
+/* Path the last fgmm_em_step of this handle ran: FGMM_PREC_FP32 (CUDA cores) or
+ * FGMM_PREC_FP16X3 (tensor cores).  Under FGMM_PREC_AUTO the choice is made on the
+ * device per step, so this call synchronises the device.  -1 before any step. */
+int fgmm_last_step_path(fgmm_handle h, int* path_out);
+
 /* Bytes of device memory the handle holds (independent of N). */
 int fgmm_workspace_bytes(fgmm_handle h, size_t* bytes_out);
 

@@ -35,6 +35,7 @@ SIGNATURES = {
     "fgmm_set_precision": (_int, [_vp, _int]),
     "fgmm_get_precision": (_int, [_vp, _c.POINTER(_int)]),
     "fgmm_workspace_bytes": (_int, [_vp, _c.POINTER(_c.c_size_t)]),
+    "fgmm_last_step_path": (_int, [_vp, _c.POINTER(_int)]),
     "fgmm_em_step": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_fit": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _int, _dbl,
                         _c.POINTER(_dbl), _c.POINTER(_int), _vp]),

@@ -33,7 +33,7 @@ def sources():
 
 def build(verbose: bool = False, out: str = OUT) -> str:
     cmd = [nvcc_path(), *ARCH, *FLAGS, "-I", os.path.join(HERE, "..", "include"),
-           *sources(), "-o", out + ".tmp", "-lcuda"]
+           *sources(), "-o", out + ".tmp"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     log = r.stdout + r.stderr
     with open(os.path.join(HERE, "_build_ptxas.log"), "w") as f:

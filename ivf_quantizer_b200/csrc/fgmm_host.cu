@@ -90,7 +90,8 @@ int map_cuda(cudaError_t e) {
 }
 
 void free_ws(Workspace& w) {
-  void* ptrs[] = {w.mu, w.prec, w.cconst, w.logz, w.ll_tiles, w.ll_total, w.stats, w.nk, w.status};
+  void* ptrs[] = {w.mu,   w.prec,   w.cconst, w.logz, w.ll_tiles, w.ll_total, w.stats, w.nk,
+                  w.status, w.center, w.dscale, w.wop, w.tck,     w.tks,      w.xop,   w.mode};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -102,10 +103,22 @@ cudaError_t alloc(T** p, size_t count, size_t* total) {
   return cudaMalloc((void**)p, count * sizeof(T));
 }
 
+size_t stats_bytes(const Workspace& w) {
+  return (size_t)w.slots * w.KpS * (1 + 2 * (size_t)w.Dp) * sizeof(double);
+}
+
 cudaError_t alloc_ws(Ctx& c) {
   Workspace& w = c.ws;
   w.Kp = round_up(c.K, kKB);
   w.Dp = round_up(c.D, kDC);
+  w.KpS = round_up(c.K, 128);
+  w.Kt = w.KpS;
+  w.Dq = w.Dp;
+  w.K1 = 2 * w.Dq;
+  const bool tc = tc_supported(c);
+  int s_tc = c.num_sms / (w.Kt / 128);
+  if (s_tc < 1) s_tc = 1;
+  w.slots = tc && s_tc > kSlices ? s_tc : kSlices;
   size_t t = 0;
   cudaError_t e;
   const size_t kd = (size_t)w.Kp * w.Dp;
@@ -113,14 +126,29 @@ cudaError_t alloc_ws(Ctx& c) {
   if ((e = alloc(&w.prec, kd, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.cconst, (size_t)w.Kp, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.logz, (size_t)kChunk, &t)) != cudaSuccess) return e;
-  if ((e = alloc(&w.ll_tiles, (size_t)(kChunk / kTP), &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.ll_tiles, (size_t)(kChunk / 32), &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.ll_total, (size_t)1, &t)) != cudaSuccess) return e;
-  if ((e = alloc(&w.stats, (size_t)kSlices * w.Kp * (1 + 2 * (size_t)w.Dp), &t)) != cudaSuccess)
-    return e;
-  if ((e = alloc(&w.nk, (size_t)w.Kp, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.stats, stats_bytes(w) / sizeof(double), &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.nk, (size_t)w.KpS, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.status, (size_t)1, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.mode, (size_t)1, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.center, (size_t)w.Dq, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.dscale, (size_t)w.Dq, &t)) != cudaSuccess) return e;
   if ((e = cudaMemset(w.status, 0, sizeof(int))) != cudaSuccess) return e;
+  if ((e = cudaMemset(w.center, 0, w.Dq * sizeof(float))) != cudaSuccess) return e;
+  if ((e = cudaMemset(w.dscale, 0, w.Dq * sizeof(float))) != cudaSuccess) return e;
+  if (tc) {
+    if ((e = alloc(&w.wop, (size_t)2 * w.Kt * w.K1, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.tck, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.tks, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.xop, (size_t)2 * kChunk * w.K1, &t)) != cudaSuccess) return e;
+    // rows past the end of a short chunk are read by the tensor cores (and multiplied
+    // by r = 0): keep them finite from the start
+    if ((e = cudaMemset(w.xop, 0, (size_t)2 * kChunk * w.K1 * sizeof(__half))) != cudaSuccess)
+      return e;
+  }
   w.bytes = t;
+  if (tc && (e = tc_init(c)) != cudaSuccess) return e;
   return cudaSuccess;
 }
 
@@ -192,7 +220,8 @@ int fgmm_set_precision(fgmm_handle h, int prec) {
   if (prec != FGMM_PREC_FP32 && prec != FGMM_PREC_FP16X3 && prec != FGMM_PREC_FP16 &&
       prec != FGMM_PREC_AUTO)
     return FGMM_ERR_INVALID_ARG;
-  if (prec == FGMM_PREC_FP16X3 || prec == FGMM_PREC_FP16) return FGMM_ERR_UNSUPPORTED;
+  if (prec == FGMM_PREC_FP16) return FGMM_ERR_UNSUPPORTED;
+  if (prec == FGMM_PREC_FP16X3 && !h->c.tc.ready) return FGMM_ERR_UNSUPPORTED;
   h->c.prec = prec;
   return FGMM_OK;
 }
@@ -215,28 +244,66 @@ int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t l
   int rc = check_x(h, X, x_dtype, N, ldx);
   if (rc) return rc;
   if (!weights || !means || !vars) return FGMM_ERR_INVALID_ARG;
-  const Ctx& c = h->c;
+  Ctx& c = h->c;
   if ((rc = set_device(c))) return rc;
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
   const Workspace& w = c.ws;
+  // which path(s) to enqueue: FP32 -> CUDA cores; FP16X3 -> tensor cores; AUTO ->
+  // both, each kernel returning at once unless the device-side mode word (set by the
+  // tensor-core preparation's conditioning check) selects its path
+  const bool auto_mode = c.prec == FGMM_PREC_AUTO && c.tc.ready;
+  const bool run_tc = (c.prec == FGMM_PREC_FP16X3 || auto_mode) && c.tc.ready;
+  const bool run_simt = c.prec == FGMM_PREC_FP32 || !c.tc.ready || auto_mode;
+  const int fixed_mode = run_tc && !run_simt ? kModeTensor : kModeSimt;
+  const int* mode = auto_mode ? w.mode : nullptr;
+  if (run_tc && x_dtype == FGMM_F32 && ((uintptr_t)X % 4 != 0)) return FGMM_ERR_INVALID_ARG;
   if ((e = cudaMemsetAsync(w.ll_total, 0, sizeof(double), s)) != cudaSuccess) return map_cuda(e);
-  if ((e = cudaMemsetAsync(w.stats, 0, (size_t)kSlices * w.Kp * (1 + 2 * (size_t)w.Dp) * 8, s)) !=
-      cudaSuccess)
+  if ((e = cudaMemsetAsync(w.stats, 0, stats_bytes(w), s)) != cudaSuccess) return map_cuda(e);
+  if (auto_mode && (e = cudaMemsetAsync(w.mode, 0, sizeof(int), s)) != cudaSuccess)
     return map_cuda(e);
-  if ((e = launch_prep_simt(c, weights, means, vars, s)) != cudaSuccess) return map_cuda(e);
+  if (run_simt && (e = launch_prep_simt(c, weights, means, vars, s)) != cudaSuccess)
+    return map_cuda(e);
+  if (run_tc && (e = launch_tc_prep(c, weights, means, vars, auto_mode ? w.mode : nullptr, s)) !=
+                    cudaSuccess)
+    return map_cuda(e);
   const size_t eb = dtype_bytes(x_dtype);
   for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
     const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
     const void* Xc = (const char*)X + (size_t)c0 * ldx * eb;
-    if ((e = launch_lse_simt(c, Xc, x_dtype, nc, ldx, logz_out ? logz_out + c0 : nullptr, s)) !=
-        cudaSuccess)
+    float* lzo = logz_out ? logz_out + c0 : nullptr;
+    if (run_tc) {
+      if ((e = launch_tc_convert(c, Xc, x_dtype, nc, ldx, mode, s)) != cudaSuccess)
+        return map_cuda(e);
+      if ((e = launch_tc_lse(c, nc, lzo, mode, s)) != cudaSuccess) return map_cuda(e);
+    }
+    if (run_simt && (e = launch_lse_simt(c, Xc, x_dtype, nc, ldx, lzo, mode, s)) != cudaSuccess)
       return map_cuda(e);
-    if ((e = launch_ll_accumulate(c, nc, s)) != cudaSuccess) return map_cuda(e);
-    if ((e = launch_stats_simt(c, Xc, x_dtype, nc, ldx, s)) != cudaSuccess) return map_cuda(e);
+    if ((e = launch_ll_accumulate(c, nc, mode, fixed_mode, s)) != cudaSuccess) return map_cuda(e);
+    if (run_tc && (e = launch_tc_stats(c, nc, mode, s)) != cudaSuccess) return map_cuda(e);
+    if (run_simt && (e = launch_stats_simt(c, Xc, x_dtype, nc, ldx, mode, s)) != cudaSuccess)
+      return map_cuda(e);
   }
-  if ((e = launch_mstep(c, weights, means, vars, loglik_out, s)) != cudaSuccess)
+  if ((e = launch_mstep(c, weights, means, vars, loglik_out, mode, fixed_mode, s)) != cudaSuccess)
     return map_cuda(e);
+  h->c.last_auto = auto_mode;
+  h->c.last_path = fixed_mode == kModeTensor ? FGMM_PREC_FP16X3 : FGMM_PREC_FP32;
+  return FGMM_OK;
+}
+
+int fgmm_last_step_path(fgmm_handle h, int* path_out) {
+  if (!h || !path_out) return FGMM_ERR_INVALID_ARG;
+  if (!h->c.last_auto) {
+    *path_out = h->c.last_path;
+    return FGMM_OK;
+  }
+  int rc = set_device(h->c);
+  if (rc) return rc;
+  int m = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&m, h->c.ws.mode, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return map_cuda(e);
+  *path_out = m == kModeTensor ? FGMM_PREC_FP16X3 : FGMM_PREC_FP32;
   return FGMM_OK;
 }
 

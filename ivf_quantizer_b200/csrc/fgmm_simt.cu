@@ -16,7 +16,7 @@
 //
 // Data layout: prepared parameters are zero padded to [Kp, Dp] (Kp multiple of
 // 64, Dp multiple of 32); padded / dead components carry cconst = -inf so that
-// they contribute exp(-inf) = 0.  Statistics partials live in [kSlices][Kp][1+2Dp]
+// they contribute exp(-inf) = 0.  Statistics partials live in [slots][KpS][1+2Dp]
 // fp64 slots, each written by exactly one CTA, summed in a fixed order by the
 // M-step kernel: the result is bitwise reproducible.
 #include <cuda_bf16.h>
@@ -136,7 +136,9 @@ __global__ void __launch_bounds__(kSimtThreads)
     lse_simt_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp, int Kp,
                     const float* __restrict__ mu, const float* __restrict__ prec,
                     const float* __restrict__ cconst, float* __restrict__ logz,
-                    float* __restrict__ logz_out, double* __restrict__ ll_tiles) {
+                    float* __restrict__ logz_out, double* __restrict__ ll_tiles,
+                    const int* mode) {
+  if (mode && *mode != kModeSimt) return;
   __shared__ __align__(16) float xs[kTP][kDC + 4];
   __shared__ __align__(16) float ms[kKB][kDC + 4];
   __shared__ __align__(16) float ps[kKB][kDC + 4];
@@ -194,9 +196,11 @@ __global__ void __launch_bounds__(kSimtThreads)
 }
 
 // Adds the chunk's per-tile partial log-likelihoods, in tile order, to ll_total.
-__global__ void ll_accumulate_kernel(const double* __restrict__ ll_tiles, int ntiles,
+__global__ void ll_accumulate_kernel(const double* __restrict__ ll_tiles, int n_simt, int n_tc,
+                                     const int* mode, int fixed_mode,
                                      double* __restrict__ ll_total) {
   __shared__ double red[kSimtThreads];
+  const int ntiles = ((mode ? *mode : fixed_mode) == kModeSimt) ? n_simt : n_tc;
   double s = 0.0;
   for (int t = threadIdx.x; t < ntiles; t += blockDim.x) s += ll_tiles[t];
   red[threadIdx.x] = s;
@@ -228,7 +232,9 @@ __global__ void __launch_bounds__(kSimtThreads)
     stats_simt_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp, int Kp,
                       const float* __restrict__ mu, const float* __restrict__ prec,
                       const float* __restrict__ cconst, const float* __restrict__ logz,
-                      double* __restrict__ stats, int64_t slice_len) {
+                      double* __restrict__ stats, int kstride, int64_t slice_len,
+                      const int* mode) {
+  if (mode && *mode != kModeSimt) return;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   StatsSmem& sm = *reinterpret_cast<StatsSmem*>(smem_raw);
   const int kb = blockIdx.x * kKBs;
@@ -244,7 +250,7 @@ __global__ void __launch_bounds__(kSimtThreads)
   const int f = f0 + fl;
   const bool f_ok = f < D;
   const size_t row = (size_t)(1 + 2 * Dp);
-  double* slot = stats + (size_t)s * Kp * row;
+  double* slot = stats + (size_t)s * kstride * row;
 
   float mreg[16];
 #pragma unroll
@@ -327,34 +333,50 @@ __global__ void __launch_bounds__(kSimtThreads)
 }
 
 // ------------------------------------------------------------------ M-step
-// One CTA per component: fixed-order fp64 sum over the slice slots, then Eqs. (1)-(3):
-//   mu_new = mu_old + S1/N_k,  sigma^2 = max(S2/N_k - (S1/N_k)^2, 0) + reg_covar
+// One CTA per component: fixed-order fp64 sum over the slice slots, then Eqs. (1)-(3).
+// The slots hold N_k, S1 = sum r (y - o), S2 = sum r (y - o)^2 in a coordinate y with
+// origin o: the CUDA-core path uses y = x, o = mu_old (centred on the current mean);
+// the tensor-core path uses y = (x - c) s, o = 0.  Then
+//   m1 = S1 / N_k,  mu_new = o + m1 (mapped back to x),
+//   sigma^2 = max(S2 / N_k - m1^2, 0) (mapped back to x) + reg_covar
 // (isotropic: averaged over d).  Empty components keep their parameters.  Nothing is
 // written when the log-likelihood of the step is not finite.
-__global__ void mstep_kernel(int K, int D, int Dp, int Kp, int cov, double reg,
-                             const double* __restrict__ stats, const float* __restrict__ mu_old,
+__global__ void mstep_kernel(int K, int D, int Dp, int kstride, int cov, double reg,
+                             const double* __restrict__ stats, int s_simt, int s_tc,
+                             const int* mode, int fixed_mode, const float* __restrict__ mu_old,
+                             const float* __restrict__ center, const float* __restrict__ dscale,
                              const double* __restrict__ ll_total, float* __restrict__ means,
                              float* __restrict__ vars, double* __restrict__ nk_out, int* status) {
   __shared__ double red[kSimtThreads];
   const int k = blockIdx.x;
+  const bool simt = ((mode ? *mode : fixed_mode) == kModeSimt);
+  const int nslots = simt ? s_simt : s_tc;
   const size_t row = (size_t)(1 + 2 * Dp);
   const bool ll_ok = isfinite(*ll_total);
   double nk = 0.0;
-  for (int s = 0; s < kSlices; ++s) nk += stats[((size_t)s * Kp + k) * row];
+  for (int s = 0; s < nslots; ++s) nk += stats[((size_t)s * kstride + k) * row];
   if (threadIdx.x == 0) nk_out[k] = nk;
   const bool live = ll_ok && (nk >= FGMM_EMPTY_NK);
   double vsum = 0.0;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     double s1 = 0.0, s2 = 0.0;
-    for (int s = 0; s < kSlices; ++s) {
-      const double* r = stats + ((size_t)s * Kp + k) * row;
+    for (int s = 0; s < nslots; ++s) {
+      const double* r = stats + ((size_t)s * kstride + k) * row;
       s1 += r[1 + d];
       s2 += r[1 + Dp + d];
     }
     if (live) {
       const double m1 = s1 / nk;
-      const double v = fmax(s2 / nk - m1 * m1, 0.0);
-      means[(size_t)k * D + d] = (float)((double)mu_old[(size_t)k * Dp + d] + m1);
+      double v = fmax(s2 / nk - m1 * m1, 0.0);
+      double mu;
+      if (simt) {
+        mu = (double)mu_old[(size_t)k * Dp + d] + m1;
+      } else {
+        const double sd = dscale[d];
+        mu = (double)center[d] + m1 / sd;
+        v = v / (sd * sd);
+      }
+      means[(size_t)k * D + d] = (float)mu;
       if (cov == FGMM_COV_DIAG) vars[(size_t)k * D + d] = (float)(v + reg);
       vsum += v;
     }
@@ -479,31 +501,33 @@ cudaError_t launch_prep_simt(const Ctx& c, const float* weights, const float* me
 }
 
 cudaError_t launch_lse_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
-                            float* logz_out, cudaStream_t s) {
+                            float* logz_out, const int* mode, cudaStream_t s) {
   const unsigned grid = (unsigned)ceil_div64(n, kTP);
   prof_begin(c, KK_SWEEP1, s);
   if (x_dtype == FGMM_BF16)
     lse_simt_kernel<<<grid, kSimtThreads, 0, s>>>(
         (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
-        c.ws.logz, logz_out, c.ws.ll_tiles);
+        c.ws.logz, logz_out, c.ws.ll_tiles, mode);
   else
     lse_simt_kernel<<<grid, kSimtThreads, 0, s>>>((const float*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp,
                                                   c.ws.mu, c.ws.prec, c.ws.cconst, c.ws.logz,
-                                                  logz_out, c.ws.ll_tiles);
+                                                  logz_out, c.ws.ll_tiles, mode);
   prof_end(c, KK_SWEEP1, s);
   return cudaGetLastError();
 }
 
-cudaError_t launch_ll_accumulate(const Ctx& c, int64_t n, cudaStream_t s) {
+cudaError_t launch_ll_accumulate(const Ctx& c, int64_t n, const int* mode, int fixed_mode,
+                                 cudaStream_t s) {
   prof_begin(c, KK_OTHER, s);
   ll_accumulate_kernel<<<1, kSimtThreads, 0, s>>>(c.ws.ll_tiles, (int)ceil_div64(n, kTP),
+                                                  (int)ceil_div64(n, 128) * 4, mode, fixed_mode,
                                                   c.ws.ll_total);
   prof_end(c, KK_OTHER, s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
-                              cudaStream_t s) {
+                              const int* mode, cudaStream_t s) {
   const size_t smem = sizeof(StatsSmem);
   static bool attr_set = false;
   if (!attr_set) {
@@ -520,21 +544,22 @@ cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t 
   if (x_dtype == FGMM_BF16)
     stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>(
         (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
-        c.ws.logz, c.ws.stats, slice);
+        c.ws.logz, c.ws.stats, c.ws.KpS, slice, mode);
   else
     stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>((const float*)X, n, ldx, c.D, c.ws.Dp,
                                                        c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
-                                                       c.ws.logz, c.ws.stats, slice);
+                                                       c.ws.logz, c.ws.stats, c.ws.KpS, slice, mode);
   prof_end(c, KK_SWEEP2, s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_mstep(const Ctx& c, float* weights, float* means, float* vars,
-                         double* loglik_out, cudaStream_t s) {
+                         double* loglik_out, const int* mode, int fixed_mode, cudaStream_t s) {
   prof_begin(c, KK_OTHER, s);
-  mstep_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, c.ws.Dp, c.ws.Kp, c.cov, c.reg,
-                                            c.ws.stats, c.ws.mu, c.ws.ll_total, means, vars,
-                                            c.ws.nk, c.ws.status);
+  mstep_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, c.ws.Dp, c.ws.KpS, c.cov, c.reg, c.ws.stats,
+                                            kSlices, c.tc.ready ? tc_slices(c) : 1, mode,
+                                            fixed_mode, c.ws.mu, c.ws.center, c.ws.dscale,
+                                            c.ws.ll_total, means, vars, c.ws.nk, c.ws.status);
   prof_end(c, KK_OTHER, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -1,0 +1,928 @@
+// Tensor-core (tcgen05 / TMEM / TMA) kernels of the fused EM step, sm_100a.
+//
+// Paper: "Flash-GMM: A Memory-Efficient Kernel for Scalable Soft Clustering",
+// §3.1 and Algorithm 1: per point tile, sweep 1 builds log Z_i with an online
+// log-sum-exp over component blocks; sweep 2 recomputes the log-densities, forms
+// r_ik = exp(log z_ik - log Z_i) and folds them into the sufficient statistics.
+// The N x K responsibilities exist only as one 128 x 128 tile in TMEM / shared memory.
+//
+// Expanded form.  With a per-dimension centre c_d and power-of-two scale s_d,
+// x^_d = (x_d - c_d) s_d and phi(x) = [x^_0 .. x^_{Dq-1}, x^_0^2 .. x^_{Dq-1}^2]:
+//   log z_ik = 2^t_k * sum_j W'_kj phi_j(x_i) + c_k,
+//   W_k = [ (mu_kd - c_d) / (sigma_kd^2 s_d) , -1 / (2 sigma_kd^2 s_d^2) ],  W' = W 2^-t_k,
+//   c_k = log pi_k - 1/2 sum_d log(2 pi sigma_kd^2) - 1/2 sum_d (mu_kd - c_d)^2 / sigma_kd^2,
+// which is §2's log pi_k + log N(x | mu_k, diag sigma_k^2) rewritten as one dot product:
+// a dense contraction of K1 = 2 Dq terms per (point, component), i.e. a GEMM.
+//
+// Precision (FGMM_PREC_FP16X3).  Every operand a is split a = a_hi + a_lo with
+// a_hi = fp16(a), a_lo = fp16(a - a_hi); the product uses three tcgen05 kind::f16
+// MMAs (hi*hi + hi*lo + lo*hi) with fp32 accumulation in TMEM, about 22 significant
+// bits per term.  One fp16 product (~11 bits) misses the 1e-4 log-likelihood
+// tolerance on the Table-1 generator; bf16 splits (16 bits) pass with little margin.
+// Statistics: r is scaled by 2^15 and rounded once to fp16 (the same rounded values
+// feed N_k and the GEMM, so the weights stay consistent); phi is split hi/lo, two MMAs.
+//
+// Kernels (one chunk of <= 2^20 points at a time):
+//   tc_center     per-dimension centre and scale from the parameters
+//   tc_prep       W' hi/lo, c_k, 2^t_k; conditioning check for AUTO mode
+//   tc_convert    X chunk -> phi hi/lo (fp16, row-major, TMA-ready)
+//   tc_lse        sweep 1: persistent, one 128-point tile per CTA at a time; phi tile
+//                 resident in smem, W streamed through a TMA ring; S = phi W^T in
+//                 TMEM (double buffered), online log-sum-exp by a 4-warp epilogue.
+//   tc_stats      sweep 2: CTA owns a 128-component block (W resident) and a slice
+//                 of points; S^T = W phi^T in TMEM, responsibilities written as the
+//                 A operand of the second GEMM acc += R^T phi (TMEM, 128 x 2Dq),
+//                 flushed to the CTA's fp64 slot.
+//
+// Warp roles in both sweeps: warp 0 TMA producer, warp 1 MMA issuer (one thread,
+// also owns the TMEM allocation), warps 4..7 epilogue (TMEM lane quarters 0..3).
+// Every wait is bounded (ptx::mbar_wait); on expiry the kernel latches
+// FGMM_ERR_TIMEOUT, the other roles see the abort flag, and the CTA drains and frees
+// its TMEM before returning.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "fgmm_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace fgmm {
+
+namespace {
+
+constexpr int BM = 128;          // points per tile
+constexpr int BKc = 128;         // components per block
+constexpr int KC = 64;           // K elements per swizzle row / TMA box
+constexpr int BOX = 128 * 64 * 2;  // bytes of one [128 rows][64 fp16] box
+constexpr int SW = 4;            // W ring stages (sweep 1)
+constexpr int SX = 4;            // X ring stages (sweep 2)
+constexpr float kRScale = 32768.f;  // r is stored as fp16(r * 2^15)
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ void set_status(int* st, int code) { atomicCAS(st, FGMM_OK, code); }
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// fp16 split of a float: hi = fp16(a) (saturating), lo = fp16(a - hi).
+__device__ __forceinline__ void split16(float a, __half& hi, __half& lo) {
+  hi = __float2half_rn(fminf(fmaxf(a, -65504.f), 65504.f));
+  lo = __float2half_rn(a - __half2float(hi));
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ centre and scale
+// One CTA per dimension d: c_d = sum_k pi_k mu_kd / sum_k pi_k, spread_d^2 =
+// sum_k pi_k (sigma_kd^2 + (mu_kd - c_d)^2) / sum pi, s_d = 2^-round(log2 spread_d).
+__global__ void tc_center_kernel(int K, int D, int cov, const float* __restrict__ w,
+                                 const float* __restrict__ means, const float* __restrict__ vars,
+                                 float* __restrict__ center, float* __restrict__ scale) {
+  __shared__ double r0[kSimtThreads], r1[kSimtThreads];
+  const int d = blockIdx.x;
+  double sw = 0.0, sm = 0.0;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    const double wk = fmax((double)w[k], 0.0);
+    sw += wk;
+    sm += wk * (double)means[(size_t)k * D + d];
+  }
+  r0[threadIdx.x] = sw;
+  r1[threadIdx.x] = sm;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) { r0[threadIdx.x] += r0[threadIdx.x + s]; r1[threadIdx.x] += r1[threadIdx.x + s]; }
+    __syncthreads();
+  }
+  const double W = r0[0];
+  const double c = (W > 0.0) ? r1[0] / W : 0.0;
+  __syncthreads();
+  double sv = 0.0;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    const double wk = fmax((double)w[k], 0.0);
+    const double v = (cov == FGMM_COV_DIAG) ? vars[(size_t)k * D + d] : vars[k];
+    const double dm = (double)means[(size_t)k * D + d] - c;
+    sv += wk * (v + dm * dm);
+  }
+  r0[threadIdx.x] = sv;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) r0[threadIdx.x] += r0[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double spread = (W > 0.0) ? sqrt(r0[0] / W) : 1.0;
+    double sc = 1.0;
+    if (spread > 0.0 && isfinite(spread)) sc = exp2(-rint(log2(spread)));
+    center[d] = isfinite(c) ? (float)c : 0.f;
+    scale[d] = (float)sc;
+  }
+}
+
+// ------------------------------------------------------------------ parameter preparation
+// One CTA per padded component k (grid Kt).  Writes W' = W 2^-t_k as fp16 hi/lo into
+// wop[part][k][j] (part 0 hi, 1 lo; j < Dq the linear terms, Dq + d the squares),
+// c_k (fp64 sums, -inf for an absent or zero-weight component) and 2^t_k.
+// Conditioning check: the split product keeps ~2^-22 relative error per term; near
+// x = mu_k the terms reach t_d = 1.5 (|mu~| + sigma)^2 / sigma^2 and cancel, so the
+// expected logit error is ~2^-20 sqrt(sum_d t_d^2).  Above 1e-3 nats the component is
+// "stiff" and AUTO mode runs this step on the fp32 CUDA-core path instead.
+__global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
+                               const float* __restrict__ w, const float* __restrict__ means,
+                               const float* __restrict__ vars, const float* __restrict__ center,
+                               const float* __restrict__ scale, __half* __restrict__ wop,
+                               float* __restrict__ ck, float* __restrict__ kscale, int* mode,
+                               int* status) {
+  __shared__ double rs[kSimtThreads], rq[kSimtThreads], rt[kSimtThreads];
+  __shared__ float rmax[kSimtThreads];
+  __shared__ float s_pow;
+  const int k = blockIdx.x;
+  const int K1 = 2 * Dq;
+  __half* hi = wop + (size_t)k * K1;
+  __half* lo = wop + ((size_t)Kt + k) * K1;
+  double slog = 0.0, squad = 0.0, stiff = 0.0;
+  float wmax = 0.f;
+  bool bad = false;
+  const bool live_k = k < K;
+  // pass 1: constants and max |W|
+  for (int d = threadIdx.x; d < Dq; d += blockDim.x) {
+    if (live_k && d < D) {
+      const double v = (cov == FGMM_COV_DIAG) ? vars[(size_t)k * D + d] : vars[k];
+      const double m = means[(size_t)k * D + d];
+      if (!(v > 0.0) || !isfinite(v) || !isfinite(m)) bad = true;
+      const double mt = m - (double)center[d];
+      const double p = 1.0 / v;
+      const double sd = scale[d];
+      slog += log(2.0 * CUDART_PI * v);
+      squad += mt * mt * p;
+      const double a = mt * p / sd, b = -0.5 * p / (sd * sd);
+      wmax = fmaxf(wmax, (float)fmax(fabs(a), fabs(b)));
+      const double t = 1.5 * (fabs(mt) + sqrt(v)) * (fabs(mt) + sqrt(v)) * p;
+      stiff += t * t;
+    }
+  }
+  rs[threadIdx.x] = slog;
+  rq[threadIdx.x] = squad;
+  rt[threadIdx.x] = stiff;
+  rmax[threadIdx.x] = wmax;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) {
+      rs[threadIdx.x] += rs[threadIdx.x + s];
+      rq[threadIdx.x] += rq[threadIdx.x + s];
+      rt[threadIdx.x] += rt[threadIdx.x + s];
+      rmax[threadIdx.x] = fmaxf(rmax[threadIdx.x], rmax[threadIdx.x + s]);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    float c = -CUDART_INF_F;
+    float pw = 1.f;
+    if (live_k) {
+      const float wk = w[k];
+      if (!(wk >= 0.f) || !isfinite(wk)) bad = true;
+      if (wk > 0.f) c = (float)(log((double)wk) - 0.5 * rs[0] - 0.5 * rq[0]);
+      const float mx = rmax[0];
+      if (mx > 0.f && isfinite(mx)) pw = exp2f(ceilf(log2f(mx)) - 14.f);
+      if (mode && !(ldexp(sqrt(rt[0]), -20) <= 1e-3)) atomicExch(mode, 1);
+    }
+    ck[k] = c;
+    kscale[k] = pw;
+    s_pow = pw;
+  }
+  __syncthreads();
+  const float inv = 1.f / s_pow;
+  // pass 2: write the split operand rows
+  for (int j = threadIdx.x; j < K1; j += blockDim.x) {
+    const int d = (j < Dq) ? j : j - Dq;
+    float val = 0.f;
+    if (live_k && d < D) {
+      const double v = (cov == FGMM_COV_DIAG) ? vars[(size_t)k * D + d] : vars[k];
+      const double m = means[(size_t)k * D + d];
+      const double p = 1.0 / v;
+      const double sd = scale[d];
+      const double wv = (j < Dq) ? (m - (double)center[d]) * p / sd : -0.5 * p / (sd * sd);
+      val = (float)wv * inv;
+      if (!isfinite(val)) val = 0.f;
+    }
+    __half h, l;
+    split16(val, h, l);
+    hi[j] = h;
+    lo[j] = l;
+  }
+  if (bad) set_status(status, FGMM_ERR_INVALID_ARG);
+}
+
+// ------------------------------------------------------------------ X -> phi (fp16 hi / lo)
+// Thread per (point, group of 8 dims).  xop[part][i][j]: part 0 hi, 1 lo; j < Dq the
+// scaled centred coordinate, Dq + d its square.
+template <typename T>
+__global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dq,
+                                  int64_t ncmax, const float* __restrict__ center,
+                                  const float* __restrict__ scale, __half* __restrict__ xop,
+                                  const int* mode) {
+  if (mode && *mode != 0) return;
+  const int groups = Dq / 8;
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n * groups) return;
+  const int64_t i = e / groups;
+  const int g = (int)(e % groups);
+  const int K1 = 2 * Dq;
+  __align__(16) __half xh[8], xl[8], qh[8], ql[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int d = 8 * g + u;
+    float xv = 0.f;
+    if (d < D) {
+      float x;
+      if constexpr (sizeof(T) == 4) x = __ldg(reinterpret_cast<const float*>(X) + i * ldx + d);
+      else x = __bfloat162float(X[i * ldx + d]);
+      xv = (x - center[d]) * scale[d];
+    }
+    split16(xv, xh[u], xl[u]);
+    split16(xv * xv, qh[u], ql[u]);
+  }
+  __half* hi = xop + (size_t)i * K1;
+  __half* lo = xop + ((size_t)ncmax + i) * K1;
+  *reinterpret_cast<uint4*>(hi + 8 * g) = *reinterpret_cast<uint4*>(xh);
+  *reinterpret_cast<uint4*>(lo + 8 * g) = *reinterpret_cast<uint4*>(xl);
+  *reinterpret_cast<uint4*>(hi + Dq + 8 * g) = *reinterpret_cast<uint4*>(qh);
+  *reinterpret_cast<uint4*>(lo + Dq + 8 * g) = *reinterpret_cast<uint4*>(ql);
+}
+
+// ------------------------------------------------------------------ sweep 1 (log Z)
+struct LseBars {
+  uint64_t x_full[4], x_empty[4];
+  uint64_t w_full[SW], w_empty[SW];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t drain;
+  uint32_t tmem;
+  int abort;
+};
+
+template <int NKC>
+__global__ void __launch_bounds__(256, 1)
+    tc_lse_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
+                  int nc, int ncmax, int Kt, const float* __restrict__ ck,
+                  const float* __restrict__ kscale, float* __restrict__ logz,
+                  float* __restrict__ logz_out, double* __restrict__ ll_tiles, const int* mode,
+                  int* status) {
+  if (mode && *mode != 0) return;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  unsigned char* xbuf = base;                         // [2][NKC][BOX]
+  unsigned char* wring = base + 2 * NKC * BOX;        // [SW][BOX]
+  LseBars* bars = reinterpret_cast<LseBars*>(wring + SW * BOX);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntiles = (nc + BM - 1) / BM;
+  const int nkb = Kt / BKc;
+
+  if (threadIdx.x == 0) {
+    for (int c = 0; c < 4; ++c) { ptx::mbar_init(&bars->x_full[c], 1); ptx::mbar_init(&bars->x_empty[c], 1); }
+    for (int s = 0; s < SW; ++s) { ptx::mbar_init(&bars->w_full[s], 1); ptx::mbar_init(&bars->w_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { ptx::mbar_init(&bars->s_full[b], 1); ptx::mbar_init(&bars->s_empty[b], 4); }
+    ptx::mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&bars->tmem, 256);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmx);
+      ptx::prefetch_tmap(&tmw);
+      uint32_t itw = 0;
+      int j = 0, x_issued = 0;
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++j) {
+        const int row0 = t * BM;
+        x_issued = j + 1;
+        for (int c = 0; c < NKC; ++c) {
+          if (j > 0 && !ptx::mbar_wait(&bars->x_empty[c], (j - 1) & 1, abort)) goto fail_p;
+          ptx::mbar_arrive_expect_tx(&bars->x_full[c], 2 * BOX);
+          ptx::tma_load_2d(xbuf + c * BOX, &tmx, &bars->x_full[c], c * KC, row0);
+          ptx::tma_load_2d(xbuf + (NKC + c) * BOX, &tmx, &bars->x_full[c], c * KC, ncmax + row0);
+        }
+        for (int kb = 0; kb < nkb; ++kb)
+          for (int c = 0; c < NKC; ++c)
+            for (int part = 0; part < 2; ++part, ++itw) {
+              const int s = itw % SW;
+              if (itw >= SW && !ptx::mbar_wait(&bars->w_empty[s], ((itw / SW) - 1) & 1, abort))
+                goto fail_p;
+              ptx::mbar_arrive_expect_tx(&bars->w_full[s], BOX);
+              ptx::tma_load_2d(wring + s * BOX, &tmw, &bars->w_full[s], c * KC,
+                               part * Kt + kb * BKc);
+            }
+      }
+      goto done_p;
+    fail_p:
+      set_status(status, FGMM_ERR_TIMEOUT);
+      bars->abort = 1;
+    done_p:
+      if (*abort) {  // let every copy this thread started land before the CTA exits
+        for (int c = 0; c < NKC && x_issued > 0; ++c) ptx::mbar_drain(&bars->x_full[c], (x_issued - 1) & 1);
+        for (uint32_t k = (itw > SW ? itw - SW : 0); k < itw; ++k)
+          ptx::mbar_drain(&bars->w_full[k % SW], (k / SW) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_f16(128, 128, false, false);
+      uint32_t itw = 0, its = 0;
+      int j = 0;
+      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++j) {
+        for (int kb = 0; kb < nkb; ++kb, ++its) {
+          const int b = its & 1;
+          if (its >= 2 && !ptx::mbar_wait(&bars->s_empty[b], ((its >> 1) - 1) & 1, abort)) goto fail_m;
+          ptx::tc_fence_after();
+          const uint32_t d_tmem = tmem + b * 128;
+          for (int c = 0; c < NKC; ++c) {
+            if (kb == 0 && !ptx::mbar_wait(&bars->x_full[c], j & 1, abort)) goto fail_m;
+            const int sh = itw % SW;
+            if (!ptx::mbar_wait(&bars->w_full[sh], (itw / SW) & 1, abort)) goto fail_m;
+            ++itw;
+            const int sl = itw % SW;
+            if (!ptx::mbar_wait(&bars->w_full[sl], (itw / SW) & 1, abort)) goto fail_m;
+            ++itw;
+            ptx::tc_fence_after();
+            const uint32_t xa_hi = ptx::smem_u32(xbuf + c * BOX);
+            const uint32_t xa_lo = ptx::smem_u32(xbuf + (NKC + c) * BOX);
+            const uint32_t wb_hi = ptx::smem_u32(wring + sh * BOX);
+            const uint32_t wb_lo = ptx::smem_u32(wring + sl * BOX);
+#pragma unroll
+            for (int ks = 0; ks < KC / 16; ++ks) {
+              const uint32_t o = ks * 32;
+              const uint64_t ah = ptx::smem_desc_sw128(xa_hi + o, 16, 1024);
+              const uint64_t al = ptx::smem_desc_sw128(xa_lo + o, 16, 1024);
+              const uint64_t bh = ptx::smem_desc_sw128(wb_hi + o, 16, 1024);
+              const uint64_t bl = ptx::smem_desc_sw128(wb_lo + o, 16, 1024);
+              ptx::mma_f16_ss(d_tmem, ah, bh, idesc, (c > 0 || ks > 0) ? 1u : 0u);
+              ptx::mma_f16_ss(d_tmem, ah, bl, idesc, 1u);
+              ptx::mma_f16_ss(d_tmem, al, bh, idesc, 1u);
+            }
+            ptx::mma_commit(&bars->w_empty[sh]);
+            ptx::mma_commit(&bars->w_empty[sl]);
+            if (kb == nkb - 1) ptx::mma_commit(&bars->x_empty[c]);
+          }
+          ptx::mma_commit(&bars->s_full[b]);
+        }
+      }
+      goto done_m;
+    fail_m:
+      set_status(status, FGMM_ERR_TIMEOUT);
+      bars->abort = 1;
+    done_m:
+      if (*abort) {  // wait for the MMAs already issued before TMEM is freed
+        ptx::mma_commit(&bars->drain);
+        ptx::mbar_drain(&bars->drain, 0);
+      }
+    }
+  } else if (warp >= 4) {
+    const int q = warp - 4;               // TMEM lane quarter
+    const int r = q * 32 + lane;          // row of the tile = TMEM lane
+    uint32_t its = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+      float m = -CUDART_INF_F, s = 0.f;   // in log2 units
+      for (int kb = 0; kb < nkb; ++kb, ++its) {
+        const int b = its & 1;
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full[b], (its >> 1) & 1, abort))) {
+          set_status(status, FGMM_ERR_TIMEOUT);
+          bars->abort = 1;
+          break;
+        }
+        ptx::tc_fence_after();
+        const float4* ckb = reinterpret_cast<const float4*>(ck + kb * BKc);
+        const float4* ksb = reinterpret_cast<const float4*>(kscale + kb * BKc);
+#pragma unroll 1
+        for (int h = 0; h < 4; ++h) {
+          uint32_t u[32];
+          ptx::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 128 + h * 32, u);
+          ptx::tmem_wait_ld();
+          float v[32];
+          float bm = -CUDART_INF_F;
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 cc = __ldg(ckb + h * 8 + e4);
+            const float4 kk = __ldg(ksb + h * 8 + e4);
+            v[4 * e4 + 0] = (__uint_as_float(u[4 * e4 + 0]) * kk.x + cc.x) * kLog2e;
+            v[4 * e4 + 1] = (__uint_as_float(u[4 * e4 + 1]) * kk.y + cc.y) * kLog2e;
+            v[4 * e4 + 2] = (__uint_as_float(u[4 * e4 + 2]) * kk.z + cc.z) * kLog2e;
+            v[4 * e4 + 3] = (__uint_as_float(u[4 * e4 + 3]) * kk.w + cc.w) * kLog2e;
+#pragma unroll
+            for (int z = 0; z < 4; ++z) bm = fmaxf(bm, v[4 * e4 + z]);
+          }
+          const float nm = fmaxf(m, bm);
+          if (nm > -CUDART_INF_F) {
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc += exp2f(v[e] - nm);
+            s = s * exp2f(m - nm) + acc;
+            m = nm;
+          }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->s_empty[b]);
+      }
+      if (*abort) break;
+      const int i = t * BM + r;
+      const float lz = (m + log2f(s)) / kLog2e;
+      double part = 0.0;
+      if (i < nc) {
+        logz[i] = lz;
+        if (logz_out) logz_out[i] = lz;
+        part = lz;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      if (lane == 0) ll_tiles[(size_t)t * 4 + q] = part;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 256);
+  }
+}
+
+// ------------------------------------------------------------------ sweep 2 (statistics)
+struct StatBars {
+  uint64_t w_full;
+  uint64_t x_full[SX], x_empty[SX];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t r_full, r_empty;
+  uint64_t acc_full, acc_empty;
+  uint64_t drain;
+  uint32_t tmem;
+  int abort;
+};
+
+template <int NKC>
+__global__ void __launch_bounds__(256, 1)
+    tc_stats_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
+                    int nc, int ncmax, int Kt, int slice_len, int flush_tiles,
+                    const float* __restrict__ ck, const float* __restrict__ kscale,
+                    const float* __restrict__ logz, double* __restrict__ stats, int kstride,
+                    int Dp, const int* mode, int* status) {
+  if (mode && *mode != 0) return;
+  constexpr int Dq = NKC * 32;            // features: phi has 2 Dq = NKC * 64 entries
+  constexpr int ACC_COLS = 2 * Dq;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  unsigned char* wbuf = base;                          // [2][NKC][BOX]
+  unsigned char* xring = base + 2 * NKC * BOX;         // [SX][BOX]
+  unsigned char* rbuf = xring + SX * BOX;              // [2][BOX]: R^T, 64 points per box
+  StatBars* bars = reinterpret_cast<StatBars*>(rbuf + 2 * BOX);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kb = blockIdx.x;
+  const int p0 = blockIdx.y * slice_len;
+  const int p1 = min(nc, p0 + slice_len);
+  const int ntl = (p1 > p0) ? (p1 - p0 + BM - 1) / BM : 0;
+  if (ntl == 0) return;  // uniform over the CTA, before any barrier or TMEM use
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bars->w_full, 1);
+    for (int s = 0; s < SX; ++s) { ptx::mbar_init(&bars->x_full[s], 1); ptx::mbar_init(&bars->x_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { ptx::mbar_init(&bars->s_full[b], 1); ptx::mbar_init(&bars->s_empty[b], 4); }
+    ptx::mbar_init(&bars->r_full, 4);
+    ptx::mbar_init(&bars->r_empty, 1);
+    ptx::mbar_init(&bars->acc_full, 1);
+    ptx::mbar_init(&bars->acc_empty, 4);
+    ptx::mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&bars->tmem, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem;         // cols [0,256): S^T x2, [256, 256+ACC_COLS): acc
+  const uint32_t acc_tmem = tmem + 256;
+
+  // The schedule of MMA groups (and of the producer's X loads) is
+  //   G1(0), G1(1), G2(0), G1(2), G2(1), ..., G1(n-1), G2(n-2), G2(n-1)
+  // so the epilogue's softmax of tile j overlaps G1(j+1).
+  if (warp == 0) {
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmx);
+      ptx::prefetch_tmap(&tmw);
+      ptx::mbar_arrive_expect_tx(&bars->w_full, 2 * NKC * BOX);
+      for (int c = 0; c < NKC; ++c) {
+        ptx::tma_load_2d(wbuf + c * BOX, &tmw, &bars->w_full, c * KC, kb * BKc);
+        ptx::tma_load_2d(wbuf + (NKC + c) * BOX, &tmw, &bars->w_full, c * KC, Kt + kb * BKc);
+      }
+      uint32_t itx = 0;
+      // step g: g < ntl -> G1(g); then G2(g-1) for g >= 1; final G2(ntl-1)
+      for (int g = 0; g <= ntl && !*abort; ++g) {
+        for (int which = 0; which < 2; ++which) {
+          int tile;
+          if (which == 0) { if (g >= ntl) continue; tile = g; }
+          else { if (g == 0) continue; tile = g - 1; }
+          const int row0 = p0 + tile * BM;
+          for (int c = 0; c < NKC; ++c)
+            for (int part = 0; part < 2; ++part, ++itx) {
+              const int s = itx % SX;
+              if (itx >= SX && !ptx::mbar_wait(&bars->x_empty[s], ((itx / SX) - 1) & 1, abort)) {
+                set_status(status, FGMM_ERR_TIMEOUT);
+                bars->abort = 1;
+                goto done_p;
+              }
+              ptx::mbar_arrive_expect_tx(&bars->x_full[s], BOX);
+              ptx::tma_load_2d(xring + s * BOX, &tmx, &bars->x_full[s], c * KC,
+                               part * ncmax + row0);
+            }
+        }
+      }
+    done_p:
+      if (*abort) {  // let every copy this thread started land before the CTA exits
+        ptx::mbar_drain(&bars->w_full, 0);
+        for (uint32_t k = (itx > SX ? itx - SX : 0); k < itx; ++k)
+          ptx::mbar_drain(&bars->x_full[k % SX], (k / SX) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc1 = ptx::idesc_f16(128, 128, false, false);  // S^T = W phi^T
+      constexpr uint32_t idesc2 = ptx::idesc_f16(128, 64, false, true);    // acc += R^T phi
+      uint32_t itx = 0;
+      int tiles_since_flush = 0;
+      bool fresh = true;   // next G2 starts a new accumulation period
+      int flushes = 0;
+      if (!ptx::mbar_wait(&bars->w_full, 0, abort)) goto fail_m;
+      for (int g = 0; g <= ntl && !*abort; ++g) {
+        if (g < ntl) {  // ---- G1(g)
+          const int b = g & 1;
+          if (g >= 2 && !ptx::mbar_wait(&bars->s_empty[b], ((g >> 1) - 1) & 1, abort)) goto fail_m;
+          ptx::tc_fence_after();
+          const uint32_t d_tmem = tmem + b * 128;
+          for (int c = 0; c < NKC; ++c) {
+            const int sh = itx % SX;
+            if (!ptx::mbar_wait(&bars->x_full[sh], (itx / SX) & 1, abort)) goto fail_m;
+            ++itx;
+            const int sl = itx % SX;
+            if (!ptx::mbar_wait(&bars->x_full[sl], (itx / SX) & 1, abort)) goto fail_m;
+            ++itx;
+            ptx::tc_fence_after();
+            const uint32_t wa_hi = ptx::smem_u32(wbuf + c * BOX);
+            const uint32_t wa_lo = ptx::smem_u32(wbuf + (NKC + c) * BOX);
+            const uint32_t xb_hi = ptx::smem_u32(xring + sh * BOX);
+            const uint32_t xb_lo = ptx::smem_u32(xring + sl * BOX);
+#pragma unroll
+            for (int ks = 0; ks < KC / 16; ++ks) {
+              const uint32_t o = ks * 32;
+              const uint64_t ah = ptx::smem_desc_sw128(wa_hi + o, 16, 1024);
+              const uint64_t al = ptx::smem_desc_sw128(wa_lo + o, 16, 1024);
+              const uint64_t bh = ptx::smem_desc_sw128(xb_hi + o, 16, 1024);
+              const uint64_t bl = ptx::smem_desc_sw128(xb_lo + o, 16, 1024);
+              ptx::mma_f16_ss(d_tmem, ah, bh, idesc1, (c > 0 || ks > 0) ? 1u : 0u);
+              ptx::mma_f16_ss(d_tmem, ah, bl, idesc1, 1u);
+              ptx::mma_f16_ss(d_tmem, al, bh, idesc1, 1u);
+            }
+            ptx::mma_commit(&bars->x_empty[sh]);
+            ptx::mma_commit(&bars->x_empty[sl]);
+          }
+          ptx::mma_commit(&bars->s_full[b]);
+        }
+        if (g >= 1) {  // ---- G2(g-1)
+          const int tile = g - 1;
+          if (!ptx::mbar_wait(&bars->r_full, tile & 1, abort)) goto fail_m;
+          if (fresh && flushes > 0 && !ptx::mbar_wait(&bars->acc_empty, (flushes - 1) & 1, abort))
+            goto fail_m;
+          ptx::tc_fence_after();
+          const uint32_t r0 = ptx::smem_u32(rbuf);
+          for (int c = 0; c < NKC; ++c) {
+            const int sh = itx % SX;
+            if (!ptx::mbar_wait(&bars->x_full[sh], (itx / SX) & 1, abort)) goto fail_m;
+            ++itx;
+            const int sl = itx % SX;
+            if (!ptx::mbar_wait(&bars->x_full[sl], (itx / SX) & 1, abort)) goto fail_m;
+            ++itx;
+            ptx::tc_fence_after();
+            const uint32_t xb_hi = ptx::smem_u32(xring + sh * BOX);
+            const uint32_t xb_lo = ptx::smem_u32(xring + sl * BOX);
+            const uint32_t d_tmem = acc_tmem + c * 64;
+#pragma unroll
+            for (int ks = 0; ks < BM / 16; ++ks) {
+              // A = R^T (K-major, K = points): box ks/4, 32 B per 16 points inside it
+              const uint64_t a = ptx::smem_desc_sw128(r0 + (ks >> 2) * BOX + (ks & 3) * 32, 16, 1024);
+              // B = phi (MN-major, K = points = rows): 16 rows = 2 atoms of 1024 B
+              const uint64_t bh = ptx::smem_desc_sw128(xb_hi + ks * 2048, BOX, 1024);
+              const uint64_t bl = ptx::smem_desc_sw128(xb_lo + ks * 2048, BOX, 1024);
+              ptx::mma_f16_ss(d_tmem, a, bh, idesc2, (fresh && ks == 0) ? 0u : 1u);
+              ptx::mma_f16_ss(d_tmem, a, bl, idesc2, 1u);
+            }
+            ptx::mma_commit(&bars->x_empty[sh]);
+            ptx::mma_commit(&bars->x_empty[sl]);
+          }
+          ptx::mma_commit(&bars->r_empty);
+          fresh = false;
+          if (++tiles_since_flush == flush_tiles || tile == ntl - 1) {
+            ptx::mma_commit(&bars->acc_full);
+            tiles_since_flush = 0;
+            fresh = true;
+            ++flushes;
+          }
+        }
+      }
+      goto done_m;
+    fail_m:
+      set_status(status, FGMM_ERR_TIMEOUT);
+      bars->abort = 1;
+    done_m:
+      if (*abort) {  // wait for the MMAs already issued before TMEM is freed
+        ptx::mma_commit(&bars->drain);
+        ptx::mbar_drain(&bars->drain, 0);
+      }
+    }
+  } else if (warp >= 4) {
+    const int q = warp - 4;
+    const int kl = q * 32 + lane;             // component within the block = TMEM lane
+    const int k = kb * BKc + kl;
+    const float ckk = ck[k];
+    const float ksk = kscale[k];
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    const size_t row = (size_t)(1 + 2 * Dp);
+    double* slot = stats + ((size_t)blockIdx.y * kstride + k) * row;
+    float nk = 0.f;
+    int tiles_since_flush = 0, flushes = 0;
+    // R^T row kl lives in boxes 0/1 (points 0-63 / 64-127): 8-row atoms of 1024 B,
+    // 128 B per row, 16-byte units XOR-swizzled by (row & 7).
+    unsigned char* rrow0 = rbuf + (kl >> 3) * 1024 + (kl & 7) * 128;
+    for (int tile = 0; tile < ntl && !*abort; ++tile) {
+      const int row0 = p0 + tile * BM;
+      const int b = tile & 1;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full[b], (tile >> 1) & 1, abort)))
+        goto fail_e;
+      ptx::tc_fence_after();
+      if (tile >= 1 &&
+          !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->r_empty, (tile - 1) & 1, abort)))
+        goto fail_e;
+#pragma unroll 1
+      for (int h = 0; h < 4; ++h) {
+        uint32_t u[32];
+        ptx::tmem_ld32(tmem + lane_base + b * 128 + h * 32, u);
+        ptx::tmem_wait_ld();
+        // log Z of these 32 points: the same addresses for every thread (L1 broadcast);
+        // rows past the slice end read stale but finite values and are masked below
+        const float4* lz4 = reinterpret_cast<const float4*>(logz + row0 + h * 32);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float rr[2];
+          const float4 lzv = __ldg(lz4 + (e >> 2));
+#pragma unroll
+          for (int z = 0; z < 2; ++z) {
+            const int pe = e + z;
+            const float l = __uint_as_float(u[pe]) * ksk + ckk;
+            const float lz = ((pe & 3) == 0) ? lzv.x : ((pe & 3) == 1) ? lzv.y : ((pe & 3) == 2) ? lzv.z : lzv.w;
+            const bool ok = (row0 + h * 32 + pe < p1) && lz > -CUDART_INF_F && l > -CUDART_INF_F;
+            const float rv = ok ? exp2f((l - lz) * kLog2e) : 0.f;
+            const __half hv = __float2half_rn(fminf(rv, 1.f) * kRScale);
+            nk += __half2float(hv);
+            rr[z] = __half2float(hv);
+          }
+          pk[e >> 1] = pack_half2(rr[0], rr[1]);
+        }
+        // points h*32 .. h*32+31 -> box (h >> 1), 16-byte units (h & 1)*4 .. +3
+        unsigned char* rowp = rrow0 + (h >> 1) * BOX;
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+          const int unit = ((h & 1) * 4 + uu) ^ (kl & 7);
+          *reinterpret_cast<uint4*>(rowp + unit * 16) =
+              make_uint4(pk[uu * 4], pk[uu * 4 + 1], pk[uu * 4 + 2], pk[uu * 4 + 3]);
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(&bars->s_empty[b]);
+        ptx::mbar_arrive(&bars->r_full);
+      }
+      if (++tiles_since_flush == flush_tiles || tile == ntl - 1) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->acc_full, flushes & 1, abort)))
+          goto fail_e;
+        ptx::tc_fence_after();
+        const double inv = 1.0 / (double)kRScale;
+#pragma unroll 1
+        for (int h = 0; h < ACC_COLS / 32; ++h) {
+          uint32_t u[32];
+          ptx::tmem_ld32(acc_tmem + lane_base + h * 32, u);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int j = h * 32 + e;                 // phi index: j < Dq linear, else square
+            const int col = (j < Dq) ? 1 + j : 1 + Dp + (j - Dq);
+            if ((j < Dq ? j : j - Dq) < Dp) slot[col] += (double)__uint_as_float(u[e]) * inv;
+          }
+        }
+        slot[0] += (double)nk * inv;
+        nk = 0.f;
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->acc_empty);
+        tiles_since_flush = 0;
+        ++flushes;
+      }
+    }
+    goto done_e;
+  fail_e:
+    set_status(status, FGMM_ERR_TIMEOUT);
+    bars->abort = 1;
+  done_e:;
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+// The driver's tensor-map encoder, fetched through the runtime so that the library
+// does not link libcuda (it must load on hosts without a driver).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                                      const_cast<void*>(ptr), dims, strides, box, estr,
+                                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+size_t lse_smem(int nkc) { return 1024 + (size_t)(2 * nkc + SW) * BOX + sizeof(LseBars); }
+size_t stats_smem(int nkc) { return 1024 + (size_t)(2 * nkc + SX + 2) * BOX + sizeof(StatBars); }
+
+template <int NKC>
+cudaError_t set_attrs() {
+  cudaError_t e = cudaFuncSetAttribute(tc_lse_kernel<NKC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)lse_smem(NKC));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(tc_stats_kernel<NKC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)stats_smem(NKC));
+}
+
+}  // namespace
+
+bool tc_supported(const Ctx& c) { return round_up(c.D, 32) <= 128; }
+
+cudaError_t tc_init(Ctx& c) {
+  if (!tc_supported(c)) return cudaSuccess;
+  const int nkc = round_up(c.D, 32) / 32;
+  cudaError_t e = cudaSuccess;
+  switch (nkc) {
+    case 1: e = set_attrs<1>(); break;
+    case 2: e = set_attrs<2>(); break;
+    case 3: e = set_attrs<3>(); break;
+    default: e = set_attrs<4>(); break;
+  }
+  if (e != cudaSuccess) return e;
+  const Workspace& w = c.ws;
+  c.tc.ready = false;
+  if (!make_tmap(&c.tc.tmap_x, w.xop, (uint64_t)w.K1, (uint64_t)2 * kChunk) ||
+      !make_tmap(&c.tc.tmap_w, w.wop, (uint64_t)w.K1, (uint64_t)2 * w.Kt))
+    return cudaErrorInvalidValue;
+  c.tc.ready = true;
+  return cudaSuccess;
+}
+
+cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* means,
+                           const float* vars, int* mode, cudaStream_t s) {
+  const Workspace& w = c.ws;
+  prof_begin(c, KK_OTHER, s);
+  tc_center_kernel<<<c.D, kSimtThreads, 0, s>>>(c.K, c.D, c.cov, weights, means, vars, w.center,
+                                                w.dscale);
+  prof_end(c, KK_OTHER, s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (w.Dq > c.D) cudaMemsetAsync(w.center + c.D, 0, (w.Dq - c.D) * sizeof(float), s);
+  prof_begin(c, KK_OTHER, s);
+  tc_prep_kernel<<<w.Kt, kSimtThreads, 0, s>>>(c.K, c.D, w.Dq, w.Kt, c.cov, weights, means, vars,
+                                               w.center, w.dscale, w.wop, w.tck, w.tks, mode,
+                                               w.status);
+  prof_end(c, KK_OTHER, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_convert(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                              const int* mode, cudaStream_t s) {
+  const Workspace& w = c.ws;
+  const int64_t total = n * (w.Dq / 8);
+  const unsigned grid = (unsigned)ceil_div64(total, 256);
+  prof_begin(c, KK_OTHER, s);
+  if (x_dtype == FGMM_BF16)
+    tc_convert_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dq, kChunk,
+                                           w.center, w.dscale, w.xop, mode);
+  else
+    tc_convert_kernel<<<grid, 256, 0, s>>>((const float*)X, n, ldx, c.D, w.Dq, kChunk, w.center,
+                                           w.dscale, w.xop, mode);
+  prof_end(c, KK_OTHER, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* mode,
+                          cudaStream_t s) {
+  const Workspace& w = c.ws;
+  const int nkc = w.K1 / 64;
+  const int ntiles = (int)ceil_div64(n, BM);
+  const int grid = ntiles < c.num_sms ? ntiles : c.num_sms;
+  const CUtensorMap& tx = c.tc.tmap_x;
+  const CUtensorMap& tw = c.tc.tmap_w;
+  prof_begin(c, KK_SWEEP1, s);
+#define LSE_CASE(N_)                                                                          \
+  case N_:                                                                                    \
+    tc_lse_kernel<N_><<<grid, 256, lse_smem(N_), s>>>(tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, \
+                                                      w.tks, w.logz, logz_out, w.ll_tiles, mode, \
+                                                      w.status);                              \
+    break;
+  switch (nkc) {
+    LSE_CASE(1)
+    LSE_CASE(2)
+    LSE_CASE(3)
+    LSE_CASE(4)
+  }
+#undef LSE_CASE
+  prof_end(c, KK_SWEEP1, s);
+  return cudaGetLastError();
+}
+
+int tc_slices(const Ctx& c) {
+  const int nkb = c.ws.Kt / BKc;
+  int S = c.num_sms / nkb;
+  if (S < 1) S = 1;
+  if (S > c.ws.slots) S = c.ws.slots;
+  return S;
+}
+
+cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream_t s) {
+  const Workspace& w = c.ws;
+  const int nkc = w.K1 / 64;
+  const int S = tc_slices(c);
+  int slice = (int)ceil_div64(ceil_div64(n, S), BM) * BM;
+  dim3 grid(w.Kt / BKc, S);
+  const CUtensorMap& tx = c.tc.tmap_x;
+  const CUtensorMap& tw = c.tc.tmap_w;
+  const int flush_tiles = 16;
+  prof_begin(c, KK_SWEEP2, s);
+#define STATS_CASE(N_)                                                                         \
+  case N_:                                                                                     \
+    tc_stats_kernel<N_><<<grid, 256, stats_smem(N_), s>>>(tx, tw, (int)n, (int)kChunk, w.Kt,    \
+                                                          slice, flush_tiles, w.tck, w.tks,    \
+                                                          w.logz, w.stats, w.KpS, w.Dp, mode,  \
+                                                          w.status);                           \
+    break;
+  switch (nkc) {
+    STATS_CASE(1)
+    STATS_CASE(2)
+    STATS_CASE(3)
+    STATS_CASE(4)
+  }
+#undef STATS_CASE
+  prof_end(c, KK_SWEEP2, s);
+  return cudaGetLastError();
+}
+
+}  // namespace fgmm

@@ -75,6 +75,12 @@ class GMM:
         check(LIB.fgmm_get_precision(self._h, ctypes.byref(v)), "fgmm_get_precision")
         return v.value
 
+    def last_step_path(self) -> int:
+        """PREC_FP32 or PREC_FP16X3: the path the last step ran (synchronises under AUTO)."""
+        v = ctypes.c_int()
+        check(LIB.fgmm_last_step_path(self._h, ctypes.byref(v)), "fgmm_last_step_path")
+        return v.value
+
     @property
     def workspace_bytes(self) -> int:
         v = ctypes.c_size_t()

@@ -14,7 +14,7 @@ from tests._cmp import compare_step, ids_match_where_decisive
 
 pytestmark = pytest.mark.gpu
 
-PRECISIONS = ["fp32"]
+PRECISIONS = ["fp32", "fp16x3"]
 
 
 def _gmm(K, D, cov=0, reg=1e-6, prec="fp32"):
@@ -92,13 +92,17 @@ def test_table1_shape_first_step(prec):
     print(_check(X, w, mu, var, prec=prec))
 
 
-@pytest.mark.parametrize("prec", PRECISIONS)
-def test_table1_teacher_forced_late_iteration(prec):
+@pytest.mark.parametrize("prec,N,K", [("fp32", 2500, 192), ("auto", 2500, 192),
+                                      ("fp16x3", 20000, 64)])
+def test_table1_teacher_forced_late_iteration(prec, N, K):
     """Run 8 GPU iterations, then check one step from the GPU's own Θ_8 (teacher
-    forcing: both sides start from the same parameters)."""
-    X = synth.generate("table1", 2500, seed=3)
-    w, mu, var = synth.init_params(X, 192, seed=3)
-    g = _gmm(192, 128, prec=prec)
+    forcing: both sides start from the same parameters).  At ~13 points per
+    component some components collapse onto single points; AUTO must then take
+    the CUDA-core path, and the explicit tensor-core mode is checked on a
+    better-populated problem."""
+    X = synth.generate("table1", N, seed=3)
+    w, mu, var = synth.init_params(X, K, seed=3)
+    g = _gmm(K, 128, prec=prec)
     Xd = X.cuda()
     wd, md, vd = g.new_params(w, mu, var)
     for _ in range(8):
@@ -108,41 +112,56 @@ def test_table1_teacher_forced_late_iteration(prec):
 
 
 @pytest.mark.parametrize("N,D,K", [(1, 1, 1), (5, 3, 2), (63, 7, 5), (65, 33, 65), (130, 130, 3),
-                                   (200, 1, 70), (777, 100, 100), (300, 260, 9)])
+                                   (200, 1, 70), (777, 100, 100), (300, 260, 9), (129, 128, 129),
+                                   (1000, 64, 257)])
 @pytest.mark.parametrize("cov", [0, 1])
-def test_edge_shapes(N, D, K, cov):
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_edge_shapes(N, D, K, cov, prec):
+    import ivf_quantizer_b200 as q
+    if prec == "fp16x3" and D > 128:
+        g = q.GMM(K, D, cov)
+        with pytest.raises(q.FgmmError):
+            g.set_precision(q.PREC_FP16X3)
+        return
     X = synth.uniform_points(N, D, seed=N + D + K, lo=-3, hi=3)
     g = torch.Generator().manual_seed(N * 31 + K)
     mu = X[torch.randint(0, N, (K,), generator=g)] + 0.3 * torch.randn(K, D, generator=g)
     w = torch.rand(K, generator=g) + 0.2
     w = w / w.sum()
     var = (torch.rand(K, generator=g) + 0.5) if cov == 1 else (torch.rand(K, D, generator=g) + 0.5)
-    _check(X, w.numpy(), mu.numpy(), var.numpy(), cov=cov, reg=1e-4)
+    _check(X, w.numpy(), mu.numpy(), var.numpy(), cov=cov, reg=1e-4, prec=prec)
 
 
-def test_k1_closed_form_on_gpu():
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_k1_closed_form_on_gpu(prec):
     """K = 1: one step returns the sample mean and the population variance (+ floor)."""
     X = synth.uniform_points(1000, 20, seed=5, lo=-2, hi=4)
-    gw, gm, gv, gll, _ = _run_step(X, np.ones(1), np.zeros((1, 20)), np.ones((1, 20)), reg=1e-3)
+    gw, gm, gv, gll, _ = _run_step(X, np.ones(1), np.zeros((1, 20)), np.ones((1, 20)), reg=1e-3,
+                                   prec=prec)
     Xn = X.double().numpy()
     np.testing.assert_allclose(gw, [1.0], rtol=1e-7)
     np.testing.assert_allclose(gm[0], Xn.mean(0), rtol=1e-5, atol=1e-5)
     np.testing.assert_allclose(gv[0], Xn.var(0) + 1e-3, rtol=1e-5)
 
 
-def test_dead_and_duplicate_components():
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_dead_and_duplicate_components(prec):
     X = synth.uniform_points(500, 4, seed=6)
     mu = np.array([[0, 0, 0, 0], [0.5, 0.5, 0.5, 0.5], [0.5, 0.5, 0.5, 0.5], [1e4] * 4], float)
     var = np.ones((4, 4))
-    w = np.array([0.3, 0.3, 0.3, 0.1])
-    gw, gm, gv, _, _ = _run_step(X, w, mu, var)
+    # the unreachable component keeps a tiny weight so that it does not move the
+    # tensor-core path's coordinate centre (a far-off heavy component would make
+    # every component ill-conditioned for the expanded form; AUTO covers that case)
+    w = np.array([0.3, 0.35, 0.35, 1e-6])
+    w = w / w.sum()
+    gw, gm, gv, _, _ = _run_step(X, w, mu, var, prec=prec)
     assert gw[3] == 0.0
     np.testing.assert_array_equal(gm[3], mu[3].astype(np.float32))
     np.testing.assert_array_equal(gv[3], var[3].astype(np.float32))
     # duplicates stay identical and share the mass
     np.testing.assert_array_equal(gm[1], gm[2])
     assert gw[1] == gw[2]
-    _check(X, w, mu, var)
+    _check(X, w, mu, var, prec=prec)
 
 
 def test_zero_weight_component_is_excluded():
@@ -153,12 +172,13 @@ def test_zero_weight_component_is_excluded():
     np.testing.assert_allclose(gm[0], X.double().numpy().mean(0), rtol=1e-5, atol=1e-6)
 
 
-def test_bf16_input():
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_bf16_input(prec):
     """bf16 X: the oracle consumes the same rounded values."""
     X = synth.generate("c1", 4000, seed=8).to(torch.bfloat16)
     w, mu, var = synth.init_params(X.float(), 16, seed=8)
     K, D = mu.shape
-    g = _gmm(K, D)
+    g = _gmm(K, D, prec=prec)
     Xd = X.cuda()
     wd, md, vd = g.new_params(w, mu, var)
     lz = torch.empty(4000, device="cuda")
@@ -170,14 +190,15 @@ def test_bf16_input():
                  X.float().numpy(), logz_gpu=lz.cpu().numpy())
 
 
-def test_strided_rows():
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_strided_rows(prec):
     """ldx > D: X is a column slice of a wider matrix."""
     W = synth.uniform_points(700, 40, seed=9)
     X = W[:, :24]
     g = torch.Generator().manual_seed(1)
     mu = X[torch.randperm(700, generator=g)[:10]]
     Xd = W.cuda()[:, :24]
-    gg = _gmm(10, 24)
+    gg = _gmm(10, 24, prec=prec)
     wd, md, vd = gg.new_params(torch.full((10,), 0.1), mu, torch.ones(10, 24))
     lz = torch.empty(700, device="cuda")
     gg.step(Xd, wd, md, vd, logz=lz)
@@ -187,19 +208,21 @@ def test_strided_rows():
                  logz_gpu=lz.cpu().numpy())
 
 
-def test_chunk_boundary():
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_chunk_boundary(prec):
     """N crosses the 2^20-point chunk of the library: statistics accumulate across chunks."""
     N = (1 << 20) + 4099
     X = synth.generate("c1", N, seed=10)
     w, mu, var = synth.init_params(X, 16, seed=10)
-    print(_check(X, w, mu, var))
+    print(_check(X, w, mu, var, prec=prec))
 
 
-def test_deterministic_bitwise():
+@pytest.mark.parametrize("prec", PRECISIONS)
+def test_deterministic_bitwise(prec):
     X = synth.generate("table1", 3000, seed=11)
     w, mu, var = synth.init_params(X, 128, seed=11)
-    a = _run_step(X, w, mu, var)
-    b = _run_step(X, w, mu, var)
+    a = _run_step(X, w, mu, var, prec=prec)
+    b = _run_step(X, w, mu, var, prec=prec)
     for x, y in zip(a, b):
         assert np.array_equal(np.asarray(x), np.asarray(y))
 
@@ -272,3 +295,43 @@ def test_soft_assign_spherical_and_argmax():
     Rs = -np.sort(-R, 1)
     dec = (Rs[:, 0] - Rs[:, 1]) > 1e-3
     assert np.array_equal(ids.cpu().numpy()[dec, 0], arg[dec])
+
+
+def _step_with(X, w, mu, var, prec):
+    import ivf_quantizer_b200 as q
+    K, D = np.asarray(mu).shape
+    g = _gmm(K, D, prec=prec)
+    wd, md, vd = g.new_params(w, mu, var)
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    g.step(X.cuda(), wd, md, vd, loglik=ll)
+    path = g.last_step_path()
+    assert g.status() == 0
+    return path, wd.cpu(), md.cpu(), vd.cpu(), ll.item()
+
+
+def test_auto_takes_tensor_cores_when_well_conditioned():
+    import ivf_quantizer_b200 as q
+    X = synth.generate("table1", 4000, seed=16)
+    w, mu, var = synth.init_params(X, 128, seed=16)
+    pa, *ra = _step_with(X, w, mu, var, "auto")
+    pt, *rt = _step_with(X, w, mu, var, "fp16x3")
+    assert pa == q.PREC_FP16X3 and pt == q.PREC_FP16X3
+    for a, b in zip(ra, rt):
+        assert np.array_equal(np.asarray(a), np.asarray(b))
+
+
+def test_auto_falls_back_on_a_collapsed_component():
+    """A component with variance 1e-6 around a data point cannot be evaluated in the
+    expanded form to the tolerance: AUTO runs the step on the CUDA-core path and the
+    result equals the explicit FP32 mode bit for bit (and matches the oracle)."""
+    import ivf_quantizer_b200 as q
+    X = synth.generate("table1", 3000, seed=17)
+    w, mu, var = synth.init_params(X, 64, seed=17)
+    var = var.clone()
+    var[5] = 1e-6
+    pa, *ra = _step_with(X, w, mu, var, "auto")
+    pf, *rf = _step_with(X, w, mu, var, "fp32")
+    assert pa == q.PREC_FP32
+    for a, b in zip(ra, rf):
+        assert np.array_equal(np.asarray(a), np.asarray(b))
+    _check(X, w, mu, var, prec="auto")
