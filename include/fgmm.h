@@ -160,6 +160,13 @@ int fgmm_profile_read(fgmm_handle h, fgmm_profile* out, int reset);
  * latched since the last call), then clear it. */
 int fgmm_get_status(fgmm_handle h, fgmm_stream_t stream);
 
+/* Self-test of the bounded device-side wait every tensor-core kernel uses: one thread
+ * waits on an mbarrier that nothing completes, with a limit of limit_ms (1..10000)
+ * milliseconds, and records FGMM_ERR_TIMEOUT when the limit expires.  Synchronises.
+ * Returns the recorded status (FGMM_ERR_TIMEOUT when the wait gave up as it must),
+ * FGMM_ERR_INVALID_ARG for a limit out of range.  It faults, traps and hangs nothing. */
+int fgmm_selftest_bounded_wait(int limit_ms);
+
 /* Static text for a status code. */
 const char* fgmm_status_string(int status);
 

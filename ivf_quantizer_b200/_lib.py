@@ -44,6 +44,7 @@ SIGNATURES = {
     "fgmm_get_status": (_int, [_vp, _vp]),
     "fgmm_status_string": (_c.c_char_p, [_int]),
     "fgmm_profile_enable": (_int, [_vp, _int]),
+    "fgmm_selftest_bounded_wait": (_int, [_int]),
     "fgmm_profile_read": (_int, [_vp, _c.POINTER(Profile), _int]),
 }
 

@@ -430,6 +430,14 @@ int fgmm_profile_read(fgmm_handle h, fgmm_profile* out, int reset) {
   return FGMM_OK;
 }
 
+int fgmm_selftest_bounded_wait(int limit_ms) {
+  if (limit_ms < 1 || limit_ms > 10000) return FGMM_ERR_INVALID_ARG;
+  int st = FGMM_OK;
+  cudaError_t e = run_bounded_wait_probe((int64_t)limit_ms * 1000000, &st);
+  if (e != cudaSuccess) return map_cuda(e);
+  return st;
+}
+
 const char* fgmm_status_string(int status) {
   switch (status) {
     case FGMM_OK: return "ok";

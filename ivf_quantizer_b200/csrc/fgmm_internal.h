@@ -115,6 +115,7 @@ cudaError_t launch_tc_convert(const Ctx& c, const void* X, int x_dtype, int64_t 
 cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* mode,
                           cudaStream_t s);
 cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream_t s);
+cudaError_t run_bounded_wait_probe(int64_t limit_ns, int* status_host);
 cudaError_t launch_soft_assign_simt(const Ctx& c, const void* X, int x_dtype, int64_t n,
                                     int64_t ldx, int top_m, float r_threshold, int32_t* ids,
                                     float* resp, cudaStream_t s);

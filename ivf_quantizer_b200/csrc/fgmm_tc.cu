@@ -755,6 +755,33 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
+// ------------------------------------------------------------------ bounded-wait self-test
+// One thread initialises an mbarrier expecting one arrival that never comes and
+// waits on it through the same bounded wait as the sweeps.
+__global__ void bounded_wait_probe_kernel(uint64_t limit_ns, int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+    const bool ok = ptx::mbar_wait(&bar, 0, &abort_flag, limit_ns);
+    *status = ok ? FGMM_OK : FGMM_ERR_TIMEOUT;
+  }
+}
+
+cudaError_t run_bounded_wait_probe(int64_t limit_ns, int* status_host) {
+  int* d = nullptr;
+  cudaError_t e = cudaMalloc(&d, sizeof(int));
+  if (e != cudaSuccess) return e;
+  bounded_wait_probe_kernel<<<1, 32>>>((uint64_t)limit_ns, d);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(status_host, d, sizeof(int), cudaMemcpyDeviceToHost);
+  cudaFree(d);
+  return e;
+}
+
 // ------------------------------------------------------------------ host side
 namespace {
 
