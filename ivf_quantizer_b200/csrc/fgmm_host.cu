@@ -268,21 +268,34 @@ int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t l
                     cudaSuccess)
     return map_cuda(e);
   const size_t eb = dtype_bytes(x_dtype);
-  for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
-    const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
-    const void* Xc = (const char*)X + (size_t)c0 * ldx * eb;
-    float* lzo = logz_out ? logz_out + c0 : nullptr;
-    if (run_tc) {
+  if (run_tc) {
+    for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
+      const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
+      const void* Xc = (const char*)X + (size_t)c0 * ldx * eb;
+      float* lzo = logz_out ? logz_out + c0 : nullptr;
       if ((e = launch_tc_convert(c, Xc, x_dtype, nc, ldx, mode, s)) != cudaSuccess)
         return map_cuda(e);
       if ((e = launch_tc_lse(c, nc, lzo, mode, s)) != cudaSuccess) return map_cuda(e);
+      if ((e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeTensor, s)) != cudaSuccess)
+        return map_cuda(e);
+      if ((e = launch_tc_stats(c, nc, mode, s)) != cudaSuccess) return map_cuda(e);
     }
-    if (run_simt && (e = launch_lse_simt(c, Xc, x_dtype, nc, ldx, lzo, mode, s)) != cudaSuccess)
-      return map_cuda(e);
-    if ((e = launch_ll_accumulate(c, nc, mode, fixed_mode, s)) != cudaSuccess) return map_cuda(e);
-    if (run_tc && (e = launch_tc_stats(c, nc, mode, s)) != cudaSuccess) return map_cuda(e);
-    if (run_simt && (e = launch_stats_simt(c, Xc, x_dtype, nc, ldx, mode, s)) != cudaSuccess)
-      return map_cuda(e);
+  }
+  // AUTO: a step whose new variances would lose accuracy to cancellation is sent back
+  // to the CUDA-core path (the kernels below run only when the mode word says so)
+  if (auto_mode && (e = launch_auto_check_and_reset(c, s)) != cudaSuccess) return map_cuda(e);
+  if (run_simt) {
+    for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
+      const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
+      const void* Xc = (const char*)X + (size_t)c0 * ldx * eb;
+      float* lzo = logz_out ? logz_out + c0 : nullptr;
+      if ((e = launch_lse_simt(c, Xc, x_dtype, nc, ldx, lzo, mode, s)) != cudaSuccess)
+        return map_cuda(e);
+      if ((e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeSimt, s)) != cudaSuccess)
+        return map_cuda(e);
+      if ((e = launch_stats_simt(c, Xc, x_dtype, nc, ldx, mode, s)) != cudaSuccess)
+        return map_cuda(e);
+    }
   }
   if ((e = launch_mstep(c, weights, means, vars, loglik_out, mode, fixed_mode, s)) != cudaSuccess)
     return map_cuda(e);

@@ -99,7 +99,10 @@ cudaError_t launch_prep_simt(const Ctx& c, const float* weights, const float* me
 cudaError_t launch_lse_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
                             float* logz_out, const int* mode, cudaStream_t s);
 cudaError_t launch_ll_accumulate(const Ctx& c, int64_t n, const int* mode, int fixed_mode,
-                                 cudaStream_t s);
+                                 int required, cudaStream_t s);
+// AUTO only: variance-cancellation check after the tensor-core sweeps, and the reset
+// of their partial results when the step is sent back to the CUDA-core path.
+cudaError_t launch_auto_check_and_reset(const Ctx& c, cudaStream_t s);
 cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
                               const int* mode, cudaStream_t s);
 cudaError_t launch_mstep(const Ctx& c, float* weights, float* means, float* vars,

@@ -196,11 +196,14 @@ __global__ void __launch_bounds__(kSimtThreads)
 }
 
 // Adds the chunk's per-tile partial log-likelihoods, in tile order, to ll_total.
+// Runs only when the step's path (device mode word, or fixed_mode when mode is null)
+// equals `required`; the partial count depends on that path's tile size.
 __global__ void ll_accumulate_kernel(const double* __restrict__ ll_tiles, int n_simt, int n_tc,
-                                     const int* mode, int fixed_mode,
+                                     const int* mode, int fixed_mode, int required,
                                      double* __restrict__ ll_total) {
   __shared__ double red[kSimtThreads];
-  const int ntiles = ((mode ? *mode : fixed_mode) == kModeSimt) ? n_simt : n_tc;
+  if ((mode ? *mode : fixed_mode) != required) return;
+  const int ntiles = (required == kModeSimt) ? n_simt : n_tc;
   double s = 0.0;
   for (int t = threadIdx.x; t < ntiles; t += blockDim.x) s += ll_tiles[t];
   red[threadIdx.x] = s;
@@ -489,6 +492,51 @@ __global__ void __launch_bounds__(kSimtThreads)
   }
 }
 
+// ------------------------------------------------------------------ AUTO: variance check
+// After the tensor-core sweeps, AUTO checks how much cancellation the variance update
+// S2/N_k - (S1/N_k)^2 suffers: the statistics are raw moments about the global centre,
+// accurate to ~6e-7 relative, so the new variance carries a relative error of about
+// A * 6e-7 with A = (S2/N_k) / variance.  A component whose A exceeds kMaxAmplification
+// (tight cluster far from the centre, or one that collapsed onto a single point this
+// step) sends the whole step back to the CUDA-core path, whose statistics are centred
+// on each component's current mean.  One CTA per component.
+constexpr double kMaxAmplification = 512.0;
+
+__global__ void tc_variance_check_kernel(int K, int D, int Dp, int kstride,
+                                         const double* __restrict__ stats, int nslots,
+                                         int* mode) {
+  if (*mode != kModeTensor) return;
+  const int k = blockIdx.x;
+  const size_t row = (size_t)(1 + 2 * Dp);
+  double nk = 0.0;
+  for (int s = 0; s < nslots; ++s) nk += stats[((size_t)s * kstride + k) * row];
+  if (!(nk >= FGMM_EMPTY_NK)) return;  // empty: parameters are kept, nothing to check
+  bool bad = false;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    double s1 = 0.0, s2 = 0.0;
+    for (int s = 0; s < nslots; ++s) {
+      const double* r = stats + ((size_t)s * kstride + k) * row;
+      s1 += r[1 + d];
+      s2 += r[1 + Dp + d];
+    }
+    const double m2 = s2 / nk, m1 = s1 / nk;
+    const double v = m2 - m1 * m1;
+    if (!(v > 0.0) || !(m2 <= kMaxAmplification * v)) bad = true;
+  }
+  if (bad) atomicExch(mode, kModeSimt);
+}
+
+// When the step was sent back to the CUDA-core path after the tensor-core sweeps ran,
+// clear what they accumulated.  Grid-stride over the statistics slots.
+__global__ void redo_reset_kernel(const int* mode, double* __restrict__ stats, size_t n,
+                                  double* __restrict__ ll_total) {
+  if (*mode != kModeSimt) return;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    stats[i] = 0.0;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ll_total = 0.0;
+}
+
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_prep_simt(const Ctx& c, const float* weights, const float* means,
                              const float* vars, cudaStream_t s) {
@@ -517,11 +565,11 @@ cudaError_t launch_lse_simt(const Ctx& c, const void* X, int x_dtype, int64_t n,
 }
 
 cudaError_t launch_ll_accumulate(const Ctx& c, int64_t n, const int* mode, int fixed_mode,
-                                 cudaStream_t s) {
+                                 int required, cudaStream_t s) {
   prof_begin(c, KK_OTHER, s);
   ll_accumulate_kernel<<<1, kSimtThreads, 0, s>>>(c.ws.ll_tiles, (int)ceil_div64(n, kTP),
                                                   (int)ceil_div64(n, 128) * 4, mode, fixed_mode,
-                                                  c.ws.ll_total);
+                                                  required, c.ws.ll_total);
   prof_end(c, KK_OTHER, s);
   return cudaGetLastError();
 }
@@ -587,4 +635,20 @@ cudaError_t launch_soft_assign_simt(const Ctx& c, const void* X, int x_dtype, in
   return cudaGetLastError();
 }
 
+}  // namespace fgmm
+
+namespace fgmm {
+cudaError_t launch_auto_check_and_reset(const Ctx& c, cudaStream_t s) {
+  prof_begin(c, KK_OTHER, s);
+  tc_variance_check_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, c.ws.Dp, c.ws.KpS, c.ws.stats,
+                                                        tc_slices(c), c.ws.mode);
+  prof_end(c, KK_OTHER, s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t n = (size_t)c.ws.slots * c.ws.KpS * (1 + 2 * (size_t)c.ws.Dp);
+  prof_begin(c, KK_OTHER, s);
+  redo_reset_kernel<<<2 * c.num_sms, 256, 0, s>>>(c.ws.mode, c.ws.stats, n, c.ws.ll_total);
+  prof_end(c, KK_OTHER, s);
+  return cudaGetLastError();
+}
 }  // namespace fgmm
