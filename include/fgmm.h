@@ -139,6 +139,37 @@ int fgmm_soft_assign(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64
                      int top_m, float r_threshold, int32_t* ids, float* resp,
                      fgmm_stream_t stream);
 
+/* Soft assignment for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart to this call; it exists for the host programs that
+ * may not call cudaMalloc or cudaFree at all: applications whose device memory is
+ * owned by one arena reserved up front (servers, engines, embedded runtimes that
+ * account for every byte), and latency-critical loops where the allocator's implicit
+ * device synchronisation is not acceptable.  fgmm_create allocates a workspace, so
+ * those callers cannot use a handle.
+ *
+ * Same result as fgmm_soft_assign (§4.2-4.3) with the same arguments, but without a
+ * handle: K, D and cov_type are passed directly.  Its scratch (padded means,
+ * precisions and per-component constants) lives in one fixed array inside the
+ * library's own device memory, which every GPU that loads the library holds until
+ * the process exits (about 2.1 MB).  Limits: padded K x padded D <= FGMM_STATIC_MAX_KD
+ * and padded K <= FGMM_STATIC_MAX_K (K rounded up to 64, D to 32); larger problems
+ * return FGMM_ERR_UNSUPPORTED and enqueue nothing.
+ *
+ * The first call on a device looks up that array's device address (once per device,
+ * with that device current), and the CUDA runtime may allocate the array then if it
+ * loads modules lazily; make this first call before any stream capture.  Every
+ * call shares the array and overwrites what the previous call left there; calls that
+ * overlap on the GPU (two streams, two host threads) race on it and must be
+ * serialised by the caller.  The call synchronises the stream and returns the device
+ * status (FGMM_ERR_INVALID_ARG for invalid parameters), or the argument error. */
+#define FGMM_STATIC_MAX_KD (1 << 18)
+#define FGMM_STATIC_MAX_K (1 << 14)
+int fgmm_soft_assign_static(int K, int D, int cov_type, const void* X, int x_dtype, int64_t N,
+                            int64_t ldx, const float* weights, const float* means,
+                            const float* vars, int top_m, float r_threshold, int32_t* ids,
+                            float* resp, fgmm_stream_t stream);
+
 /* Kernel timing, for benchmarks.  When enabled, the library records a CUDA
  * event pair on the call's stream around every kernel it launches and keeps a
  * launch counter; fgmm_profile_read synchronises the device, sums the elapsed

@@ -17,6 +17,8 @@ PREC_FP32, PREC_FP16X3, PREC_FP16, PREC_AUTO = 0, 1, 2, 3
 F32, BF16 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_OOM, ERR_NUMERIC, ERR_TIMEOUT = range(7)
 MAX_TOP_M = 16
+STATIC_MAX_KD = 1 << 18
+STATIC_MAX_K = 1 << 14
 EMPTY_NK = 1e-6
 
 class Profile(ctypes.Structure):
@@ -45,6 +47,8 @@ SIGNATURES = {
     "fgmm_status_string": (_c.c_char_p, [_int]),
     "fgmm_profile_enable": (_int, [_vp, _int]),
     "fgmm_selftest_bounded_wait": (_int, [_int]),
+    "fgmm_soft_assign_static": (_int, [_int, _int, _int, _vp, _int, _i64, _i64, _vp, _vp, _vp,
+                                       _int, _flt, _vp, _vp, _vp]),
     "fgmm_profile_read": (_int, [_vp, _c.POINTER(Profile), _int]),
 }
 

@@ -119,6 +119,14 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
                           cudaStream_t s);
 cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream_t s);
 cudaError_t run_bounded_wait_probe(int64_t limit_ns, int* status_host);
+// soft assignment on caller-provided scratch (allocation-free entry point)
+cudaError_t launch_prep_simt_raw(int K, int D, int Kp, int Dp, int cov, const float* weights,
+                                 const float* means, const float* vars, float* mu, float* prec,
+                                 float* cconst, int* status, cudaStream_t s);
+cudaError_t launch_soft_assign_simt_raw(const void* X, int x_dtype, int64_t n, int64_t ldx, int K,
+                                        int D, int Kp, int Dp, const float* mu, const float* prec,
+                                        const float* cconst, int top_m, float r_threshold,
+                                        int32_t* ids, float* resp, cudaStream_t s);
 cudaError_t launch_soft_assign_simt(const Ctx& c, const void* X, int x_dtype, int64_t n,
                                     int64_t ldx, int top_m, float r_threshold, int32_t* ids,
                                     float* resp, cudaStream_t s);

@@ -652,3 +652,30 @@ cudaError_t launch_auto_check_and_reset(const Ctx& c, cudaStream_t s) {
   return cudaGetLastError();
 }
 }  // namespace fgmm
+
+namespace fgmm {
+// Launchers on explicit buffers (no handle), for the allocation-free entry point.
+cudaError_t launch_prep_simt_raw(int K, int D, int Kp, int Dp, int cov, const float* weights,
+                                 const float* means, const float* vars, float* mu, float* prec,
+                                 float* cconst, int* status, cudaStream_t s) {
+  prep_simt_kernel<<<Kp, kSimtThreads, 0, s>>>(K, D, Kp, Dp, cov, weights, means, vars, mu, prec,
+                                               cconst, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_soft_assign_simt_raw(const void* X, int x_dtype, int64_t n, int64_t ldx, int K,
+                                        int D, int Kp, int Dp, const float* mu, const float* prec,
+                                        const float* cconst, int top_m, float r_threshold,
+                                        int32_t* ids, float* resp, cudaStream_t s) {
+  const unsigned grid = (unsigned)ceil_div64(n, kTP);
+  if (x_dtype == FGMM_BF16)
+    soft_assign_simt_kernel<<<grid, kSimtThreads, 0, s>>>((const __nv_bfloat16*)X, n, ldx, D, Dp,
+                                                          Kp, K, mu, prec, cconst, top_m,
+                                                          r_threshold, ids, resp);
+  else
+    soft_assign_simt_kernel<<<grid, kSimtThreads, 0, s>>>((const float*)X, n, ldx, D, Dp, Kp, K,
+                                                          mu, prec, cconst, top_m, r_threshold,
+                                                          ids, resp);
+  return cudaGetLastError();
+}
+}  // namespace fgmm
