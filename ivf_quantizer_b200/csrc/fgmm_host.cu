@@ -90,8 +90,10 @@ int map_cuda(cudaError_t e) {
 }
 
 void free_ws(Workspace& w) {
-  void* ptrs[] = {w.mu,   w.prec,   w.cconst, w.logz, w.ll_tiles, w.ll_total, w.stats, w.nk,
-                  w.status, w.center, w.dscale, w.wop, w.tck,     w.tks,      w.xop,   w.mode};
+  void* ptrs[] = {w.mu,     w.prec,   w.cconst, w.logz, w.ll_tiles, w.ll_total,
+                  w.stats,  w.nk,     w.status, w.center, w.dscale, w.wop,
+                  w.tck,    w.tks,    w.xop,    w.mode, w.stiff,    w.stiff_list, w.n_stiff,
+                  w.side_part};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -137,7 +139,17 @@ cudaError_t alloc_ws(Ctx& c) {
   if ((e = cudaMemset(w.status, 0, sizeof(int))) != cudaSuccess) return e;
   if ((e = cudaMemset(w.center, 0, w.Dq * sizeof(float))) != cudaSuccess) return e;
   if ((e = cudaMemset(w.dscale, 0, w.Dq * sizeof(float))) != cudaSuccess) return e;
+  // the previous step's N_k feeds AUTO's "about to collapse" test: start far above it
+  if ((e = cudaMemset(w.nk, 0x7F, (size_t)w.KpS * sizeof(double))) != cudaSuccess) return e;
   if (tc) {
+    if ((e = alloc(&w.stiff, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.stiff_list, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.n_stiff, (size_t)1, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.side_part, (size_t)kSideParts * kSideMaxStiff * (1 + 2 * (size_t)w.Dp), &t)) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaMemset(w.stiff, 0, (size_t)w.Kt * sizeof(int))) != cudaSuccess) return e;
+    if ((e = cudaMemset(w.n_stiff, 0, sizeof(int))) != cudaSuccess) return e;
     if ((e = alloc(&w.wop, (size_t)2 * w.Kt * w.K1, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.tck, (size_t)w.Kt, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.tks, (size_t)w.Kt, &t)) != cudaSuccess) return e;
@@ -185,7 +197,7 @@ int fgmm_create(int K, int D, int cov_type, double reg_covar, fgmm_handle* out) 
   h->c.D = D;
   h->c.cov = cov_type;
   h->c.reg = reg_covar;
-  h->c.prec = FGMM_PREC_FP32;
+  h->c.prec = FGMM_PREC_AUTO;
   if (cudaGetDevice(&h->c.device) != cudaSuccess ||
       cudaDeviceGetAttribute(&h->c.num_sms, cudaDevAttrMultiProcessorCount, h->c.device) !=
           cudaSuccess) {
@@ -264,9 +276,12 @@ int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t l
     return map_cuda(e);
   if (run_simt && (e = launch_prep_simt(c, weights, means, vars, s)) != cudaSuccess)
     return map_cuda(e);
-  if (run_tc && (e = launch_tc_prep(c, weights, means, vars, auto_mode ? w.mode : nullptr, s)) !=
-                    cudaSuccess)
-    return map_cuda(e);
+  if (run_tc) {
+    if ((e = launch_tc_prep(c, weights, means, vars, auto_mode, s)) != cudaSuccess)
+      return map_cuda(e);
+    if ((e = launch_stiff_compact(c, auto_mode ? w.mode : nullptr, s)) != cudaSuccess)
+      return map_cuda(e);
+  }
   const size_t eb = dtype_bytes(x_dtype);
   if (run_tc) {
     for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
@@ -276,9 +291,14 @@ int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t l
       if ((e = launch_tc_convert(c, Xc, x_dtype, nc, ldx, mode, s)) != cudaSuccess)
         return map_cuda(e);
       if ((e = launch_tc_lse(c, nc, lzo, mode, s)) != cudaSuccess) return map_cuda(e);
+      // stiff components (AUTO) join log Z here; then the chunk's log-likelihood
+      if ((e = launch_side_lse(c, Xc, x_dtype, nc, ldx, lzo, mode, s)) != cudaSuccess)
+        return map_cuda(e);
       if ((e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeTensor, s)) != cudaSuccess)
         return map_cuda(e);
       if ((e = launch_tc_stats(c, nc, mode, s)) != cudaSuccess) return map_cuda(e);
+      if ((e = launch_side_stats(c, Xc, x_dtype, nc, ldx, mode, s)) != cudaSuccess)
+        return map_cuda(e);
     }
   }
   // AUTO: a step whose new variances would lose accuracy to cancellation is sent back

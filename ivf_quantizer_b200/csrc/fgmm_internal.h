@@ -22,6 +22,8 @@ constexpr int kFC = 128;       // features per CTA in the statistics sweep
 constexpr int kSlices = 16;    // point slices of a chunk in the statistics sweep
 constexpr int kFlushTiles = 64;  // fp32 run length (tiles) before an fp64 flush
 constexpr int64_t kChunk = 1 << 20;  // points per chunk: bounds every N-sized buffer
+constexpr int kSideMaxStiff = 256;   // AUTO side path: most stiff components per step
+constexpr int kSideParts = 64;       // AUTO side path: point ranges per chunk
 
 static inline int round_up(int a, int b) { return (a + b - 1) / b * b; }
 static inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -46,6 +48,10 @@ struct Workspace {
   float* tks = nullptr;     // [Kt] 2^t_k
   __half* xop = nullptr;    // [2][kChunk][K1] phi(x) hi / lo of the current chunk
   int* mode = nullptr;      // [1] path of the current step: 0 tensor cores, 1 CUDA cores
+  int* stiff = nullptr;     // [Kt] AUTO: 1 = component handled by the CUDA-core side path
+  int* stiff_list = nullptr;  // [Kt] stiff components in index order
+  int* n_stiff = nullptr;   // [1]
+  double* side_part = nullptr;  // [kSideParts][kSideMaxStiff][1 + 2 Dp] side-path partial rows
   // prepared parameters (CUDA-core path)
   float* mu = nullptr;     // [Kp, Dp] means, zero padded
   float* prec = nullptr;   // [Kp, Dp] -1/(2 sigma^2), zero padded
@@ -112,7 +118,13 @@ bool tc_supported(const Ctx& c);
 cudaError_t tc_init(Ctx& c);
 int tc_slices(const Ctx& c);
 cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* means,
-                           const float* vars, int* mode, cudaStream_t s);
+                           const float* vars, bool auto_mode, cudaStream_t s);
+// AUTO side path for stiff components (fgmm_side.cu)
+cudaError_t launch_stiff_compact(const Ctx& c, int* mode, cudaStream_t s);
+cudaError_t launch_side_lse(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                            float* logz_out, const int* mode, cudaStream_t s);
+cudaError_t launch_side_stats(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                              const int* mode, cudaStream_t s);
 cudaError_t launch_tc_convert(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
                               const int* mode, cudaStream_t s);
 cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* mode,

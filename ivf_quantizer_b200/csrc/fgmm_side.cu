@@ -1,0 +1,286 @@
+// Side path of the AUTO mode: the few components that the tensor-core expanded form
+// cannot evaluate accurately ("stiff": collapsed onto a point, very few effective
+// points, or tight and far from the coordinate centre) are taken out of the tensor-core
+// sweeps (their c_k is -inf there) and handled here on CUDA cores in the direct form
+// sum_d -(x_d - mu_kd)^2 / (2 sigma_kd^2), with statistics centred on their current mean
+// ("Flash-GMM: A Memory-Efficient Kernel for Scalable Soft Clustering", §2 for the
+// density and Eqs. (1)-(3); the same quantities as the tensor-core sweeps, exactly).
+//
+//   stiff_compact      ordered list of the stiff components (deterministic)
+//   side_lse           per point: log Z <- logsumexp(log Z_tensor, log z_ik for stiff k)
+//   ll_partials        per-block fp64 sums of the chunk's log Z (fixed order)
+//   side_stats         per stiff component: N_k, sum r (x - mu), sum r (x - mu)^2
+//
+// A stiff component's log-density is evaluated dimension by dimension and abandoned
+// as soon as its upper bound (the constant plus the partial sum, every remaining term
+// being <= 0) falls more than kCut nats below the point's log Z: its responsibility
+// would be exp(-kCut) < 1e-52, zero in fp32.  A collapsed component costs one or two
+// dimensions per point.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "fgmm_internal.h"
+
+namespace fgmm {
+namespace {
+
+constexpr float kCut = 120.f;
+
+__device__ __forceinline__ float ldx_f(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float ldx_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+// Direct-form log z for one point and one component, abandoned (returns -inf) once the
+// bound drops below `floor`.
+template <typename T>
+__device__ __forceinline__ float stiff_logit(const T* __restrict__ x, int D,
+                                             const float* __restrict__ mu,
+                                             const float* __restrict__ prec, float c,
+                                             float floor) {
+  if (!(c > floor)) return -CUDART_INF_F;
+  float acc = 0.f;  // sum of prec (x - mu)^2, prec = -1/(2 sigma^2) <= 0
+  int d = 0;
+  for (; d < D; ++d) {
+    const float t = ldx_f(x + d) - mu[d];
+    acc = fmaf(prec[d] * t, t, acc);
+    if ((d & 3) == 3 && c + acc < floor) return -CUDART_INF_F;
+  }
+  return c + acc;
+}
+
+}  // namespace
+
+// One CTA: stiff_list = the stiff components in increasing index order, n = their count.
+// More than kMaxStiff stiff components: the side path would cost as much as the
+// CUDA-core path, so the whole step goes there (mode word).
+constexpr int kMaxStiff = kSideMaxStiff;
+
+__global__ void stiff_compact_kernel(const int* __restrict__ stiff, int K, int* __restrict__ list,
+                                     int* __restrict__ n_out, int* mode) {
+  if (mode && *mode != kModeTensor) return;
+  __shared__ int base;
+  if (threadIdx.x == 0) base = 0;
+  __syncthreads();
+  for (int k0 = 0; k0 < K; k0 += blockDim.x) {
+    const int k = k0 + threadIdx.x;
+    const int f = (k < K) ? stiff[k] : 0;
+    // block-wide exclusive scan of f by warp ballots (order = component index)
+    const unsigned m = __ballot_sync(0xffffffffu, f);
+    __shared__ int wsum[32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    if (lane == 0) wsum[w] = __popc(m);
+    __syncthreads();
+    int off = base;
+    for (int i = 0; i < w; ++i) off += wsum[i];
+    if (f) list[off + __popc(m & ((1u << lane) - 1u))] = k;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int t = 0;
+      for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += wsum[i];
+      base += t;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    *n_out = base;
+    if (mode && base > kMaxStiff) *mode = kModeSimt;
+  }
+}
+
+// Thread per point: merge the stiff components' log-densities into log Z.
+template <typename T>
+__global__ void side_lse_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp,
+                                const float* __restrict__ mu, const float* __restrict__ prec,
+                                const float* __restrict__ cconst, const int* __restrict__ list,
+                                const int* __restrict__ n_stiff, float* __restrict__ logz,
+                                float* __restrict__ logz_out, const int* mode) {
+  if (mode && *mode != kModeTensor) return;
+  const int ns = *n_stiff;
+  if (ns == 0) return;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const T* x = X + i * ldx;
+  float lz = logz[i];
+  for (int j = 0; j < ns; ++j) {
+    const int k = list[j];
+    const float l = stiff_logit(x, D, mu + (size_t)k * Dp, prec + (size_t)k * Dp, cconst[k],
+                                lz - kCut);
+    if (l > -CUDART_INF_F) {
+      const float m = fmaxf(lz, l);
+      lz = (lz > -CUDART_INF_F) ? m + log1pf(expf(fminf(lz, l) - m)) : l;
+    }
+  }
+  logz[i] = lz;
+  if (logz_out) logz_out[i] = lz;
+}
+
+// Fixed-order per-block fp64 sums of log Z over [b * 4096, (b + 1) * 4096).
+__global__ void ll_partials_kernel(const float* __restrict__ logz, int64_t n,
+                                   double* __restrict__ part, const int* mode) {
+  if (mode && *mode != kModeTensor) return;
+  __shared__ double red[256];
+  const int64_t b0 = (int64_t)blockIdx.x * 4096;
+  double s = 0.0;
+  for (int e = threadIdx.x; e < 4096; e += 256) {
+    const int64_t i = b0 + e;
+    if (i < n) s += (double)logz[i];
+  }
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) part[blockIdx.x] = red[0];
+}
+
+// Grid (kSideMaxStiff, kSideParts): CTA (j, p) folds stiff component list[j] over the
+// p-th of kSideParts equal point ranges of the chunk.  Each warp takes a contiguous part
+// of the range; for a batch of 32 points the lanes evaluate r = exp(log z - log Z), and
+// the points with r > 0 are folded into the warp's shared-memory sums by the whole warp
+// (lanes over dimensions, points in index order).  The 8 warp sums are combined in warp
+// order and written as this CTA's partial row; side_reduce adds the partial rows, in p
+// order, to the component's statistics.  Everything is deterministic.
+struct SideAcc {
+  float s1[128];   // the tensor-core path (and so this side path) has D <= 128
+  float s2[128];
+  float nk;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    side_stats_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp,
+                      const float* __restrict__ mu, const float* __restrict__ prec,
+                      const float* __restrict__ cconst, const int* __restrict__ list,
+                      const int* __restrict__ n_stiff, const float* __restrict__ logz,
+                      double* __restrict__ part, const int* mode) {
+  if (mode && *mode != kModeTensor) return;
+  const int j = blockIdx.x;
+  if (j >= *n_stiff) return;
+  __shared__ SideAcc acc[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = list[j];
+  const float* muk = mu + (size_t)k * Dp;
+  const float* pk = prec + (size_t)k * Dp;
+  const float ck = cconst[k];
+  const int64_t range = (n + kSideParts - 1) / kSideParts;
+  const int64_t p0 = (int64_t)blockIdx.y * range, p1 = min(n, p0 + range);
+  const int64_t wlen = (range + 7) / 8;
+  const int64_t w0 = p0 + warp * wlen, w1 = min(p1, w0 + wlen);
+  SideAcc& a = acc[warp];
+  for (int d = lane; d < 128; d += 32) { a.s1[d] = 0.f; a.s2[d] = 0.f; }
+  float nk = 0.f;
+  __syncwarp();
+  for (int64_t b = w0; b < w1; b += 32) {
+    const int64_t i = b + lane;
+    float r = 0.f;
+    if (i < w1) {
+      const float lz = logz[i];
+      const float l = stiff_logit(X + i * ldx, D, muk, pk, ck, lz - kCut);
+      if (l > -CUDART_INF_F && lz > -CUDART_INF_F) r = fminf(expf(l - lz), 1.f);
+    }
+    unsigned live = __ballot_sync(0xffffffffu, r > 0.f);
+    while (live) {
+      const int src = __ffs(live) - 1;
+      live &= live - 1;
+      const float rr = __shfl_sync(0xffffffffu, r, src);
+      const T* x = X + (b + src) * ldx;
+      for (int d = lane; d < D; d += 32) {
+        const float t = ldx_f(x + d) - muk[d];
+        const float rt = rr * t;
+        a.s1[d] += rt;
+        a.s2[d] = fmaf(rt, t, a.s2[d]);
+      }
+      nk += rr;   // the same running sum in every lane
+    }
+  }
+  if (lane == 0) a.nk = nk;
+  __syncthreads();
+  const size_t row = (size_t)(1 + 2 * Dp);
+  double* dst = part + ((size_t)blockIdx.y * kSideMaxStiff + j) * row;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float s1 = 0.f, s2 = 0.f;
+    for (int w = 0; w < 8; ++w) { s1 += acc[w].s1[d]; s2 += acc[w].s2[d]; }
+    dst[1 + d] = (double)s1;
+    dst[1 + Dp + d] = (double)s2;
+  }
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < 8; ++w) t += acc[w].nk;
+    dst[0] = (double)t;
+  }
+}
+
+// One CTA per stiff slot j: the kSideParts partial rows, summed in p order, are added to
+// the statistics of component list[j] (slot 0 of the point slices; the tensor-core
+// sweep added zeros there, the component being masked out of it).
+__global__ void side_reduce_kernel(const double* __restrict__ part, const int* __restrict__ list,
+                                   const int* __restrict__ n_stiff, int D, int Dp,
+                                   double* __restrict__ stats, const int* mode) {
+  if (mode && *mode != kModeTensor) return;
+  const int j = blockIdx.x;
+  if (j >= *n_stiff) return;
+  const size_t row = (size_t)(1 + 2 * Dp);
+  double* dst = stats + (size_t)list[j] * row;
+  for (int c = threadIdx.x; c < (int)row; c += blockDim.x) {
+    const int d = (c == 0) ? 0 : (c <= Dp ? c - 1 : c - 1 - Dp);
+    if (c != 0 && d >= D) continue;
+    double s = 0.0;
+    for (int p = 0; p < kSideParts; ++p) s += part[((size_t)p * kSideMaxStiff + j) * row + c];
+    dst[c] += s;
+  }
+}
+
+// ------------------------------------------------------------------ launchers
+cudaError_t launch_stiff_compact(const Ctx& c, int* mode, cudaStream_t s) {
+  prof_begin(c, KK_OTHER, s);
+  stiff_compact_kernel<<<1, 256, 0, s>>>(c.ws.stiff, c.K, c.ws.stiff_list, c.ws.n_stiff, mode);
+  prof_end(c, KK_OTHER, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_side_lse(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                            float* logz_out, const int* mode, cudaStream_t s) {
+  const unsigned grid = (unsigned)ceil_div64(n, 128);
+  const Workspace& w = c.ws;
+  prof_begin(c, KK_OTHER, s);
+  if (x_dtype == FGMM_BF16)
+    side_lse_kernel<<<grid, 128, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
+                                         w.cconst, w.stiff_list, w.n_stiff, w.logz, logz_out,
+                                         mode);
+  else
+    side_lse_kernel<<<grid, 128, 0, s>>>((const float*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
+                                         w.cconst, w.stiff_list, w.n_stiff, w.logz, logz_out,
+                                         mode);
+  prof_end(c, KK_OTHER, s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  prof_begin(c, KK_OTHER, s);
+  ll_partials_kernel<<<(unsigned)ceil_div64(n, 4096), 256, 0, s>>>(w.logz, n, w.ll_tiles, mode);
+  prof_end(c, KK_OTHER, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_side_stats(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                              const int* mode, cudaStream_t s) {
+  const Workspace& w = c.ws;
+  dim3 grid(kSideMaxStiff, kSideParts);
+  prof_begin(c, KK_OTHER, s);
+  if (x_dtype == FGMM_BF16)
+    side_stats_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dp, w.mu,
+                                           w.prec, w.cconst, w.stiff_list, w.n_stiff, w.logz,
+                                           w.side_part, mode);
+  else
+    side_stats_kernel<<<grid, 256, 0, s>>>((const float*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
+                                           w.cconst, w.stiff_list, w.n_stiff, w.logz,
+                                           w.side_part, mode);
+  prof_end(c, KK_OTHER, s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  prof_begin(c, KK_OTHER, s);
+  side_reduce_kernel<<<kSideMaxStiff, 256, 0, s>>>(w.side_part, w.stiff_list, w.n_stiff, c.D,
+                                                   w.Dp, w.stats, mode);
+  prof_end(c, KK_OTHER, s);
+  return cudaGetLastError();
+}
+
+}  // namespace fgmm

@@ -75,7 +75,10 @@ __global__ void prep_simt_kernel(int K, int D, int Kp, int Dp, int cov, const fl
 // ------------------------------------------------------------------ shared logit tile
 // Computes acc[j][q] = sum_d prec_kd (x_id - mu_kd)^2 for points r = ty + 16 j of the
 // tile and components kb + tx + 16 q, looping over the features in chunks of kDC staged
-// in shared memory.  NJ points x NQ components per thread.
+// in shared memory.  NJ points x NQ components per thread.  Each chunk's 32 terms are
+// summed in fp32 and the chunk sums in fp64, so that the rounding of the sum does not
+// grow with D (at D = 960 a plain fp32 sum of log-densities near -2700 carries ~5e-3
+// nats of error, enough to move the responsibilities of shared points by 0.5%).
 template <int NQ, typename T>
 __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, int64_t ldx, int D,
                                            int Dp, int64_t i0, int kb,
@@ -85,11 +88,16 @@ __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, i
                                            float (*ps)[kDC + 4], float (&acc)[4][NQ]) {
   constexpr int KBLK = 16 * NQ;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  double dacc[4][NQ];
 #pragma unroll
   for (int j = 0; j < 4; ++j)
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) acc[j][q] = 0.f;
+    for (int q = 0; q < NQ; ++q) dacc[j][q] = 0.0;
   for (int d0 = 0; d0 < Dp; d0 += kDC) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) acc[j][q] = 0.f;
     for (int e = threadIdx.x; e < kTP * kDC; e += kSimtThreads) {
       const int r = e / kDC, cx = e % kDC;
       const int64_t i = i0 + r;
@@ -124,7 +132,15 @@ __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, i
         }
     }
     __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) dacc[j][q] += (double)acc[j][q];
   }
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) acc[j][q] = (float)dacc[j][q];
 }
 
 // ------------------------------------------------------------------ sweep 1: log Z_i
@@ -346,14 +362,18 @@ __global__ void __launch_bounds__(kSimtThreads)
 // written when the log-likelihood of the step is not finite.
 __global__ void mstep_kernel(int K, int D, int Dp, int kstride, int cov, double reg,
                              const double* __restrict__ stats, int s_simt, int s_tc,
-                             const int* mode, int fixed_mode, const float* __restrict__ mu_old,
+                             const int* mode, int fixed_mode, const int* __restrict__ stiff,
+                             const float* __restrict__ mu_old,
                              const float* __restrict__ center, const float* __restrict__ dscale,
                              const double* __restrict__ ll_total, float* __restrict__ means,
                              float* __restrict__ vars, double* __restrict__ nk_out, int* status) {
   __shared__ double red[kSimtThreads];
   const int k = blockIdx.x;
-  const bool simt = ((mode ? *mode : fixed_mode) == kModeSimt);
-  const int nslots = simt ? s_simt : s_tc;
+  const bool simt_step = ((mode ? *mode : fixed_mode) == kModeSimt);
+  const int nslots = simt_step ? s_simt : s_tc;
+  // a stiff component of a tensor-core step was handled by the side path, whose
+  // statistics are centred on the current mean like the CUDA-core path's
+  const bool simt = simt_step || (stiff && stiff[k]);
   const size_t row = (size_t)(1 + 2 * Dp);
   const bool ll_ok = isfinite(*ll_total);
   double nk = 0.0;
@@ -494,19 +514,22 @@ __global__ void __launch_bounds__(kSimtThreads)
 
 // ------------------------------------------------------------------ AUTO: variance check
 // After the tensor-core sweeps, AUTO checks how much cancellation the variance update
-// S2/N_k - (S1/N_k)^2 suffers: the statistics are raw moments about the global centre,
-// accurate to ~6e-7 relative, so the new variance carries a relative error of about
-// A * 6e-7 with A = (S2/N_k) / variance.  A component whose A exceeds kMaxAmplification
-// (tight cluster far from the centre, or one that collapsed onto a single point this
-// step) sends the whole step back to the CUDA-core path, whose statistics are centred
-// on each component's current mean.  One CTA per component.
-constexpr double kMaxAmplification = 512.0;
+// S2/N_k - (S1/N_k)^2 suffers.  The statistics are raw moments about the global centre,
+// accumulated in fp32 for 8 tiles (64 MMA steps) before each fp64 flush: about
+// 2^-24 sqrt(64/3) sqrt(2) = 3.9e-7 relative (rms) on S1 and S2, so the new variance
+// carries a relative error of about 3.9e-7 A with A = (S2/N_k) / variance.  A component
+// whose A exceeds kMaxAmplification (a tight cluster far from the centre, or one that
+// collapsed onto a single point this step) sends the whole step back to the CUDA-core
+// path, whose statistics are centred on each component's current mean.  At the bound
+// the expected error is 3.5e-4, a third of the 1e-3 tolerance.  One CTA per component.
+constexpr double kMaxAmplification = 900.0;
 
 __global__ void tc_variance_check_kernel(int K, int D, int Dp, int kstride,
                                          const double* __restrict__ stats, int nslots,
-                                         int* mode) {
+                                         const int* __restrict__ stiff, int* mode) {
   if (*mode != kModeTensor) return;
   const int k = blockIdx.x;
+  if (stiff[k]) return;  // the side path's statistics are centred on the mean: exact
   const size_t row = (size_t)(1 + 2 * Dp);
   double nk = 0.0;
   for (int s = 0; s < nslots; ++s) nk += stats[((size_t)s * kstride + k) * row];
@@ -568,7 +591,7 @@ cudaError_t launch_ll_accumulate(const Ctx& c, int64_t n, const int* mode, int f
                                  int required, cudaStream_t s) {
   prof_begin(c, KK_OTHER, s);
   ll_accumulate_kernel<<<1, kSimtThreads, 0, s>>>(c.ws.ll_tiles, (int)ceil_div64(n, kTP),
-                                                  (int)ceil_div64(n, 128) * 4, mode, fixed_mode,
+                                                  (int)ceil_div64(n, 4096), mode, fixed_mode,
                                                   required, c.ws.ll_total);
   prof_end(c, KK_OTHER, s);
   return cudaGetLastError();
@@ -606,7 +629,8 @@ cudaError_t launch_mstep(const Ctx& c, float* weights, float* means, float* vars
   prof_begin(c, KK_OTHER, s);
   mstep_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, c.ws.Dp, c.ws.KpS, c.cov, c.reg, c.ws.stats,
                                             kSlices, c.tc.ready ? tc_slices(c) : 1, mode,
-                                            fixed_mode, c.ws.mu, c.ws.center, c.ws.dscale,
+                                            fixed_mode, c.tc.ready ? c.ws.stiff : nullptr,
+                                            c.ws.mu, c.ws.center, c.ws.dscale,
                                             c.ws.ll_total, means, vars, c.ws.nk, c.ws.status);
   prof_end(c, KK_OTHER, s);
   cudaError_t e = cudaGetLastError();
@@ -641,7 +665,7 @@ namespace fgmm {
 cudaError_t launch_auto_check_and_reset(const Ctx& c, cudaStream_t s) {
   prof_begin(c, KK_OTHER, s);
   tc_variance_check_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, c.ws.Dp, c.ws.KpS, c.ws.stats,
-                                                        tc_slices(c), c.ws.mode);
+                                                        tc_slices(c), c.ws.stiff, c.ws.mode);
   prof_end(c, KK_OTHER, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -21,6 +21,9 @@
 // tolerance on the Table-1 generator; bf16 splits (16 bits) pass with little margin.
 // Statistics: r is scaled by 2^15 and rounded once to fp16 (the same rounded values
 // feed N_k and the GEMM, so the weights stay consistent); phi is split hi/lo, two MMAs.
+// The moments are raw (about the global centre): the variance of a component whose
+// spread is small next to its distance from the centre loses accuracy to cancellation,
+// which AUTO detects after the sweeps (see the M-step kernels).
 //
 // Kernels (one chunk of <= 2^20 points at a time):
 //   tc_center     per-dimension centre and scale from the parameters
@@ -125,28 +128,33 @@ __global__ void tc_center_kernel(int K, int D, int cov, const float* __restrict_
 // One CTA per padded component k (grid Kt).  Writes W' = W 2^-t_k as fp16 hi/lo into
 // wop[part][k][j] (part 0 hi, 1 lo; j < Dq the linear terms, Dq + d the squares),
 // c_k (fp64 sums, -inf for an absent or zero-weight component) and 2^t_k.
-// Conditioning check: the split product keeps ~2^-22 relative error per term; near
-// x = mu_k the terms reach t_d = 1.5 (|mu~| + sigma)^2 / sigma^2 and cancel, so the
-// expected logit error is ~2^-20 sqrt(sum_d t_d^2).  Above 1e-3 nats the component is
-// "stiff" and AUTO mode runs this step on the fp32 CUDA-core path instead.
+// Stiff components (AUTO only, when `stiff` is non-null) are left to the CUDA-core
+// side path: their c_k here is -inf, so the tensor-core sweeps ignore them.  A live
+// component is stiff when
+//   * its expanded-form logit error, ~2^-20 sqrt(sum_d t_d^2) with
+//     t_d = 1.5 (|mu~| + sigma)^2 / sigma^2 (the size of the cancelling terms near
+//     its mean), exceeds 1e-3 nats (a collapsed or very tight component);
+//   * its variance update would cancel: A_d = 1 + mu~_d^2 / sigma_d^2 > 900 for some d;
+//   * it had fewer than 4 effective points in the previous step (about to collapse).
 __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
                                const float* __restrict__ w, const float* __restrict__ means,
                                const float* __restrict__ vars, const float* __restrict__ center,
-                               const float* __restrict__ scale, __half* __restrict__ wop,
-                               float* __restrict__ ck, float* __restrict__ kscale, int* mode,
+                               const float* __restrict__ scale, const double* __restrict__ nk_prev,
+                               __half* __restrict__ wop, float* __restrict__ ck,
+                               float* __restrict__ kscale, int* __restrict__ stiff,
                                int* status) {
   __shared__ double rs[kSimtThreads], rq[kSimtThreads], rt[kSimtThreads];
-  __shared__ float rmax[kSimtThreads];
+  __shared__ float rmax[kSimtThreads], amax[kSimtThreads];
   __shared__ float s_pow;
   const int k = blockIdx.x;
   const int K1 = 2 * Dq;
   __half* hi = wop + (size_t)k * K1;
   __half* lo = wop + ((size_t)Kt + k) * K1;
-  double slog = 0.0, squad = 0.0, stiff = 0.0;
-  float wmax = 0.f;
+  double slog = 0.0, squad = 0.0, stf = 0.0;
+  float wmax = 0.f, amp = 0.f;
   bool bad = false;
   const bool live_k = k < K;
-  // pass 1: constants and max |W|
+  // pass 1: constants, max |W|, conditioning
   for (int d = threadIdx.x; d < Dq; d += blockDim.x) {
     if (live_k && d < D) {
       const double v = (cov == FGMM_COV_DIAG) ? vars[(size_t)k * D + d] : vars[k];
@@ -160,13 +168,15 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
       const double a = mt * p / sd, b = -0.5 * p / (sd * sd);
       wmax = fmaxf(wmax, (float)fmax(fabs(a), fabs(b)));
       const double t = 1.5 * (fabs(mt) + sqrt(v)) * (fabs(mt) + sqrt(v)) * p;
-      stiff += t * t;
+      stf += t * t;
+      amp = fmaxf(amp, (float)(1.0 + mt * mt * p));
     }
   }
   rs[threadIdx.x] = slog;
   rq[threadIdx.x] = squad;
-  rt[threadIdx.x] = stiff;
+  rt[threadIdx.x] = stf;
   rmax[threadIdx.x] = wmax;
+  amax[threadIdx.x] = amp;
   __syncthreads();
   for (int s = blockDim.x / 2; s > 0; s >>= 1) {
     if (threadIdx.x < s) {
@@ -174,19 +184,27 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
       rq[threadIdx.x] += rq[threadIdx.x + s];
       rt[threadIdx.x] += rt[threadIdx.x + s];
       rmax[threadIdx.x] = fmaxf(rmax[threadIdx.x], rmax[threadIdx.x + s]);
+      amax[threadIdx.x] = fmaxf(amax[threadIdx.x], amax[threadIdx.x + s]);
     }
     __syncthreads();
   }
   if (threadIdx.x == 0) {
     float c = -CUDART_INF_F;
     float pw = 1.f;
+    int is_stiff = 0;
     if (live_k) {
       const float wk = w[k];
       if (!(wk >= 0.f) || !isfinite(wk)) bad = true;
       if (wk > 0.f) c = (float)(log((double)wk) - 0.5 * rs[0] - 0.5 * rq[0]);
       const float mx = rmax[0];
       if (mx > 0.f && isfinite(mx)) pw = exp2f(ceilf(log2f(mx)) - 14.f);
-      if (mode && !(ldexp(sqrt(rt[0]), -20) <= 1e-3)) atomicExch(mode, 1);
+      if (stiff && wk > 0.f)
+        is_stiff = !(ldexp(sqrt(rt[0]), -20) <= 1e-3) || !(amax[0] <= 900.f) ||
+                   (nk_prev[k] < 4.0);
+    }
+    if (stiff) {
+      stiff[k] = is_stiff;
+      if (is_stiff) c = -CUDART_INF_F;
     }
     ck[k] = c;
     kscale[k] = pw;
@@ -253,28 +271,39 @@ __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ld
 }
 
 // ------------------------------------------------------------------ sweep 1 (log Z)
+// 384 threads: warp 0 TMA producer, warp 1 MMA issuer, warps 4..11 epilogue.  The two
+// epilogue warpgroups split each 128-column S tile in halves (columns 64g .. 64g+63) and
+// keep a running (max, sum) per row; at the end of a tile the upper half hands its
+// pair to the lower half through shared memory, which writes log Z.
+constexpr int kEpiWarps = 8;
+constexpr int kTcThreads = 128 + 32 * kEpiWarps;
+
 struct LseBars {
   uint64_t x_full[4], x_empty[4];
   uint64_t w_full[SW], w_empty[SW];
   uint64_t s_full[2], s_empty[2];
+  uint64_t xc_full[2], xc_empty[2];
   uint64_t drain;
   uint32_t tmem;
   int abort;
+  float xm[2][BM], xs[2][BM];
 };
 
 template <int NKC>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
     tc_lse_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                   int nc, int ncmax, int Kt, const float* __restrict__ ck,
-                  const float* __restrict__ kscale, float* __restrict__ logz,
+                  const float* __restrict__ kscale, int params_in_smem, float* __restrict__ logz,
                   float* __restrict__ logz_out, double* __restrict__ ll_tiles, const int* mode,
                   int* status) {
-  if (mode && *mode != 0) return;
+  if (mode && *mode != kModeTensor) return;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   unsigned char* xbuf = base;                         // [2][NKC][BOX]
   unsigned char* wring = base + 2 * NKC * BOX;        // [SW][BOX]
   LseBars* bars = reinterpret_cast<LseBars*>(wring + SW * BOX);
+  float* ckl = reinterpret_cast<float*>(bars + 1);    // [Kt] c_k log2(e)   (if staged)
+  float* ksl = ckl + Kt;                              // [Kt] 2^t_k log2(e) (if staged)
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -284,11 +313,21 @@ __global__ void __launch_bounds__(256, 1)
   if (threadIdx.x == 0) {
     for (int c = 0; c < 4; ++c) { ptx::mbar_init(&bars->x_full[c], 1); ptx::mbar_init(&bars->x_empty[c], 1); }
     for (int s = 0; s < SW; ++s) { ptx::mbar_init(&bars->w_full[s], 1); ptx::mbar_init(&bars->w_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { ptx::mbar_init(&bars->s_full[b], 1); ptx::mbar_init(&bars->s_empty[b], 4); }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&bars->s_full[b], 1);
+      ptx::mbar_init(&bars->s_empty[b], kEpiWarps);
+      ptx::mbar_init(&bars->xc_full[b], kEpiWarps / 2);
+      ptx::mbar_init(&bars->xc_empty[b], kEpiWarps / 2);
+    }
     ptx::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
+  if (params_in_smem)
+    for (int k = threadIdx.x; k < Kt; k += blockDim.x) {
+      ckl[k] = ck[k] * kLog2e;
+      ksl[k] = kscale[k] * kLog2e;
+    }
   if (warp == 1) {
     ptx::tmem_alloc(&bars->tmem, 256);
     ptx::tmem_relinquish();
@@ -388,10 +427,13 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   } else if (warp >= 4) {
-    const int q = warp - 4;               // TMEM lane quarter
-    const int r = q * 32 + lane;          // row of the tile = TMEM lane
+    const int g = (warp - 4) >> 2;         // column half of the S tile
+    const int q = warp & 3;                // TMEM lane quarter
+    const int r = q * 32 + lane;           // row of the tile = TMEM lane
+    const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     uint32_t its = 0;
-    for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x) {
+    int jt = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++jt) {
       float m = -CUDART_INF_F, s = 0.f;   // in log2 units
       for (int kb = 0; kb < nkb; ++kb, ++its) {
         const int b = its & 1;
@@ -401,23 +443,31 @@ __global__ void __launch_bounds__(256, 1)
           break;
         }
         ptx::tc_fence_after();
-        const float4* ckb = reinterpret_cast<const float4*>(ck + kb * BKc);
-        const float4* ksb = reinterpret_cast<const float4*>(kscale + kb * BKc);
 #pragma unroll 1
-        for (int h = 0; h < 4; ++h) {
+        for (int h = 0; h < 2; ++h) {
+          const int col = 64 * g + 32 * h;   // column within the 128-component block
           uint32_t u[32];
-          ptx::tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 128 + h * 32, u);
+          ptx::tmem_ld32(tmem + lane_base + b * 128 + col, u);
           ptx::tmem_wait_ld();
           float v[32];
           float bm = -CUDART_INF_F;
+          const int k0 = kb * BKc + col;
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 cc = __ldg(ckb + h * 8 + e4);
-            const float4 kk = __ldg(ksb + h * 8 + e4);
-            v[4 * e4 + 0] = (__uint_as_float(u[4 * e4 + 0]) * kk.x + cc.x) * kLog2e;
-            v[4 * e4 + 1] = (__uint_as_float(u[4 * e4 + 1]) * kk.y + cc.y) * kLog2e;
-            v[4 * e4 + 2] = (__uint_as_float(u[4 * e4 + 2]) * kk.z + cc.z) * kLog2e;
-            v[4 * e4 + 3] = (__uint_as_float(u[4 * e4 + 3]) * kk.w + cc.w) * kLog2e;
+            float4 cc, kk;
+            if (params_in_smem) {
+              cc = *reinterpret_cast<const float4*>(ckl + k0 + 4 * e4);
+              kk = *reinterpret_cast<const float4*>(ksl + k0 + 4 * e4);
+            } else {
+              cc = __ldg(reinterpret_cast<const float4*>(ck + k0) + e4);
+              kk = __ldg(reinterpret_cast<const float4*>(kscale + k0) + e4);
+              cc.x *= kLog2e; cc.y *= kLog2e; cc.z *= kLog2e; cc.w *= kLog2e;
+              kk.x *= kLog2e; kk.y *= kLog2e; kk.z *= kLog2e; kk.w *= kLog2e;
+            }
+            v[4 * e4 + 0] = fmaf(__uint_as_float(u[4 * e4 + 0]), kk.x, cc.x);
+            v[4 * e4 + 1] = fmaf(__uint_as_float(u[4 * e4 + 1]), kk.y, cc.y);
+            v[4 * e4 + 2] = fmaf(__uint_as_float(u[4 * e4 + 2]), kk.z, cc.z);
+            v[4 * e4 + 3] = fmaf(__uint_as_float(u[4 * e4 + 3]), kk.w, cc.w);
 #pragma unroll
             for (int z = 0; z < 4; ++z) bm = fmaxf(bm, v[4 * e4 + z]);
           }
@@ -435,17 +485,43 @@ __global__ void __launch_bounds__(256, 1)
         if (lane == 0) ptx::mbar_arrive(&bars->s_empty[b]);
       }
       if (*abort) break;
-      const int i = t * BM + r;
-      const float lz = (m + log2f(s)) / kLog2e;
-      double part = 0.0;
-      if (i < nc) {
-        logz[i] = lz;
-        if (logz_out) logz_out[i] = lz;
-        part = lz;
-      }
+      // combine the two column halves of each row
+      const int xb = jt & 1, use = jt >> 1;
+      if (g == 1) {
+        if (use >= 1 &&
+            !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->xc_empty[xb], (use - 1) & 1, abort))) {
+          set_status(status, FGMM_ERR_TIMEOUT);
+          bars->abort = 1;
+          break;
+        }
+        bars->xm[xb][r] = m;
+        bars->xs[xb][r] = s;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->xc_full[xb]);
+      } else {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->xc_full[xb], use & 1, abort))) {
+          set_status(status, FGMM_ERR_TIMEOUT);
+          bars->abort = 1;
+          break;
+        }
+        const float m2 = bars->xm[xb][r], s2 = bars->xs[xb][r];
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->xc_empty[xb]);
+        const float M = fmaxf(m, m2);
+        float S = 0.f;
+        if (M > -CUDART_INF_F) S = s * exp2f(m - M) + s2 * exp2f(m2 - M);
+        const int i = t * BM + r;
+        const float lz = (M + log2f(S)) / kLog2e;
+        double part = 0.0;
+        if (i < nc) {
+          logz[i] = lz;
+          if (logz_out) logz_out[i] = lz;
+          part = lz;
+        }
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-      if (lane == 0) ll_tiles[(size_t)t * 4 + q] = part;
+        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        if (lane == 0) ll_tiles[(size_t)t * 4 + q] = part;
+      }
     }
   }
   ptx::tc_fence_before();
@@ -457,27 +533,36 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 // ------------------------------------------------------------------ sweep 2 (statistics)
+// 384 threads: warp 0 TMA producer (W block once, phi boxes, log Z tiles by bulk copy),
+// warp 1 MMA issuer, warps 4..11 epilogue.  Epilogue warpgroup g handles points
+// 64g .. 64g+63 of each tile (and, when flushing, accumulator columns g*Dq .. g*Dq+Dq-1:
+// g = 0 the linear moments, g = 1 the squares).  Each statistic of the CTA's fp64 slot
+// has exactly one writing thread, whose fire-and-forget reductions land in program
+// order: the sums stay bitwise reproducible.
 struct StatBars {
   uint64_t w_full;
   uint64_t x_full[SX], x_empty[SX];
   uint64_t s_full[2], s_empty[2];
   uint64_t r_full, r_empty;
   uint64_t acc_full, acc_empty;
+  uint64_t lz_full[2], lz_empty[2];
+  uint64_t nk_full;
   uint64_t drain;
   uint32_t tmem;
   int abort;
+  float lz[2][BM];
+  float nkx[BKc];
 };
 
 template <int NKC>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
     tc_stats_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                     int nc, int ncmax, int Kt, int slice_len, int flush_tiles,
                     const float* __restrict__ ck, const float* __restrict__ kscale,
                     const float* __restrict__ logz, double* __restrict__ stats, int kstride,
                     int Dp, const int* mode, int* status) {
-  if (mode && *mode != 0) return;
+  if (mode && *mode != kModeTensor) return;
   constexpr int Dq = NKC * 32;            // features: phi has 2 Dq = NKC * 64 entries
-  constexpr int ACC_COLS = 2 * Dq;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   unsigned char* wbuf = base;                          // [2][NKC][BOX]
@@ -496,11 +581,17 @@ __global__ void __launch_bounds__(256, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bars->w_full, 1);
     for (int s = 0; s < SX; ++s) { ptx::mbar_init(&bars->x_full[s], 1); ptx::mbar_init(&bars->x_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { ptx::mbar_init(&bars->s_full[b], 1); ptx::mbar_init(&bars->s_empty[b], 4); }
-    ptx::mbar_init(&bars->r_full, 4);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&bars->s_full[b], 1);
+      ptx::mbar_init(&bars->s_empty[b], kEpiWarps);
+      ptx::mbar_init(&bars->lz_full[b], 1);
+      ptx::mbar_init(&bars->lz_empty[b], kEpiWarps);
+    }
+    ptx::mbar_init(&bars->r_full, kEpiWarps);
     ptx::mbar_init(&bars->r_empty, 1);
     ptx::mbar_init(&bars->acc_full, 1);
-    ptx::mbar_init(&bars->acc_empty, 4);
+    ptx::mbar_init(&bars->acc_empty, kEpiWarps);
+    ptx::mbar_init(&bars->nk_full, kEpiWarps / 2);
     ptx::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
@@ -512,10 +603,10 @@ __global__ void __launch_bounds__(256, 1)
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  const uint32_t tmem = bars->tmem;         // cols [0,256): S^T x2, [256, 256+ACC_COLS): acc
+  const uint32_t tmem = bars->tmem;         // cols [0,256): S^T x2, [256, 256 + 2 Dq): acc
   const uint32_t acc_tmem = tmem + 256;
 
-  // The schedule of MMA groups (and of the producer's X loads) is
+  // The schedule of MMA groups (and of the producer's loads) is
   //   G1(0), G1(1), G2(0), G1(2), G2(1), ..., G1(n-1), G2(n-2), G2(n-1)
   // so the epilogue's softmax of tile j overlaps G1(j+1).
   if (warp == 0) {
@@ -528,13 +619,25 @@ __global__ void __launch_bounds__(256, 1)
         ptx::tma_load_2d(wbuf + (NKC + c) * BOX, &tmw, &bars->w_full, c * KC, Kt + kb * BKc);
       }
       uint32_t itx = 0;
-      // step g: g < ntl -> G1(g); then G2(g-1) for g >= 1; final G2(ntl-1)
+      int lz_issued = 0;
       for (int g = 0; g <= ntl && !*abort; ++g) {
         for (int which = 0; which < 2; ++which) {
           int tile;
           if (which == 0) { if (g >= ntl) continue; tile = g; }
           else { if (g == 0) continue; tile = g - 1; }
           const int row0 = p0 + tile * BM;
+          if (which == 0) {  // log Z of the tile's points, for the epilogue
+            const int lb = tile & 1;
+            if (tile >= 2 &&
+                !ptx::mbar_wait(&bars->lz_empty[lb], ((tile >> 1) - 1) & 1, abort)) {
+              set_status(status, FGMM_ERR_TIMEOUT);
+              bars->abort = 1;
+              goto done_p;
+            }
+            ptx::mbar_arrive_expect_tx(&bars->lz_full[lb], BM * sizeof(float));
+            ptx::bulk_load(bars->lz[lb], logz + row0, BM * sizeof(float), &bars->lz_full[lb]);
+            lz_issued = tile + 1;
+          }
           for (int c = 0; c < NKC; ++c)
             for (int part = 0; part < 2; ++part, ++itx) {
               const int s = itx % SX;
@@ -554,6 +657,8 @@ __global__ void __launch_bounds__(256, 1)
         ptx::mbar_drain(&bars->w_full, 0);
         for (uint32_t k = (itx > SX ? itx - SX : 0); k < itx; ++k)
           ptx::mbar_drain(&bars->x_full[k % SX], (k / SX) & 1);
+        for (int t = (lz_issued > 2 ? lz_issued - 2 : 0); t < lz_issued; ++t)
+          ptx::mbar_drain(&bars->lz_full[t & 1], (t >> 1) & 1);
       }
     }
   } else if (warp == 1) {
@@ -651,60 +756,64 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   } else if (warp >= 4) {
-    const int q = warp - 4;
+    const int g = (warp - 4) >> 2;            // point half of each tile / moment half of acc
+    const int q = warp & 3;
     const int kl = q * 32 + lane;             // component within the block = TMEM lane
     const int k = kb * BKc + kl;
-    const float ckk = ck[k];
-    const float ksk = kscale[k];
+    // log2(e)-scaled epilogue constants; fp16(r 2^15) = exp2(v ksl + ckl - log Z log2(e))
+    const float ksl = kscale[k] * kLog2e;
+    const float ckl = ck[k] * kLog2e + 15.f;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const size_t row = (size_t)(1 + 2 * Dp);
     double* slot = stats + ((size_t)blockIdx.y * kstride + k) * row;
     float nk = 0.f;
     int tiles_since_flush = 0, flushes = 0;
-    // R^T row kl lives in boxes 0/1 (points 0-63 / 64-127): 8-row atoms of 1024 B,
-    // 128 B per row, 16-byte units XOR-swizzled by (row & 7).
-    unsigned char* rrow0 = rbuf + (kl >> 3) * 1024 + (kl & 7) * 128;
+    // R^T row kl, points 64g .. 64g+63 = box g: 8-row atoms of 1024 B, 128 B per row,
+    // 16-byte units XOR-swizzled by (row & 7).
+    unsigned char* rrow = rbuf + g * BOX + (kl >> 3) * 1024 + (kl & 7) * 128;
     for (int tile = 0; tile < ntl && !*abort; ++tile) {
       const int row0 = p0 + tile * BM;
       const int b = tile & 1;
+      const int nvalid = p1 - row0;            // points of this tile inside the slice
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full[b], (tile >> 1) & 1, abort)))
+        goto fail_e;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->lz_full[b], (tile >> 1) & 1, abort)))
         goto fail_e;
       ptx::tc_fence_after();
       if (tile >= 1 &&
           !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->r_empty, (tile - 1) & 1, abort)))
         goto fail_e;
+      const float* lzt = bars->lz[b];
 #pragma unroll 1
-      for (int h = 0; h < 4; ++h) {
+      for (int h = 0; h < 2; ++h) {
+        const int pb = 64 * g + 32 * h;        // first point of this 32-column group
         uint32_t u[32];
-        ptx::tmem_ld32(tmem + lane_base + b * 128 + h * 32, u);
+        ptx::tmem_ld32(tmem + lane_base + b * 128 + pb, u);
         ptx::tmem_wait_ld();
-        // log Z of these 32 points: the same addresses for every thread (L1 broadcast);
-        // rows past the slice end read stale but finite values and are masked below
-        const float4* lz4 = reinterpret_cast<const float4*>(logz + row0 + h * 32);
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float rr[2];
-          const float4 lzv = __ldg(lz4 + (e >> 2));
+        for (int e = 0; e < 32; e += 4) {
+          const float4 lz4 = *reinterpret_cast<const float4*>(lzt + pb + e);
+          const float lzv[4] = {lz4.x, lz4.y, lz4.z, lz4.w};
+          float rr[4];
 #pragma unroll
-          for (int z = 0; z < 2; ++z) {
-            const int pe = e + z;
-            const float l = __uint_as_float(u[pe]) * ksk + ckk;
-            const float lz = ((pe & 3) == 0) ? lzv.x : ((pe & 3) == 1) ? lzv.y : ((pe & 3) == 2) ? lzv.z : lzv.w;
-            const bool ok = (row0 + h * 32 + pe < p1) && lz > -CUDART_INF_F && l > -CUDART_INF_F;
-            const float rv = ok ? exp2f((l - lz) * kLog2e) : 0.f;
-            const __half hv = __float2half_rn(fminf(rv, 1.f) * kRScale);
-            nk += __half2float(hv);
-            rr[z] = __half2float(hv);
+          for (int z = 0; z < 4; ++z) {
+            // t = log2(r 2^15); r <= 1 up to rounding, and the clamp keeps fp16(r 2^15)
+            // finite even where the two sweeps' roundings disagree
+            const float t = fminf(fmaf(__uint_as_float(u[e + z]), ksl, fmaf(-lzv[z], kLog2e, ckl)), 15.f);
+            rr[z] = exp2f(pb + e + z < nvalid ? t : -CUDART_INF_F);
           }
-          pk[e >> 1] = pack_half2(rr[0], rr[1]);
+          const __half2 h01 = __floats2half2_rn(rr[0], rr[1]);
+          const __half2 h23 = __floats2half2_rn(rr[2], rr[3]);
+          const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+          nk += (f01.x + f01.y) + (f23.x + f23.y);
+          pk[e >> 1] = *reinterpret_cast<const uint32_t*>(&h01);
+          pk[(e >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&h23);
         }
-        // points h*32 .. h*32+31 -> box (h >> 1), 16-byte units (h & 1)*4 .. +3
-        unsigned char* rowp = rrow0 + (h >> 1) * BOX;
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu) {
-          const int unit = ((h & 1) * 4 + uu) ^ (kl & 7);
-          *reinterpret_cast<uint4*>(rowp + unit * 16) =
+          const int unit = (h * 4 + uu) ^ (kl & 7);
+          *reinterpret_cast<uint4*>(rrow + unit * 16) =
               make_uint4(pk[uu * 4], pk[uu * 4 + 1], pk[uu * 4 + 2], pk[uu * 4 + 3]);
         }
       }
@@ -713,6 +822,7 @@ __global__ void __launch_bounds__(256, 1)
       __syncwarp();
       if (lane == 0) {
         ptx::mbar_arrive(&bars->s_empty[b]);
+        ptx::mbar_arrive(&bars->lz_empty[b]);
         ptx::mbar_arrive(&bars->r_full);
       }
       if (++tiles_since_flush == flush_tiles || tile == ntl - 1) {
@@ -720,19 +830,25 @@ __global__ void __launch_bounds__(256, 1)
           goto fail_e;
         ptx::tc_fence_after();
         const double inv = 1.0 / (double)kRScale;
+        double* dst = slot + 1 + (g == 0 ? 0 : Dp);   // g 0: linear moments, g 1: squares
 #pragma unroll 1
-        for (int h = 0; h < ACC_COLS / 32; ++h) {
+        for (int h = 0; h < NKC; ++h) {
           uint32_t u[32];
-          ptx::tmem_ld32(acc_tmem + lane_base + h * 32, u);
+          ptx::tmem_ld32(acc_tmem + lane_base + g * Dq + h * 32, u);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int j = h * 32 + e;                 // phi index: j < Dq linear, else square
-            const int col = (j < Dq) ? 1 + j : 1 + Dp + (j - Dq);
-            if ((j < Dq ? j : j - Dq) < Dp) slot[col] += (double)__uint_as_float(u[e]) * inv;
-          }
+          for (int e = 0; e < 32; ++e) atomicAdd(dst + h * 32 + e, (double)__uint_as_float(u[e]) * inv);
         }
-        slot[0] += (double)nk * inv;
+        // N_k: the upper half hands its partial sum to the lower half
+        if (g == 1) {
+          bars->nkx[kl] = nk;
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&bars->nk_full);
+        } else {
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->nk_full, flushes & 1, abort)))
+            goto fail_e;
+          atomicAdd(slot, ((double)nk + (double)bars->nkx[kl]) * inv);
+        }
         nk = 0.f;
         ptx::tc_fence_before();
         __syncwarp();
@@ -820,13 +936,17 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows) {
   return r == CUDA_SUCCESS;
 }
 
-size_t lse_smem(int nkc) { return 1024 + (size_t)(2 * nkc + SW) * BOX + sizeof(LseBars); }
+size_t lse_smem(int nkc, int Kt, bool params) {
+  return 1024 + (size_t)(2 * nkc + SW) * BOX + sizeof(LseBars) +
+         (params ? 2 * (size_t)Kt * sizeof(float) : 0);
+}
+constexpr size_t kMaxDynSmem = 232448;  // 227 KB per block on sm_100
 size_t stats_smem(int nkc) { return 1024 + (size_t)(2 * nkc + SX + 2) * BOX + sizeof(StatBars); }
 
 template <int NKC>
 cudaError_t set_attrs() {
   cudaError_t e = cudaFuncSetAttribute(tc_lse_kernel<NKC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)lse_smem(NKC));
+                                       (int)kMaxDynSmem);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(tc_stats_kernel<NKC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)stats_smem(NKC));
@@ -857,7 +977,7 @@ cudaError_t tc_init(Ctx& c) {
 }
 
 cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* means,
-                           const float* vars, int* mode, cudaStream_t s) {
+                           const float* vars, bool auto_mode, cudaStream_t s) {
   const Workspace& w = c.ws;
   prof_begin(c, KK_OTHER, s);
   tc_center_kernel<<<c.D, kSimtThreads, 0, s>>>(c.K, c.D, c.cov, weights, means, vars, w.center,
@@ -866,10 +986,11 @@ cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* mean
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (w.Dq > c.D) cudaMemsetAsync(w.center + c.D, 0, (w.Dq - c.D) * sizeof(float), s);
+  if (!auto_mode) cudaMemsetAsync(w.stiff, 0, w.Kt * sizeof(int), s);
   prof_begin(c, KK_OTHER, s);
   tc_prep_kernel<<<w.Kt, kSimtThreads, 0, s>>>(c.K, c.D, w.Dq, w.Kt, c.cov, weights, means, vars,
-                                               w.center, w.dscale, w.wop, w.tck, w.tks, mode,
-                                               w.status);
+                                               w.center, w.dscale, w.nk, w.wop, w.tck, w.tks,
+                                               auto_mode ? w.stiff : nullptr, w.status);
   prof_end(c, KK_OTHER, s);
   return cudaGetLastError();
 }
@@ -898,12 +1019,14 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
   const int grid = ntiles < c.num_sms ? ntiles : c.num_sms;
   const CUtensorMap& tx = c.tc.tmap_x;
   const CUtensorMap& tw = c.tc.tmap_w;
+  const bool params = lse_smem(nkc, w.Kt, true) <= kMaxDynSmem;
+  const size_t smem = lse_smem(nkc, w.Kt, params);
   prof_begin(c, KK_SWEEP1, s);
 #define LSE_CASE(N_)                                                                          \
   case N_:                                                                                    \
-    tc_lse_kernel<N_><<<grid, 256, lse_smem(N_), s>>>(tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, \
-                                                      w.tks, w.logz, logz_out, w.ll_tiles, mode, \
-                                                      w.status);                              \
+    tc_lse_kernel<N_><<<grid, kTcThreads, smem, s>>>(tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, \
+                                                     w.tks, params ? 1 : 0, w.logz, logz_out,   \
+                                                     w.ll_tiles, mode, w.status);             \
     break;
   switch (nkc) {
     LSE_CASE(1)
@@ -932,11 +1055,12 @@ cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream
   dim3 grid(w.Kt / BKc, S);
   const CUtensorMap& tx = c.tc.tmap_x;
   const CUtensorMap& tw = c.tc.tmap_w;
-  const int flush_tiles = 16;
+  const int flush_tiles = 8;  // fp32 runs of 1024 points (64 MMA steps) between fp64 flushes
   prof_begin(c, KK_SWEEP2, s);
 #define STATS_CASE(N_)                                                                         \
   case N_:                                                                                     \
-    tc_stats_kernel<N_><<<grid, 256, stats_smem(N_), s>>>(tx, tw, (int)n, (int)kChunk, w.Kt,    \
+    tc_stats_kernel<N_><<<grid, kTcThreads, stats_smem(N_), s>>>(tx, tw, (int)n, (int)kChunk, \
+                                                                 w.Kt,                        \
                                                           slice, flush_tiles, w.tck, w.tks,    \
                                                           w.logz, w.stats, w.KpS, w.Dp, mode,  \
                                                           w.status);                           \

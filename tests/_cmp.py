@@ -52,16 +52,20 @@ def compare_step(gpu, ref, X, cov_spherical=False, logz_gpu=None, loglik_gpu=Non
 
 def ids_match_where_decisive(ids_gpu, ids_ref, resp_ref, R_full, thr, gap=1e-3):
     """Soft-assign ids must be bit-exact wherever the decision is not within `gap`:
-    adjacent sorted responsibilities differ by > gap and |r - thr| > gap."""
+    rank 1 is unique (r_1 - r_2 > gap); every rank 2..m is clear of the threshold
+    (|r_j - thr| > gap); and among the kept ranks the order, and which one is the
+    m-th, is clear (r_j - r_{j+1} > gap).  The order of dropped ranks is irrelevant."""
     ids_gpu = np.asarray(ids_gpu)
     ids_ref = np.asarray(ids_ref)
     m = ids_ref.shape[1]
     Rs = -np.sort(-R_full, axis=1)
     N, K = R_full.shape
-    decisive = np.ones(N, dtype=bool)
-    for j in range(min(m, K - 1)):
-        decisive &= (Rs[:, j] - Rs[:, j + 1]) > gap
+    pad = np.zeros((N, 1))
+    Rs = np.concatenate([Rs, pad], axis=1)          # r_{K+1} = 0
+    decisive = (Rs[:, 0] - Rs[:, 1]) > gap
     for j in range(1, min(m, K)):
         decisive &= np.abs(Rs[:, j] - thr) > gap
+        kept = Rs[:, j] > thr
+        decisive &= ~kept | ((Rs[:, j] - Rs[:, j + 1]) > gap)
     bad = np.nonzero(decisive & np.any(ids_gpu != ids_ref, axis=1))[0]
     return decisive, bad

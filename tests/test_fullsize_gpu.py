@@ -40,6 +40,10 @@ def test_full_size_step(big_x, prec):
     wd, md, vd = g.new_params(w, mu, var)
     ll = torch.zeros(1, dtype=torch.float64, device="cuda")
     lz = torch.empty(N, dtype=torch.float32, device="cuda")
+    # a first step on a small slice loads every kernel (lazy module loading allocates
+    # then); the full-size step must not change device memory after that
+    w2, m2, v2 = wd.clone(), md.clone(), vd.clone()
+    g.step(X[:8192], w2, m2, v2)
     torch.cuda.synchronize()
     free0 = torch.cuda.mem_get_info()[0]
     g.step(X, wd, md, vd, loglik=ll, logz=lz)
