@@ -93,7 +93,7 @@ void free_ws(Workspace& w) {
   void* ptrs[] = {w.mu,     w.prec,   w.cconst, w.logz, w.ll_tiles, w.ll_total,
                   w.stats,  w.nk,     w.status, w.center, w.dscale, w.wop,
                   w.tck,    w.tks,    w.xop,    w.mode, w.stiff,    w.stiff_list, w.n_stiff,
-                  w.side_part};
+                  w.side_part, w.mode2};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -134,6 +134,7 @@ cudaError_t alloc_ws(Ctx& c) {
   if ((e = alloc(&w.nk, (size_t)w.KpS, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.status, (size_t)1, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.mode, (size_t)1, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.mode2, (size_t)1, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.center, (size_t)w.Dq, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.dscale, (size_t)w.Dq, &t)) != cudaSuccess) return e;
   if ((e = cudaMemset(w.status, 0, sizeof(int))) != cudaSuccess) return e;
@@ -279,31 +280,41 @@ int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t l
   if (run_tc) {
     if ((e = launch_tc_prep(c, weights, means, vars, auto_mode, s)) != cudaSuccess)
       return map_cuda(e);
-    if ((e = launch_stiff_compact(c, auto_mode ? w.mode : nullptr, s)) != cudaSuccess)
+    if ((e = launch_stiff_compact(c, auto_mode ? w.mode : nullptr, w.mode, s)) != cudaSuccess)
       return map_cuda(e);
   }
   const size_t eb = dtype_bytes(x_dtype);
-  if (run_tc) {
-    for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
+  // one tensor-core pass over all chunks, its kernels gated on the word `gate`
+  auto tc_pass = [&](const int* gate) -> cudaError_t {
+    cudaError_t r = cudaSuccess;
+    for (int64_t c0 = 0; c0 < N && r == cudaSuccess; c0 += kChunk) {
       const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
       const void* Xc = (const char*)X + (size_t)c0 * ldx * eb;
       float* lzo = logz_out ? logz_out + c0 : nullptr;
-      if ((e = launch_tc_convert(c, Xc, x_dtype, nc, ldx, mode, s)) != cudaSuccess)
-        return map_cuda(e);
-      if ((e = launch_tc_lse(c, nc, lzo, mode, s)) != cudaSuccess) return map_cuda(e);
+      if ((r = launch_tc_convert(c, Xc, x_dtype, nc, ldx, gate, s)) != cudaSuccess) break;
+      if ((r = launch_tc_lse(c, nc, lzo, gate, s)) != cudaSuccess) break;
       // stiff components (AUTO) join log Z here; then the chunk's log-likelihood
-      if ((e = launch_side_lse(c, Xc, x_dtype, nc, ldx, lzo, mode, s)) != cudaSuccess)
-        return map_cuda(e);
-      if ((e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeTensor, s)) != cudaSuccess)
-        return map_cuda(e);
-      if ((e = launch_tc_stats(c, nc, mode, s)) != cudaSuccess) return map_cuda(e);
-      if ((e = launch_side_stats(c, Xc, x_dtype, nc, ldx, mode, s)) != cudaSuccess)
-        return map_cuda(e);
+      if ((r = launch_side_lse(c, Xc, x_dtype, nc, ldx, lzo, gate, s)) != cudaSuccess) break;
+      if ((r = launch_ll_accumulate(c, nc, gate, fixed_mode, kModeTensor, s)) != cudaSuccess) break;
+      if ((r = launch_tc_stats(c, nc, gate, s)) != cudaSuccess) break;
+      r = launch_side_stats(c, Xc, x_dtype, nc, ldx, gate, s);
+    }
+    return r;
+  };
+  if (run_tc) {
+    if (auto_mode && (e = cudaMemsetAsync(w.mode2, 0xFF, sizeof(int), s)) != cudaSuccess)
+      return map_cuda(e);
+    if ((e = tc_pass(mode)) != cudaSuccess) return map_cuda(e);
+    if (auto_mode) {
+      // AUTO: components whose new variance would lose accuracy to cancellation move to
+      // the side path and the pass is redone (gated on mode2); a failure after that sends
+      // the step to the CUDA-core kernels below (gated on mode)
+      if ((e = launch_auto_check(c, 0, s)) != cudaSuccess) return map_cuda(e);
+      if ((e = launch_stiff_compact(c, w.mode2, w.mode, s)) != cudaSuccess) return map_cuda(e);
+      if ((e = tc_pass(w.mode2)) != cudaSuccess) return map_cuda(e);
+      if ((e = launch_auto_check(c, 1, s)) != cudaSuccess) return map_cuda(e);
     }
   }
-  // AUTO: a step whose new variances would lose accuracy to cancellation is sent back
-  // to the CUDA-core path (the kernels below run only when the mode word says so)
-  if (auto_mode && (e = launch_auto_check_and_reset(c, s)) != cudaSuccess) return map_cuda(e);
   if (run_simt) {
     for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
       const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;

@@ -48,6 +48,7 @@ struct Workspace {
   float* tks = nullptr;     // [Kt] 2^t_k
   __half* xop = nullptr;    // [2][kChunk][K1] phi(x) hi / lo of the current chunk
   int* mode = nullptr;      // [1] path of the current step: 0 tensor cores, 1 CUDA cores
+  int* mode2 = nullptr;     // [1] AUTO: tensor when the hybrid redo pass must run
   int* stiff = nullptr;     // [Kt] AUTO: 1 = component handled by the CUDA-core side path
   int* stiff_list = nullptr;  // [Kt] stiff components in index order
   int* n_stiff = nullptr;   // [1]
@@ -106,9 +107,11 @@ cudaError_t launch_lse_simt(const Ctx& c, const void* X, int x_dtype, int64_t n,
                             float* logz_out, const int* mode, cudaStream_t s);
 cudaError_t launch_ll_accumulate(const Ctx& c, int64_t n, const int* mode, int fixed_mode,
                                  int required, cudaStream_t s);
-// AUTO only: variance-cancellation check after the tensor-core sweeps, and the reset
-// of their partial results when the step is sent back to the CUDA-core path.
-cudaError_t launch_auto_check_and_reset(const Ctx& c, cudaStream_t s);
+// AUTO only: variance-cancellation check after a tensor-core pass.  Stage 0: failing
+// components become stiff and a hybrid redo pass is enabled (mode2 word); stage 1: a
+// failure after the redo sends the step to the CUDA-core path.  Each stage clears the
+// partial results it invalidates.
+cudaError_t launch_auto_check(const Ctx& c, int stage, cudaStream_t s);
 cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
                               const int* mode, cudaStream_t s);
 cudaError_t launch_mstep(const Ctx& c, float* weights, float* means, float* vars,
@@ -120,7 +123,7 @@ int tc_slices(const Ctx& c);
 cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* means,
                            const float* vars, bool auto_mode, cudaStream_t s);
 // AUTO side path for stiff components (fgmm_side.cu)
-cudaError_t launch_stiff_compact(const Ctx& c, int* mode, cudaStream_t s);
+cudaError_t launch_stiff_compact(const Ctx& c, int* gate, int* mode, cudaStream_t s);
 cudaError_t launch_side_lse(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
                             float* logz_out, const int* mode, cudaStream_t s);
 cudaError_t launch_side_stats(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,

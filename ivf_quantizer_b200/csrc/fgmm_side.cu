@@ -54,9 +54,11 @@ __device__ __forceinline__ float stiff_logit(const T* __restrict__ x, int D,
 // CUDA-core path, so the whole step goes there (mode word).
 constexpr int kMaxStiff = kSideMaxStiff;
 
+// Runs when *gate is tensor (or gate is null); on overflow the step goes to the CUDA-core
+// path (*mode) and the gated pass is switched off (*gate).
 __global__ void stiff_compact_kernel(const int* __restrict__ stiff, int K, int* __restrict__ list,
-                                     int* __restrict__ n_out, int* mode) {
-  if (mode && *mode != kModeTensor) return;
+                                     int* __restrict__ n_out, int* gate, int* mode) {
+  if (gate && *gate != kModeTensor) return;
   __shared__ int base;
   if (threadIdx.x == 0) base = 0;
   __syncthreads();
@@ -82,7 +84,10 @@ __global__ void stiff_compact_kernel(const int* __restrict__ stiff, int K, int* 
   }
   if (threadIdx.x == 0) {
     *n_out = base;
-    if (mode && base > kMaxStiff) *mode = kModeSimt;
+    if (gate && base > kMaxStiff) {
+      *mode = kModeSimt;
+      *gate = kModeSimt;
+    }
   }
 }
 
@@ -231,9 +236,10 @@ __global__ void side_reduce_kernel(const double* __restrict__ part, const int* _
 }
 
 // ------------------------------------------------------------------ launchers
-cudaError_t launch_stiff_compact(const Ctx& c, int* mode, cudaStream_t s) {
+cudaError_t launch_stiff_compact(const Ctx& c, int* gate, int* mode, cudaStream_t s) {
   prof_begin(c, KK_OTHER, s);
-  stiff_compact_kernel<<<1, 256, 0, s>>>(c.ws.stiff, c.K, c.ws.stiff_list, c.ws.n_stiff, mode);
+  stiff_compact_kernel<<<1, 256, 0, s>>>(c.ws.stiff, c.K, c.ws.stiff_list, c.ws.n_stiff, gate,
+                                         mode);
   prof_end(c, KK_OTHER, s);
   return cudaGetLastError();
 }

@@ -524,16 +524,25 @@ __global__ void __launch_bounds__(kSimtThreads)
 // the expected error is 3.5e-4, a third of the 1e-3 tolerance.  One CTA per component.
 constexpr double kMaxAmplification = 900.0;
 
+// Stage 0 (after the first tensor-core pass, gated on *gate == tensor): a failing
+// component becomes stiff (it will be evaluated on the side path) and *redo is set to
+// tensor, which enables a second, hybrid pass with the enlarged stiff set.  Stage 1
+// (after that pass, gated on *gate = the redo word): any remaining failure sends the
+// step to the CUDA-core path (*mode = CUDA cores).
 __global__ void tc_variance_check_kernel(int K, int D, int Dp, int kstride,
                                          const double* __restrict__ stats, int nslots,
-                                         const int* __restrict__ stiff, int* mode) {
-  if (*mode != kModeTensor) return;
+                                         int* __restrict__ stiff, const int* gate, int* redo,
+                                         int* mode, int stage) {
+  if (*gate != kModeTensor || *mode != kModeTensor) return;
   const int k = blockIdx.x;
   if (stiff[k]) return;  // the side path's statistics are centred on the mean: exact
   const size_t row = (size_t)(1 + 2 * Dp);
   double nk = 0.0;
   for (int s = 0; s < nslots; ++s) nk += stats[((size_t)s * kstride + k) * row];
   if (!(nk >= FGMM_EMPTY_NK)) return;  // empty: parameters are kept, nothing to check
+  __shared__ int bad_any;
+  if (threadIdx.x == 0) bad_any = 0;
+  __syncthreads();
   bool bad = false;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     double s1 = 0.0, s2 = 0.0;
@@ -546,18 +555,36 @@ __global__ void tc_variance_check_kernel(int K, int D, int Dp, int kstride,
     const double v = m2 - m1 * m1;
     if (!(v > 0.0) || !(m2 <= kMaxAmplification * v)) bad = true;
   }
-  if (bad) atomicExch(mode, kModeSimt);
+  if (bad) atomicExch(&bad_any, 1);
+  __syncthreads();
+  if (threadIdx.x == 0 && bad_any) {
+    if (stage == 0) {
+      stiff[k] = 1;
+      atomicExch(redo, kModeTensor);
+    } else {
+      atomicExch(mode, kModeSimt);
+    }
+  }
 }
 
-// When the step was sent back to the CUDA-core path after the tensor-core sweeps ran,
-// clear what they accumulated.  Grid-stride over the statistics slots.
-__global__ void redo_reset_kernel(const int* mode, double* __restrict__ stats, size_t n,
-                                  double* __restrict__ ll_total) {
-  if (*mode != kModeSimt) return;
+// Clears the statistics and the log-likelihood when *flag == value (a pass is about to be
+// redone).  Grid-stride over the statistics slots.
+__global__ void redo_reset_kernel(const int* flag, int value, double* __restrict__ stats,
+                                  size_t n, double* __restrict__ ll_total) {
+  if (*flag != value) return;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x)
     stats[i] = 0.0;
   if (blockIdx.x == 0 && threadIdx.x == 0) *ll_total = 0.0;
+}
+
+// Before the hybrid redo pass: components made stiff by the stage-0 check leave the
+// tensor-core sweeps (c_k = -inf there).
+__global__ void remask_kernel(const int* redo, const int* __restrict__ stiff, int Kt,
+                              float* __restrict__ tck) {
+  if (*redo != kModeTensor) return;
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k < Kt && stiff[k]) tck[k] = -CUDART_INF_F;
 }
 
 // ------------------------------------------------------------------ launchers
@@ -662,16 +689,27 @@ cudaError_t launch_soft_assign_simt(const Ctx& c, const void* X, int x_dtype, in
 }  // namespace fgmm
 
 namespace fgmm {
-cudaError_t launch_auto_check_and_reset(const Ctx& c, cudaStream_t s) {
+cudaError_t launch_auto_check(const Ctx& c, int stage, cudaStream_t s) {
+  const Workspace& w = c.ws;
+  const size_t n = (size_t)w.slots * w.KpS * (1 + 2 * (size_t)w.Dp);
   prof_begin(c, KK_OTHER, s);
-  tc_variance_check_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, c.ws.Dp, c.ws.KpS, c.ws.stats,
-                                                        tc_slices(c), c.ws.stiff, c.ws.mode);
+  tc_variance_check_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, w.Dp, w.KpS, w.stats,
+                                                        tc_slices(c), w.stiff,
+                                                        stage == 0 ? w.mode : w.mode2, w.mode2,
+                                                        w.mode, stage);
   prof_end(c, KK_OTHER, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t n = (size_t)c.ws.slots * c.ws.KpS * (1 + 2 * (size_t)c.ws.Dp);
   prof_begin(c, KK_OTHER, s);
-  redo_reset_kernel<<<2 * c.num_sms, 256, 0, s>>>(c.ws.mode, c.ws.stats, n, c.ws.ll_total);
+  if (stage == 0)
+    redo_reset_kernel<<<2 * c.num_sms, 256, 0, s>>>(w.mode2, kModeTensor, w.stats, n, w.ll_total);
+  else
+    redo_reset_kernel<<<2 * c.num_sms, 256, 0, s>>>(w.mode, kModeSimt, w.stats, n, w.ll_total);
+  prof_end(c, KK_OTHER, s);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || stage != 0) return e;
+  prof_begin(c, KK_OTHER, s);
+  remask_kernel<<<(w.Kt + 255) / 256, 256, 0, s>>>(w.mode2, w.stiff, w.Kt, w.tck);
   prof_end(c, KK_OTHER, s);
   return cudaGetLastError();
 }

@@ -59,7 +59,7 @@ constexpr int BKc = 128;         // components per block
 constexpr int KC = 64;           // K elements per swizzle row / TMA box
 constexpr int BOX = 128 * 64 * 2;  // bytes of one [128 rows][64 fp16] box
 constexpr int SW = 4;            // W ring stages (sweep 1)
-constexpr int SX = 4;            // X ring stages (sweep 2)
+constexpr int SX = 8;            // X ring stages (sweep 2)
 constexpr float kRScale = 32768.f;  // r is stored as fp16(r * 2^15)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -286,7 +286,8 @@ struct LseBars {
   uint64_t drain;
   uint32_t tmem;
   int abort;
-  float xm[2][BM], xs[2][BM];
+  alignas(16) float xm[2][BM];   // bulk-copy destinations: 16-byte aligned
+  alignas(16) float xs[2][BM];
 };
 
 template <int NKC>
@@ -540,9 +541,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // has exactly one writing thread, whose fire-and-forget reductions land in program
 // order: the sums stay bitwise reproducible.
 struct StatBars {
-  uint64_t w_full;
+  uint64_t w_full, wlo_ready;
   uint64_t x_full[SX], x_empty[SX];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full, s_empty;
   uint64_t r_full, r_empty;
   uint64_t acc_full, acc_empty;
   uint64_t lz_full[2], lz_empty[2];
@@ -550,9 +551,10 @@ struct StatBars {
   uint64_t drain;
   uint32_t tmem;
   int abort;
-  float lz[2][BM];
+  alignas(16) float lz[2][BM];   // bulk-copy destination, read as float4: 16-byte aligned
   float nkx[BKc];
 };
+static_assert(offsetof(StatBars, lz) % 16 == 0, "log Z tiles must be 16-byte aligned");
 
 template <int NKC>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -560,13 +562,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     int nc, int ncmax, int Kt, int slice_len, int flush_tiles,
                     const float* __restrict__ ck, const float* __restrict__ kscale,
                     const float* __restrict__ logz, double* __restrict__ stats, int kstride,
-                    int Dp, const int* mode, int* status) {
+                    int Dp, const __half* __restrict__ wop, const int* mode, int* status) {
   if (mode && *mode != kModeTensor) return;
   constexpr int Dq = NKC * 32;            // features: phi has 2 Dq = NKC * 64 entries
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  unsigned char* wbuf = base;                          // [2][NKC][BOX]
-  unsigned char* xring = base + 2 * NKC * BOX;         // [SX][BOX]
+  unsigned char* wbuf = base;                          // [NKC][BOX]: W' hi of the block
+  unsigned char* xring = base + NKC * BOX;             // [SX][BOX]
   unsigned char* rbuf = xring + SX * BOX;              // [2][BOX]: R^T, 64 points per box
   StatBars* bars = reinterpret_cast<StatBars*>(rbuf + 2 * BOX);
   volatile int* abort = &bars->abort;
@@ -580,10 +582,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bars->w_full, 1);
+    ptx::mbar_init(&bars->wlo_ready, kEpiWarps);
     for (int s = 0; s < SX; ++s) { ptx::mbar_init(&bars->x_full[s], 1); ptx::mbar_init(&bars->x_empty[s], 1); }
+    ptx::mbar_init(&bars->s_full, 1);
+    ptx::mbar_init(&bars->s_empty, kEpiWarps);
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(&bars->s_full[b], 1);
-      ptx::mbar_init(&bars->s_empty[b], kEpiWarps);
       ptx::mbar_init(&bars->lz_full[b], 1);
       ptx::mbar_init(&bars->lz_empty[b], kEpiWarps);
     }
@@ -603,7 +606,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  const uint32_t tmem = bars->tmem;         // cols [0,256): S^T x2, [256, 256 + 2 Dq): acc
+  // TMEM columns: [0,128) S^T, [128, 128 + Dq) W' lo of the block (A operand of the
+  // third product, two fp16 per column), [256, 256 + 2 Dq) the statistics accumulator
+  const uint32_t tmem = bars->tmem;
+  const uint32_t wlo_tmem = tmem + 128;
   const uint32_t acc_tmem = tmem + 256;
 
   // The schedule of MMA groups (and of the producer's loads) is
@@ -613,11 +619,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       ptx::prefetch_tmap(&tmx);
       ptx::prefetch_tmap(&tmw);
-      ptx::mbar_arrive_expect_tx(&bars->w_full, 2 * NKC * BOX);
-      for (int c = 0; c < NKC; ++c) {
+      ptx::mbar_arrive_expect_tx(&bars->w_full, NKC * BOX);
+      for (int c = 0; c < NKC; ++c)
         ptx::tma_load_2d(wbuf + c * BOX, &tmw, &bars->w_full, c * KC, kb * BKc);
-        ptx::tma_load_2d(wbuf + (NKC + c) * BOX, &tmw, &bars->w_full, c * KC, Kt + kb * BKc);
-      }
       uint32_t itx = 0;
       int lz_issued = 0;
       for (int g = 0; g <= ntl && !*abort; ++g) {
@@ -670,12 +674,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool fresh = true;   // next G2 starts a new accumulation period
       int flushes = 0;
       if (!ptx::mbar_wait(&bars->w_full, 0, abort)) goto fail_m;
+      if (!ptx::mbar_wait(&bars->wlo_ready, 0, abort)) goto fail_m;
       for (int g = 0; g <= ntl && !*abort; ++g) {
-        if (g < ntl) {  // ---- G1(g)
-          const int b = g & 1;
-          if (g >= 2 && !ptx::mbar_wait(&bars->s_empty[b], ((g >> 1) - 1) & 1, abort)) goto fail_m;
+        if (g < ntl) {  // ---- G1(g): S^T is single-buffered, released once loaded
+          if (g >= 1 && !ptx::mbar_wait(&bars->s_empty, (g - 1) & 1, abort)) goto fail_m;
           ptx::tc_fence_after();
-          const uint32_t d_tmem = tmem + b * 128;
+          const uint32_t d_tmem = tmem;
           for (int c = 0; c < NKC; ++c) {
             const int sh = itx % SX;
             if (!ptx::mbar_wait(&bars->x_full[sh], (itx / SX) & 1, abort)) goto fail_m;
@@ -685,24 +689,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ++itx;
             ptx::tc_fence_after();
             const uint32_t wa_hi = ptx::smem_u32(wbuf + c * BOX);
-            const uint32_t wa_lo = ptx::smem_u32(wbuf + (NKC + c) * BOX);
             const uint32_t xb_hi = ptx::smem_u32(xring + sh * BOX);
             const uint32_t xb_lo = ptx::smem_u32(xring + sl * BOX);
 #pragma unroll
             for (int ks = 0; ks < KC / 16; ++ks) {
               const uint32_t o = ks * 32;
               const uint64_t ah = ptx::smem_desc_sw128(wa_hi + o, 16, 1024);
-              const uint64_t al = ptx::smem_desc_sw128(wa_lo + o, 16, 1024);
               const uint64_t bh = ptx::smem_desc_sw128(xb_hi + o, 16, 1024);
               const uint64_t bl = ptx::smem_desc_sw128(xb_lo + o, 16, 1024);
               ptx::mma_f16_ss(d_tmem, ah, bh, idesc1, (c > 0 || ks > 0) ? 1u : 0u);
               ptx::mma_f16_ss(d_tmem, ah, bl, idesc1, 1u);
-              ptx::mma_f16_ss(d_tmem, al, bh, idesc1, 1u);
+              // W' lo from TMEM: K elements c*64 + ks*16 .. +15 = columns c*32 + ks*8 .. +7
+              ptx::mma_f16_ts(d_tmem, wlo_tmem + c * 32 + ks * 8, bh, idesc1, 1u);
             }
             ptx::mma_commit(&bars->x_empty[sh]);
             ptx::mma_commit(&bars->x_empty[sl]);
           }
-          ptx::mma_commit(&bars->s_full[b]);
+          ptx::mma_commit(&bars->s_full);
         }
         if (g >= 1) {  // ---- G2(g-1)
           const int tile = g - 1;
@@ -771,26 +774,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // R^T row kl, points 64g .. 64g+63 = box g: 8-row atoms of 1024 B, 128 B per row,
     // 16-byte units XOR-swizzled by (row & 7).
     unsigned char* rrow = rbuf + g * BOX + (kl >> 3) * 1024 + (kl & 7) * 128;
+    // W' lo of this component into TMEM (the third product's A operand): this
+    // warpgroup writes K elements g*Dq .. g*Dq+Dq-1 = columns g*Dq/2 .. +Dq/2-1
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(wop + ((size_t)Kt + k) * (2 * Dq) + g * Dq);
+#pragma unroll 1
+      for (int c8 = 0; c8 < Dq / 16; ++c8) {   // 8 columns = 16 fp16 per store
+        const uint4 v0 = __ldg(src + 2 * c8), v1 = __ldg(src + 2 * c8 + 1);
+        const uint32_t r8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        ptx::tmem_st8(wlo_tmem + lane_base + g * (Dq / 2) + c8 * 8, r8);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bars->wlo_ready);
+    }
     for (int tile = 0; tile < ntl && !*abort; ++tile) {
       const int row0 = p0 + tile * BM;
       const int b = tile & 1;
       const int nvalid = p1 - row0;            // points of this tile inside the slice
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full[b], (tile >> 1) & 1, abort)))
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full, tile & 1, abort)))
         goto fail_e;
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->lz_full[b], (tile >> 1) & 1, abort)))
         goto fail_e;
       ptx::tc_fence_after();
-      if (tile >= 1 &&
-          !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->r_empty, (tile - 1) & 1, abort)))
-        goto fail_e;
+      // load this warpgroup's 64 columns of S^T, then free the buffer for G1(tile + 1)
+      uint32_t u[2][32];
+      ptx::tmem_ld32(tmem + lane_base + 64 * g, u[0]);
+      ptx::tmem_ld32(tmem + lane_base + 64 * g + 32, u[1]);
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bars->s_empty);
       const float* lzt = bars->lz[b];
-#pragma unroll 1
+      uint32_t pk[2][16];
+#pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int pb = 64 * g + 32 * h;        // first point of this 32-column group
-        uint32_t u[32];
-        ptx::tmem_ld32(tmem + lane_base + b * 128 + pb, u);
-        ptx::tmem_wait_ld();
-        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float4 lz4 = *reinterpret_cast<const float4*>(lzt + pb + e);
@@ -800,28 +820,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int z = 0; z < 4; ++z) {
             // t = log2(r 2^15); r <= 1 up to rounding, and the clamp keeps fp16(r 2^15)
             // finite even where the two sweeps' roundings disagree
-            const float t = fminf(fmaf(__uint_as_float(u[e + z]), ksl, fmaf(-lzv[z], kLog2e, ckl)), 15.f);
+            const float t = fminf(fmaf(__uint_as_float(u[h][e + z]), ksl, fmaf(-lzv[z], kLog2e, ckl)), 15.f);
             rr[z] = exp2f(pb + e + z < nvalid ? t : -CUDART_INF_F);
           }
           const __half2 h01 = __floats2half2_rn(rr[0], rr[1]);
           const __half2 h23 = __floats2half2_rn(rr[2], rr[3]);
           const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
           nk += (f01.x + f01.y) + (f23.x + f23.y);
-          pk[e >> 1] = *reinterpret_cast<const uint32_t*>(&h01);
-          pk[(e >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+          pk[h][e >> 1] = *reinterpret_cast<const uint32_t*>(&h01);
+          pk[h][(e >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&h23);
         }
+      }
+      // R^T of the previous tile must have been consumed by G2 before it is overwritten
+      if (tile >= 1 &&
+          !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->r_empty, (tile - 1) & 1, abort)))
+        goto fail_e;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu) {
           const int unit = (h * 4 + uu) ^ (kl & 7);
           *reinterpret_cast<uint4*>(rrow + unit * 16) =
-              make_uint4(pk[uu * 4], pk[uu * 4 + 1], pk[uu * 4 + 2], pk[uu * 4 + 3]);
+              make_uint4(pk[h][uu * 4], pk[h][uu * 4 + 1], pk[h][uu * 4 + 2], pk[h][uu * 4 + 3]);
         }
-      }
-      ptx::tc_fence_before();
       ptx::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        ptx::mbar_arrive(&bars->s_empty[b]);
         ptx::mbar_arrive(&bars->lz_empty[b]);
         ptx::mbar_arrive(&bars->r_full);
       }
@@ -941,7 +965,7 @@ size_t lse_smem(int nkc, int Kt, bool params) {
          (params ? 2 * (size_t)Kt * sizeof(float) : 0);
 }
 constexpr size_t kMaxDynSmem = 232448;  // 227 KB per block on sm_100
-size_t stats_smem(int nkc) { return 1024 + (size_t)(2 * nkc + SX + 2) * BOX + sizeof(StatBars); }
+size_t stats_smem(int nkc) { return 1024 + (size_t)(nkc + SX + 2) * BOX + sizeof(StatBars); }
 
 template <int NKC>
 cudaError_t set_attrs() {
@@ -1062,8 +1086,8 @@ cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream
     tc_stats_kernel<N_><<<grid, kTcThreads, stats_smem(N_), s>>>(tx, tw, (int)n, (int)kChunk, \
                                                                  w.Kt,                        \
                                                           slice, flush_tiles, w.tck, w.tks,    \
-                                                          w.logz, w.stats, w.KpS, w.Dp, mode,  \
-                                                          w.status);                           \
+                                                          w.logz, w.stats, w.KpS, w.Dp, w.wop, \
+                                                          mode, w.status);                     \
     break;
   switch (nkc) {
     STATS_CASE(1)
