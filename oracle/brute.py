@@ -81,3 +81,18 @@ def top_m_assign(X, w, mu, var, top_m, r_threshold, spherical=False):
         ids.append(row_i)
         resp.append(row_r)
     return ids, resp
+
+
+def shard_statistics(X, w, mu, var, spherical=False):
+    """Per component [N_k, Σ r (x_d − μ_kd) for each d, Σ r (x_d − μ_kd)² for each d]
+    about the input means, flattened, then Σ log Z (scalar loops, math.fsum)."""
+    N, K, D = len(X), len(mu), len(X[0])
+    *_, logZ, R = em_step(X, w, mu, var, spherical)
+    out = []
+    for k in range(K):
+        out.append(math.fsum(R[i][k] for i in range(N)))
+        out.extend(math.fsum(R[i][k] * (X[i][d] - mu[k][d]) for i in range(N)) for d in range(D))
+        out.extend(math.fsum(R[i][k] * (X[i][d] - mu[k][d]) ** 2 for i in range(N))
+                   for d in range(D))
+    out.append(math.fsum(logZ))
+    return out

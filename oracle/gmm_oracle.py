@@ -204,6 +204,76 @@ def em_step(X, weights, means, variances, cov_type=COV_DIAG, reg_covar=1e-6):
     return StepResult(w_new, mu_new, var_new, loglik, logZ, Nk, empty)
 
 
+def shard_statistics(X, weights, means, variances, cov_type=COV_DIAG):
+    """The sufficient statistics one shard of the rows contributes to an EM step.
+
+    Layout (fp64, length K (1 + 2D) + 1), per component k at offset k (1 + 2D):
+      N_k = Σ_i r_ik,   Σ_i r_ik (x_id − μ_kd),   Σ_i r_ik (x_id − μ_kd)²   (d < D)
+    about the INPUT means μ_k, then Σ_i log Z_i.  Every entry is a sum over rows, so
+    the statistics of disjoint shards add up to those of their union; §2's M-step
+    (Eqs. (1)-(3)) is a function of the sums alone (m_step_from_statistics).
+    """
+    X = _as_f64(X)
+    N, D = X.shape
+    mu = _as_f64(means)
+    K = mu.shape[0]
+    row = 1 + 2 * D
+    out = np.zeros(K * row + 1, dtype=np.float64)
+    st = out[:K * row].reshape(K, row)
+    ll = 0.0
+    for s, e in _row_chunks(N, K):
+        lz, R = e_step(X[s:e], weights, mu, variances, cov_type)
+        ll += float(np.sum(lz))
+        st[:, 0] += R.sum(axis=0)
+        for k in range(K):
+            diff = X[s:e] - mu[k]
+            st[k, 1:1 + D] += R[:, k] @ diff
+            st[k, 1 + D:] += R[:, k] @ (diff * diff)
+    out[K * row] = ll
+    return out
+
+
+def m_step_from_statistics(stats, weights, means, variances, cov_type=COV_DIAG,
+                           reg_covar=1e-6):
+    """§2's M-step from summed shard statistics (layout of shard_statistics).
+
+    With S1 = Σ r (x − μ) and S2 = Σ r (x − μ)² about the input mean μ:
+      μ_new = μ + S1 / N_k                                           (Eq. (2))
+      Σ r (x − μ_new)² = S2 − S1² / N_k, so σ² = S2 / N_k − (S1 / N_k)²  (Eq. (3))
+    plus the same readings as em_step (weights over live components, additive floor,
+    empty components kept).  Returns a StepResult with logZ = None.
+    """
+    stats = _as_f64(stats)
+    mu_in = _as_f64(means)
+    K, D = mu_in.shape
+    row = 1 + 2 * D
+    st = stats[:K * row].reshape(K, row)
+    loglik = float(stats[K * row])
+    if not np.isfinite(loglik):
+        raise FloatingPointError("non-finite log-likelihood")
+    Nk = st[:, 0].copy()
+    empty = Nk < EMPTY_NK
+    if np.all(empty):
+        raise FloatingPointError("every component is empty")
+    live = ~empty
+    m1 = np.zeros((K, D))
+    m1[live] = st[live, 1:1 + D] / Nk[live, None]
+    v = np.zeros((K, D))
+    v[live] = np.maximum(st[live, 1 + D:] / Nk[live, None] - m1[live] ** 2, 0.0)
+    mu_new = mu_in.copy()
+    mu_new[live] = mu_in[live] + m1[live]
+    var_in = _as_f64(variances)
+    if cov_type == COV_DIAG:
+        var_new = var_in.reshape(K, D).copy()
+        var_new[live] = v[live] + reg_covar
+    else:
+        var_new = var_in.reshape(K).copy()
+        var_new[live] = v[live].mean(axis=1) + reg_covar
+    w_new = np.zeros(K)
+    w_new[live] = Nk[live] / np.sum(Nk[live])
+    return StepResult(w_new, mu_new, var_new, loglik, None, Nk, empty)
+
+
 def fit(X, weights, means, variances, cov_type=COV_DIAG, reg_covar=1e-6,
         max_iters=100, tol=0.0):
     """Repeat em_step; stop after max_iters or when |L_t − L_{t−1}| / N < tol.

@@ -298,3 +298,71 @@ def test_recovers_well_separated_mixture():
         assert np.all(np.abs(mu[k] - true_mu[k]) < 4 * true_s[k] / math.sqrt(nk))
         assert abs(w[k] - true_w[k]) < 3 * math.sqrt(true_w[k] / N) + 1e-3
         np.testing.assert_allclose(np.sqrt(var[k]), true_s[k], rtol=0.1)
+
+
+# ------------------------------------------------------------------ sharded statistics
+@pytest.mark.parametrize("spherical", [False, True])
+def test_shard_statistics_match_brute_force(spherical):
+    """The exchanged statistics (N_k, Σ r (x − μ), Σ r (x − μ)² about the input
+    mean, Σ log Z) against the pure-Python statement on a tiny input."""
+    rng = np.random.default_rng(11)
+    N, K, D = 23, 3, 2
+    X = rng.normal(size=(N, D)) * 2.0
+    w = np.array([0.5, 0.3, 0.2])
+    mu = rng.normal(size=(K, D))
+    var = rng.uniform(0.5, 2.0, size=K) if spherical else rng.uniform(0.5, 2.0, size=(K, D))
+    cov = O.COV_SPHERICAL if spherical else O.COV_DIAG
+    got = O.shard_statistics(X, w, mu, var, cov)
+    ref = brute.shard_statistics(X.tolist(), w.tolist(), mu.tolist(), var.tolist(), spherical)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_shard_statistics_are_additive_over_row_partitions():
+    """Every entry is a sum over rows: three uneven shards add up to the whole."""
+    rng = np.random.default_rng(12)
+    X = rng.normal(size=(700, 6))
+    K = 5
+    w = rng.dirichlet(np.ones(K))
+    mu = X[rng.choice(700, K, replace=False)]
+    var = rng.uniform(0.5, 2.0, size=(K, 6))
+    parts = [X[:1], X[1:333], X[333:]]
+    tot = sum(O.shard_statistics(p, w, mu, var) for p in parts)
+    np.testing.assert_allclose(tot, O.shard_statistics(X, w, mu, var), rtol=1e-12, atol=1e-9)
+
+
+@pytest.mark.parametrize("cov", [O.COV_DIAG, O.COV_SPHERICAL])
+def test_m_step_from_statistics_equals_em_step(cov):
+    """Eq. (3) about the updated mean follows from the sums about the input mean:
+    the M-step on summed shard statistics equals the one-pass em_step."""
+    rng = np.random.default_rng(13)
+    X = np.concatenate([rng.normal(-3, 1, size=(300, 4)), rng.normal(2, 0.5, size=(200, 4))])
+    K = 3
+    w = np.full(K, 1 / K)
+    mu = X[[0, 1, 350]]
+    var = np.ones(K) if cov == O.COV_SPHERICAL else np.ones((K, 4))
+    st = O.shard_statistics(X[:137], w, mu, var, cov) + O.shard_statistics(X[137:], w, mu, var, cov)
+    a = O.m_step_from_statistics(st, w, mu, var, cov)
+    b = O.em_step(X, w, mu, var, cov)
+    np.testing.assert_allclose(a.means, b.means, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(a.variances, b.variances, rtol=1e-10)
+    np.testing.assert_allclose(a.weights, b.weights, rtol=1e-12)
+    assert abs(a.loglik - b.loglik) <= 1e-12 * abs(b.loglik)
+
+
+def test_m_step_from_statistics_keeps_empty_components():
+    """A component with N_k below the empty threshold keeps μ, σ² and gets π = 0."""
+    K, D = 2, 3
+    st = np.zeros(K * (1 + 2 * D) + 1)
+    st[0] = 10.0
+    st[1:1 + D] = [1.0, 2.0, 3.0]
+    st[1 + D:1 + 2 * D] = [10.0, 10.0, 10.0]
+    st[-1] = -5.0
+    mu = np.array([[0.0, 0.0, 0.0], [7.0, 8.0, 9.0]])
+    var = np.array([[1.0, 1.0, 1.0], [4.0, 5.0, 6.0]])
+    r = O.m_step_from_statistics(st, np.array([0.5, 0.5]), mu, var, reg_covar=0.0)
+    np.testing.assert_allclose(r.means[0], [0.1, 0.2, 0.3])
+    np.testing.assert_allclose(r.variances[0], [1 - 0.01, 1 - 0.04, 1 - 0.09])
+    np.testing.assert_array_equal(r.means[1], mu[1])
+    np.testing.assert_array_equal(r.variances[1], var[1])
+    np.testing.assert_array_equal(r.weights, [1.0, 0.0])
+    assert r.loglik == -5.0
