@@ -8,9 +8,12 @@ of synth/ with seed = rank.  Prints one JSON line on rank 0.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload table1-1e8|table1-1e6|c1] [--prec auto|fp32|fp16x3]
 
-Multi-GPU (torchrun, one process per GPU): each rank fits its own independent
-mixture problem of the full per-rank size (weak scaling, no data-path
-collective); only the timing is reduced (max over ranks).
+Multi-GPU (torchrun, one process per GPU): the ranks fit ONE mixture to the union
+of their row shards, each rank holding the full per-rank size (weak scaling).  A
+step is fgmm_em_partial on every shard, one NCCL all-gather of the statistics
+vectors (K (1 + 2D) + 1 doubles), a rank-ordered sum and fgmm_em_finish on every
+rank; the timing is reduced as the max over ranks, and one step over W ranks counts
+as W units of the per-GPU metric.
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload (rank 0 only) and scales it to the metric.
 """
@@ -243,7 +246,9 @@ def main():
     prec = {"auto": q.PREC_AUTO, "fp32": q.PREC_FP32, "fp16x3": q.PREC_FP16X3}[args.prec]
     X = torch.empty(N, D, device=dev, dtype=torch.float32)
     synth.generate(w["gen"], N, seed=rank, device=dev, out=X)
-    wt, mu, var = synth.init_params(X, K, seed=rank)
+    # every rank starts from rank 0's initial parameters: the ranks fit ONE mixture to
+    # the union of their shards (one statistics exchange per step)
+    wt, mu, var = synth.init_params(X, K, seed=0)
     g = q.GMM(K, D)
     try:
         g.set_precision(prec)
@@ -251,14 +256,23 @@ def main():
         g.set_precision(q.PREC_FP32)
     prec_set = {q.PREC_FP32: "fp32", q.PREC_FP16X3: "fp16x3", q.PREC_AUTO: "auto"}[g.precision]
     wd, md, vd = g.new_params(wt, mu, var)
+    if world > 1:
+        for t in (wd, md, vd):
+            dist.broadcast(t, src=0)
     ll = torch.zeros(1, dtype=torch.float64, device=dev)
+    from ivf_quantizer_b200 import dist as shard
+
+    def em_step(Xs, w_, m_, v_):
+        if world > 1:
+            shard.sharded_step(g, Xs, w_, m_, v_, loglik=ll)
+        else:
+            g.step(Xs, w_, m_, v_, loglik=ll)
 
     for _ in range(args.warmup):
-        g.step(X, wd, md, vd, loglik=ll)
+        em_step(X, wd, md, vd)
     torch.cuda.synchronize()
     g.check_status()
     barrier()
-    paths = set()
 
     sampler = ClockSampler(gpu_id_for(local))
     sampler.start()
@@ -272,10 +286,8 @@ def main():
     barrier()
     t0.record(stream)
     for _ in range(args.steps):
-        g.step(X, wd, md, vd, loglik=ll)
+        em_step(X, wd, md, vd)
     t1.record(stream)
-    torch.cuda.synchronize()
-    paths.add(g.last_step_path())
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
@@ -290,17 +302,21 @@ def main():
     iters_per_s = world * args.steps / (ms_max / 1e3)
 
     # ---- roofline of the dominant kernel (per launch, live CUDA-event durations)
+    # Under AUTO a step enqueues both paths' kernels and the other path's return at
+    # their gate; only the launches that did work ("active") enter the per-launch time.
     peaks, peak_src = measured_peaks()
-    s1, s2 = prof["sweep1_ms"], prof["sweep2_ms"]
-    dom = "sweep2" if s2 >= s1 else "sweep1"
-    launches = prof[f"{dom}_launches"]
-    avg_ms = prof[f"{dom}_ms"] / max(1, launches)
-    pts_per_launch = N * args.steps / max(1, launches)
+    kern = prof["kernels"]
+    sweeps = {"tc_lse": "sweep1", "tc_stats": "sweep2", "lse_simt": "sweep1",
+              "stats_simt": "sweep2"}
+    dom = max(sweeps, key=lambda k: kern.get(k, {}).get("active_ms", 0.0))
+    kd = kern.get(dom, {"active": 0, "active_ms": 0.0})
+    launches = kd["active"]
+    avg_ms = kd["active_ms"] / max(1, launches)
+    n_chunks = -(-N // q.CHUNK_POINTS)
+    pts_per_launch = N / n_chunks                       # one launch = one chunk of points
     flops_per_launch = 4.0 * D * K * pts_per_launch     # each sweep: 4*D flops per (point, comp)
-    achieved = flops_per_launch / (avg_ms / 1e3) / 1e12
-    # the path the timed steps ran (AUTO decides per step on the device; the timed
-    # region's last step is representative once warm-up has passed)
-    prec_used = "fp16x3" if paths == {q.PREC_FP16X3} else "fp32"
+    achieved = flops_per_launch / (avg_ms / 1e3) / 1e12 if launches else 0.0
+    prec_used = "fp16x3" if dom.startswith("tc_") else "fp32"
     if prec_used == "fp32":
         clk = float(peaks.get("sm_max_mhz", 1965.0))
         peak = 148 * 128 * 2 * clk * 1e6 / 1e12
@@ -313,24 +329,40 @@ def main():
                 f"(4*D per point-component per sweep), the three-product split and the "
                 f"recompute are not counted"}
     traffic = recorded_traffic(dom, prec_used)
-    roof.update({"kernel": dom, "achieved": achieved, "peak": peak, "frac": achieved / peak,
-                 "traffic": traffic, "peak_source": peak_src,
+    roof.update({"kernel": dom, "achieved": achieved, "peak": peak,
+                 "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                  "launches": launches, "avg_launch_ms": avg_ms,
-                 "share_of_step": prof[f"{dom}_ms"] / max(1e-9, ms)})
+                 "flops_per_launch": flops_per_launch,
+                 "share_of_step": kd["active_ms"] / max(1e-9, ms)})
+    # where a step's time goes: active time per kernel per step, and how many passes
+    # over the data each path made per step (an AUTO redo shows as > 1)
+    breakdown = {k: round(v["active_ms"] / args.steps, 3) for k, v in
+                 sorted(kern.items(), key=lambda kv: -kv[1]["active_ms"]) if v["active"]}
+    passes = {"tensor": kern.get("tc_stats", {}).get("active", 0) / (args.steps * n_chunks),
+              "cuda_core": kern.get("stats_simt", {}).get("active", 0) / (args.steps * n_chunks)}
 
     # ---- end to end through the public API from pinned host memory
+    # All ranks agree first on whether the pinned copy of X could be made, so that they
+    # all take the same collective steps below.
     e2e = None
     if not args.no_e2e:
+        err = None
         try:
             Xh = torch.empty(N, D, dtype=torch.float32, pin_memory=True)
             Xh.copy_(X)
+        except Exception as ex:  # pinned allocation of X may fail on small hosts
+            Xh, err = None, str(ex)[:200]
+        ok = torch.tensor([0 if err else 1], dtype=torch.int32, device=dev)
+        if world > 1:
+            dist.all_reduce(ok, op=dist.ReduceOp.MIN)
+        if int(ok.item()) == 1:
             # continue from the warmed-up parameters: the same steady-state step as above
             wd2, md2, vd2 = wd.clone(), md.clone(), vd.clone()
             llh = torch.zeros(1, dtype=torch.float64, pin_memory=True)
 
             def e2e_step():
                 X.copy_(Xh, non_blocking=True)
-                g.step(X, wd2, md2, vd2, loglik=ll)
+                em_step(X, wd2, md2, vd2)
                 llh.copy_(ll, non_blocking=True)
                 torch.cuda.current_stream().synchronize()
                 return float(llh.item())
@@ -350,9 +382,9 @@ def main():
             e2e = {"value": world * args.e2e_steps / (float(e_ms.item()) / 1e3), "unit": "iters/s",
                    "h2d_bytes_per_step": N * D * 4, "d2h_bytes_per_step": 8,
                    "steps": args.e2e_steps}
-            del Xh
-        except Exception as ex:  # pinned allocation of X may fail on small hosts
-            e2e = {"value": None, "unit": "iters/s", "error": str(ex)[:200]}
+        else:
+            e2e = {"value": None, "unit": "iters/s", "error": err or "pinned copy failed on a rank"}
+        del Xh
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -372,9 +404,12 @@ def main():
                        "precision_setting": prec_set,
                        "l2": f"inputs larger than L2 (X = {N * D * 4 / 1e9:.1f} GB per GPU)"
                        if N * D * 4 > 126e6 else "inputs smaller than L2",
-                       "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
+                       "parallelism": (f"dp{world}: row shards of one mixture fit, one all-gather "
+                                       f"of the {g.stats_len}-double statistics vector per step"
+                                       if world > 1 else "single GPU")},
             "evals_per_s": iters_per_s * N * K,
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "step_ms_by_kernel": breakdown, "passes_per_step": passes,
             "gpu_launches": int(prof["launches"]),
             "workspace_bytes": g.workspace_bytes,
             "clocks": clocks,

@@ -76,6 +76,10 @@ enum fgmm_status {
 /* A component with responsibility mass N_k below this is treated as empty:
  * its mean and variance are kept and its weight becomes 0. */
 #define FGMM_EMPTY_NK 1e-6
+/* A step walks X in chunks of this many points (the last one ragged); each sweep
+ * kernel is launched once per chunk, and every buffer the handle holds that grows
+ * with the point count is sized for one chunk. */
+#define FGMM_CHUNK_POINTS (1 << 20)
 
 /* Create a handle for K components in D dimensions.
  * reg_covar >= 0 is added to every variance after each M-step (variance floor).
@@ -114,6 +118,46 @@ int fgmm_workspace_bytes(fgmm_handle h, size_t* bytes_out);
 int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
                  float* weights, float* means, float* vars,
                  double* loglik_out, float* logz_out, fgmm_stream_t stream);
+
+/* Data-parallel EM over row shards of X (one exchange per iteration).  Each entry
+ * of the M-step's input is a sum over rows (§2, Eqs. (1)-(3)), so an iteration over
+ * shards held by several handles, devices or processes is: fgmm_em_partial on every
+ * shard with the same parameters, an elementwise sum of the statistics vectors (a
+ * collective such as an all-reduce, or an all-gather and fgmm_stats_sum), then
+ * fgmm_em_finish with the sum on every shard.  fgmm_em_step is exactly
+ * fgmm_em_partial followed by fgmm_em_finish on one shard.
+ *
+ * Statistics vector: device double[FGMM_STATS_LEN(K, D)], for component k at offset
+ * k (1 + 2D):  N_k = sum_i r_ik,  then D entries sum_i r_ik (x_id - mu_kd),  then D
+ * entries sum_i r_ik (x_id - mu_kd)^2, about the means passed to fgmm_em_partial; last
+ * entry sum_i log Z_i (this shard's log-likelihood).  The same layout serves both
+ * covariance types. */
+#define FGMM_STATS_LEN(K, D) ((int64_t)(K) * (1 + 2 * (int64_t)(D)) + 1)
+
+/* E-step and statistics sweep of one EM iteration on this shard.  weights, means,
+ * vars are read, not changed; stats_out receives the statistics vector (device,
+ * caller-owned, FGMM_STATS_LEN(K, D) doubles); logz_out as in fgmm_em_step.  Same
+ * precision modes, paths and status handling as fgmm_em_step.  Asynchronous. */
+int fgmm_em_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                    const float* weights, const float* means, const float* vars,
+                    double* stats_out, float* logz_out, fgmm_stream_t stream);
+
+/* M-step (Eqs. (1)-(3), the variance floor and the empty-component rule) from a
+ * statistics vector summed over every shard.  weights, means, vars: in/out, the
+ * parameters the statistics were taken about, replaced by Theta_out.  loglik_out:
+ * optional device double, receives the summed log-likelihood.  A non-finite
+ * log-likelihood or an all-empty mixture leaves the parameters unchanged and sets
+ * FGMM_ERR_NUMERIC in the status word.  Asynchronous. */
+int fgmm_em_finish(fgmm_handle h, const double* stats, float* weights, float* means,
+                   float* vars, double* loglik_out, fgmm_stream_t stream);
+
+/* out[j] = sum_{p = 0 .. n_parts-1} parts[p * len + j], summed in part order, so the
+ * result does not depend on how the parts arrived (device buffers; out may not
+ * overlap parts).  For combining gathered statistics vectors bit-reproducibly.
+ * FGMM_ERR_INVALID_ARG for NULL pointers, n_parts < 1 or len < 1.  Asynchronous on
+ * `stream` of the current device. */
+int fgmm_stats_sum(const double* parts, int n_parts, int64_t len, double* out,
+                   fgmm_stream_t stream);
 
 /* Repeat fgmm_em_step up to max_iters times (§2, stopping rule).  With tol > 0
  * it stops early once |L_t - L_{t-1}| / N < tol, which needs one 8-byte
@@ -173,8 +217,14 @@ int fgmm_soft_assign_static(int K, int D, int cov_type, const void* X, int x_dty
 /* Kernel timing, for benchmarks.  When enabled, the library records a CUDA
  * event pair on the call's stream around every kernel it launches and keeps a
  * launch counter; fgmm_profile_read synchronises the device, sums the elapsed
- * times per kernel kind and (if reset != 0) clears the record.  Disabled by
- * default; costs two event records per launch when enabled. */
+ * times per kernel and per kernel kind and (if reset != 0) clears the record.
+ * Under FGMM_PREC_AUTO a step enqueues the kernels of both paths and those of the
+ * path it does not take return at once; for each launch the library also copies
+ * the device word that decides this (stream-ordered, 4 bytes into pinned host
+ * memory), so that launches which did work are counted apart ("active").
+ * Disabled by default; costs two event records per launch, and one 4-byte copy
+ * per gated launch, when enabled. */
+#define FGMM_PROF_KERNELS 21
 typedef struct fgmm_profile {
   int64_t launches;          /* kernels launched while enabled (all kinds) */
   int64_t sweep1_launches;   /* log-sum-exp sweep (first pass over the components) */
@@ -183,7 +233,15 @@ typedef struct fgmm_profile {
   double sweep2_ms;
   int64_t other_launches;    /* preparation, reductions, M-step, soft assignment */
   double other_ms;
+  /* per kernel, indexed as fgmm_profile_kernel_name: every launch, and the launches
+   * that passed their path gate and did work */
+  int64_t kernel_launches[FGMM_PROF_KERNELS];
+  double kernel_ms[FGMM_PROF_KERNELS];
+  int64_t kernel_active[FGMM_PROF_KERNELS];
+  double kernel_active_ms[FGMM_PROF_KERNELS];
 } fgmm_profile;
+/* Name of kernel `index` of fgmm_profile's arrays; NULL outside [0, FGMM_PROF_KERNELS). */
+const char* fgmm_profile_kernel_name(int index);
 int fgmm_profile_enable(fgmm_handle h, int enable);
 int fgmm_profile_read(fgmm_handle h, fgmm_profile* out, int reset);
 

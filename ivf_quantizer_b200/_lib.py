@@ -20,12 +20,20 @@ MAX_TOP_M = 16
 STATIC_MAX_KD = 1 << 18
 STATIC_MAX_K = 1 << 14
 EMPTY_NK = 1e-6
+CHUNK_POINTS = 1 << 20
+
+PROF_KERNELS = 21
+
 
 class Profile(ctypes.Structure):
     _fields_ = [("launches", ctypes.c_int64), ("sweep1_launches", ctypes.c_int64),
                 ("sweep1_ms", ctypes.c_double), ("sweep2_launches", ctypes.c_int64),
                 ("sweep2_ms", ctypes.c_double), ("other_launches", ctypes.c_int64),
-                ("other_ms", ctypes.c_double)]
+                ("other_ms", ctypes.c_double),
+                ("kernel_launches", ctypes.c_int64 * PROF_KERNELS),
+                ("kernel_ms", ctypes.c_double * PROF_KERNELS),
+                ("kernel_active", ctypes.c_int64 * PROF_KERNELS),
+                ("kernel_active_ms", ctypes.c_double * PROF_KERNELS)]
 
 
 # every exported symbol of include/fgmm.h with (restype, argtypes)
@@ -50,6 +58,10 @@ SIGNATURES = {
     "fgmm_soft_assign_static": (_int, [_int, _int, _int, _vp, _int, _i64, _i64, _vp, _vp, _vp,
                                        _int, _flt, _vp, _vp, _vp]),
     "fgmm_profile_read": (_int, [_vp, _c.POINTER(Profile), _int]),
+    "fgmm_profile_kernel_name": (_c.c_char_p, [_int]),
+    "fgmm_em_partial": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_em_finish": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_stats_sum": (_int, [_vp, _int, _i64, _vp, _vp]),
 }
 
 

@@ -28,17 +28,24 @@ struct fgmm_ctx {
 };
 
 // Optional per-launch event timing (fgmm_profile_*).  Events are pooled and
-// reused after each read.
+// reused after each read; gate snapshots go to pinned host blocks.
 struct fgmm::Profiler {
+  static constexpr int kSnapBlock = 4096;
   bool enabled = false;
   int64_t launches = 0;
   struct Rec {
     cudaEvent_t a, b;
-    int kind;
+    int kernel;
+    int64_t snap;  // index of the gate snapshot, -1 for an ungated launch
+    int required;
   };
   std::vector<Rec> recs;
   std::vector<cudaEvent_t> pool;
+  std::vector<int*> snaps;  // pinned blocks of kSnapBlock words
+  int64_t nsnap = 0;
   cudaEvent_t pending = nullptr;
+  int64_t pending_snap = -1;
+  int pending_required = 0;
   cudaEvent_t get() {
     if (!pool.empty()) {
       cudaEvent_t e = pool.back();
@@ -49,6 +56,17 @@ struct fgmm::Profiler {
     cudaEventCreate(&e);
     return e;
   }
+  int* snap_slot(int64_t i) { return snaps[i / kSnapBlock] + i % kSnapBlock; }
+  int64_t new_snap() {
+    if (nsnap == (int64_t)snaps.size() * kSnapBlock) {
+      int* blk = nullptr;
+      if (cudaHostAlloc((void**)&blk, kSnapBlock * sizeof(int), cudaHostAllocDefault) !=
+          cudaSuccess)
+        return -1;
+      snaps.push_back(blk);
+    }
+    return nsnap++;
+  }
   ~Profiler() {
     for (auto& r : recs) {
       cudaEventDestroy(r.a);
@@ -56,24 +74,44 @@ struct fgmm::Profiler {
     }
     for (auto e : pool) cudaEventDestroy(e);
     if (pending) cudaEventDestroy(pending);
+    for (int* blk : snaps) cudaFreeHost(blk);
   }
 };
 
+namespace {
+const char* const kKernelNames[fgmm::KI_COUNT] = {
+    "tc_center",   "tc_prep",   "tc_convert",  "tc_lse",         "tc_stats",
+    "prep_simt",   "lse_simt",  "ll_accumulate", "stats_simt",   "reduce_stats", "mstep",
+    "finalize",    "soft_assign", "auto_check", "redo_reset",    "remask",
+    "stiff_compact", "side_lse", "ll_partials", "side_stats",    "side_reduce"};
+static_assert(fgmm::KI_COUNT == FGMM_PROF_KERNELS, "kernel table and public arrays differ");
+}  // namespace
+
 namespace fgmm {
-void prof_begin(const Ctx& c, KernelKind, cudaStream_t s) {
+void prof_begin(const Ctx& c, KernelId, cudaStream_t s, const int* gate, int required) {
   Profiler* p = c.prof;
   if (!p) return;
   ++p->launches;
   if (!p->enabled) return;
+  p->pending_snap = -1;
+  if (gate) {
+    const int64_t i = p->new_snap();
+    if (i >= 0 &&
+        cudaMemcpyAsync(p->snap_slot(i), gate, sizeof(int), cudaMemcpyDeviceToHost, s) ==
+            cudaSuccess) {
+      p->pending_snap = i;
+      p->pending_required = required;
+    }
+  }
   p->pending = p->get();
   cudaEventRecord(p->pending, s);
 }
-void prof_end(const Ctx& c, KernelKind k, cudaStream_t s) {
+void prof_end(const Ctx& c, KernelId k, cudaStream_t s) {
   Profiler* p = c.prof;
   if (!p || !p->enabled || !p->pending) return;
   cudaEvent_t b = p->get();
   cudaEventRecord(b, s);
-  p->recs.push_back({p->pending, b, (int)k});
+  p->recs.push_back({p->pending, b, (int)k, p->pending_snap, p->pending_required});
   p->pending = nullptr;
 }
 }  // namespace fgmm
@@ -93,7 +131,8 @@ void free_ws(Workspace& w) {
   void* ptrs[] = {w.mu,     w.prec,   w.cconst, w.logz, w.ll_tiles, w.ll_total,
                   w.stats,  w.nk,     w.status, w.center, w.dscale, w.wop,
                   w.tck,    w.tks,    w.xop,    w.mode, w.stiff,    w.stiff_list, w.n_stiff,
-                  w.side_part, w.mode2};
+                  w.side_part, w.mode2, w.canon, w.tcraw, w.tcm, w.tcpk, w.tckf, w.lzlow,
+                  w.side_flag};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -130,6 +169,7 @@ cudaError_t alloc_ws(Ctx& c) {
   if ((e = alloc(&w.logz, (size_t)kChunk, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.ll_tiles, (size_t)(kChunk / 32), &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.ll_total, (size_t)1, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.canon, (size_t)c.K * (1 + 2 * (size_t)c.D) + 1, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.stats, stats_bytes(w) / sizeof(double), &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.nk, (size_t)w.KpS, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.status, (size_t)1, &t)) != cudaSuccess) return e;
@@ -154,6 +194,13 @@ cudaError_t alloc_ws(Ctx& c) {
     if ((e = alloc(&w.wop, (size_t)2 * w.Kt * w.K1, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.tck, (size_t)w.Kt, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.tks, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.tcraw, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.tcm, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.tcpk, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.tckf, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.lzlow, (size_t)1, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.side_flag, (size_t)kChunk, &t)) != cudaSuccess) return e;
+    if ((e = cudaMemset(w.side_flag, 0, (size_t)kChunk)) != cudaSuccess) return e;
     if ((e = alloc(&w.xop, (size_t)2 * kChunk * w.K1, &t)) != cudaSuccess) return e;
     // rows past the end of a short chunk are read by the tensor cores (and multiplied
     // by r = 0): keep them finite from the start
@@ -251,9 +298,12 @@ int fgmm_workspace_bytes(fgmm_handle h, size_t* bytes_out) {
   return FGMM_OK;
 }
 
-int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
-                 float* weights, float* means, float* vars, double* loglik_out, float* logz_out,
-                 fgmm_stream_t stream) {
+namespace {
+// Everything of one EM iteration up to the exchange-form statistics (written to `st`):
+// preparation, both sweeps over all chunks on the selected path(s), slot reduction.
+int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                const float* weights, const float* means, const float* vars, double* st,
+                float* logz_out, fgmm_stream_t stream) {
   int rc = check_x(h, X, x_dtype, N, ldx);
   if (rc) return rc;
   if (!weights || !means || !vars) return FGMM_ERR_INVALID_ARG;
@@ -328,11 +378,44 @@ int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t l
         return map_cuda(e);
     }
   }
-  if ((e = launch_mstep(c, weights, means, vars, loglik_out, mode, fixed_mode, s)) != cudaSuccess)
+  if ((e = launch_reduce_stats(c, means, st, mode, fixed_mode, s)) != cudaSuccess)
     return map_cuda(e);
   h->c.last_auto = auto_mode;
   h->c.last_path = fixed_mode == kModeTensor ? FGMM_PREC_FP16X3 : FGMM_PREC_FP32;
   return FGMM_OK;
+}
+}  // namespace
+
+int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                 float* weights, float* means, float* vars, double* loglik_out, float* logz_out,
+                 fgmm_stream_t stream) {
+  int rc = run_partial(h, X, x_dtype, N, ldx, weights, means, vars,
+                       h ? h->c.ws.canon : nullptr, logz_out, stream);
+  if (rc) return rc;
+  return map_cuda(launch_finish(h->c, h->c.ws.canon, weights, means, vars, loglik_out,
+                                (cudaStream_t)stream));
+}
+
+int fgmm_em_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                    const float* weights, const float* means, const float* vars,
+                    double* stats_out, float* logz_out, fgmm_stream_t stream) {
+  if (!stats_out) return FGMM_ERR_INVALID_ARG;
+  return run_partial(h, X, x_dtype, N, ldx, weights, means, vars, stats_out, logz_out, stream);
+}
+
+int fgmm_em_finish(fgmm_handle h, const double* stats, float* weights, float* means,
+                   float* vars, double* loglik_out, fgmm_stream_t stream) {
+  if (!h || !stats || !weights || !means || !vars) return FGMM_ERR_INVALID_ARG;
+  int rc = set_device(h->c);
+  if (rc) return rc;
+  return map_cuda(launch_finish(h->c, stats, weights, means, vars, loglik_out,
+                                (cudaStream_t)stream));
+}
+
+int fgmm_stats_sum(const double* parts, int n_parts, int64_t len, double* out,
+                   fgmm_stream_t stream) {
+  if (!parts || !out || n_parts < 1 || len < 1) return FGMM_ERR_INVALID_ARG;
+  return map_cuda(launch_stats_sum(parts, n_parts, len, out, (cudaStream_t)stream));
 }
 
 int fgmm_last_step_path(fgmm_handle h, int* path_out) {
@@ -458,8 +541,15 @@ int fgmm_profile_read(fgmm_handle h, fgmm_profile* out, int reset) {
   for (auto& rec : p->recs) {
     float ms = 0.f;
     if ((e = cudaEventElapsedTime(&ms, rec.a, rec.b)) != cudaSuccess) return map_cuda(e);
-    if (rec.kind == KK_SWEEP1) { r.sweep1_launches++; r.sweep1_ms += ms; }
-    else if (rec.kind == KK_SWEEP2) { r.sweep2_launches++; r.sweep2_ms += ms; }
+    const bool active = rec.snap < 0 || *p->snap_slot(rec.snap) == rec.required;
+    r.kernel_launches[rec.kernel]++;
+    r.kernel_ms[rec.kernel] += ms;
+    if (active) {
+      r.kernel_active[rec.kernel]++;
+      r.kernel_active_ms[rec.kernel] += ms;
+    }
+    if (rec.kernel == KI_TC_LSE || rec.kernel == KI_LSE_SIMT) { r.sweep1_launches++; r.sweep1_ms += ms; }
+    else if (rec.kernel == KI_TC_STATS || rec.kernel == KI_STATS_SIMT) { r.sweep2_launches++; r.sweep2_ms += ms; }
     else { r.other_launches++; r.other_ms += ms; }
   }
   *out = r;
@@ -470,8 +560,13 @@ int fgmm_profile_read(fgmm_handle h, fgmm_profile* out, int reset) {
     }
     p->recs.clear();
     p->launches = 0;
+    p->nsnap = 0;
   }
   return FGMM_OK;
+}
+
+const char* fgmm_profile_kernel_name(int index) {
+  return (index >= 0 && index < FGMM_PROF_KERNELS) ? kKernelNames[index] : nullptr;
 }
 
 int fgmm_selftest_bounded_wait(int limit_ms) {

@@ -21,11 +21,25 @@ constexpr int kDC = 32;        // feature chunk staged in shared memory
 constexpr int kFC = 128;       // features per CTA in the statistics sweep
 constexpr int kSlices = 16;    // point slices of a chunk in the statistics sweep
 constexpr int kFlushTiles = 64;  // fp32 run length (tiles) before an fp64 flush
-constexpr int64_t kChunk = 1 << 20;  // points per chunk: bounds every N-sized buffer
+constexpr int64_t kChunk = FGMM_CHUNK_POINTS;  // points per chunk: bounds every N-sized buffer
 constexpr int kSideMaxStiff = 256;   // AUTO side path: most stiff components per step
 constexpr int kSideParts = 64;       // AUTO side path: point ranges per chunk
+// AUTO side path: a stiff component whose log-density is more than this many nats below
+// a point's log Z has responsibility exp(-120) < 1e-52 there (zero in fp32)
+constexpr float kSideCut = 120.f;
 
 static inline int round_up(int a, int b) { return (a + b - 1) / b * b; }
+
+// Index of statistic c (0: N_k, 1 + d: first moment, 1 + Dp + d: second moment) of
+// component k in slot s.  The CUDA-core kernels use [slot][component][row] (a component's
+// row contiguous); the tensor-core kernels use [slot][row][component] (consecutive
+// components contiguous, so that the 32 lanes of a flushing warp, 32 components, reduce
+// into 32 consecutive doubles).  kstride = components per slot, row = 1 + 2 Dp.
+__host__ __device__ __forceinline__ size_t stat_idx(bool tc_layout, int s, int k, int c,
+                                                    int kstride, size_t row) {
+  return tc_layout ? ((size_t)s * row + (size_t)c) * (size_t)kstride + (size_t)k
+                   : ((size_t)s * (size_t)kstride + (size_t)k) * row + (size_t)c;
+}
 static inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Device-side status word values are the public fgmm_status codes.
@@ -46,6 +60,14 @@ struct Workspace {
   __half* wop = nullptr;    // [2][Kt][K1] W' hi / lo
   float* tck = nullptr;     // [Kt] c_k
   float* tks = nullptr;     // [Kt] 2^t_k
+  // AUTO side-path filter: a stiff component's tensor-core logit is only an estimate, but
+  // with a per-component error bound E_k it tells which points can need the side path
+  float* tcraw = nullptr;   // [Kt] c_k before masking
+  float* tcm = nullptr;     // [Kt] M_k = sum_d (mu_kd - c_d)^2 / sigma_kd^2
+  float* tcpk = nullptr;    // [Kt] P_k = log pi_k + log N(mu_k | mu_k, Sigma_k), the peak
+  float* tckf = nullptr;    // [Kt] c_k + E_k for stiff components, -inf otherwise
+  float* lzlow = nullptr;   // [1] log Z below which a point is always flagged
+  uint8_t* side_flag = nullptr;  // [kChunk] 1: the point may have a stiff component within kCut
   __half* xop = nullptr;    // [2][kChunk][K1] phi(x) hi / lo of the current chunk
   int* mode = nullptr;      // [1] path of the current step: 0 tensor cores, 1 CUDA cores
   int* mode2 = nullptr;     // [1] AUTO: tensor when the hybrid redo pass must run
@@ -61,6 +83,7 @@ struct Workspace {
   float* logz = nullptr;   // [kChunk] log Z_i of the chunk being processed
   double* ll_tiles = nullptr;  // [kChunk / 32] partial log-likelihoods of the chunk
   double* ll_total = nullptr;  // [1]
+  double* canon = nullptr;  // [K (1 + 2D) + 1] exchange-form statistics of the step
   // statistics partials, one slot per point slice: [slots][KpS][1 + 2 Dp]
   double* stats = nullptr;
   double* nk = nullptr;    // [Kp] reduced N_k of the last step
@@ -68,8 +91,16 @@ struct Workspace {
   size_t bytes = 0;
 };
 
-// Kernel kinds for the optional event timing (fgmm_profile_*).
-enum KernelKind { KK_SWEEP1 = 0, KK_SWEEP2 = 1, KK_OTHER = 2 };
+// Kernels, for the optional event timing (fgmm_profile_*); the order is the index into
+// fgmm_profile's per-kernel arrays and must match the names in fgmm_host.cu.
+enum KernelId {
+  KI_TC_CENTER = 0, KI_TC_PREP, KI_TC_CONVERT, KI_TC_LSE, KI_TC_STATS,
+  KI_PREP_SIMT, KI_LSE_SIMT, KI_LL_ACCUMULATE, KI_STATS_SIMT, KI_REDUCE_STATS, KI_MSTEP,
+  KI_FINALIZE,
+  KI_SOFT_ASSIGN, KI_AUTO_CHECK, KI_REDO_RESET, KI_REMASK,
+  KI_STIFF_COMPACT, KI_SIDE_LSE, KI_LL_PARTIALS, KI_SIDE_STATS, KI_SIDE_REDUCE,
+  KI_COUNT
+};
 
 struct Profiler;  // defined in fgmm_host.cu
 
@@ -95,8 +126,13 @@ constexpr int kModeTensor = 0;
 constexpr int kModeSimt = 1;
 
 // Brackets one kernel launch with profiling events when profiling is enabled.
-void prof_begin(const Ctx& c, KernelKind k, cudaStream_t s);
-void prof_end(const Ctx& c, KernelKind k, cudaStream_t s);
+// Brackets one launch with events when profiling is enabled.  A launch whose kernel
+// returns at once unless *gate == required passes gate (else nullptr): the profiler then
+// snapshots the word in stream order, so that it can tell launches that did work from
+// launches that returned at their gate.
+void prof_begin(const Ctx& c, KernelId k, cudaStream_t s, const int* gate = nullptr,
+                int required = 0);
+void prof_end(const Ctx& c, KernelId k, cudaStream_t s);
 
 // ---------------------------------------------------------------- launchers
 // `mode` arguments: nullptr runs the kernel unconditionally; otherwise the kernel
@@ -114,8 +150,14 @@ cudaError_t launch_ll_accumulate(const Ctx& c, int64_t n, const int* mode, int f
 cudaError_t launch_auto_check(const Ctx& c, int stage, cudaStream_t s);
 cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
                               const int* mode, cudaStream_t s);
-cudaError_t launch_mstep(const Ctx& c, float* weights, float* means, float* vars,
-                         double* loglik_out, const int* mode, int fixed_mode, cudaStream_t s);
+// Slot sums -> exchange-form statistics (out: [K (1 + 2D) + 1], about `means`).
+cudaError_t launch_reduce_stats(const Ctx& c, const float* means, double* out, const int* mode,
+                                int fixed_mode, cudaStream_t s);
+// M-step and weights from exchange-form statistics; parameters updated in place.
+cudaError_t launch_finish(const Ctx& c, const double* st, float* weights, float* means,
+                          float* vars, double* loglik_out, cudaStream_t s);
+cudaError_t launch_stats_sum(const double* parts, int n_parts, int64_t len, double* out,
+                             cudaStream_t s);
 // tensor-core path (fgmm_tc.cu)
 bool tc_supported(const Ctx& c);
 cudaError_t tc_init(Ctx& c);

@@ -24,7 +24,9 @@
 namespace fgmm {
 namespace {
 
-constexpr float kCut = 120.f;
+constexpr float kCut = kSideCut;
+constexpr double kErrRel = 2e-5;      // tensor-core logit error per unit of sum |W' phi|
+constexpr float kLzMargin = 5000.f;   // nats below the lowest component peak
 
 __device__ __forceinline__ float ldx_f(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float ldx_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
@@ -56,8 +58,11 @@ constexpr int kMaxStiff = kSideMaxStiff;
 
 // Runs when *gate is tensor (or gate is null); on overflow the step goes to the CUDA-core
 // path (*mode) and the gated pass is switched off (*gate).
-__global__ void stiff_compact_kernel(const int* __restrict__ stiff, int K, int* __restrict__ list,
-                                     int* __restrict__ n_out, int* gate, int* mode) {
+__global__ void stiff_compact_kernel(const int* __restrict__ stiff, int K, int Kt,
+                                     int* __restrict__ list, int* __restrict__ n_out,
+                                     const float* __restrict__ craw, const float* __restrict__ mq,
+                                     const float* __restrict__ peak, float* __restrict__ ckf,
+                                     float* __restrict__ lzlow, int* gate, int* mode) {
   if (gate && *gate != kModeTensor) return;
   __shared__ int base;
   if (threadIdx.x == 0) base = 0;
@@ -89,6 +94,37 @@ __global__ void stiff_compact_kernel(const int* __restrict__ stiff, int K, int* 
       *gate = kModeSimt;
     }
   }
+  // Filter constants.  The tensor-core logit of component k at x is exact up to
+  // |err| <= kErrRel * sum_j |W'_kj phi_j(x)| (three-product split: 3 * 2^-22 per product;
+  // fp32 accumulation over at most 64 steps: 64 * 2^-23; kErrRel carries a factor 2.4 of
+  // margin).  With M_k = sum_d p_d mu~_d^2 (p = 1/sigma^2, mu~ = mu - c) and
+  // s = sum_d p_d (x_d - mu_d)^2, that sum is at most 1.5 M + 2 sqrt(M s) + s / 2.  A point
+  // with log Z >= L for which k matters (log z_k >= log Z - kCut) has
+  // s = 2 (P_k - log z_k) <= Q_k = 2 (P_k - L + kCut), so its estimate exceeds
+  // log Z - kCut - E_k, E_k = kErrRel (1.5 M + 2 sqrt(M Q) + Q / 2) + 1.  L = the lowest
+  // peak minus kLzMargin; points below L are always flagged.
+  __shared__ float red[256];
+  float pm = CUDART_INF_F;
+  for (int k = threadIdx.x; k < K; k += blockDim.x)
+    if (peak[k] > -CUDART_INF_F) pm = fminf(pm, peak[k]);
+  red[threadIdx.x] = pm;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] = fminf(red[threadIdx.x], red[threadIdx.x + s]);
+    __syncthreads();
+  }
+  const float low = red[0] - kLzMargin;
+  if (threadIdx.x == 0) *lzlow = low;
+  for (int k = threadIdx.x; k < Kt; k += blockDim.x) {
+    float f = -CUDART_INF_F;
+    if (k < K && stiff[k] && craw[k] > -CUDART_INF_F) {
+      const double M = mq[k];
+      const double Q = fmax(2.0 * ((double)peak[k] - (double)low + (double)kCut), 0.0);
+      const double E = kErrRel * (1.5 * M + 2.0 * sqrt(M * Q) + 0.5 * Q) + 1.0;
+      f = (float)((double)craw[k] + E);
+    }
+    ckf[k] = f;
+  }
 }
 
 // Thread per point: merge the stiff components' log-densities into log Z.
@@ -96,13 +132,14 @@ template <typename T>
 __global__ void side_lse_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp,
                                 const float* __restrict__ mu, const float* __restrict__ prec,
                                 const float* __restrict__ cconst, const int* __restrict__ list,
-                                const int* __restrict__ n_stiff, float* __restrict__ logz,
-                                float* __restrict__ logz_out, const int* mode) {
+                                const int* __restrict__ n_stiff, const uint8_t* __restrict__ flag,
+                                float* __restrict__ logz, float* __restrict__ logz_out,
+                                const int* mode) {
   if (mode && *mode != kModeTensor) return;
   const int ns = *n_stiff;
   if (ns == 0) return;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
+  if (i >= n || !flag[i]) return;  // unflagged: no stiff component within kCut of log Z
   const T* x = X + i * ldx;
   float lz = logz[i];
   for (int j = 0; j < ns; ++j) {
@@ -156,8 +193,8 @@ __global__ void __launch_bounds__(256)
     side_stats_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp,
                       const float* __restrict__ mu, const float* __restrict__ prec,
                       const float* __restrict__ cconst, const int* __restrict__ list,
-                      const int* __restrict__ n_stiff, const float* __restrict__ logz,
-                      double* __restrict__ part, const int* mode) {
+                      const int* __restrict__ n_stiff, const uint8_t* __restrict__ flag,
+                      const float* __restrict__ logz, double* __restrict__ part, const int* mode) {
   if (mode && *mode != kModeTensor) return;
   const int j = blockIdx.x;
   if (j >= *n_stiff) return;
@@ -178,7 +215,7 @@ __global__ void __launch_bounds__(256)
   for (int64_t b = w0; b < w1; b += 32) {
     const int64_t i = b + lane;
     float r = 0.f;
-    if (i < w1) {
+    if (i < w1 && flag[i]) {
       const float lz = logz[i];
       const float l = stiff_logit(X + i * ldx, D, muk, pk, ck, lz - kCut);
       if (l > -CUDART_INF_F && lz > -CUDART_INF_F) r = fminf(expf(l - lz), 1.f);
@@ -216,31 +253,32 @@ __global__ void __launch_bounds__(256)
 }
 
 // One CTA per stiff slot j: the kSideParts partial rows, summed in p order, are added to
-// the statistics of component list[j] (slot 0 of the point slices; the tensor-core
-// sweep added zeros there, the component being masked out of it).
+// the statistics of component list[j] (slot 0 of the point slices, in the tensor-core
+// layout; the tensor-core sweep added zeros there, the component being masked out of it).
 __global__ void side_reduce_kernel(const double* __restrict__ part, const int* __restrict__ list,
-                                   const int* __restrict__ n_stiff, int D, int Dp,
+                                   const int* __restrict__ n_stiff, int D, int Dp, int kstride,
                                    double* __restrict__ stats, const int* mode) {
   if (mode && *mode != kModeTensor) return;
   const int j = blockIdx.x;
   if (j >= *n_stiff) return;
   const size_t row = (size_t)(1 + 2 * Dp);
-  double* dst = stats + (size_t)list[j] * row;
+  const int k = list[j];
   for (int c = threadIdx.x; c < (int)row; c += blockDim.x) {
     const int d = (c == 0) ? 0 : (c <= Dp ? c - 1 : c - 1 - Dp);
     if (c != 0 && d >= D) continue;
     double s = 0.0;
     for (int p = 0; p < kSideParts; ++p) s += part[((size_t)p * kSideMaxStiff + j) * row + c];
-    dst[c] += s;
+    stats[stat_idx(true, 0, k, c, kstride, row)] += s;
   }
 }
 
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_stiff_compact(const Ctx& c, int* gate, int* mode, cudaStream_t s) {
-  prof_begin(c, KK_OTHER, s);
-  stiff_compact_kernel<<<1, 256, 0, s>>>(c.ws.stiff, c.K, c.ws.stiff_list, c.ws.n_stiff, gate,
-                                         mode);
-  prof_end(c, KK_OTHER, s);
+  prof_begin(c, KI_STIFF_COMPACT, s);
+  const Workspace& w = c.ws;
+  stiff_compact_kernel<<<1, 256, 0, s>>>(w.stiff, c.K, w.Kt, w.stiff_list, w.n_stiff, w.tcraw,
+                                         w.tcm, w.tcpk, w.tckf, w.lzlow, gate, mode);
+  prof_end(c, KI_STIFF_COMPACT, s);
   return cudaGetLastError();
 }
 
@@ -248,21 +286,23 @@ cudaError_t launch_side_lse(const Ctx& c, const void* X, int x_dtype, int64_t n,
                             float* logz_out, const int* mode, cudaStream_t s) {
   const unsigned grid = (unsigned)ceil_div64(n, 128);
   const Workspace& w = c.ws;
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_SIDE_LSE, s, mode, kModeTensor);
   if (x_dtype == FGMM_BF16)
     side_lse_kernel<<<grid, 128, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
-                                         w.cconst, w.stiff_list, w.n_stiff, w.logz, logz_out,
+                                         w.cconst, w.stiff_list, w.n_stiff, w.side_flag, w.logz,
+                                         logz_out,
                                          mode);
   else
     side_lse_kernel<<<grid, 128, 0, s>>>((const float*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
-                                         w.cconst, w.stiff_list, w.n_stiff, w.logz, logz_out,
+                                         w.cconst, w.stiff_list, w.n_stiff, w.side_flag, w.logz,
+                                         logz_out,
                                          mode);
-  prof_end(c, KK_OTHER, s);
+  prof_end(c, KI_SIDE_LSE, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_LL_PARTIALS, s, mode, kModeTensor);
   ll_partials_kernel<<<(unsigned)ceil_div64(n, 4096), 256, 0, s>>>(w.logz, n, w.ll_tiles, mode);
-  prof_end(c, KK_OTHER, s);
+  prof_end(c, KI_LL_PARTIALS, s);
   return cudaGetLastError();
 }
 
@@ -270,22 +310,22 @@ cudaError_t launch_side_stats(const Ctx& c, const void* X, int x_dtype, int64_t 
                               const int* mode, cudaStream_t s) {
   const Workspace& w = c.ws;
   dim3 grid(kSideMaxStiff, kSideParts);
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_SIDE_STATS, s, mode, kModeTensor);
   if (x_dtype == FGMM_BF16)
     side_stats_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dp, w.mu,
-                                           w.prec, w.cconst, w.stiff_list, w.n_stiff, w.logz,
-                                           w.side_part, mode);
+                                           w.prec, w.cconst, w.stiff_list, w.n_stiff, w.side_flag,
+                                           w.logz, w.side_part, mode);
   else
     side_stats_kernel<<<grid, 256, 0, s>>>((const float*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
-                                           w.cconst, w.stiff_list, w.n_stiff, w.logz,
-                                           w.side_part, mode);
-  prof_end(c, KK_OTHER, s);
+                                           w.cconst, w.stiff_list, w.n_stiff, w.side_flag,
+                                           w.logz, w.side_part, mode);
+  prof_end(c, KI_SIDE_STATS, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_SIDE_REDUCE, s, mode, kModeTensor);
   side_reduce_kernel<<<kSideMaxStiff, 256, 0, s>>>(w.side_part, w.stiff_list, w.n_stiff, c.D,
-                                                   w.Dp, w.stats, mode);
-  prof_end(c, KK_OTHER, s);
+                                                   w.Dp, w.KpS, w.stats, mode);
+  prof_end(c, KI_SIDE_REDUCE, s);
   return cudaGetLastError();
 }
 

@@ -351,59 +351,75 @@ __global__ void __launch_bounds__(kSimtThreads)
   flush();
 }
 
-// ------------------------------------------------------------------ M-step
-// One CTA per component: fixed-order fp64 sum over the slice slots, then Eqs. (1)-(3).
-// The slots hold N_k, S1 = sum r (y - o), S2 = sum r (y - o)^2 in a coordinate y with
-// origin o: the CUDA-core path uses y = x, o = mu_old (centred on the current mean);
-// the tensor-core path uses y = (x - c) s, o = 0.  Then
-//   m1 = S1 / N_k,  mu_new = o + m1 (mapped back to x),
-//   sigma^2 = max(S2 / N_k - m1^2, 0) (mapped back to x) + reg_covar
-// (isotropic: averaged over d).  Empty components keep their parameters.  Nothing is
-// written when the log-likelihood of the step is not finite.
-__global__ void mstep_kernel(int K, int D, int Dp, int kstride, int cov, double reg,
-                             const double* __restrict__ stats, int s_simt, int s_tc,
-                             const int* mode, int fixed_mode, const int* __restrict__ stiff,
-                             const float* __restrict__ mu_old,
-                             const float* __restrict__ center, const float* __restrict__ dscale,
-                             const double* __restrict__ ll_total, float* __restrict__ means,
-                             float* __restrict__ vars, double* __restrict__ nk_out, int* status) {
-  __shared__ double red[kSimtThreads];
+// ------------------------------------------------------------------ reduction and M-step
+// Fixed-order sum of the statistics slots and conversion to the exchange form: per
+// component [N_k, sum r (x - mu_k), sum r (x - mu_k)^2] about the step's input means
+// (data units), then sum log Z.  A CUDA-core step, or a stiff component of a
+// tensor-core step (side path), accumulated about the input mean already; the tensor
+// cores accumulated moments of x^ = (x - c) s about the centre c, which are unscaled
+// and shifted here in fp64.  One CTA per component.
+__global__ void reduce_stats_kernel(int K, int D, int Dp, int kstride,
+                                    const double* __restrict__ stats, int s_simt, int s_tc,
+                                    const int* mode, int fixed_mode, const int* __restrict__ stiff,
+                                    const float* __restrict__ means,
+                                    const float* __restrict__ center,
+                                    const float* __restrict__ dscale,
+                                    const double* __restrict__ ll_total, double* __restrict__ out) {
   const int k = blockIdx.x;
   const bool simt_step = ((mode ? *mode : fixed_mode) == kModeSimt);
   const int nslots = simt_step ? s_simt : s_tc;
-  // a stiff component of a tensor-core step was handled by the side path, whose
-  // statistics are centred on the current mean like the CUDA-core path's
   const bool simt = simt_step || (stiff && stiff[k]);
   const size_t row = (size_t)(1 + 2 * Dp);
-  const bool ll_ok = isfinite(*ll_total);
+  const size_t orow = (size_t)(1 + 2 * D);
   double nk = 0.0;
-  for (int s = 0; s < nslots; ++s) nk += stats[((size_t)s * kstride + k) * row];
-  if (threadIdx.x == 0) nk_out[k] = nk;
-  const bool live = ll_ok && (nk >= FGMM_EMPTY_NK);
-  double vsum = 0.0;
+  for (int s = 0; s < nslots; ++s) nk += stats[stat_idx(!simt_step, s, k, 0, kstride, row)];
+  double* o = out + (size_t)k * orow;
+  if (threadIdx.x == 0) o[0] = nk;
+  if (k == 0 && threadIdx.x == 0) out[(size_t)K * orow] = *ll_total;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     double s1 = 0.0, s2 = 0.0;
     for (int s = 0; s < nslots; ++s) {
-      const double* r = stats + ((size_t)s * kstride + k) * row;
-      s1 += r[1 + d];
-      s2 += r[1 + Dp + d];
+      s1 += stats[stat_idx(!simt_step, s, k, 1 + d, kstride, row)];
+      s2 += stats[stat_idx(!simt_step, s, k, 1 + Dp + d, kstride, row)];
     }
-    if (live) {
-      const double m1 = s1 / nk;
-      double v = fmax(s2 / nk - m1 * m1, 0.0);
-      double mu;
-      if (simt) {
-        mu = (double)mu_old[(size_t)k * Dp + d] + m1;
-      } else {
-        const double sd = dscale[d];
-        mu = (double)center[d] + m1 / sd;
-        v = v / (sd * sd);
-      }
-      means[(size_t)k * D + d] = (float)mu;
+    if (!simt) {
+      // about c in scaled units -> about c in data units -> about mu_k
+      const double sd = dscale[d];
+      const double s1c = s1 / sd, s2c = s2 / (sd * sd);
+      const double del = (double)means[(size_t)k * D + d] - (double)center[d];
+      s1 = s1c - nk * del;
+      s2 = s2c - 2.0 * del * s1c + nk * del * del;
+    }
+    o[1 + d] = s1;
+    o[1 + D + d] = s2;
+  }
+}
+
+// M-step Eqs. (1)-(3) from exchange-form statistics (summed over every shard of the
+// rows): mu_new = mu + S1/N_k, sigma^2 = S2/N_k - (S1/N_k)^2 (+ floor; spherical: mean
+// over d).  Empty components keep mu and sigma^2.  Parameters are updated in place; the
+// means passed in must be those the statistics were taken about.  One CTA per component.
+__global__ void finish_kernel(int K, int D, int cov, double reg, const double* __restrict__ st,
+                              float* __restrict__ means, float* __restrict__ vars,
+                              double* __restrict__ nk_out, int* status) {
+  __shared__ double red[kSimtThreads];
+  const int k = blockIdx.x;
+  const size_t orow = (size_t)(1 + 2 * D);
+  const double* o = st + (size_t)k * orow;
+  const double nk = o[0];
+  const bool ll_ok = isfinite(st[(size_t)K * orow]);
+  if (threadIdx.x == 0) nk_out[k] = nk;
+  const bool live = ll_ok && (nk >= FGMM_EMPTY_NK);
+  double vsum = 0.0;
+  if (live)
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+      const double m1 = o[1 + d] / nk;
+      const double v = fmax(o[1 + D + d] / nk - m1 * m1, 0.0);
+      float* mp = means + (size_t)k * D + d;
+      *mp = (float)((double)*mp + m1);
       if (cov == FGMM_COV_DIAG) vars[(size_t)k * D + d] = (float)(v + reg);
       vsum += v;
     }
-  }
   if (cov == FGMM_COV_SPHERICAL) {
     red[threadIdx.x] = vsum;
     __syncthreads();
@@ -414,6 +430,17 @@ __global__ void mstep_kernel(int K, int D, int Dp, int kstride, int cov, double 
     if (threadIdx.x == 0 && live) vars[k] = (float)(red[0] / D + reg);
   }
   if (threadIdx.x == 0 && !isfinite(nk)) set_status(status, FGMM_ERR_NUMERIC);
+}
+
+// Sum of n_parts exchange-form statistics vectors, in part order.
+__global__ void stats_sum_kernel(const double* __restrict__ parts, int n_parts, int64_t len,
+                                 double* __restrict__ out) {
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < len;
+       j += (int64_t)gridDim.x * blockDim.x) {
+    double acc = 0.0;
+    for (int p = 0; p < n_parts; ++p) acc += parts[(size_t)p * len + j];
+    out[j] = acc;
+  }
 }
 
 // Weights pi_k = N_k / sum_{live k'} N_k' (Alg. 1, final step), log-likelihood output,
@@ -537,8 +564,8 @@ __global__ void tc_variance_check_kernel(int K, int D, int Dp, int kstride,
   const int k = blockIdx.x;
   if (stiff[k]) return;  // the side path's statistics are centred on the mean: exact
   const size_t row = (size_t)(1 + 2 * Dp);
-  double nk = 0.0;
-  for (int s = 0; s < nslots; ++s) nk += stats[((size_t)s * kstride + k) * row];
+  double nk = 0.0;  // tensor-core slot layout (this check runs after tensor-core passes only)
+  for (int s = 0; s < nslots; ++s) nk += stats[stat_idx(true, s, k, 0, kstride, row)];
   if (!(nk >= FGMM_EMPTY_NK)) return;  // empty: parameters are kept, nothing to check
   __shared__ int bad_any;
   if (threadIdx.x == 0) bad_any = 0;
@@ -547,9 +574,8 @@ __global__ void tc_variance_check_kernel(int K, int D, int Dp, int kstride,
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     double s1 = 0.0, s2 = 0.0;
     for (int s = 0; s < nslots; ++s) {
-      const double* r = stats + ((size_t)s * kstride + k) * row;
-      s1 += r[1 + d];
-      s2 += r[1 + Dp + d];
+      s1 += stats[stat_idx(true, s, k, 1 + d, kstride, row)];
+      s2 += stats[stat_idx(true, s, k, 1 + Dp + d, kstride, row)];
     }
     const double m2 = s2 / nk, m1 = s1 / nk;
     const double v = m2 - m1 * m1;
@@ -590,18 +616,18 @@ __global__ void remask_kernel(const int* redo, const int* __restrict__ stiff, in
 // ------------------------------------------------------------------ launchers
 cudaError_t launch_prep_simt(const Ctx& c, const float* weights, const float* means,
                              const float* vars, cudaStream_t s) {
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_PREP_SIMT, s);
   prep_simt_kernel<<<c.ws.Kp, kSimtThreads, 0, s>>>(c.K, c.D, c.ws.Kp, c.ws.Dp, c.cov, weights,
                                                     means, vars, c.ws.mu, c.ws.prec,
                                                     c.ws.cconst, c.ws.status);
-  prof_end(c, KK_OTHER, s);
+  prof_end(c, KI_PREP_SIMT, s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_lse_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
                             float* logz_out, const int* mode, cudaStream_t s) {
   const unsigned grid = (unsigned)ceil_div64(n, kTP);
-  prof_begin(c, KK_SWEEP1, s);
+  prof_begin(c, KI_LSE_SIMT, s, mode, kModeSimt);
   if (x_dtype == FGMM_BF16)
     lse_simt_kernel<<<grid, kSimtThreads, 0, s>>>(
         (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
@@ -610,17 +636,17 @@ cudaError_t launch_lse_simt(const Ctx& c, const void* X, int x_dtype, int64_t n,
     lse_simt_kernel<<<grid, kSimtThreads, 0, s>>>((const float*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp,
                                                   c.ws.mu, c.ws.prec, c.ws.cconst, c.ws.logz,
                                                   logz_out, c.ws.ll_tiles, mode);
-  prof_end(c, KK_SWEEP1, s);
+  prof_end(c, KI_LSE_SIMT, s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ll_accumulate(const Ctx& c, int64_t n, const int* mode, int fixed_mode,
                                  int required, cudaStream_t s) {
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_LL_ACCUMULATE, s, mode, required);
   ll_accumulate_kernel<<<1, kSimtThreads, 0, s>>>(c.ws.ll_tiles, (int)ceil_div64(n, kTP),
                                                   (int)ceil_div64(n, 4096), mode, fixed_mode,
                                                   required, c.ws.ll_total);
-  prof_end(c, KK_OTHER, s);
+  prof_end(c, KI_LL_ACCUMULATE, s);
   return cudaGetLastError();
 }
 
@@ -638,7 +664,7 @@ cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t 
   int64_t slice = ceil_div64(n, kSlices);
   slice = ceil_div64(slice, kTP) * kTP;
   dim3 grid(c.ws.Kp / kKBs, kSlices, (unsigned)ceil_div64(c.ws.Dp, kFC));
-  prof_begin(c, KK_SWEEP2, s);
+  prof_begin(c, KI_STATS_SIMT, s, mode, kModeSimt);
   if (x_dtype == FGMM_BF16)
     stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>(
         (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
@@ -647,25 +673,41 @@ cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t 
     stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>((const float*)X, n, ldx, c.D, c.ws.Dp,
                                                        c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
                                                        c.ws.logz, c.ws.stats, c.ws.KpS, slice, mode);
-  prof_end(c, KK_SWEEP2, s);
+  prof_end(c, KI_STATS_SIMT, s);
   return cudaGetLastError();
 }
 
-cudaError_t launch_mstep(const Ctx& c, float* weights, float* means, float* vars,
-                         double* loglik_out, const int* mode, int fixed_mode, cudaStream_t s) {
-  prof_begin(c, KK_OTHER, s);
-  mstep_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, c.ws.Dp, c.ws.KpS, c.cov, c.reg, c.ws.stats,
-                                            kSlices, c.tc.ready ? tc_slices(c) : 1, mode,
-                                            fixed_mode, c.tc.ready ? c.ws.stiff : nullptr,
-                                            c.ws.mu, c.ws.center, c.ws.dscale,
-                                            c.ws.ll_total, means, vars, c.ws.nk, c.ws.status);
-  prof_end(c, KK_OTHER, s);
+cudaError_t launch_reduce_stats(const Ctx& c, const float* means, double* out, const int* mode,
+                                int fixed_mode, cudaStream_t s) {
+  prof_begin(c, KI_REDUCE_STATS, s);
+  reduce_stats_kernel<<<c.K, kSimtThreads, 0, s>>>(
+      c.K, c.D, c.ws.Dp, c.ws.KpS, c.ws.stats, kSlices, c.tc.ready ? tc_slices(c) : 1, mode,
+      fixed_mode, c.tc.ready ? c.ws.stiff : nullptr, means, c.ws.center, c.ws.dscale,
+      c.ws.ll_total, out);
+  prof_end(c, KI_REDUCE_STATS, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finish(const Ctx& c, const double* st, float* weights, float* means,
+                          float* vars, double* loglik_out, cudaStream_t s) {
+  prof_begin(c, KI_MSTEP, s);
+  finish_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, c.cov, c.reg, st, means, vars, c.ws.nk,
+                                             c.ws.status);
+  prof_end(c, KI_MSTEP, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  prof_begin(c, KK_OTHER, s);
-  finalize_kernel<<<1, kSimtThreads, 0, s>>>(c.K, c.ws.nk, c.ws.ll_total, weights, loglik_out,
-                                             c.ws.status);
-  prof_end(c, KK_OTHER, s);
+  prof_begin(c, KI_FINALIZE, s);
+  finalize_kernel<<<1, kSimtThreads, 0, s>>>(c.K, c.ws.nk, st + (size_t)c.K * (1 + 2 * c.D),
+                                             weights, loglik_out, c.ws.status);
+  prof_end(c, KI_FINALIZE, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats_sum(const double* parts, int n_parts, int64_t len, double* out,
+                             cudaStream_t s) {
+  const int64_t blocks = (len + 255) / 256;
+  stats_sum_kernel<<<(unsigned)(blocks < 1024 ? blocks : 1024), 256, 0, s>>>(parts, n_parts, len,
+                                                                             out);
   return cudaGetLastError();
 }
 
@@ -673,7 +715,7 @@ cudaError_t launch_soft_assign_simt(const Ctx& c, const void* X, int x_dtype, in
                                     int64_t ldx, int top_m, float r_threshold, int32_t* ids,
                                     float* resp, cudaStream_t s) {
   const unsigned grid = (unsigned)ceil_div64(n, kTP);
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_SOFT_ASSIGN, s);
   if (x_dtype == FGMM_BF16)
     soft_assign_simt_kernel<<<grid, kSimtThreads, 0, s>>>(
         (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.K, c.ws.mu, c.ws.prec,
@@ -682,7 +724,7 @@ cudaError_t launch_soft_assign_simt(const Ctx& c, const void* X, int x_dtype, in
     soft_assign_simt_kernel<<<grid, kSimtThreads, 0, s>>>(
         (const float*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.K, c.ws.mu, c.ws.prec, c.ws.cconst,
         top_m, r_threshold, ids, resp);
-  prof_end(c, KK_OTHER, s);
+  prof_end(c, KI_SOFT_ASSIGN, s);
   return cudaGetLastError();
 }
 
@@ -692,25 +734,25 @@ namespace fgmm {
 cudaError_t launch_auto_check(const Ctx& c, int stage, cudaStream_t s) {
   const Workspace& w = c.ws;
   const size_t n = (size_t)w.slots * w.KpS * (1 + 2 * (size_t)w.Dp);
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_AUTO_CHECK, s);
   tc_variance_check_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, w.Dp, w.KpS, w.stats,
                                                         tc_slices(c), w.stiff,
                                                         stage == 0 ? w.mode : w.mode2, w.mode2,
                                                         w.mode, stage);
-  prof_end(c, KK_OTHER, s);
+  prof_end(c, KI_AUTO_CHECK, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_REDO_RESET, s);
   if (stage == 0)
     redo_reset_kernel<<<2 * c.num_sms, 256, 0, s>>>(w.mode2, kModeTensor, w.stats, n, w.ll_total);
   else
     redo_reset_kernel<<<2 * c.num_sms, 256, 0, s>>>(w.mode, kModeSimt, w.stats, n, w.ll_total);
-  prof_end(c, KK_OTHER, s);
+  prof_end(c, KI_REDO_RESET, s);
   e = cudaGetLastError();
   if (e != cudaSuccess || stage != 0) return e;
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_REMASK, s);
   remask_kernel<<<(w.Kt + 255) / 256, 256, 0, s>>>(w.mode2, w.stiff, w.Kt, w.tck);
-  prof_end(c, KK_OTHER, s);
+  prof_end(c, KI_REMASK, s);
   return cudaGetLastError();
 }
 }  // namespace fgmm

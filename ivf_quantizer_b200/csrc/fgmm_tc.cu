@@ -58,7 +58,7 @@ constexpr int BM = 128;          // points per tile
 constexpr int BKc = 128;         // components per block
 constexpr int KC = 64;           // K elements per swizzle row / TMA box
 constexpr int BOX = 128 * 64 * 2;  // bytes of one [128 rows][64 fp16] box
-constexpr int SW = 4;            // W ring stages (sweep 1)
+constexpr int SW = 8;            // W ring stages (sweep 1)
 constexpr int SX = 8;            // X ring stages (sweep 2)
 constexpr float kRScale = 32768.f;  // r is stored as fp16(r * 2^15)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -142,7 +142,8 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
                                const float* __restrict__ scale, const double* __restrict__ nk_prev,
                                __half* __restrict__ wop, float* __restrict__ ck,
                                float* __restrict__ kscale, int* __restrict__ stiff,
-                               int* status) {
+                               float* __restrict__ craw, float* __restrict__ mq,
+                               float* __restrict__ peak, int* status) {
   __shared__ double rs[kSimtThreads], rq[kSimtThreads], rt[kSimtThreads];
   __shared__ float rmax[kSimtThreads], amax[kSimtThreads];
   __shared__ float s_pow;
@@ -202,6 +203,9 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
         is_stiff = !(ldexp(sqrt(rt[0]), -20) <= 1e-3) || !(amax[0] <= 900.f) ||
                    (nk_prev[k] < 4.0);
     }
+    craw[k] = c;
+    mq[k] = live_k ? (float)rq[0] : 0.f;
+    peak[k] = (live_k && w[k] > 0.f) ? (float)(log((double)w[k]) - 0.5 * rs[0]) : -CUDART_INF_F;
     if (stiff) {
       stiff[k] = is_stiff;
       if (is_stiff) c = -CUDART_INF_F;
@@ -275,11 +279,15 @@ __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ld
 // epilogue warpgroups split each 128-column S tile in halves (columns 64g .. 64g+63) and
 // keep a running (max, sum) per row; at the end of a tile the upper half hands its
 // pair to the lower half through shared memory, which writes log Z.
+// phi hi of the point tile sits in shared memory (A operand of two products); phi lo
+// sits in tensor memory (A operand of the third), written there by the epilogue warps
+// one tile ahead, so that shared memory holds an 8-stage ring of W' boxes.
 constexpr int kEpiWarps = 8;
 constexpr int kTcThreads = 128 + 32 * kEpiWarps;
 
 struct LseBars {
   uint64_t x_full[4], x_empty[4];
+  uint64_t xlo_ready[2];
   uint64_t w_full[SW], w_empty[SW];
   uint64_t s_full[2], s_empty[2];
   uint64_t xc_full[2], xc_empty[2];
@@ -288,6 +296,7 @@ struct LseBars {
   int abort;
   alignas(16) float xm[2][BM];   // bulk-copy destinations: 16-byte aligned
   alignas(16) float xs[2][BM];
+  float xf[2][BM];
 };
 
 template <int NKC>
@@ -295,16 +304,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_lse_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                   int nc, int ncmax, int Kt, const float* __restrict__ ck,
                   const float* __restrict__ kscale, int params_in_smem, float* __restrict__ logz,
-                  float* __restrict__ logz_out, double* __restrict__ ll_tiles, const int* mode,
-                  int* status) {
+                  float* __restrict__ logz_out, double* __restrict__ ll_tiles,
+                  const __half* __restrict__ xop, const float* __restrict__ ckf,
+                  const float* __restrict__ lzlow, uint8_t* __restrict__ side_flag,
+                  const int* mode, int* status) {
   if (mode && *mode != kModeTensor) return;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  unsigned char* xbuf = base;                         // [2][NKC][BOX]
-  unsigned char* wring = base + 2 * NKC * BOX;        // [SW][BOX]
+  unsigned char* xbuf = base;                         // [NKC][BOX]: phi hi of the tile
+  unsigned char* wring = base + NKC * BOX;            // [SW][BOX]
   LseBars* bars = reinterpret_cast<LseBars*>(wring + SW * BOX);
   float* ckl = reinterpret_cast<float*>(bars + 1);    // [Kt] c_k log2(e)   (if staged)
   float* ksl = ckl + Kt;                              // [Kt] 2^t_k log2(e) (if staged)
+  float* cfl = ksl + Kt;                              // [Kt] (c_k + E_k) log2(e) (if staged)
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -317,6 +329,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&bars->s_full[b], 1);
       ptx::mbar_init(&bars->s_empty[b], kEpiWarps);
+      ptx::mbar_init(&bars->xlo_ready[b], kEpiWarps);
       ptx::mbar_init(&bars->xc_full[b], kEpiWarps / 2);
       ptx::mbar_init(&bars->xc_empty[b], kEpiWarps / 2);
     }
@@ -328,15 +341,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int k = threadIdx.x; k < Kt; k += blockDim.x) {
       ckl[k] = ck[k] * kLog2e;
       ksl[k] = kscale[k] * kLog2e;
+      cfl[k] = ckf[k] * kLog2e;
     }
   if (warp == 1) {
-    ptx::tmem_alloc(&bars->tmem, 256);
+    ptx::tmem_alloc(&bars->tmem, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  // TMEM columns: [0, 256) S double-buffered, [256 + 128 b, ...) phi lo of tile buffer b
+  // (two fp16 per column, 2 Dq / 2 = NKC * 32 columns)
   const uint32_t tmem = bars->tmem;
+  const uint32_t xlo_tmem = tmem + 256;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -349,9 +366,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         x_issued = j + 1;
         for (int c = 0; c < NKC; ++c) {
           if (j > 0 && !ptx::mbar_wait(&bars->x_empty[c], (j - 1) & 1, abort)) goto fail_p;
-          ptx::mbar_arrive_expect_tx(&bars->x_full[c], 2 * BOX);
+          ptx::mbar_arrive_expect_tx(&bars->x_full[c], BOX);
           ptx::tma_load_2d(xbuf + c * BOX, &tmx, &bars->x_full[c], c * KC, row0);
-          ptx::tma_load_2d(xbuf + (NKC + c) * BOX, &tmx, &bars->x_full[c], c * KC, ncmax + row0);
         }
         for (int kb = 0; kb < nkb; ++kb)
           for (int c = 0; c < NKC; ++c)
@@ -386,6 +402,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (its >= 2 && !ptx::mbar_wait(&bars->s_empty[b], ((its >> 1) - 1) & 1, abort)) goto fail_m;
           ptx::tc_fence_after();
           const uint32_t d_tmem = tmem + b * 128;
+          if (kb == 0 && !ptx::mbar_wait(&bars->xlo_ready[j & 1], (j >> 1) & 1, abort)) goto fail_m;
+          const uint32_t xl_tmem = xlo_tmem + (j & 1) * 128;
           for (int c = 0; c < NKC; ++c) {
             if (kb == 0 && !ptx::mbar_wait(&bars->x_full[c], j & 1, abort)) goto fail_m;
             const int sh = itw % SW;
@@ -396,19 +414,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ++itw;
             ptx::tc_fence_after();
             const uint32_t xa_hi = ptx::smem_u32(xbuf + c * BOX);
-            const uint32_t xa_lo = ptx::smem_u32(xbuf + (NKC + c) * BOX);
             const uint32_t wb_hi = ptx::smem_u32(wring + sh * BOX);
             const uint32_t wb_lo = ptx::smem_u32(wring + sl * BOX);
 #pragma unroll
             for (int ks = 0; ks < KC / 16; ++ks) {
               const uint32_t o = ks * 32;
               const uint64_t ah = ptx::smem_desc_sw128(xa_hi + o, 16, 1024);
-              const uint64_t al = ptx::smem_desc_sw128(xa_lo + o, 16, 1024);
               const uint64_t bh = ptx::smem_desc_sw128(wb_hi + o, 16, 1024);
               const uint64_t bl = ptx::smem_desc_sw128(wb_lo + o, 16, 1024);
               ptx::mma_f16_ss(d_tmem, ah, bh, idesc, (c > 0 || ks > 0) ? 1u : 0u);
               ptx::mma_f16_ss(d_tmem, ah, bl, idesc, 1u);
-              ptx::mma_f16_ss(d_tmem, al, bh, idesc, 1u);
+              // phi lo from TMEM: K elements c*64 + ks*16 .. +15 = columns c*32 + ks*8 .. +7
+              ptx::mma_f16_ts(d_tmem, xl_tmem + c * 32 + ks * 8, bh, idesc, 1u);
             }
             ptx::mma_commit(&bars->w_empty[sh]);
             ptx::mma_commit(&bars->w_empty[sl]);
@@ -432,10 +449,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q = warp & 3;                // TMEM lane quarter
     const int r = q * 32 + lane;           // row of the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    // phi lo of tile t into TMEM buffer b: this thread's row, K elements
+    // g*NKC*32 .. +NKC*32-1 = columns g*NKC*16 .. +NKC*16-1 (row t*BM + r < ncmax)
+    auto put_xlo = [&](int t, int b) {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          xop + ((size_t)ncmax + (size_t)t * BM + r) * (NKC * 64) + g * (NKC * 32));
+#pragma unroll
+      for (int c8 = 0; c8 < NKC * 2; ++c8) {   // 8 columns = 16 fp16 per store
+        const uint4 v0 = __ldg(src + 2 * c8), v1 = __ldg(src + 2 * c8 + 1);
+        const uint32_t r8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        ptx::tmem_st8(xlo_tmem + b * 128 + lane_base + g * (NKC * 16) + c8 * 8, r8);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bars->xlo_ready[b]);
+    };
+    if (blockIdx.x < ntiles) put_xlo(blockIdx.x, 0);
     uint32_t its = 0;
     int jt = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++jt) {
+      // the next tile's phi lo goes into the buffer of tile jt - 1, whose MMAs have all
+      // completed: this thread has consumed every S block they produced
+      if (t + (int)gridDim.x < ntiles) put_xlo(t + gridDim.x, (jt + 1) & 1);
       float m = -CUDART_INF_F, s = 0.f;   // in log2 units
+      float fm = -CUDART_INF_F;            // max over stiff components of estimate + E_k
       for (int kb = 0; kb < nkb; ++kb, ++its) {
         const int b = its & 1;
         if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full[b], (its >> 1) & 1, abort))) {
@@ -455,20 +493,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int k0 = kb * BKc + col;
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
-            float4 cc, kk;
+            float4 cc, kk, cf;
             if (params_in_smem) {
               cc = *reinterpret_cast<const float4*>(ckl + k0 + 4 * e4);
               kk = *reinterpret_cast<const float4*>(ksl + k0 + 4 * e4);
+              cf = *reinterpret_cast<const float4*>(cfl + k0 + 4 * e4);
             } else {
               cc = __ldg(reinterpret_cast<const float4*>(ck + k0) + e4);
               kk = __ldg(reinterpret_cast<const float4*>(kscale + k0) + e4);
+              cf = __ldg(reinterpret_cast<const float4*>(ckf + k0) + e4);
               cc.x *= kLog2e; cc.y *= kLog2e; cc.z *= kLog2e; cc.w *= kLog2e;
               kk.x *= kLog2e; kk.y *= kLog2e; kk.z *= kLog2e; kk.w *= kLog2e;
+              cf.x *= kLog2e; cf.y *= kLog2e; cf.z *= kLog2e; cf.w *= kLog2e;
             }
-            v[4 * e4 + 0] = fmaf(__uint_as_float(u[4 * e4 + 0]), kk.x, cc.x);
-            v[4 * e4 + 1] = fmaf(__uint_as_float(u[4 * e4 + 1]), kk.y, cc.y);
-            v[4 * e4 + 2] = fmaf(__uint_as_float(u[4 * e4 + 2]), kk.z, cc.z);
-            v[4 * e4 + 3] = fmaf(__uint_as_float(u[4 * e4 + 3]), kk.w, cc.w);
+            const float uu[4] = {__uint_as_float(u[4 * e4 + 0]), __uint_as_float(u[4 * e4 + 1]),
+                                 __uint_as_float(u[4 * e4 + 2]), __uint_as_float(u[4 * e4 + 3])};
+            v[4 * e4 + 0] = fmaf(uu[0], kk.x, cc.x);
+            v[4 * e4 + 1] = fmaf(uu[1], kk.y, cc.y);
+            v[4 * e4 + 2] = fmaf(uu[2], kk.z, cc.z);
+            v[4 * e4 + 3] = fmaf(uu[3], kk.w, cc.w);
+            // stiff components (c_k = -inf above): estimate + error bound, for the filter
+            fm = fmaxf(fm, fmaxf(fmaxf(fmaf(uu[0], kk.x, cf.x), fmaf(uu[1], kk.y, cf.y)),
+                                 fmaxf(fmaf(uu[2], kk.z, cf.z), fmaf(uu[3], kk.w, cf.w))));
 #pragma unroll
             for (int z = 0; z < 4; ++z) bm = fmaxf(bm, v[4 * e4 + z]);
           }
@@ -497,6 +543,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         bars->xm[xb][r] = m;
         bars->xs[xb][r] = s;
+        bars->xf[xb][r] = fm;
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&bars->xc_full[xb]);
       } else {
@@ -506,18 +553,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         const float m2 = bars->xm[xb][r], s2 = bars->xs[xb][r];
+        const float f2 = fmaxf(fm, bars->xf[xb][r]);
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&bars->xc_empty[xb]);
         const float M = fmaxf(m, m2);
         float S = 0.f;
         if (M > -CUDART_INF_F) S = s * exp2f(m - M) + s2 * exp2f(m2 - M);
         const int i = t * BM + r;
-        const float lz = (M + log2f(S)) / kLog2e;
+        const float lz2 = M + log2f(S);
+        const float lz = lz2 / kLog2e;
         double part = 0.0;
         if (i < nc) {
           logz[i] = lz;
           if (logz_out) logz_out[i] = lz;
           part = lz;
+          // may a stiff component come within kSideCut nats of log Z here?
+          side_flag[i] = (f2 > lz2 - kSideCut * kLog2e) || !(lz >= *lzlow);
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
@@ -529,7 +580,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, 256);
+    ptx::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -768,7 +819,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const float ckl = ck[k] * kLog2e + 15.f;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const size_t row = (size_t)(1 + 2 * Dp);
-    double* slot = stats + ((size_t)blockIdx.y * kstride + k) * row;
+    // this CTA's slot, [row][kstride] layout: statistic c of component k at c * kstride + k
+    double* slot = stats + stat_idx(true, blockIdx.y, k, 0, kstride, row);
     float nk = 0.f;
     int tiles_since_flush = 0, flushes = 0;
     // R^T row kl, points 64g .. 64g+63 = box g: 8-row atoms of 1024 B, 128 B per row,
@@ -854,14 +906,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           goto fail_e;
         ptx::tc_fence_after();
         const double inv = 1.0 / (double)kRScale;
-        double* dst = slot + 1 + (g == 0 ? 0 : Dp);   // g 0: linear moments, g 1: squares
+        // g 0: linear moments, g 1: squares; the warp's 32 lanes (components) add into
+        // 32 consecutive doubles per statistic
+        double* dst = slot + (size_t)(1 + (g == 0 ? 0 : Dp)) * kstride;
 #pragma unroll 1
         for (int h = 0; h < NKC; ++h) {
           uint32_t u[32];
           ptx::tmem_ld32(acc_tmem + lane_base + g * Dq + h * 32, u);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) atomicAdd(dst + h * 32 + e, (double)__uint_as_float(u[e]) * inv);
+          for (int e = 0; e < 32; ++e)
+            atomicAdd(dst + (size_t)(h * 32 + e) * kstride, (double)__uint_as_float(u[e]) * inv);
         }
         // N_k: the upper half hands its partial sum to the lower half
         if (g == 1) {
@@ -961,8 +1016,8 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows) {
 }
 
 size_t lse_smem(int nkc, int Kt, bool params) {
-  return 1024 + (size_t)(2 * nkc + SW) * BOX + sizeof(LseBars) +
-         (params ? 2 * (size_t)Kt * sizeof(float) : 0);
+  return 1024 + (size_t)(nkc + SW) * BOX + sizeof(LseBars) +
+         (params ? 3 * (size_t)Kt * sizeof(float) : 0);
 }
 constexpr size_t kMaxDynSmem = 232448;  // 227 KB per block on sm_100
 size_t stats_smem(int nkc) { return 1024 + (size_t)(nkc + SX + 2) * BOX + sizeof(StatBars); }
@@ -1003,19 +1058,20 @@ cudaError_t tc_init(Ctx& c) {
 cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* means,
                            const float* vars, bool auto_mode, cudaStream_t s) {
   const Workspace& w = c.ws;
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_TC_CENTER, s);
   tc_center_kernel<<<c.D, kSimtThreads, 0, s>>>(c.K, c.D, c.cov, weights, means, vars, w.center,
                                                 w.dscale);
-  prof_end(c, KK_OTHER, s);
+  prof_end(c, KI_TC_CENTER, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (w.Dq > c.D) cudaMemsetAsync(w.center + c.D, 0, (w.Dq - c.D) * sizeof(float), s);
   if (!auto_mode) cudaMemsetAsync(w.stiff, 0, w.Kt * sizeof(int), s);
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_TC_PREP, s);
   tc_prep_kernel<<<w.Kt, kSimtThreads, 0, s>>>(c.K, c.D, w.Dq, w.Kt, c.cov, weights, means, vars,
                                                w.center, w.dscale, w.nk, w.wop, w.tck, w.tks,
-                                               auto_mode ? w.stiff : nullptr, w.status);
-  prof_end(c, KK_OTHER, s);
+                                               auto_mode ? w.stiff : nullptr, w.tcraw, w.tcm,
+                                               w.tcpk, w.status);
+  prof_end(c, KI_TC_PREP, s);
   return cudaGetLastError();
 }
 
@@ -1024,14 +1080,14 @@ cudaError_t launch_tc_convert(const Ctx& c, const void* X, int x_dtype, int64_t 
   const Workspace& w = c.ws;
   const int64_t total = n * (w.Dq / 8);
   const unsigned grid = (unsigned)ceil_div64(total, 256);
-  prof_begin(c, KK_OTHER, s);
+  prof_begin(c, KI_TC_CONVERT, s, mode, kModeTensor);
   if (x_dtype == FGMM_BF16)
     tc_convert_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dq, kChunk,
                                            w.center, w.dscale, w.xop, mode);
   else
     tc_convert_kernel<<<grid, 256, 0, s>>>((const float*)X, n, ldx, c.D, w.Dq, kChunk, w.center,
                                            w.dscale, w.xop, mode);
-  prof_end(c, KK_OTHER, s);
+  prof_end(c, KI_TC_CONVERT, s);
   return cudaGetLastError();
 }
 
@@ -1045,12 +1101,13 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
   const CUtensorMap& tw = c.tc.tmap_w;
   const bool params = lse_smem(nkc, w.Kt, true) <= kMaxDynSmem;
   const size_t smem = lse_smem(nkc, w.Kt, params);
-  prof_begin(c, KK_SWEEP1, s);
+  prof_begin(c, KI_TC_LSE, s, mode, kModeTensor);
 #define LSE_CASE(N_)                                                                          \
   case N_:                                                                                    \
     tc_lse_kernel<N_><<<grid, kTcThreads, smem, s>>>(tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, \
                                                      w.tks, params ? 1 : 0, w.logz, logz_out,   \
-                                                     w.ll_tiles, mode, w.status);             \
+                                                     w.ll_tiles, w.xop, w.tckf, w.lzlow,       \
+                                                     w.side_flag, mode, w.status);            \
     break;
   switch (nkc) {
     LSE_CASE(1)
@@ -1059,7 +1116,7 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
     LSE_CASE(4)
   }
 #undef LSE_CASE
-  prof_end(c, KK_SWEEP1, s);
+  prof_end(c, KI_TC_LSE, s);
   return cudaGetLastError();
 }
 
@@ -1080,7 +1137,7 @@ cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream
   const CUtensorMap& tx = c.tc.tmap_x;
   const CUtensorMap& tw = c.tc.tmap_w;
   const int flush_tiles = 8;  // fp32 runs of 1024 points (64 MMA steps) between fp64 flushes
-  prof_begin(c, KK_SWEEP2, s);
+  prof_begin(c, KI_TC_STATS, s, mode, kModeTensor);
 #define STATS_CASE(N_)                                                                         \
   case N_:                                                                                     \
     tc_stats_kernel<N_><<<grid, kTcThreads, stats_smem(N_), s>>>(tx, tw, (int)n, (int)kChunk, \
@@ -1096,7 +1153,7 @@ cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream
     STATS_CASE(4)
   }
 #undef STATS_CASE
-  prof_end(c, KK_SWEEP2, s);
+  prof_end(c, KI_TC_STATS, s);
   return cudaGetLastError();
 }
 

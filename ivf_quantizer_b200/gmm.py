@@ -123,6 +123,51 @@ class GMM:
                                _ptr(variances), _ptr(loglik), _ptr(logz), _stream()),
               "fgmm_em_step")
 
+    # ---------------------------------------------------------------- sharded EM
+    @property
+    def stats_len(self) -> int:
+        """Length of the statistics vector exchanged between shards: K (1 + 2D) + 1."""
+        return self.K * (1 + 2 * self.D) + 1
+
+    def partial(self, X, weights, means, variances, stats=None, logz=None):
+        """E-step and statistics of one EM iteration on this shard of the rows.
+
+        Returns the statistics vector (CUDA float64 [stats_len]: per component N_k,
+        Σ r (x − μ_k), Σ r (x − μ_k)², then Σ log Z); the parameters are not changed.
+        Vectors of disjoint shards add up to the vector of their union.
+        """
+        self._check_params(weights, means, variances)
+        xp, dt, n, ldx = _x_args(X)
+        if stats is None:
+            stats = torch.empty(self.stats_len, dtype=torch.float64, device=X.device)
+        elif not (stats.is_cuda and stats.dtype == torch.float64 and stats.is_contiguous()
+                  and stats.numel() == self.stats_len):
+            raise ValueError("stats must be a contiguous CUDA float64 tensor of stats_len")
+        if logz is not None and not (logz.is_cuda and logz.dtype == torch.float32
+                                     and logz.numel() >= n):
+            raise ValueError("logz must be a CUDA float32 tensor with N elements")
+        check(LIB.fgmm_em_partial(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means),
+                                  _ptr(variances), _ptr(stats), _ptr(logz), _stream()),
+              "fgmm_em_partial")
+        return stats
+
+    def finish(self, stats, weights, means, variances, loglik=None):
+        """M-step from a statistics vector summed over every shard; updates the
+        parameters (those the statistics were taken about) in place."""
+        self._check_params(weights, means, variances)
+        if not (stats.is_cuda and stats.dtype == torch.float64 and stats.is_contiguous()
+                and stats.numel() == self.stats_len):
+            raise ValueError("stats must be a contiguous CUDA float64 tensor of stats_len")
+        if loglik is not None and not (loglik.is_cuda and loglik.dtype == torch.float64):
+            raise ValueError("loglik must be a CUDA float64 tensor")
+        check(LIB.fgmm_em_finish(self._h, _ptr(stats), _ptr(weights), _ptr(means),
+                                 _ptr(variances), _ptr(loglik), _stream()), "fgmm_em_finish")
+
+    def combine(self, parts):
+        """Sum of gathered statistics vectors ([n, stats_len]) in row order."""
+        return stats_sum(parts)
+
+
     def fit(self, X, weights, means, variances, max_iters=100, tol=0.0):
         """Repeat step up to max_iters times; returns (final_loglik, iters_done)."""
         self._check_params(weights, means, variances)
@@ -152,9 +197,18 @@ class GMM:
         check(LIB.fgmm_profile_enable(self._h, int(enable)), "fgmm_profile_enable")
 
     def profile_read(self, reset: bool = True) -> dict:
+        """Event timings since the last reset: totals per kernel kind, and under
+        ``"kernels"`` per kernel name {launches, ms, active, active_ms}, where the
+        active launches are those that passed their path gate and did work."""
         p = _lib.Profile()
         check(LIB.fgmm_profile_read(self._h, ctypes.byref(p), int(reset)), "fgmm_profile_read")
-        return {f: getattr(p, f) for f, _ in _lib.Profile._fields_}
+        out = {f: getattr(p, f) for f, _ in _lib.Profile._fields_ if not f.startswith("kernel_")}
+        out["kernels"] = {
+            LIB.fgmm_profile_kernel_name(i).decode(): {
+                "launches": p.kernel_launches[i], "ms": p.kernel_ms[i],
+                "active": p.kernel_active[i], "active_ms": p.kernel_active_ms[i]}
+            for i in range(_lib.PROF_KERNELS) if p.kernel_launches[i]}
+        return out
 
     def status(self) -> int:
         """Synchronise and return (then clear) the device status word."""
@@ -162,3 +216,16 @@ class GMM:
 
     def check_status(self):
         check(self.status(), "device status")
+
+
+def stats_sum(parts, out=None):
+    """Sum of statistics vectors stacked as rows of ``parts`` ([n, len] CUDA float64),
+    in row order (bit-reproducible whatever order they were gathered in)."""
+    if not (parts.is_cuda and parts.dtype == torch.float64 and parts.dim() == 2
+            and parts.is_contiguous()):
+        raise ValueError("parts must be a contiguous [n, len] CUDA float64 tensor")
+    n, length = parts.shape
+    if out is None:
+        out = torch.empty(length, dtype=torch.float64, device=parts.device)
+    check(LIB.fgmm_stats_sum(_ptr(parts), n, length, _ptr(out), _stream()), "fgmm_stats_sum")
+    return out

@@ -76,3 +76,19 @@ def test_package_has_no_fallback(monkeypatch, tmp_path):
     from ivf_quantizer_b200 import _lib
     with pytest.raises(ImportError):
         _lib.load(str(tmp_path / "missing.so"))
+
+
+def test_profile_layout_and_kernel_names():
+    """The ctypes mirror of fgmm_profile matches the header's array length, and every
+    per-kernel slot has a distinct name; indices outside the table give NULL."""
+    import re
+    from ivf_quantizer_b200 import _lib
+    hdr = open(os.path.join(ROOT, "include", "fgmm.h")).read()
+    assert int(re.search(r"#define FGMM_PROF_KERNELS (\d+)", hdr).group(1)) == _lib.PROF_KERNELS
+    assert re.search(r"#define FGMM_CHUNK_POINTS \(1 << (\d+)\)", hdr).group(1) == "20"
+    assert _lib.CHUNK_POINTS == 1 << 20
+    names = [_lib.LIB.fgmm_profile_kernel_name(i) for i in range(_lib.PROF_KERNELS)]
+    assert all(n for n in names) and len(set(names)) == len(names)
+    assert b"tc_lse" in names and b"tc_stats" in names and b"stats_simt" in names
+    assert _lib.LIB.fgmm_profile_kernel_name(-1) is None
+    assert _lib.LIB.fgmm_profile_kernel_name(_lib.PROF_KERNELS) is None
