@@ -65,11 +65,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ void set_status(int* st, int code) { atomicCAS(st, FGMM_OK, code); }
 
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
 // fp16 split of a float: hi = fp16(a) (saturating), lo = fp16(a - hi).
 __device__ __forceinline__ void split16(float a, __half& hi, __half& lo) {
   hi = __float2half_rn(fminf(fmaxf(a, -65504.f), 65504.f));
@@ -275,15 +270,18 @@ __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ld
 }
 
 // ------------------------------------------------------------------ sweep 1 (log Z)
-// 384 threads: warp 0 TMA producer, warp 1 MMA issuer, warps 4..11 epilogue.  The two
-// epilogue warpgroups split each 128-column S tile in halves (columns 64g .. 64g+63) and
-// keep a running (max, sum) per row; at the end of a tile the upper half hands its
-// pair to the lower half through shared memory, which writes log Z.
+// 640 threads: warp 0 TMA producer, warp 1 MMA issuer, warps 4..19 epilogue.  The four
+// epilogue warpgroups split each 128-column S tile in quarters (columns 32g .. 32g+31;
+// four warps per scheduler hide the TMEM-load and exp latencies) and keep a running
+// (max, sum) per row; at the end of a tile groups 1..3 hand their pairs to group 0
+// through shared memory, which writes log Z.
 // phi hi of the point tile sits in shared memory (A operand of two products); phi lo
 // sits in tensor memory (A operand of the third), written there by the epilogue warps
 // one tile ahead, so that shared memory holds an 8-stage ring of W' boxes.
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 8;                        // statistics sweep
 constexpr int kTcThreads = 128 + 32 * kEpiWarps;
+constexpr int kLseEpiWarps = 16;                    // log-sum-exp sweep
+constexpr int kLseThreads = 128 + 32 * kLseEpiWarps;
 
 struct LseBars {
   uint64_t x_full[4], x_empty[4];
@@ -294,17 +292,17 @@ struct LseBars {
   uint64_t drain;
   uint32_t tmem;
   int abort;
-  alignas(16) float xm[2][BM];   // bulk-copy destinations: 16-byte aligned
-  alignas(16) float xs[2][BM];
-  float xf[2][BM];
+  float xm[2][3][BM];   // (max, sum, filter max) of column groups 1..3, per tile buffer
+  float xs[2][3][BM];
+  float xf[2][3][BM];
 };
 
 template <int NKC>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kLseThreads, 1)
     tc_lse_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                   int nc, int ncmax, int Kt, const float* __restrict__ ck,
                   const float* __restrict__ kscale, int params_in_smem, float* __restrict__ logz,
-                  float* __restrict__ logz_out, double* __restrict__ ll_tiles,
+                  float* __restrict__ logz_out,
                   const __half* __restrict__ xop, const float* __restrict__ ckf,
                   const float* __restrict__ lzlow, uint8_t* __restrict__ side_flag,
                   const int* mode, int* status) {
@@ -328,10 +326,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int s = 0; s < SW; ++s) { ptx::mbar_init(&bars->w_full[s], 1); ptx::mbar_init(&bars->w_empty[s], 1); }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&bars->s_full[b], 1);
-      ptx::mbar_init(&bars->s_empty[b], kEpiWarps);
-      ptx::mbar_init(&bars->xlo_ready[b], kEpiWarps);
-      ptx::mbar_init(&bars->xc_full[b], kEpiWarps / 2);
-      ptx::mbar_init(&bars->xc_empty[b], kEpiWarps / 2);
+      ptx::mbar_init(&bars->s_empty[b], kLseEpiWarps);
+      ptx::mbar_init(&bars->xlo_ready[b], kLseEpiWarps);
+      ptx::mbar_init(&bars->xc_full[b], 3 * kLseEpiWarps / 4);
+      ptx::mbar_init(&bars->xc_empty[b], kLseEpiWarps / 4);
     }
     ptx::mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -445,7 +443,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   } else if (warp >= 4) {
-    const int g = (warp - 4) >> 2;         // column half of the S tile
+    const int g = (warp - 4) >> 2;         // column quarter of the S tile
     const int q = warp & 3;                // TMEM lane quarter
     const int r = q * 32 + lane;           // row of the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
@@ -453,12 +451,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // g*NKC*32 .. +NKC*32-1 = columns g*NKC*16 .. +NKC*16-1 (row t*BM + r < ncmax)
     auto put_xlo = [&](int t, int b) {
       const uint4* src = reinterpret_cast<const uint4*>(
-          xop + ((size_t)ncmax + (size_t)t * BM + r) * (NKC * 64) + g * (NKC * 32));
+          xop + ((size_t)ncmax + (size_t)t * BM + r) * (NKC * 64) + g * (NKC * 16));
 #pragma unroll
-      for (int c8 = 0; c8 < NKC * 2; ++c8) {   // 8 columns = 16 fp16 per store
+      for (int c8 = 0; c8 < NKC; ++c8) {   // 8 columns = 16 fp16 per store
         const uint4 v0 = __ldg(src + 2 * c8), v1 = __ldg(src + 2 * c8 + 1);
         const uint32_t r8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        ptx::tmem_st8(xlo_tmem + b * 128 + lane_base + g * (NKC * 16) + c8 * 8, r8);
+        ptx::tmem_st8(xlo_tmem + b * 128 + lane_base + g * (NKC * 8) + c8 * 8, r8);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -482,9 +480,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         ptx::tc_fence_after();
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          const int col = 64 * g + 32 * h;   // column within the 128-component block
+        {
+          const int col = 32 * g;            // column within the 128-component block
           uint32_t u[32];
           ptx::tmem_ld32(tmem + lane_base + b * 128 + col, u);
           ptx::tmem_wait_ld();
@@ -532,18 +529,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) ptx::mbar_arrive(&bars->s_empty[b]);
       }
       if (*abort) break;
-      // combine the two column halves of each row
+      // combine the four column quarters of each row
       const int xb = jt & 1, use = jt >> 1;
-      if (g == 1) {
+      if (g >= 1) {
         if (use >= 1 &&
             !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->xc_empty[xb], (use - 1) & 1, abort))) {
           set_status(status, FGMM_ERR_TIMEOUT);
           bars->abort = 1;
           break;
         }
-        bars->xm[xb][r] = m;
-        bars->xs[xb][r] = s;
-        bars->xf[xb][r] = fm;
+        bars->xm[xb][g - 1][r] = m;
+        bars->xs[xb][g - 1][r] = s;
+        bars->xf[xb][g - 1][r] = fm;
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&bars->xc_full[xb]);
       } else {
@@ -552,27 +549,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           bars->abort = 1;
           break;
         }
-        const float m2 = bars->xm[xb][r], s2 = bars->xs[xb][r];
-        const float f2 = fmaxf(fm, bars->xf[xb][r]);
+        float mq[4] = {m, 0.f, 0.f, 0.f}, sq[4] = {s, 0.f, 0.f, 0.f};
+        float f2 = fm;
+#pragma unroll
+        for (int o = 0; o < 3; ++o) {
+          mq[o + 1] = bars->xm[xb][o][r];
+          sq[o + 1] = bars->xs[xb][o][r];
+          f2 = fmaxf(f2, bars->xf[xb][o][r]);
+        }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&bars->xc_empty[xb]);
-        const float M = fmaxf(m, m2);
+        const float M = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
         float S = 0.f;
-        if (M > -CUDART_INF_F) S = s * exp2f(m - M) + s2 * exp2f(m2 - M);
+        if (M > -CUDART_INF_F)
+#pragma unroll
+          for (int o = 0; o < 4; ++o) S += sq[o] * exp2f(mq[o] - M);
         const int i = t * BM + r;
         const float lz2 = M + log2f(S);
         const float lz = lz2 / kLog2e;
-        double part = 0.0;
         if (i < nc) {
           logz[i] = lz;
           if (logz_out) logz_out[i] = lz;
-          part = lz;
           // may a stiff component come within kSideCut nats of log Z here?
           side_flag[i] = (f2 > lz2 - kSideCut * kLog2e) || !(lz >= *lzlow);
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-        if (lane == 0) ll_tiles[(size_t)t * 4 + q] = part;
       }
     }
   }
@@ -1104,9 +1104,9 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
   prof_begin(c, KI_TC_LSE, s, mode, kModeTensor);
 #define LSE_CASE(N_)                                                                          \
   case N_:                                                                                    \
-    tc_lse_kernel<N_><<<grid, kTcThreads, smem, s>>>(tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, \
+    tc_lse_kernel<N_><<<grid, kLseThreads, smem, s>>>(tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, \
                                                      w.tks, params ? 1 : 0, w.logz, logz_out,   \
-                                                     w.ll_tiles, w.xop, w.tckf, w.lzlow,       \
+                                                     w.xop, w.tckf, w.lzlow,                  \
                                                      w.side_flag, mode, w.status);            \
     break;
   switch (nkc) {
