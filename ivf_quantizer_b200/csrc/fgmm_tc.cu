@@ -719,7 +719,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc1 = ptx::idesc_f16(128, 128, false, false);  // S^T = W phi^T
-      constexpr uint32_t idesc2 = ptx::idesc_f16(128, 64, false, true);    // acc += R^T phi
       uint32_t itx = 0;
       int tiles_since_flush = 0;
       bool fresh = true;   // next G2 starts a new accumulation period
@@ -765,29 +764,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             goto fail_m;
           ptx::tc_fence_after();
           const uint32_t r0 = ptx::smem_u32(rbuf);
-          for (int c = 0; c < NKC; ++c) {
-            const int sh = itx % SX;
-            if (!ptx::mbar_wait(&bars->x_full[sh], (itx / SX) & 1, abort)) goto fail_m;
-            ++itx;
-            const int sl = itx % SX;
-            if (!ptx::mbar_wait(&bars->x_full[sl], (itx / SX) & 1, abort)) goto fail_m;
-            ++itx;
+          // A phase's phi boxes sit in ring slots hi(0), lo(0), hi(1), lo(1), ...; when a
+          // phase starts at a multiple of its size the hi boxes of chunks c and c + 1 are
+          // two slots apart without wrapping, and one MMA with N = 128 features (leading
+          // byte offset 2 BOX between the two 64-feature atoms) covers both chunks.
+          constexpr int CP = (NKC % 2 == 0 && SX % (2 * NKC) == 0) ? 2 : 1;
+          constexpr uint32_t idesc2 = ptx::idesc_f16(128, 64 * CP, false, true);
+          for (int c = 0; c < NKC; c += CP) {
+            const uint32_t it0 = itx;
+            for (int i = 0; i < 2 * CP; ++i, ++itx)
+              if (!ptx::mbar_wait(&bars->x_full[itx % SX], (itx / SX) & 1, abort)) goto fail_m;
             ptx::tc_fence_after();
-            const uint32_t xb_hi = ptx::smem_u32(xring + sh * BOX);
-            const uint32_t xb_lo = ptx::smem_u32(xring + sl * BOX);
+            const uint32_t xb_hi = ptx::smem_u32(xring + (it0 % SX) * BOX);
+            const uint32_t xb_lo = ptx::smem_u32(xring + ((it0 + 1) % SX) * BOX);
             const uint32_t d_tmem = acc_tmem + c * 64;
 #pragma unroll
             for (int ks = 0; ks < BM / 16; ++ks) {
               // A = R^T (K-major, K = points): box ks/4, 32 B per 16 points inside it
               const uint64_t a = ptx::smem_desc_sw128(r0 + (ks >> 2) * BOX + (ks & 3) * 32, 16, 1024);
               // B = phi (MN-major, K = points = rows): 16 rows = 2 atoms of 1024 B
-              const uint64_t bh = ptx::smem_desc_sw128(xb_hi + ks * 2048, BOX, 1024);
-              const uint64_t bl = ptx::smem_desc_sw128(xb_lo + ks * 2048, BOX, 1024);
+              const uint64_t bh = ptx::smem_desc_sw128(xb_hi + ks * 2048, 2 * BOX, 1024);
+              const uint64_t bl = ptx::smem_desc_sw128(xb_lo + ks * 2048, 2 * BOX, 1024);
               ptx::mma_f16_ss(d_tmem, a, bh, idesc2, (fresh && ks == 0) ? 0u : 1u);
               ptx::mma_f16_ss(d_tmem, a, bl, idesc2, 1u);
             }
-            ptx::mma_commit(&bars->x_empty[sh]);
-            ptx::mma_commit(&bars->x_empty[sl]);
+            for (uint32_t i = it0; i < itx; ++i) ptx::mma_commit(&bars->x_empty[i % SX]);
           }
           ptx::mma_commit(&bars->r_empty);
           fresh = false;
