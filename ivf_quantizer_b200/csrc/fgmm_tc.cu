@@ -764,11 +764,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             goto fail_m;
           ptx::tc_fence_after();
           const uint32_t r0 = ptx::smem_u32(rbuf);
-          // A phase's phi boxes sit in ring slots hi(0), lo(0), hi(1), lo(1), ...; when a
-          // phase starts at a multiple of its size the hi boxes of chunks c and c + 1 are
-          // two slots apart without wrapping, and one MMA with N = 128 features (leading
-          // byte offset 2 BOX between the two 64-feature atoms) covers both chunks.
-          constexpr int CP = (NKC % 2 == 0 && SX % (2 * NKC) == 0) ? 2 : 1;
+          // A phase's phi boxes sit in ring slots hi(0), lo(0), hi(1), lo(1), ...; when the
+          // ring holds a whole number of phases, every phase starts at a multiple of its
+          // size, its hi boxes are two slots apart without wrapping, and one MMA with
+          // N = 64 NKC features (leading byte offset 2 BOX between the 64-feature atoms)
+          // covers all chunks.
+          constexpr int CP = (SX % (2 * NKC) == 0) ? NKC : 1;
           constexpr uint32_t idesc2 = ptx::idesc_f16(128, 64 * CP, false, true);
           for (int c = 0; c < NKC; c += CP) {
             const uint32_t it0 = itx;
