@@ -119,6 +119,21 @@ int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t l
                  float* weights, float* means, float* vars,
                  double* loglik_out, float* logz_out, fgmm_stream_t stream);
 
+/* fgmm_em_step with X in host memory: rows are copied to the device one chunk
+ * (FGMM_CHUNK_POINTS points) at a time into two device staging buffers, the copy of
+ * the next chunk overlapping the sweeps of the current one on an internal copy stream,
+ * so N is not limited by device memory (the paper's path to N beyond HBM, §6).  X_host
+ * should be pinned (page-locked) for the copies to overlap; pageable memory works but
+ * serialises them.  The staging buffers (2 x FGMM_CHUNK_POINTS x D x 4 bytes) are
+ * allocated by the first call and kept by the handle.  Under FGMM_PREC_AUTO the
+ * device's path decision is read back (one synchronisation per decision) so that only
+ * the passes that run copy X.  Other arguments as fgmm_em_step (weights, means, vars,
+ * loglik_out and logz_out are device memory).  The call returns when the last copy has
+ * been enqueued; X_host must stay valid until the stream reaches the step's end. */
+int fgmm_em_step_host(fgmm_handle h, const void* X_host, int x_dtype, int64_t N, int64_t ldx,
+                      float* weights, float* means, float* vars, double* loglik_out,
+                      float* logz_out, fgmm_stream_t stream);
+
 /* Data-parallel EM over row shards of X (one exchange per iteration).  Each entry
  * of the M-step's input is a sum over rows (§2, Eqs. (1)-(3)), so an iteration over
  * shards held by several handles, devices or processes is: fgmm_em_partial on every
@@ -141,6 +156,12 @@ int fgmm_em_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t l
 int fgmm_em_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
                     const float* weights, const float* means, const float* vars,
                     double* stats_out, float* logz_out, fgmm_stream_t stream);
+
+/* fgmm_em_partial with X in host memory, streamed as in fgmm_em_step_host. */
+int fgmm_em_partial_host(fgmm_handle h, const void* X_host, int x_dtype, int64_t N,
+                         int64_t ldx, const float* weights, const float* means,
+                         const float* vars, double* stats_out, float* logz_out,
+                         fgmm_stream_t stream);
 
 /* M-step (Eqs. (1)-(3), the variance floor and the empty-component rule) from a
  * statistics vector summed over every shard.  weights, means, vars: in/out, the
@@ -214,6 +235,39 @@ int fgmm_soft_assign_static(int K, int D, int cov_type, const void* X, int x_dty
                             const float* vars, int top_m, float r_threshold, int32_t* ids,
                             float* resp, fgmm_stream_t stream);
 
+/* k-means warm start ("Flash-GMM", §4.4: k-means, then soft EM from its centroids;
+ * the initialisation appendix: k-means++ seeding).  Both use the handle's K and D (and
+ * its workspace; they may not run concurrently with another call on the same handle).
+ * Decisions that floating point turns into indices are taken in a fixed precision so
+ * that they are reproducible: squared distances are fp32, summed over dimensions in
+ * increasing order with every subtraction, product and sum rounded separately (no
+ * fused multiply-add); ties go to the lower centroid index.  Results are bitwise
+ * reproducible run to run.
+ *
+ * fgmm_kmeans_step: one Lloyd iteration on device X.  centroids: device float [K][D],
+ * in/out (an empty cluster keeps its centroid).  assign_out: optional device int32[N],
+ * the argmin per point for the INPUT centroids.  counts_out: optional device int64[K].
+ * inertia_out: optional device double, sum of the points' squared distances to their
+ * assigned input centroid (fp64 sum of the fp32 distances).  Cluster sums are exact
+ * 64-bit fixed-point sums (scale from the data's largest |x| and N).  Asynchronous. */
+int fgmm_kmeans_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                     float* centroids, int32_t* assign_out, int64_t* counts_out,
+                     double* inertia_out, fgmm_stream_t stream);
+
+/* k-means++ seeding on device X (N >= 1).  first: index of the first centre (0 <= first
+ * < N).  u: device double[K-1], the uniforms in [0, 1) of draws 1 .. K-1 (the caller
+ * draws them; the method's randomness is an input).  Draw t weighs point i by
+ * w_i = floor(D_i * 2^s), D_i its fp32 squared distance to the nearest chosen centre and
+ * 2^s the power of two bringing the largest D to [2^29, 2^30), and picks the smallest i
+ * whose running sum of w exceeds floor(u_t * sum w) (fp64 product); when every w is 0
+ * it repeats the previous centre.  centroids: device float [K][D] out; idx_out: device
+ * int64[K] out (required).  scratch: device memory of fgmm_kmeans_seed_scratch_bytes(N)
+ * bytes, caller-owned.  K sequential draws, each a pass over X.  Asynchronous. */
+int fgmm_kmeans_seed(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                     int64_t first, const double* u, float* centroids, int64_t* idx_out,
+                     void* scratch, fgmm_stream_t stream);
+size_t fgmm_kmeans_seed_scratch_bytes(int64_t N);
+
 /* Kernel timing, for benchmarks.  When enabled, the library records a CUDA
  * event pair on the call's stream around every kernel it launches and keeps a
  * launch counter; fgmm_profile_read synchronises the device, sums the elapsed
@@ -224,7 +278,7 @@ int fgmm_soft_assign_static(int K, int D, int cov_type, const void* X, int x_dty
  * memory), so that launches which did work are counted apart ("active").
  * Disabled by default; costs two event records per launch, and one 4-byte copy
  * per gated launch, when enabled. */
-#define FGMM_PROF_KERNELS 21
+#define FGMM_PROF_KERNELS 23
 typedef struct fgmm_profile {
   int64_t launches;          /* kernels launched while enabled (all kinds) */
   int64_t sweep1_launches;   /* log-sum-exp sweep (first pass over the components) */

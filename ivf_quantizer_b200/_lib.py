@@ -22,7 +22,7 @@ STATIC_MAX_K = 1 << 14
 EMPTY_NK = 1e-6
 CHUNK_POINTS = 1 << 20
 
-PROF_KERNELS = 21
+PROF_KERNELS = 23
 
 
 class Profile(ctypes.Structure):
@@ -62,6 +62,11 @@ SIGNATURES = {
     "fgmm_em_partial": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_em_finish": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_stats_sum": (_int, [_vp, _int, _i64, _vp, _vp]),
+    "fgmm_kmeans_step": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_kmeans_seed": (_int, [_vp, _vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_kmeans_seed_scratch_bytes": (_c.c_size_t, [_i64]),
+    "fgmm_em_step_host": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_em_partial_host": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
 
 

@@ -23,8 +23,30 @@
 
 using namespace fgmm;
 
+// Streaming of X from host memory (fgmm_em_step_host): two device staging buffers of
+// one chunk each, filled on a copy stream while the compute stream works on the other.
+struct HostStaging {
+  void* buf[2] = {nullptr, nullptr};
+  cudaStream_t cs = nullptr;
+  cudaEvent_t copied[2] = {nullptr, nullptr};
+  cudaEvent_t consumed[2] = {nullptr, nullptr};
+  uint64_t seq = 0;
+  void release() {
+    for (int b = 0; b < 2; ++b) {
+      if (buf[b]) cudaFree(buf[b]);
+      if (copied[b]) cudaEventDestroy(copied[b]);
+      if (consumed[b]) cudaEventDestroy(consumed[b]);
+      buf[b] = nullptr;
+      copied[b] = consumed[b] = nullptr;
+    }
+    if (cs) cudaStreamDestroy(cs);
+    cs = nullptr;
+  }
+};
+
 struct fgmm_ctx {
-  Ctx c;
+  fgmm::Ctx c;
+  HostStaging hs;
 };
 
 // Optional per-launch event timing (fgmm_profile_*).  Events are pooled and
@@ -83,7 +105,8 @@ const char* const kKernelNames[fgmm::KI_COUNT] = {
     "tc_center",   "tc_prep",   "tc_convert",  "tc_lse",         "tc_stats",
     "prep_simt",   "lse_simt",  "ll_accumulate", "stats_simt",   "reduce_stats", "mstep",
     "finalize",    "soft_assign", "auto_check", "redo_reset",    "remask",
-    "stiff_compact", "side_lse", "ll_partials", "side_stats",    "side_reduce"};
+    "stiff_compact", "side_lse", "ll_partials", "side_stats",    "side_reduce",
+    "km_assign",   "km_seed_update"};
 static_assert(fgmm::KI_COUNT == FGMM_PROF_KERNELS, "kernel table and public arrays differ");
 }  // namespace
 
@@ -132,7 +155,7 @@ void free_ws(Workspace& w) {
                   w.stats,  w.nk,     w.status, w.center, w.dscale, w.wop,
                   w.tck,    w.tks,    w.xop,    w.mode, w.stiff,    w.stiff_list, w.n_stiff,
                   w.side_part, w.mode2, w.canon, w.tcraw, w.tcm, w.tcpk, w.tckf, w.lzlow,
-                  w.side_flag};
+                  w.side_flag, w.km_word};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -173,6 +196,7 @@ cudaError_t alloc_ws(Ctx& c) {
   if ((e = alloc(&w.stats, stats_bytes(w) / sizeof(double), &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.nk, (size_t)w.KpS, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.status, (size_t)1, &t)) != cudaSuccess) return e;
+  if ((e = alloc(&w.km_word, (size_t)2, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.mode, (size_t)1, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.mode2, (size_t)1, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.center, (size_t)w.Dq, &t)) != cudaSuccess) return e;
@@ -270,6 +294,7 @@ int fgmm_destroy(fgmm_handle h) {
   int rc = set_device(h->c);
   cudaDeviceSynchronize();
   free_ws(h->c.ws);
+  h->hs.release();
   delete h->c.prof;
   delete h;
   return rc;
@@ -301,9 +326,31 @@ int fgmm_workspace_bytes(fgmm_handle h, size_t* bytes_out) {
 namespace {
 // Everything of one EM iteration up to the exchange-form statistics (written to `st`):
 // preparation, both sweeps over all chunks on the selected path(s), slot reduction.
+// Device staging for host-resident X: buffers, copy stream and events, made on first use.
+cudaError_t ensure_staging(fgmm_ctx* h) {
+  HostStaging& hs = h->hs;
+  if (hs.cs) return cudaSuccess;
+  const size_t bytes = (size_t)kChunk * h->c.D * sizeof(float);
+  cudaError_t e;
+  for (int b = 0; b < 2; ++b) {
+    if ((e = cudaMalloc(&hs.buf[b], bytes)) != cudaSuccess) break;
+    if ((e = cudaEventCreateWithFlags(&hs.copied[b], cudaEventDisableTiming)) != cudaSuccess) break;
+    if ((e = cudaEventCreateWithFlags(&hs.consumed[b], cudaEventDisableTiming)) != cudaSuccess) break;
+  }
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hs.cs, cudaStreamNonBlocking);
+  if (e != cudaSuccess) hs.release();
+  return e;
+}
+
+int read_word(const int* dev, int* out, cudaStream_t s) {
+  cudaError_t e = cudaMemcpyAsync(out, dev, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return map_cuda(e);
+}
+
 int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
                 const float* weights, const float* means, const float* vars, double* st,
-                float* logz_out, fgmm_stream_t stream) {
+                float* logz_out, fgmm_stream_t stream, bool host_x = false) {
   int rc = check_x(h, X, x_dtype, N, ldx);
   if (rc) return rc;
   if (!weights || !means || !vars) return FGMM_ERR_INVALID_ARG;
@@ -312,6 +359,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
   const Workspace& w = c.ws;
+  if (host_x && (e = ensure_staging(h)) != cudaSuccess) return map_cuda(e);
   // which path(s) to enqueue: FP32 -> CUDA cores; FP16X3 -> tensor cores; AUTO ->
   // both, each kernel returning at once unless the device-side mode word (set by the
   // tensor-core preparation's conditioning check) selects its path
@@ -320,7 +368,8 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
   const bool run_simt = c.prec == FGMM_PREC_FP32 || !c.tc.ready || auto_mode;
   const int fixed_mode = run_tc && !run_simt ? kModeTensor : kModeSimt;
   const int* mode = auto_mode ? w.mode : nullptr;
-  if (run_tc && x_dtype == FGMM_F32 && ((uintptr_t)X % 4 != 0)) return FGMM_ERR_INVALID_ARG;
+  if (run_tc && !host_x && x_dtype == FGMM_F32 && ((uintptr_t)X % 4 != 0))
+    return FGMM_ERR_INVALID_ARG;
   if ((e = cudaMemsetAsync(w.ll_total, 0, sizeof(double), s)) != cudaSuccess) return map_cuda(e);
   if ((e = cudaMemsetAsync(w.stats, 0, stats_bytes(w), s)) != cudaSuccess) return map_cuda(e);
   if (auto_mode && (e = cudaMemsetAsync(w.mode, 0, sizeof(int), s)) != cudaSuccess)
@@ -334,48 +383,89 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       return map_cuda(e);
   }
   const size_t eb = dtype_bytes(x_dtype);
+  // The rows of chunk [c0, c0 + nc) on the device: X itself, or (host X) a staging
+  // buffer filled on the copy stream once the kernels that last read it are done; the
+  // copy of the next chunk overlaps the kernels of this one.
+  HostStaging& hs = h->hs;
+  cudaError_t copy_err = cudaSuccess;
+  auto acquire = [&](int64_t c0, int64_t nc, const void** Xc, int64_t* ldc) -> int {
+    if (!host_x) {
+      *Xc = (const char*)X + (size_t)c0 * ldx * eb;
+      *ldc = ldx;
+      return -1;
+    }
+    const int b = (int)(hs.seq++ & 1);
+    cudaError_t r = cudaStreamWaitEvent(hs.cs, hs.consumed[b], 0);
+    if (r == cudaSuccess)
+      r = cudaMemcpy2DAsync(hs.buf[b], (size_t)c.D * eb, (const char*)X + (size_t)c0 * ldx * eb,
+                            (size_t)ldx * eb, (size_t)c.D * eb, (size_t)nc,
+                            cudaMemcpyHostToDevice, hs.cs);
+    if (r == cudaSuccess) r = cudaEventRecord(hs.copied[b], hs.cs);
+    if (r == cudaSuccess) r = cudaStreamWaitEvent(s, hs.copied[b], 0);
+    if (r != cudaSuccess && copy_err == cudaSuccess) copy_err = r;
+    *Xc = hs.buf[b];
+    *ldc = c.D;
+    return b;
+  };
+  auto release = [&](int b) {
+    if (b >= 0) cudaEventRecord(hs.consumed[b], s);
+  };
   // one tensor-core pass over all chunks, its kernels gated on the word `gate`
   auto tc_pass = [&](const int* gate) -> cudaError_t {
     cudaError_t r = cudaSuccess;
     for (int64_t c0 = 0; c0 < N && r == cudaSuccess; c0 += kChunk) {
       const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
-      const void* Xc = (const char*)X + (size_t)c0 * ldx * eb;
+      const void* Xc;
+      int64_t ldc;
+      const int b = acquire(c0, nc, &Xc, &ldc);
       float* lzo = logz_out ? logz_out + c0 : nullptr;
-      if ((r = launch_tc_convert(c, Xc, x_dtype, nc, ldx, gate, s)) != cudaSuccess) break;
-      if ((r = launch_tc_lse(c, nc, lzo, gate, s)) != cudaSuccess) break;
-      // stiff components (AUTO) join log Z here; then the chunk's log-likelihood
-      if ((r = launch_side_lse(c, Xc, x_dtype, nc, ldx, lzo, gate, s)) != cudaSuccess) break;
-      if ((r = launch_ll_accumulate(c, nc, gate, fixed_mode, kModeTensor, s)) != cudaSuccess) break;
-      if ((r = launch_tc_stats(c, nc, gate, s)) != cudaSuccess) break;
-      r = launch_side_stats(c, Xc, x_dtype, nc, ldx, gate, s);
+      if ((r = launch_tc_convert(c, Xc, x_dtype, nc, ldc, gate, s)) == cudaSuccess &&
+          (r = launch_tc_lse(c, nc, lzo, gate, s)) == cudaSuccess &&
+          // stiff components (AUTO) join log Z here; then the chunk's log-likelihood
+          (r = launch_side_lse(c, Xc, x_dtype, nc, ldc, lzo, gate, s)) == cudaSuccess &&
+          (r = launch_ll_accumulate(c, nc, gate, fixed_mode, kModeTensor, s)) == cudaSuccess &&
+          (r = launch_tc_stats(c, nc, gate, s)) == cudaSuccess)
+        r = launch_side_stats(c, Xc, x_dtype, nc, ldc, gate, s);
+      release(b);
+      if (r == cudaSuccess) r = copy_err;
     }
     return r;
   };
   if (run_tc) {
     if (auto_mode && (e = cudaMemsetAsync(w.mode2, 0xFF, sizeof(int), s)) != cudaSuccess)
       return map_cuda(e);
-    if ((e = tc_pass(mode)) != cudaSuccess) return map_cuda(e);
+    // With host X a pass whose gate is off would still copy every chunk, so under AUTO
+    // the gate words are read back (one synchronisation each) before such a pass.
+    int word = kModeTensor;
+    if (host_x && auto_mode && (rc = read_word(w.mode, &word, s))) return rc;
+    if (word == kModeTensor && (e = tc_pass(mode)) != cudaSuccess) return map_cuda(e);
     if (auto_mode) {
       // AUTO: components whose new variance would lose accuracy to cancellation move to
       // the side path and the pass is redone (gated on mode2); a failure after that sends
       // the step to the CUDA-core kernels below (gated on mode)
       if ((e = launch_auto_check(c, 0, s)) != cudaSuccess) return map_cuda(e);
       if ((e = launch_stiff_compact(c, w.mode2, w.mode, s)) != cudaSuccess) return map_cuda(e);
-      if ((e = tc_pass(w.mode2)) != cudaSuccess) return map_cuda(e);
+      word = kModeTensor;
+      if (host_x && (rc = read_word(w.mode2, &word, s))) return rc;
+      if (word == kModeTensor && (e = tc_pass(w.mode2)) != cudaSuccess) return map_cuda(e);
       if ((e = launch_auto_check(c, 1, s)) != cudaSuccess) return map_cuda(e);
     }
   }
-  if (run_simt) {
+  int simt_word = kModeSimt;
+  if (run_simt && host_x && auto_mode && (rc = read_word(w.mode, &simt_word, s))) return rc;
+  if (run_simt && simt_word == kModeSimt) {
     for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
       const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
-      const void* Xc = (const char*)X + (size_t)c0 * ldx * eb;
+      const void* Xc;
+      int64_t ldc;
+      const int b = acquire(c0, nc, &Xc, &ldc);
       float* lzo = logz_out ? logz_out + c0 : nullptr;
-      if ((e = launch_lse_simt(c, Xc, x_dtype, nc, ldx, lzo, mode, s)) != cudaSuccess)
-        return map_cuda(e);
-      if ((e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeSimt, s)) != cudaSuccess)
-        return map_cuda(e);
-      if ((e = launch_stats_simt(c, Xc, x_dtype, nc, ldx, mode, s)) != cudaSuccess)
-        return map_cuda(e);
+      if ((e = launch_lse_simt(c, Xc, x_dtype, nc, ldc, lzo, mode, s)) == cudaSuccess &&
+          (e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeSimt, s)) == cudaSuccess)
+        e = launch_stats_simt(c, Xc, x_dtype, nc, ldc, mode, s);
+      release(b);
+      if (e == cudaSuccess) e = copy_err;
+      if (e != cudaSuccess) return map_cuda(e);
     }
   }
   if ((e = launch_reduce_stats(c, means, st, mode, fixed_mode, s)) != cudaSuccess)
@@ -401,6 +491,25 @@ int fgmm_em_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_
                     double* stats_out, float* logz_out, fgmm_stream_t stream) {
   if (!stats_out) return FGMM_ERR_INVALID_ARG;
   return run_partial(h, X, x_dtype, N, ldx, weights, means, vars, stats_out, logz_out, stream);
+}
+
+int fgmm_em_step_host(fgmm_handle h, const void* X_host, int x_dtype, int64_t N, int64_t ldx,
+                      float* weights, float* means, float* vars, double* loglik_out,
+                      float* logz_out, fgmm_stream_t stream) {
+  int rc = run_partial(h, X_host, x_dtype, N, ldx, weights, means, vars,
+                       h ? h->c.ws.canon : nullptr, logz_out, stream, true);
+  if (rc) return rc;
+  return map_cuda(launch_finish(h->c, h->c.ws.canon, weights, means, vars, loglik_out,
+                                (cudaStream_t)stream));
+}
+
+int fgmm_em_partial_host(fgmm_handle h, const void* X_host, int x_dtype, int64_t N,
+                         int64_t ldx, const float* weights, const float* means,
+                         const float* vars, double* stats_out, float* logz_out,
+                         fgmm_stream_t stream) {
+  if (!stats_out) return FGMM_ERR_INVALID_ARG;
+  return run_partial(h, X_host, x_dtype, N, ldx, weights, means, vars, stats_out, logz_out,
+                     stream, true);
 }
 
 int fgmm_em_finish(fgmm_handle h, const double* stats, float* weights, float* means,
@@ -563,6 +672,34 @@ int fgmm_profile_read(fgmm_handle h, fgmm_profile* out, int reset) {
     p->nsnap = 0;
   }
   return FGMM_OK;
+}
+
+int fgmm_kmeans_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                     float* centroids, int32_t* assign_out, int64_t* counts_out,
+                     double* inertia_out, fgmm_stream_t stream) {
+  int rc = check_x(h, X, x_dtype, N, ldx);
+  if (rc) return rc;
+  if (!centroids) return FGMM_ERR_INVALID_ARG;
+  if ((rc = set_device(h->c))) return rc;
+  return map_cuda(launch_kmeans_step(h->c, X, x_dtype, N, ldx, centroids, assign_out,
+                                     counts_out, inertia_out, (cudaStream_t)stream));
+}
+
+int fgmm_kmeans_seed(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                     int64_t first, const double* u, float* centroids, int64_t* idx_out,
+                     void* scratch, fgmm_stream_t stream) {
+  int rc = check_x(h, X, x_dtype, N, ldx);
+  if (rc) return rc;
+  if (!centroids || !idx_out || !scratch || first < 0 || first >= N ||
+      (h->c.K > 1 && !u))
+    return FGMM_ERR_INVALID_ARG;
+  if ((rc = set_device(h->c))) return rc;
+  return map_cuda(launch_kmeans_seed(h->c, X, x_dtype, N, ldx, first, u, centroids, idx_out,
+                                     scratch, (cudaStream_t)stream));
+}
+
+size_t fgmm_kmeans_seed_scratch_bytes(int64_t N) {
+  return N > 0 ? kmeans_seed_scratch_bytes(N) : 0;
 }
 
 const char* fgmm_profile_kernel_name(int index) {

@@ -88,6 +88,7 @@ struct Workspace {
   double* stats = nullptr;
   double* nk = nullptr;    // [Kp] reduced N_k of the last step
   int* status = nullptr;   // [1]
+  unsigned int* km_word = nullptr;  // [2] k-means: largest |x| (float bits), fixed-point exponent
   size_t bytes = 0;
 };
 
@@ -99,6 +100,7 @@ enum KernelId {
   KI_FINALIZE,
   KI_SOFT_ASSIGN, KI_AUTO_CHECK, KI_REDO_RESET, KI_REMASK,
   KI_STIFF_COMPACT, KI_SIDE_LSE, KI_LL_PARTIALS, KI_SIDE_STATS, KI_SIDE_REDUCE,
+  KI_KM_ASSIGN, KI_KM_SEED,
   KI_COUNT
 };
 
@@ -158,6 +160,14 @@ cudaError_t launch_finish(const Ctx& c, const double* st, float* weights, float*
                           float* vars, double* loglik_out, cudaStream_t s);
 cudaError_t launch_stats_sum(const double* parts, int n_parts, int64_t len, double* out,
                              cudaStream_t s);
+// k-means warm start (fgmm_kmeans.cu)
+size_t kmeans_seed_scratch_bytes(int64_t n);
+cudaError_t launch_kmeans_step(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                               float* centroids, int32_t* assign_out, int64_t* counts_out,
+                               double* inertia_out, cudaStream_t s);
+cudaError_t launch_kmeans_seed(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                               int64_t first, const double* u, float* centroids,
+                               int64_t* idx_out, void* scratch, cudaStream_t s);
 // tensor-core path (fgmm_tc.cu)
 bool tc_supported(const Ctx& c);
 cudaError_t tc_init(Ctx& c);

@@ -23,9 +23,9 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
-def _x_args(X: torch.Tensor):
-    if X.dim() != 2 or not X.is_cuda:
-        raise ValueError("X must be a 2-D CUDA tensor")
+def _x_args(X: torch.Tensor, allow_host: bool = False):
+    if X.dim() != 2 or not (X.is_cuda or (allow_host and X.device.type == "cpu")):
+        raise ValueError("X must be a 2-D CUDA tensor" + (" or CPU tensor" if allow_host else ""))
     if X.dtype == torch.float32:
         dt = _lib.F32
     elif X.dtype == torch.bfloat16:
@@ -109,19 +109,21 @@ class GMM:
     def step(self, X, weights, means, variances, loglik=None, logz=None):
         """One fused EM iteration; updates the parameters in place.
 
+        X: CUDA tensor, or CPU tensor (ideally pinned), which is streamed to the device
+        chunk by chunk with the copies overlapping the sweeps (fgmm_em_step_host).
         loglik: optional CUDA float64 tensor [1] receiving log p(X | Θ_in).
         logz:   optional CUDA float32 tensor [N] receiving per-point log p(x_i | Θ_in).
         """
         self._check_params(weights, means, variances)
-        xp, dt, n, ldx = _x_args(X)
+        xp, dt, n, ldx = _x_args(X, allow_host=True)
         if loglik is not None and not (loglik.is_cuda and loglik.dtype == torch.float64):
             raise ValueError("loglik must be a CUDA float64 tensor")
         if logz is not None and not (logz.is_cuda and logz.dtype == torch.float32
                                      and logz.numel() >= n):
             raise ValueError("logz must be a CUDA float32 tensor with N elements")
-        check(LIB.fgmm_em_step(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means),
-                               _ptr(variances), _ptr(loglik), _ptr(logz), _stream()),
-              "fgmm_em_step")
+        fn = LIB.fgmm_em_step if X.is_cuda else LIB.fgmm_em_step_host
+        check(fn(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means), _ptr(variances),
+                 _ptr(loglik), _ptr(logz), _stream()), "fgmm_em_step")
 
     # ---------------------------------------------------------------- sharded EM
     @property
@@ -137,18 +139,18 @@ class GMM:
         Vectors of disjoint shards add up to the vector of their union.
         """
         self._check_params(weights, means, variances)
-        xp, dt, n, ldx = _x_args(X)
+        xp, dt, n, ldx = _x_args(X, allow_host=True)
         if stats is None:
-            stats = torch.empty(self.stats_len, dtype=torch.float64, device=X.device)
+            stats = torch.empty(self.stats_len, dtype=torch.float64, device=weights.device)
         elif not (stats.is_cuda and stats.dtype == torch.float64 and stats.is_contiguous()
                   and stats.numel() == self.stats_len):
             raise ValueError("stats must be a contiguous CUDA float64 tensor of stats_len")
         if logz is not None and not (logz.is_cuda and logz.dtype == torch.float32
                                      and logz.numel() >= n):
             raise ValueError("logz must be a CUDA float32 tensor with N elements")
-        check(LIB.fgmm_em_partial(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means),
-                                  _ptr(variances), _ptr(stats), _ptr(logz), _stream()),
-              "fgmm_em_partial")
+        fn = LIB.fgmm_em_partial if X.is_cuda else LIB.fgmm_em_partial_host
+        check(fn(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means), _ptr(variances),
+                 _ptr(stats), _ptr(logz), _stream()), "fgmm_em_partial")
         return stats
 
     def finish(self, stats, weights, means, variances, loglik=None):
@@ -167,6 +169,33 @@ class GMM:
         """Sum of gathered statistics vectors ([n, stats_len]) in row order."""
         return stats_sum(parts)
 
+
+    # ---------------------------------------------------------------- k-means warm start
+    def kmeans_step(self, X, centroids, assign=None, counts=None, inertia=None):
+        """One Lloyd iteration (fgmm_kmeans_step); centroids [K, D] float32 CUDA, in/out.
+        assign: optional int32 [N], counts: optional int64 [K], inertia: optional
+        float64 [1] (all CUDA) receive the assignment to the input centroids."""
+        xp, dt, n, ldx = _x_args(X)
+        if not (centroids.is_cuda and centroids.dtype == torch.float32 and centroids.is_contiguous()
+                and tuple(centroids.shape) == (self.K, self.D)):
+            raise ValueError("centroids must be a contiguous [K, D] float32 CUDA tensor")
+        check(LIB.fgmm_kmeans_step(self._h, xp, dt, n, ldx, _ptr(centroids), _ptr(assign),
+                                   _ptr(counts), _ptr(inertia), _stream()), "fgmm_kmeans_step")
+
+    def kmeans_seed(self, X, first, u):
+        """k-means++ seeding (fgmm_kmeans_seed) from the first index and the K-1 uniforms
+        u (float64, any device).  Returns (centroids [K, D] float32, indices int64 [K])."""
+        xp, dt, n, ldx = _x_args(X)
+        u = torch.as_tensor(u, dtype=torch.float64).to(X.device).contiguous()
+        if u.numel() != max(self.K - 1, 0):
+            raise ValueError("u must hold K - 1 uniforms")
+        C = torch.empty(self.K, self.D, dtype=torch.float32, device=X.device)
+        idx = torch.empty(self.K, dtype=torch.int64, device=X.device)
+        scratch = torch.empty(int(LIB.fgmm_kmeans_seed_scratch_bytes(n)), dtype=torch.uint8,
+                              device=X.device)
+        check(LIB.fgmm_kmeans_seed(self._h, xp, dt, n, ldx, int(first), _ptr(u), _ptr(C),
+                                   _ptr(idx), _ptr(scratch), _stream()), "fgmm_kmeans_seed")
+        return C, idx
 
     def fit(self, X, weights, means, variances, max_iters=100, tol=0.0):
         """Repeat step up to max_iters times; returns (final_loglik, iters_done)."""
