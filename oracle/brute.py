@@ -96,3 +96,21 @@ def shard_statistics(X, w, mu, var, spherical=False):
                    for d in range(D))
     out.append(math.fsum(logZ))
     return out
+
+
+def fisher_vector(X, w, mu, var, spherical=False):
+    """Fisher vector [G_mu, G_sigma] by scalar loops (same definition as the NumPy oracle)."""
+    N, K, D = len(X), len(mu), len(X[0])
+    *_, R = em_step(X, w, mu, var, spherical)
+    gm, gs = [], []
+    for k in range(K):
+        for d in range(D):
+            sd = math.sqrt(var[k] if spherical else var[k][d])
+            gm.append(math.fsum(R[i][k] * (X[i][d] - mu[k][d]) / sd for i in range(N))
+                      / (N * math.sqrt(w[k])))
+    for k in range(K):
+        for d in range(D):
+            sd = math.sqrt(var[k] if spherical else var[k][d])
+            gs.append(math.fsum(R[i][k] * (((X[i][d] - mu[k][d]) / sd) ** 2 - 1.0)
+                                for i in range(N)) / (N * math.sqrt(2.0 * w[k])))
+    return gm + gs

@@ -274,6 +274,50 @@ def m_step_from_statistics(stats, weights, means, variances, cov_type=COV_DIAG,
     return StepResult(w_new, mu_new, var_new, loglik, None, Nk, empty)
 
 
+def fisher_vector(X, weights, means, variances, cov_type=COV_DIAG, normalize=False):
+    """Fisher-vector encoding of the set X under the mixture (gradients of the average
+    log-likelihood with respect to the means and standard deviations, whitened by the
+    diagonal Fisher information: Perronnin & Dance 2007; Sanchez et al. 2013).  The
+    paper names the encoding as a use of the same fused E-step and weighted statistics
+    (§6) without defining it; this is the textbook definition:
+
+      G_mu_kd    = 1 / (N sqrt(pi_k))   sum_i r_ik (x_id - mu_kd) / sigma_kd
+      G_sigma_kd = 1 / (N sqrt(2 pi_k)) sum_i r_ik ((x_id - mu_kd)^2 / sigma_kd^2 - 1)
+
+    returned as [G_mu (K x D, row-major), G_sigma (K x D)] (length 2 K D).  With
+    normalize, the "improved" encoding: z <- sign(z) sqrt(|z|), then z / ||z||_2.
+    Components with pi_k = 0 contribute zeros.
+    """
+    X = _as_f64(X)
+    N, D = X.shape
+    mu = _as_f64(means)
+    K = mu.shape[0]
+    w = _as_f64(weights)
+    var = _as_f64(variances)
+    sig = np.sqrt(var.reshape(K, 1) * np.ones((1, D)) if cov_type == COV_SPHERICAL
+                  else var.reshape(K, D))
+    gm = np.zeros((K, D))
+    gs = np.zeros((K, D))
+    for s, e in _row_chunks(N, K):
+        _, R = e_step(X[s:e], w, mu, var, cov_type)
+        for k in range(K):
+            z = (X[s:e] - mu[k]) / sig[k]
+            gm[k] += R[:, k] @ z
+            gs[k] += R[:, k] @ (z * z - 1.0)
+    live = w > 0
+    gm[live] /= (N * np.sqrt(w[live]))[:, None]
+    gs[live] /= (N * np.sqrt(2.0 * w[live]))[:, None]
+    gm[~live] = 0.0
+    gs[~live] = 0.0
+    fv = np.concatenate([gm.ravel(), gs.ravel()])
+    if normalize:
+        fv = np.sign(fv) * np.sqrt(np.abs(fv))
+        nrm = np.linalg.norm(fv)
+        if nrm > 0:
+            fv = fv / nrm
+    return fv
+
+
 def fit(X, weights, means, variances, cov_type=COV_DIAG, reg_covar=1e-6,
         max_iters=100, tol=0.0):
     """Repeat em_step; stop after max_iters or when |L_t − L_{t−1}| / N < tol.

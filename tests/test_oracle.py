@@ -366,3 +366,41 @@ def test_m_step_from_statistics_keeps_empty_components():
     np.testing.assert_array_equal(r.variances[1], var[1])
     np.testing.assert_array_equal(r.weights, [1.0, 0.0])
     assert r.loglik == -5.0
+
+
+# ------------------------------------------------------------------ Fisher vectors
+@pytest.mark.parametrize("spherical", [False, True])
+def test_fisher_vector_matches_brute_force(spherical):
+    rng = np.random.default_rng(31)
+    N, K, D = 17, 3, 2
+    X = rng.normal(size=(N, D)) * 2
+    w = np.array([0.2, 0.5, 0.3])
+    mu = rng.normal(size=(K, D))
+    var = rng.uniform(0.5, 2.0, size=K) if spherical else rng.uniform(0.5, 2.0, size=(K, D))
+    cov = O.COV_SPHERICAL if spherical else O.COV_DIAG
+    got = O.fisher_vector(X, w, mu, var, cov)
+    ref = brute.fisher_vector(X.tolist(), w.tolist(), mu.tolist(), var.tolist(), spherical)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_fisher_vector_single_gaussian_closed_form():
+    """K = 1 at the sample mean: G_mu = 0; G_sigma_d = (s_d^2 / sigma_d^2 - 1) / sqrt(2),
+    with s_d^2 the (1/N) sample variance."""
+    rng = np.random.default_rng(32)
+    X = rng.normal(size=(400, 3)) * [1.0, 2.0, 0.5] + [3.0, -1.0, 0.0]
+    mu = X.mean(0, keepdims=True)
+    var = np.array([[1.5, 3.0, 0.2]])
+    fv = O.fisher_vector(X, np.array([1.0]), mu, var)
+    np.testing.assert_allclose(fv[:3], 0.0, atol=1e-12)
+    np.testing.assert_allclose(fv[3:], (X.var(0) / var[0] - 1.0) / np.sqrt(2.0), rtol=1e-12)
+
+
+def test_fisher_vector_normalisation():
+    rng = np.random.default_rng(33)
+    X = rng.normal(size=(50, 2))
+    w, mu, var = np.array([0.5, 0.5]), np.array([[-1.0, 0.0], [1.0, 0.0]]), np.ones((2, 2))
+    raw = O.fisher_vector(X, w, mu, var)
+    fv = O.fisher_vector(X, w, mu, var, normalize=True)
+    assert abs(np.linalg.norm(fv) - 1.0) < 1e-12
+    np.testing.assert_allclose(fv * np.linalg.norm(np.sqrt(np.abs(raw))),
+                               np.sign(raw) * np.sqrt(np.abs(raw)), rtol=1e-12, atol=1e-15)
