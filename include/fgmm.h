@@ -235,6 +235,30 @@ int fgmm_soft_assign_static(int K, int D, int cov_type, const void* X, int x_dty
                             const float* vars, int top_m, float r_threshold, int32_t* ids,
                             float* resp, fgmm_stream_t stream);
 
+/* Per-point log-density log p(x_i | Theta) = log sum_k pi_k N(x_i | mu_k, Sigma_k) (the
+ * first sweep of fgmm_em_step alone: no statistics, parameters unchanged).  With equal
+ * weights, the points of a sample as means and a shared isotropic bandwidth this is a
+ * Gaussian kernel density estimate (the paper, §6, names KDE as a use of the same
+ * kernel).  logz_out: device float[N] (may be NULL if loglik_out is given); loglik_out:
+ * optional device double, the sum.  Precision modes as fgmm_em_step.  Asynchronous. */
+int fgmm_score_samples(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                       const float* weights, const float* means, const float* vars,
+                       float* logz_out, double* loglik_out, fgmm_stream_t stream);
+
+/* Fisher-vector encoding of the point set X (N points) under the mixture: the
+ * gradients of the average log-likelihood with respect to the means and the standard
+ * deviations, whitened by the diagonal Fisher information (Perronnin & Dance 2007;
+ * the paper, §6, names the encoding as a use of the same E-step and weighted
+ * statistics):  G_mu_kd = sum_i r_ik (x_id - mu_kd) / sigma_kd / (N sqrt(pi_k)),
+ * G_sigma_kd = sum_i r_ik ((x_id - mu_kd)^2 / sigma_kd^2 - 1) / (N sqrt(2 pi_k)).
+ * fv_out: device float[2 K D] = [G_mu (K x D, row-major), G_sigma (K x D)]; components
+ * with pi_k = 0 give zeros.  normalize != 0: power (sign(z) sqrt|z|) and L2
+ * normalisation.  Runs the E-step and statistics sweep of fgmm_em_step (same precision
+ * modes); K <= 32768 (FGMM_ERR_UNSUPPORTED otherwise).  Asynchronous. */
+int fgmm_fisher_vector(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                       const float* weights, const float* means, const float* vars,
+                       int normalize, float* fv_out, fgmm_stream_t stream);
+
 /* k-means warm start ("Flash-GMM", §4.4: k-means, then soft EM from its centroids;
  * the initialisation appendix: k-means++ seeding).  Both use the handle's K and D (and
  * its workspace; they may not run concurrently with another call on the same handle).

@@ -62,6 +62,8 @@ SIGNATURES = {
     "fgmm_em_partial": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_em_finish": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_stats_sum": (_int, [_vp, _int, _i64, _vp, _vp]),
+    "fgmm_score_samples": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_fisher_vector": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _int, _vp, _vp]),
     "fgmm_kmeans_step": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_kmeans_seed": (_int, [_vp, _vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_kmeans_seed_scratch_bytes": (_c.c_size_t, [_i64]),

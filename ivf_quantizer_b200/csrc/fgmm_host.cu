@@ -155,7 +155,7 @@ void free_ws(Workspace& w) {
                   w.stats,  w.nk,     w.status, w.center, w.dscale, w.wop,
                   w.tck,    w.tks,    w.xop,    w.mode, w.stiff,    w.stiff_list, w.n_stiff,
                   w.side_part, w.mode2, w.canon, w.tcraw, w.tcm, w.tcpk, w.tckf, w.lzlow,
-                  w.side_flag, w.km_word};
+                  w.side_flag, w.km_word, w.grey, w.grey_pos, w.grey_stats};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -209,12 +209,18 @@ cudaError_t alloc_ws(Ctx& c) {
   if (tc) {
     if ((e = alloc(&w.stiff, (size_t)w.Kt, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.stiff_list, (size_t)w.Kt, &t)) != cudaSuccess) return e;
-    if ((e = alloc(&w.n_stiff, (size_t)1, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.n_stiff, (size_t)2, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.grey, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.grey_pos, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.grey_stats, (size_t)kSideMaxStiff * (1 + 2 * (size_t)w.Dp), &t)) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaMemset(w.grey, 0, (size_t)w.Kt * sizeof(int))) != cudaSuccess) return e;
     if ((e = alloc(&w.side_part, (size_t)kSideParts * kSideMaxStiff * (1 + 2 * (size_t)w.Dp), &t)) !=
         cudaSuccess)
       return e;
     if ((e = cudaMemset(w.stiff, 0, (size_t)w.Kt * sizeof(int))) != cudaSuccess) return e;
-    if ((e = cudaMemset(w.n_stiff, 0, sizeof(int))) != cudaSuccess) return e;
+    if ((e = cudaMemset(w.n_stiff, 0, 2 * sizeof(int))) != cudaSuccess) return e;
     if ((e = alloc(&w.wop, (size_t)2 * w.Kt * w.K1, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.tck, (size_t)w.Kt, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.tks, (size_t)w.Kt, &t)) != cudaSuccess) return e;
@@ -350,7 +356,8 @@ int read_word(const int* dev, int* out, cudaStream_t s) {
 
 int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
                 const float* weights, const float* means, const float* vars, double* st,
-                float* logz_out, fgmm_stream_t stream, bool host_x = false) {
+                float* logz_out, fgmm_stream_t stream, bool host_x = false,
+                bool want_stats = true) {
   int rc = check_x(h, X, x_dtype, N, ldx);
   if (rc) return rc;
   if (!weights || !means || !vars) return FGMM_ERR_INVALID_ARG;
@@ -412,7 +419,9 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
   };
   // one tensor-core pass over all chunks, its kernels gated on the word `gate`
   auto tc_pass = [&](const int* gate) -> cudaError_t {
-    cudaError_t r = cudaSuccess;
+    // the grey components' side-path statistics of this pass accumulate from zero
+    cudaError_t r = cudaMemsetAsync(w.grey_stats, 0,
+                                    (size_t)kSideMaxStiff * (1 + 2 * (size_t)w.Dp) * sizeof(double), s);
     for (int64_t c0 = 0; c0 < N && r == cudaSuccess; c0 += kChunk) {
       const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
       const void* Xc;
@@ -424,7 +433,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
           // stiff components (AUTO) join log Z here; then the chunk's log-likelihood
           (r = launch_side_lse(c, Xc, x_dtype, nc, ldc, lzo, gate, s)) == cudaSuccess &&
           (r = launch_ll_accumulate(c, nc, gate, fixed_mode, kModeTensor, s)) == cudaSuccess &&
-          (r = launch_tc_stats(c, nc, gate, s)) == cudaSuccess)
+          want_stats && (r = launch_tc_stats(c, nc, gate, s)) == cudaSuccess)
         r = launch_side_stats(c, Xc, x_dtype, nc, ldc, gate, s);
       release(b);
       if (r == cudaSuccess) r = copy_err;
@@ -439,7 +448,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
     int word = kModeTensor;
     if (host_x && auto_mode && (rc = read_word(w.mode, &word, s))) return rc;
     if (word == kModeTensor && (e = tc_pass(mode)) != cudaSuccess) return map_cuda(e);
-    if (auto_mode) {
+    if (auto_mode && want_stats) {
       // AUTO: components whose new variance would lose accuracy to cancellation move to
       // the side path and the pass is redone (gated on mode2); a failure after that sends
       // the step to the CUDA-core kernels below (gated on mode)
@@ -461,14 +470,15 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       const int b = acquire(c0, nc, &Xc, &ldc);
       float* lzo = logz_out ? logz_out + c0 : nullptr;
       if ((e = launch_lse_simt(c, Xc, x_dtype, nc, ldc, lzo, mode, s)) == cudaSuccess &&
-          (e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeSimt, s)) == cudaSuccess)
+          (e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeSimt, s)) == cudaSuccess &&
+          want_stats)
         e = launch_stats_simt(c, Xc, x_dtype, nc, ldc, mode, s);
       release(b);
       if (e == cudaSuccess) e = copy_err;
       if (e != cudaSuccess) return map_cuda(e);
     }
   }
-  if ((e = launch_reduce_stats(c, means, st, mode, fixed_mode, s)) != cudaSuccess)
+  if (want_stats && (e = launch_reduce_stats(c, means, st, mode, fixed_mode, s)) != cudaSuccess)
     return map_cuda(e);
   h->c.last_auto = auto_mode;
   h->c.last_path = fixed_mode == kModeTensor ? FGMM_PREC_FP16X3 : FGMM_PREC_FP32;
@@ -672,6 +682,29 @@ int fgmm_profile_read(fgmm_handle h, fgmm_profile* out, int reset) {
     p->nsnap = 0;
   }
   return FGMM_OK;
+}
+
+int fgmm_score_samples(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                       const float* weights, const float* means, const float* vars,
+                       float* logz_out, double* loglik_out, fgmm_stream_t stream) {
+  if (!logz_out && !loglik_out) return FGMM_ERR_INVALID_ARG;
+  int rc = run_partial(h, X, x_dtype, N, ldx, weights, means, vars, nullptr, logz_out, stream,
+                       false, false);
+  if (rc || !loglik_out) return rc;
+  return map_cuda(cudaMemcpyAsync(loglik_out, h->c.ws.ll_total, sizeof(double),
+                                  cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+}
+
+int fgmm_fisher_vector(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
+                       const float* weights, const float* means, const float* vars,
+                       int normalize, float* fv_out, fgmm_stream_t stream) {
+  if (!fv_out) return FGMM_ERR_INVALID_ARG;
+  if (h && h->c.K > (int)(kChunk / 32)) return FGMM_ERR_UNSUPPORTED;
+  int rc = run_partial(h, X, x_dtype, N, ldx, weights, means, vars, h ? h->c.ws.canon : nullptr,
+                       nullptr, stream);
+  if (rc) return rc;
+  return map_cuda(launch_fisher(h->c, weights, vars, (double)N, h->c.ws.canon, normalize,
+                                fv_out, (cudaStream_t)stream));
 }
 
 int fgmm_kmeans_step(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,

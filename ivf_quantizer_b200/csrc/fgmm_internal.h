@@ -24,9 +24,13 @@ constexpr int kFlushTiles = 64;  // fp32 run length (tiles) before an fp64 flush
 constexpr int64_t kChunk = FGMM_CHUNK_POINTS;  // points per chunk: bounds every N-sized buffer
 constexpr int kSideMaxStiff = 256;   // AUTO side path: most stiff components per step
 constexpr int kSideParts = 64;       // AUTO side path: point ranges per chunk
-// AUTO side path: a stiff component whose log-density is more than this many nats below
-// a point's log Z has responsibility exp(-120) < 1e-52 there (zero in fp32)
-constexpr float kSideCut = 120.f;
+// AUTO side path: a stiff or grey component whose log-density is more than this many
+// nats below a point's log Z is skipped there: its responsibility is below
+// exp(-40) = 4e-18, far under fp32 resolution of log Z and under what the tensor-core
+// statistics keep (they store r as fp16(r 2^15), which drops r below ~1e-12)
+constexpr float kSideCut = 40.f;
+// AUTO: a component with fewer effective points than this in the previous step is grey
+constexpr double kGreyNk = 8.0;
 
 static inline int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
@@ -73,7 +77,12 @@ struct Workspace {
   int* mode2 = nullptr;     // [1] AUTO: tensor when the hybrid redo pass must run
   int* stiff = nullptr;     // [Kt] AUTO: 1 = component handled by the CUDA-core side path
   int* stiff_list = nullptr;  // [Kt] stiff components in index order
-  int* n_stiff = nullptr;   // [1]
+  int* n_stiff = nullptr;   // [2] stiff count, grey count (the grey follow the stiff in the list)
+  // AUTO grey components: kept on the tensor cores, but their statistics are also taken
+  // on the side path, to be swapped in should the variance check fail
+  int* grey = nullptr;      // [Kt] 1: grey
+  int* grey_pos = nullptr;  // [Kt] index among the grey of this pass, -1 if none
+  double* grey_stats = nullptr;  // [kSideMaxStiff][1 + 2 Dp] side-path statistics of the grey
   double* side_part = nullptr;  // [kSideParts][kSideMaxStiff][1 + 2 Dp] side-path partial rows
   // prepared parameters (CUDA-core path)
   float* mu = nullptr;     // [Kp, Dp] means, zero padded
@@ -158,6 +167,9 @@ cudaError_t launch_reduce_stats(const Ctx& c, const float* means, double* out, c
 // M-step and weights from exchange-form statistics; parameters updated in place.
 cudaError_t launch_finish(const Ctx& c, const double* st, float* weights, float* means,
                           float* vars, double* loglik_out, cudaStream_t s);
+// Fisher vector from exchange-form statistics (fv: [2 K D]); uses ll_tiles (K <= kChunk/32).
+cudaError_t launch_fisher(const Ctx& c, const float* weights, const float* vars, double n_points,
+                          const double* st, int normalize, float* fv, cudaStream_t s);
 cudaError_t launch_stats_sum(const double* parts, int n_parts, int64_t len, double* out,
                              cudaStream_t s);
 // k-means warm start (fgmm_kmeans.cu)

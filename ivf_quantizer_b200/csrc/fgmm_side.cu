@@ -14,7 +14,7 @@
 // A stiff component's log-density is evaluated dimension by dimension and abandoned
 // as soon as its upper bound (the constant plus the partial sum, every remaining term
 // being <= 0) falls more than kCut nats below the point's log Z: its responsibility
-// would be exp(-kCut) < 1e-52, zero in fp32.  A collapsed component costs one or two
+// would be below exp(-kCut) (see kSideCut).  A collapsed component costs one or two
 // dimensions per point.
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -51,49 +51,69 @@ __device__ __forceinline__ float stiff_logit(const T* __restrict__ x, int D,
 
 }  // namespace
 
-// One CTA: stiff_list = the stiff components in increasing index order, n = their count.
-// More than kMaxStiff stiff components: the side path would cost as much as the
-// CUDA-core path, so the whole step goes there (mode word).
-constexpr int kMaxStiff = kSideMaxStiff;
+constexpr int kMaxStiff = kSideMaxStiff;   // stiff + grey components of one pass
 
-// Runs when *gate is tensor (or gate is null); on overflow the step goes to the CUDA-core
-// path (*mode) and the gated pass is switched off (*gate).
-__global__ void stiff_compact_kernel(const int* __restrict__ stiff, int K, int Kt,
-                                     int* __restrict__ list, int* __restrict__ n_out,
-                                     const float* __restrict__ craw, const float* __restrict__ mq,
-                                     const float* __restrict__ peak, float* __restrict__ ckf,
-                                     float* __restrict__ lzlow, int* gate, int* mode) {
-  if (gate && *gate != kModeTensor) return;
-  __shared__ int base;
-  if (threadIdx.x == 0) base = 0;
-  __syncthreads();
+// Block-wide, order-preserving append of the components k < K with sel(k) != 0 to
+// list[*base ..], by warp ballots; entries at or beyond cap are dropped (pos = -1).
+// pos (optional) receives the index relative to `start`.  Returns through *base the
+// uncapped count.  Every thread of the CTA must call it.
+template <typename Sel>
+__device__ void append_list(Sel sel, int K, int* __restrict__ list, int* base, int start, int cap,
+                            int* __restrict__ pos) {
+  __shared__ int wsum[32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   for (int k0 = 0; k0 < K; k0 += blockDim.x) {
     const int k = k0 + threadIdx.x;
-    const int f = (k < K) ? stiff[k] : 0;
-    // block-wide exclusive scan of f by warp ballots (order = component index)
+    const int f = (k < K) ? sel(k) : 0;
     const unsigned m = __ballot_sync(0xffffffffu, f);
-    __shared__ int wsum[32];
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     if (lane == 0) wsum[w] = __popc(m);
     __syncthreads();
-    int off = base;
+    int off = *base;
     for (int i = 0; i < w; ++i) off += wsum[i];
-    if (f) list[off + __popc(m & ((1u << lane) - 1u))] = k;
+    const int at = off + __popc(m & ((1u << lane) - 1u));
+    if (f && at < cap) list[at] = k;
+    if (pos && k < K) pos[k] = (f && at < cap) ? at - start : -1;
     __syncthreads();
     if (threadIdx.x == 0) {
       int t = 0;
       for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += wsum[i];
-      base += t;
+      *base += t;
     }
     __syncthreads();
   }
+}
+
+// One CTA: the stiff components (list[0 .. n_stiff)), then the grey ones that fit
+// (list[n_stiff .. n_stiff + n_grey), at most kMaxStiff in all), the filter constants.
+// More than kMaxStiff stiff components: the side path would cost as much as the
+// CUDA-core path, so the whole step goes there (*mode), and the gated pass is switched
+// off (*gate).  Runs when *gate is tensor (or gate is null).
+__global__ void stiff_compact_kernel(const int* __restrict__ stiff, const int* __restrict__ grey,
+                                     int K, int Kt, int* __restrict__ list,
+                                     int* __restrict__ n_out, int* __restrict__ grey_pos,
+                                     const float* __restrict__ craw, const float* __restrict__ mq,
+                                     const float* __restrict__ peak, float* __restrict__ ckf,
+                                     float* __restrict__ lzlow, int* gate, int* mode) {
+  if (gate && *gate != kModeTensor) return;
+  __shared__ int base, nst;
+  if (threadIdx.x == 0) base = 0;
+  __syncthreads();
+  append_list([&](int k) { return stiff[k]; }, K, list, &base, 0, Kt, nullptr);
+  if (threadIdx.x == 0) nst = base;
+  __syncthreads();
+  const int n_st = nst;
+  append_list([&](int k) { return grey[k] && !stiff[k]; }, K, list, &base, n_st,
+              max(n_st, kMaxStiff), grey_pos);
+  for (int k = K + threadIdx.x; k < Kt; k += blockDim.x) grey_pos[k] = -1;
   if (threadIdx.x == 0) {
-    *n_out = base;
-    if (gate && base > kMaxStiff) {
+    n_out[0] = n_st;
+    n_out[1] = (n_st < kMaxStiff) ? min(base, kMaxStiff) - n_st : 0;
+    if (gate && n_st > kMaxStiff) {
       *mode = kModeSimt;
       *gate = kModeSimt;
     }
   }
+  __syncthreads();
   // Filter constants.  The tensor-core logit of component k at x is exact up to
   // |err| <= kErrRel * sum_j |W'_kj phi_j(x)| (three-product split: 3 * 2^-22 per product;
   // fp32 accumulation over at most 64 steps: 64 * 2^-23; kErrRel carries a factor 2.4 of
@@ -117,7 +137,7 @@ __global__ void stiff_compact_kernel(const int* __restrict__ stiff, int K, int K
   if (threadIdx.x == 0) *lzlow = low;
   for (int k = threadIdx.x; k < Kt; k += blockDim.x) {
     float f = -CUDART_INF_F;
-    if (k < K && stiff[k] && craw[k] > -CUDART_INF_F) {
+    if (k < K && (stiff[k] || grey_pos[k] >= 0) && craw[k] > -CUDART_INF_F) {
       const double M = mq[k];
       const double Q = fmax(2.0 * ((double)peak[k] - (double)low + (double)kCut), 0.0);
       const double E = kErrRel * (1.5 * M + 2.0 * sqrt(M * Q) + 0.5 * Q) + 1.0;
@@ -197,7 +217,7 @@ __global__ void __launch_bounds__(256)
                       const float* __restrict__ logz, double* __restrict__ part, const int* mode) {
   if (mode && *mode != kModeTensor) return;
   const int j = blockIdx.x;
-  if (j >= *n_stiff) return;
+  if (j >= n_stiff[0] + n_stiff[1]) return;   // stiff, then grey components
   __shared__ SideAcc acc[8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = list[j];
@@ -255,12 +275,15 @@ __global__ void __launch_bounds__(256)
 // One CTA per stiff slot j: the kSideParts partial rows, summed in p order, are added to
 // the statistics of component list[j] (slot 0 of the point slices, in the tensor-core
 // layout; the tensor-core sweep added zeros there, the component being masked out of it).
+// A grey component's row goes to grey_stats (its statistics in waiting) instead.
 __global__ void side_reduce_kernel(const double* __restrict__ part, const int* __restrict__ list,
                                    const int* __restrict__ n_stiff, int D, int Dp, int kstride,
-                                   double* __restrict__ stats, const int* mode) {
+                                   double* __restrict__ stats, double* __restrict__ grey_stats,
+                                   const int* mode) {
   if (mode && *mode != kModeTensor) return;
   const int j = blockIdx.x;
-  if (j >= *n_stiff) return;
+  const int ns = n_stiff[0];
+  if (j >= ns + n_stiff[1]) return;
   const size_t row = (size_t)(1 + 2 * Dp);
   const int k = list[j];
   for (int c = threadIdx.x; c < (int)row; c += blockDim.x) {
@@ -268,7 +291,10 @@ __global__ void side_reduce_kernel(const double* __restrict__ part, const int* _
     if (c != 0 && d >= D) continue;
     double s = 0.0;
     for (int p = 0; p < kSideParts; ++p) s += part[((size_t)p * kSideMaxStiff + j) * row + c];
-    stats[stat_idx(true, 0, k, c, kstride, row)] += s;
+    if (j < ns)
+      stats[stat_idx(true, 0, k, c, kstride, row)] += s;
+    else
+      grey_stats[(size_t)(j - ns) * row + c] += s;
   }
 }
 
@@ -276,8 +302,9 @@ __global__ void side_reduce_kernel(const double* __restrict__ part, const int* _
 cudaError_t launch_stiff_compact(const Ctx& c, int* gate, int* mode, cudaStream_t s) {
   prof_begin(c, KI_STIFF_COMPACT, s);
   const Workspace& w = c.ws;
-  stiff_compact_kernel<<<1, 256, 0, s>>>(w.stiff, c.K, w.Kt, w.stiff_list, w.n_stiff, w.tcraw,
-                                         w.tcm, w.tcpk, w.tckf, w.lzlow, gate, mode);
+  stiff_compact_kernel<<<1, 256, 0, s>>>(w.stiff, w.grey, c.K, w.Kt, w.stiff_list, w.n_stiff,
+                                         w.grey_pos, w.tcraw, w.tcm, w.tcpk, w.tckf, w.lzlow,
+                                         gate, mode);
   prof_end(c, KI_STIFF_COMPACT, s);
   return cudaGetLastError();
 }
@@ -324,7 +351,7 @@ cudaError_t launch_side_stats(const Ctx& c, const void* X, int x_dtype, int64_t 
   if (e != cudaSuccess) return e;
   prof_begin(c, KI_SIDE_REDUCE, s, mode, kModeTensor);
   side_reduce_kernel<<<kSideMaxStiff, 256, 0, s>>>(w.side_part, w.stiff_list, w.n_stiff, c.D,
-                                                   w.Dp, w.KpS, w.stats, mode);
+                                                   w.Dp, w.KpS, w.stats, w.grey_stats, mode);
   prof_end(c, KI_SIDE_REDUCE, s);
   return cudaGetLastError();
 }

@@ -432,6 +432,62 @@ __global__ void finish_kernel(int K, int D, int cov, double reg, const double* _
   if (threadIdx.x == 0 && !isfinite(nk)) set_status(status, FGMM_ERR_NUMERIC);
 }
 
+// Fisher vector of the set from exchange-form statistics about the input means:
+//   G_mu_kd = S1_kd / (N sqrt(pi_k) sigma_kd),
+//   G_sigma_kd = (S2_kd / sigma_kd^2 - N_k) / (N sqrt(2 pi_k)),
+// written as [G_mu (K x D), G_sigma (K x D)]; with normalize, sign(z) sqrt(|z|) and the
+// block's fp64 sum of squares for the L2 norm.  One CTA per component.
+__global__ void fisher_kernel(int K, int D, int cov, double n_points, const float* __restrict__ w,
+                              const float* __restrict__ vars, const double* __restrict__ st,
+                              int normalize, float* __restrict__ fv, double* __restrict__ part) {
+  __shared__ double red[kSimtThreads];
+  const int k = blockIdx.x;
+  const size_t orow = (size_t)(1 + 2 * D);
+  const double* o = st + (size_t)k * orow;
+  const double pk = w[k];
+  double sq = 0.0;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    double gm = 0.0, gs = 0.0;
+    if (pk > 0.0) {
+      const double v = (cov == FGMM_COV_DIAG) ? (double)vars[(size_t)k * D + d] : (double)vars[k];
+      gm = o[1 + d] / (n_points * sqrt(pk) * sqrt(v));
+      gs = (o[1 + D + d] / v - o[0]) / (n_points * sqrt(2.0 * pk));
+    }
+    if (normalize) {
+      gm = copysign(sqrt(fabs(gm)), gm);
+      gs = copysign(sqrt(fabs(gs)), gs);
+      sq += gm * gm + gs * gs;
+    }
+    fv[(size_t)k * D + d] = (float)gm;
+    fv[(size_t)K * D + (size_t)k * D + d] = (float)gs;
+  }
+  red[threadIdx.x] = sq;
+  __syncthreads();
+  for (int r = blockDim.x / 2; r > 0; r >>= 1) {
+    if (threadIdx.x < r) red[threadIdx.x] += red[threadIdx.x + r];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) part[k] = red[0];
+}
+
+// L2 normalisation of the Fisher vector: fixed-order sum of the per-component squares.
+__global__ void fisher_norm_kernel(int K, int64_t len, const double* __restrict__ part,
+                                   float* __restrict__ fv) {
+  __shared__ double red[kSimtThreads];
+  double s = 0.0;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) s += part[k];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int r = blockDim.x / 2; r > 0; r >>= 1) {
+    if (threadIdx.x < r) red[threadIdx.x] += red[threadIdx.x + r];
+    __syncthreads();
+  }
+  const double tot = red[0];
+  if (!(tot > 0.0)) return;
+  const float inv = (float)(1.0 / sqrt(tot));
+  for (int64_t i = threadIdx.x; i < len; i += blockDim.x) fv[i] *= inv;
+}
+
 // Sum of n_parts exchange-form statistics vectors, in part order.
 __global__ void stats_sum_kernel(const double* __restrict__ parts, int n_parts, int64_t len,
                                  double* __restrict__ out) {
@@ -550,6 +606,7 @@ __global__ void __launch_bounds__(kSimtThreads)
 // path, whose statistics are centred on each component's current mean.  At the bound
 // the expected error is 3.5e-4, a third of the 1e-3 tolerance.  One CTA per component.
 constexpr double kMaxAmplification = 900.0;
+constexpr double kCheckMinNk = 1.0;      // effective points below which nothing is checked
 
 // Stage 0 (after the first tensor-core pass, gated on *gate == tensor): a failing
 // component becomes stiff (it will be evaluated on the side path) and *redo is set to
@@ -557,16 +614,20 @@ constexpr double kMaxAmplification = 900.0;
 // (after that pass, gated on *gate = the redo word): any remaining failure sends the
 // step to the CUDA-core path (*mode = CUDA cores).
 __global__ void tc_variance_check_kernel(int K, int D, int Dp, int kstride,
-                                         const double* __restrict__ stats, int nslots,
+                                         double* __restrict__ stats, int nslots,
                                          int* __restrict__ stiff, const int* gate, int* redo,
-                                         int* mode, int stage) {
+                                         int* mode, int stage, const int* __restrict__ grey_pos,
+                                         const double* __restrict__ grey_stats) {
   if (*gate != kModeTensor || *mode != kModeTensor) return;
   const int k = blockIdx.x;
   if (stiff[k]) return;  // the side path's statistics are centred on the mean: exact
   const size_t row = (size_t)(1 + 2 * Dp);
   double nk = 0.0;  // tensor-core slot layout (this check runs after tensor-core passes only)
   for (int s = 0; s < nslots; ++s) nk += stats[stat_idx(true, s, k, 0, kstride, row)];
-  if (!(nk >= FGMM_EMPTY_NK)) return;  // empty: parameters are kept, nothing to check
+  // Below one effective point the new mean and variance rest on far-tail
+  // responsibilities and are outside the accuracy contract; the variance is floored
+  // (never negative) whatever the cancellation, so such a component is not checked.
+  if (!(nk >= kCheckMinNk)) return;
   __shared__ int bad_any;
   if (threadIdx.x == 0) bad_any = 0;
   __syncthreads();
@@ -583,7 +644,16 @@ __global__ void tc_variance_check_kernel(int K, int D, int Dp, int kstride,
   }
   if (bad) atomicExch(&bad_any, 1);
   __syncthreads();
-  if (threadIdx.x == 0 && bad_any) {
+  if (!bad_any) return;
+  const int gp = grey_pos[k];
+  if (gp >= 0) {
+    // a grey component: its side-path statistics (centred on the mean, exact) replace
+    // the tensor-core ones in slot 0, the other slots are cleared; no pass is redone
+    for (int c = threadIdx.x; c < (int)row; c += blockDim.x)
+      for (int s = 0; s < nslots; ++s)
+        stats[stat_idx(true, s, k, c, kstride, row)] = (s == 0) ? grey_stats[(size_t)gp * row + c] : 0.0;
+    if (threadIdx.x == 0) stiff[k] = 1;
+  } else if (threadIdx.x == 0) {
     if (stage == 0) {
       stiff[k] = 1;
       atomicExch(redo, kModeTensor);
@@ -703,6 +773,16 @@ cudaError_t launch_finish(const Ctx& c, const double* st, float* weights, float*
   return cudaGetLastError();
 }
 
+cudaError_t launch_fisher(const Ctx& c, const float* weights, const float* vars, double n_points,
+                          const double* st, int normalize, float* fv, cudaStream_t s) {
+  fisher_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, c.cov, n_points, weights, vars, st,
+                                             normalize, fv, c.ws.ll_tiles);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || !normalize) return e;
+  fisher_norm_kernel<<<1, kSimtThreads, 0, s>>>(c.K, (int64_t)2 * c.K * c.D, c.ws.ll_tiles, fv);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_stats_sum(const double* parts, int n_parts, int64_t len, double* out,
                              cudaStream_t s) {
   const int64_t blocks = (len + 255) / 256;
@@ -738,7 +818,8 @@ cudaError_t launch_auto_check(const Ctx& c, int stage, cudaStream_t s) {
   tc_variance_check_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, w.Dp, w.KpS, w.stats,
                                                         tc_slices(c), w.stiff,
                                                         stage == 0 ? w.mode : w.mode2, w.mode2,
-                                                        w.mode, stage);
+                                                        w.mode, stage, w.grey_pos,
+                                                        w.grey_stats);
   prof_end(c, KI_AUTO_CHECK, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

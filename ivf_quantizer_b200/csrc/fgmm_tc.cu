@@ -138,7 +138,7 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
                                __half* __restrict__ wop, float* __restrict__ ck,
                                float* __restrict__ kscale, int* __restrict__ stiff,
                                float* __restrict__ craw, float* __restrict__ mq,
-                               float* __restrict__ peak, int* status) {
+                               float* __restrict__ peak, int* __restrict__ grey, int* status) {
   __shared__ double rs[kSimtThreads], rq[kSimtThreads], rt[kSimtThreads];
   __shared__ float rmax[kSimtThreads], amax[kSimtThreads];
   __shared__ float s_pow;
@@ -187,7 +187,7 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
   if (threadIdx.x == 0) {
     float c = -CUDART_INF_F;
     float pw = 1.f;
-    int is_stiff = 0;
+    int is_stiff = 0, is_grey = 0;
     if (live_k) {
       const float wk = w[k];
       if (!(wk >= 0.f) || !isfinite(wk)) bad = true;
@@ -197,12 +197,16 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
       if (stiff && wk > 0.f)
         is_stiff = !(ldexp(sqrt(rt[0]), -20) <= 1e-3) || !(amax[0] <= 900.f) ||
                    (nk_prev[k] < 4.0);
+      // few points last step: the variance check may fail, so its side-path statistics
+      // are taken as well (AUTO; swapped in instead of redoing the pass)
+      if (stiff && wk > 0.f && !is_stiff) is_grey = nk_prev[k] < kGreyNk;
     }
     craw[k] = c;
     mq[k] = live_k ? (float)rq[0] : 0.f;
     peak[k] = (live_k && w[k] > 0.f) ? (float)(log((double)w[k]) - 0.5 * rs[0]) : -CUDART_INF_F;
     if (stiff) {
       stiff[k] = is_stiff;
+      grey[k] = is_grey;
       if (is_stiff) c = -CUDART_INF_F;
     }
     ck[k] = c;
@@ -1067,12 +1071,15 @@ cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* mean
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (w.Dq > c.D) cudaMemsetAsync(w.center + c.D, 0, (w.Dq - c.D) * sizeof(float), s);
-  if (!auto_mode) cudaMemsetAsync(w.stiff, 0, w.Kt * sizeof(int), s);
+  if (!auto_mode) {
+    cudaMemsetAsync(w.stiff, 0, w.Kt * sizeof(int), s);
+    cudaMemsetAsync(w.grey, 0, w.Kt * sizeof(int), s);
+  }
   prof_begin(c, KI_TC_PREP, s);
   tc_prep_kernel<<<w.Kt, kSimtThreads, 0, s>>>(c.K, c.D, w.Dq, w.Kt, c.cov, weights, means, vars,
                                                w.center, w.dscale, w.nk, w.wop, w.tck, w.tks,
                                                auto_mode ? w.stiff : nullptr, w.tcraw, w.tcm,
-                                               w.tcpk, w.status);
+                                               w.tcpk, w.grey, w.status);
   prof_end(c, KI_TC_PREP, s);
   return cudaGetLastError();
 }

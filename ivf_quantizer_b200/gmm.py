@@ -170,6 +170,29 @@ class GMM:
         return stats_sum(parts)
 
 
+    # ---------------------------------------------------------------- scoring, encoding
+    def score_samples(self, X, weights, means, variances, loglik=None):
+        """Per-point log-density under the mixture (fgmm_score_samples); returns float32
+        [N] on the GPU.  loglik: optional CUDA float64 [1] receiving the sum."""
+        self._check_params(weights, means, variances)
+        xp, dt, n, ldx = _x_args(X)
+        logz = torch.empty(n, dtype=torch.float32, device=X.device)
+        check(LIB.fgmm_score_samples(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means),
+                                     _ptr(variances), _ptr(logz), _ptr(loglik), _stream()),
+              "fgmm_score_samples")
+        return logz
+
+    def fisher_vector(self, X, weights, means, variances, normalize=False):
+        """Fisher-vector encoding of the point set X (fgmm_fisher_vector): float32
+        [2 K D] = [G_mu, G_sigma] on the GPU."""
+        self._check_params(weights, means, variances)
+        xp, dt, n, ldx = _x_args(X)
+        fv = torch.empty(2 * self.K * self.D, dtype=torch.float32, device=X.device)
+        check(LIB.fgmm_fisher_vector(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means),
+                                     _ptr(variances), int(bool(normalize)), _ptr(fv), _stream()),
+              "fgmm_fisher_vector")
+        return fv
+
     # ---------------------------------------------------------------- k-means warm start
     def kmeans_step(self, X, centroids, assign=None, counts=None, inertia=None):
         """One Lloyd iteration (fgmm_kmeans_step); centroids [K, D] float32 CUDA, in/out.
