@@ -119,13 +119,18 @@ def measured_peaks():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the sources that define the tensor-core sweep kernels: recorded ncu
-    traffic is only reported while these are unchanged."""
+    """Hash of the source text of the two tensor-core sweep kernels (the part of
+    fgmm_tc.cu from the sweep-1 section to the end of the sweep-2 section) and of the
+    PTX wrappers they use: recorded ncu traffic is reported only while these match."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ivf_quantizer_b200", "csrc")
-    for f in ("fgmm_tc.cu", "sm100_ptx.cuh"):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+    with open(os.path.join(csrc, "fgmm_tc.cu")) as fh:
+        text = fh.read()
+    a = text.find("// ------------------------------------------------------------------ sweep 1")
+    b = text.find("// ------------------------------------------------------------------ bounded-wait")
+    h.update(text[a:b].encode())
+    with open(os.path.join(csrc, "sm100_ptx.cuh"), "rb") as fh:
+        h.update(fh.read())
     return h.hexdigest()[:16]
 
 
