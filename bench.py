@@ -37,6 +37,8 @@ WORKLOADS = {
     "table1-1e6": dict(gen="table1", N=1_000_000, D=128, K=1024),
     "table1-1e5": dict(gen="table1", N=100_000, D=128, K=1024),
     "c1": dict(gen="c1", N=10_000, D=16, K=16),
+    "ivf-1e7": dict(gen="ivf", N=10_000_000, D=128, K=4096),
+    "border-1e6": dict(gen="border", N=1_000_000, D=960, K=256),
 }
 METRIC = "EM iters/s at N=100M,K=1024,D=128 fp32"
 
@@ -192,8 +194,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
-    ap.add_argument("--mode", default="em", choices=["em", "kmeans"],
-                    help="kmeans: time Lloyd iterations of the warm start instead of EM steps")
+    ap.add_argument("--mode", default="em", choices=["em", "kmeans", "assign"],
+                    help="kmeans: time Lloyd iterations of the warm start; assign: time the "
+                         "top-2 soft assignment (r > 0.1) after the EM steps")
     return ap.parse_args()
 
 
@@ -279,6 +282,60 @@ def run_kmeans(args, w):
     return 0
 
 
+def run_assign(args, w):
+    """fgmm_soft_assign (top_m = 2, r_threshold = 0.1, the IVF multi-assignment) timed on
+    the workload after `warmup` EM steps (rank 0 only).  One step = one assignment of
+    all N points."""
+    import torch
+
+    import ivf_quantizer_b200 as q
+    import synth
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    N, D, K = w["N"], w["D"], w["K"]
+    X = torch.empty(N, D, device="cuda", dtype=torch.float32)
+    synth.generate(w["gen"], N, seed=0, device="cuda", out=X)
+    wt, mu, var = synth.init_params(X, K, seed=0)
+    g = q.GMM(K, D)
+    wd, md, vd = g.new_params(wt, mu, var)
+    for _ in range(args.warmup):
+        g.step(X, wd, md, vd)
+    ids = torch.empty(N, 2, dtype=torch.int32, device="cuda")
+    resp = torch.empty(N, 2, dtype=torch.float32, device="cuda")
+    g.soft_assign(X, wd, md, vd, top_m=2, r_threshold=0.1, ids=ids, resp=resp)
+    torch.cuda.synchronize()
+    g.check_status()
+    sampler = ClockSampler(gpu_id_for(0))
+    sampler.start()
+    time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        g.soft_assign(X, wd, md, vd, top_m=2, r_threshold=0.1, ids=ids, resp=resp)
+    b.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = a.elapsed_time(b) / args.steps
+    peaks, _ = measured_peaks()
+    clk = float(peaks.get("sm_max_mhz", 1965.0))
+    flops = 3.0 * N * K * D                      # subtract, multiply-add per (point, component, dim)
+    peak = 148 * 128 * 2 * clk * 1e6 / 1e12
+    multi = float((ids[:, 1] >= 0).float().mean().item())
+    line = {"metric": f"soft assignments/s ({args.workload}, top_m=2, r>0.1)",
+            "value": N / (ms / 1e3), "unit": "points/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": workload_name(w), "mode": "assign"},
+            "roofline": {"bound": "alu", "kernel": "soft_assign", "unit": "TFLOP/s",
+                         "achieved": flops / (ms / 1e3) / 1e12, "peak": peak,
+                         "frac": flops / (ms / 1e3) / 1e12 / peak,
+                         "peak_note": f"fp32 FMA: 148 SMs x 128 lanes x 2 x {clk:.0f} MHz; "
+                                      f"3 flops per (point, component, dim) counted"},
+            "second_assignment_fraction": multi, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+    g.close()
+    return 0
+
+
 def main():
     args = parse()
     w = WORKLOADS[args.workload]
@@ -286,6 +343,8 @@ def main():
         return run_reference(args, w)
     if args.mode == "kmeans":
         return run_kmeans(args, w)
+    if args.mode == "assign":
+        return run_assign(args, w)
 
     import torch
     import torch.distributed as dist
