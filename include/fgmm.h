@@ -292,6 +292,35 @@ int fgmm_kmeans_seed(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64
                      void* scratch, fgmm_stream_t stream);
 size_t fgmm_kmeans_seed_scratch_bytes(int64_t N);
 
+/* IVF application (the paper, §4): posting lists from the soft-assignment ids and nprobe
+ * search.  Stateless (no handle); device pointers; asynchronous on `stream`.
+ *
+ * fgmm_ivf_build: ids = device int32 [N][top_m] from fgmm_soft_assign (-1 = none); a
+ * vector goes to the list of every cluster it is assigned to (§4.3).  offsets: device
+ * int64[K + 1]; entries: device int64 with room for N * top_m (the list of cluster k is
+ * entries[offsets[k] .. offsets[k+1]), vector indices in increasing order); n_entries:
+ * optional device int64, the total.  scratch: device memory of
+ * fgmm_ivf_build_scratch_bytes(N, K) bytes.  Deterministic.  K * 4 bytes must fit in
+ * shared memory (FGMM_ERR_UNSUPPORTED otherwise).
+ *
+ * fgmm_ivf_search: for each of the nq queries (device float [nq][ldq]) the nprobe
+ * centroids (device float [K][D]) nearest by squared L2, then exact squared L2 to every
+ * entry of their lists (X: device float [N][ldx], the indexed vectors), the topk nearest
+ * distinct vectors (ids into out_ids int64 [nq][topk], -1 padded; distances into out_dist
+ * float [nq][topk], +inf padded), and the entries scanned per query (distance
+ * computations, "DCO") into dco_out (optional int64 [nq]).  Distances are fp32 with
+ * dimensions in increasing order, each subtraction, product and sum rounded
+ * separately; ties go to the lower index (centroid or vector).  1 <= nprobe <= K,
+ * 1 <= topk <= FGMM_IVF_MAX_TOPK. */
+#define FGMM_IVF_MAX_TOPK 32
+size_t fgmm_ivf_build_scratch_bytes(int64_t N, int K);
+int fgmm_ivf_build(int K, const int32_t* ids, int64_t N, int top_m, int64_t* offsets,
+                   int64_t* entries, int64_t* n_entries, void* scratch, fgmm_stream_t stream);
+int fgmm_ivf_search(int K, int D, const float* centroids, const int64_t* offsets,
+                    const int64_t* entries, const float* X, int64_t ldx, const float* Q,
+                    int64_t nq, int64_t ldq, int nprobe, int topk, int64_t* out_ids,
+                    float* out_dist, int64_t* dco_out, fgmm_stream_t stream);
+
 /* Kernel timing, for benchmarks.  When enabled, the library records a CUDA
  * event pair on the call's stream around every kernel it launches and keeps a
  * launch counter; fgmm_profile_read synchronises the device, sums the elapsed

@@ -17,6 +17,7 @@ PREC_FP32, PREC_FP16X3, PREC_FP16, PREC_AUTO = 0, 1, 2, 3
 F32, BF16 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_OOM, ERR_NUMERIC, ERR_TIMEOUT = range(7)
 MAX_TOP_M = 16
+IVF_MAX_TOPK = 32
 STATIC_MAX_KD = 1 << 18
 STATIC_MAX_K = 1 << 14
 EMPTY_NK = 1e-6
@@ -64,6 +65,10 @@ SIGNATURES = {
     "fgmm_stats_sum": (_int, [_vp, _int, _i64, _vp, _vp]),
     "fgmm_score_samples": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_fisher_vector": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _int, _vp, _vp]),
+    "fgmm_ivf_build_scratch_bytes": (_c.c_size_t, [_i64, _int]),
+    "fgmm_ivf_build": (_int, [_int, _vp, _i64, _int, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_ivf_search": (_int, [_int, _int, _vp, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _int, _int,
+                               _vp, _vp, _vp, _vp]),
     "fgmm_kmeans_step": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_kmeans_seed": (_int, [_vp, _vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_kmeans_seed_scratch_bytes": (_c.c_size_t, [_i64]),

@@ -735,6 +735,33 @@ size_t fgmm_kmeans_seed_scratch_bytes(int64_t N) {
   return N > 0 ? kmeans_seed_scratch_bytes(N) : 0;
 }
 
+size_t fgmm_ivf_build_scratch_bytes(int64_t N, int K) {
+  return (N > 0 && K > 0) ? ivf_build_scratch_bytes(N, K) : 0;
+}
+
+int fgmm_ivf_build(int K, const int32_t* ids, int64_t N, int top_m, int64_t* offsets,
+                   int64_t* entries, int64_t* n_entries, void* scratch, fgmm_stream_t stream) {
+  if (K < 1 || N < 1 || top_m < 1 || !ids || !offsets || !entries || !scratch)
+    return FGMM_ERR_INVALID_ARG;
+  if ((size_t)K * sizeof(int) > 227 * 1024) return FGMM_ERR_UNSUPPORTED;
+  return map_cuda(launch_ivf_build(K, ids, N, top_m, offsets, entries, n_entries, scratch,
+                                   (cudaStream_t)stream));
+}
+
+int fgmm_ivf_search(int K, int D, const float* centroids, const int64_t* offsets,
+                    const int64_t* entries, const float* X, int64_t ldx, const float* Q,
+                    int64_t nq, int64_t ldq, int nprobe, int topk, int64_t* out_ids,
+                    float* out_dist, int64_t* dco_out, fgmm_stream_t stream) {
+  if (K < 1 || D < 1 || nq < 0 || ldx < D || ldq < D || nprobe < 1 || nprobe > K ||
+      topk < 1 || topk > FGMM_IVF_MAX_TOPK || !centroids || !offsets || !entries || !X || !Q ||
+      !out_ids || !out_dist)
+    return FGMM_ERR_INVALID_ARG;
+  if (ivf_search_smem(K, D, nprobe, topk) > 227 * 1024) return FGMM_ERR_UNSUPPORTED;
+  if (nq == 0) return FGMM_OK;
+  return map_cuda(launch_ivf_search(K, D, centroids, offsets, entries, X, ldx, Q, nq, ldq, nprobe,
+                                    topk, out_ids, out_dist, dco_out, (cudaStream_t)stream));
+}
+
 const char* fgmm_profile_kernel_name(int index) {
   return (index >= 0 && index < FGMM_PROF_KERNELS) ? kKernelNames[index] : nullptr;
 }

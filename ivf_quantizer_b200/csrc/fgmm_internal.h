@@ -172,6 +172,15 @@ cudaError_t launch_fisher(const Ctx& c, const float* weights, const float* vars,
                           const double* st, int normalize, float* fv, cudaStream_t s);
 cudaError_t launch_stats_sum(const double* parts, int n_parts, int64_t len, double* out,
                              cudaStream_t s);
+// IVF application (fgmm_ivf.cu)
+size_t ivf_build_scratch_bytes(int64_t n, int K);
+cudaError_t launch_ivf_build(int K, const int32_t* ids, int64_t n, int m, int64_t* offsets,
+                             int64_t* entries, int64_t* n_entries, void* scratch, cudaStream_t s);
+size_t ivf_search_smem(int K, int D, int nprobe, int topk);
+cudaError_t launch_ivf_search(int K, int D, const float* C, const int64_t* offsets,
+                              const int64_t* entries, const float* X, int64_t ldx, const float* Q,
+                              int64_t nq, int64_t ldq, int nprobe, int topk, int64_t* out_i,
+                              float* out_d, int64_t* dco, cudaStream_t s);
 // k-means warm start (fgmm_kmeans.cu)
 size_t kmeans_seed_scratch_bytes(int64_t n);
 cudaError_t launch_kmeans_step(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
