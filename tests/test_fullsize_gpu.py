@@ -67,3 +67,54 @@ def test_full_size_step(big_x, prec):
     assert abs(wn.sum() - 1.0) < 1e-5 and np.all(wn >= 0)
     assert torch.isfinite(md).all() and torch.isfinite(vd).all() and bool((vd > 0).all())
     g.close()
+
+
+# ------------------------------------------------------------------ other full-size shapes
+@pytest.mark.parametrize("gen,N,D,K,dtype", [
+    ("ivf", 10_000_000, 128, 4096, torch.float32),       # IVF coarse-quantizer shape
+    ("border", 1_000_000, 960, 256, torch.float32),      # high-dimension shape
+    ("border", 1_000_000, 960, 256, torch.bfloat16),     # ... with bf16 input
+])
+def test_full_size_other_shapes_sampled(gen, N, D, K, dtype):
+    """One AUTO step at the full size of the other benchmark shapes: sampled per-point
+    log-likelihoods against the oracle one by one, the log-likelihood equals the sum of
+    the per-point values, valid parameters, and (IVF shape) the top-2 assignment of the
+    sampled rows where the responsibility gap is decisive."""
+    import ivf_quantizer_b200 as q
+    X = torch.empty(N, D, device="cuda", dtype=torch.float32)
+    synth.generate(gen, N, seed=1, device="cuda", out=X)
+    Xd = X.to(dtype) if dtype != torch.float32 else X
+    w, mu, var = synth.init_params(X, K, seed=1)
+    g = q.GMM(K, D)
+    wd, md, vd = g.new_params(w, mu, var)
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    lz = torch.empty(N, dtype=torch.float32, device="cuda")
+    g.step(Xd, wd, md, vd, loglik=ll, logz=lz)
+    torch.cuda.synchronize()
+    assert g.status() == 0
+    gen_ = torch.Generator().manual_seed(7)
+    rows = torch.cat([torch.randint(0, N, (500,), generator=gen_), torch.tensor([0, N - 1])])
+    xs = Xd[rows.cuda()].float().double().cpu().numpy()
+    L = O.log_joint(xs, w.double().numpy(), mu.double().numpy(), var.double().numpy())
+    ref = O.logsumexp_rows(L)
+    got = lz[rows.cuda()].double().cpu().numpy()
+    assert (np.abs(got - ref) / np.abs(ref)).max() <= 1e-4
+    total = float(lz.double().sum().item())
+    assert abs(total - ll.item()) <= 1e-9 * abs(total)
+    assert torch.isfinite(md).all() and bool((vd > 0).all())
+    if gen == "ivf":
+        ids, resp = g.soft_assign(Xd[rows.cuda()].contiguous(), wd, md, vd, top_m=2,
+                                  r_threshold=0.1)
+        ref_ids, ref_r = O.soft_assign(xs, wd.double().cpu().numpy(), md.double().cpu().numpy(),
+                                       vd.double().cpu().numpy(), top_m=2, r_threshold=0.1)
+        ids = ids.cpu().numpy()
+        # compare where the ranking is decisive (responsibility gaps above 1e-3)
+        Lp = O.log_joint(xs, wd.double().cpu().numpy(), md.double().cpu().numpy(),
+                         vd.double().cpu().numpy())
+        R = np.exp(Lp - O.logsumexp_rows(Lp)[:, None])
+        Rs = -np.sort(-R, axis=1)
+        decisive = (Rs[:, 0] - Rs[:, 1] > 1e-3) & (Rs[:, 1] - Rs[:, 2] > 1e-3) & \
+                   (np.abs(Rs[:, 1] - 0.1) > 1e-3)
+        assert decisive.sum() >= 100
+        np.testing.assert_array_equal(ids[decisive], ref_ids[decisive])
+    g.close()
