@@ -93,23 +93,45 @@ __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, i
   for (int j = 0; j < 4; ++j)
 #pragma unroll
     for (int q = 0; q < NQ; ++q) dacc[j][q] = 0.0;
+  // the next feature chunk is fetched into registers while the current one is used
+  constexpr int XPT = kTP * kDC / kSimtThreads, MPT = KBLK * kDC / kSimtThreads;
+  float xr[XPT], mr[MPT], pr[MPT];
+  auto fetch = [&](int d0) {
+#pragma unroll
+    for (int u = 0; u < XPT; ++u) {
+      const int e = threadIdx.x + u * kSimtThreads;
+      const int r = e / kDC, cx = e % kDC;
+      const int64_t i = i0 + r;
+      const int d = d0 + cx;
+      xr[u] = (i < n && d < D) ? ld_x(X + i * ldx + d) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < MPT; ++u) {
+      const int e = threadIdx.x + u * kSimtThreads;
+      const int r = e / kDC, cx = e % kDC;
+      mr[u] = mu[(size_t)(kb + r) * Dp + d0 + cx];
+      pr[u] = prec[(size_t)(kb + r) * Dp + d0 + cx];
+    }
+  };
+  fetch(0);
   for (int d0 = 0; d0 < Dp; d0 += kDC) {
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
       for (int q = 0; q < NQ; ++q) acc[j][q] = 0.f;
-    for (int e = threadIdx.x; e < kTP * kDC; e += kSimtThreads) {
-      const int r = e / kDC, cx = e % kDC;
-      const int64_t i = i0 + r;
-      const int d = d0 + cx;
-      xs[r][cx] = (i < n && d < D) ? ld_x(X + i * ldx + d) : 0.f;
+#pragma unroll
+    for (int u = 0; u < XPT; ++u) {
+      const int e = threadIdx.x + u * kSimtThreads;
+      xs[e / kDC][e % kDC] = xr[u];
     }
-    for (int e = threadIdx.x; e < KBLK * kDC; e += kSimtThreads) {
-      const int r = e / kDC, cx = e % kDC;
-      ms[r][cx] = mu[(size_t)(kb + r) * Dp + d0 + cx];
-      ps[r][cx] = prec[(size_t)(kb + r) * Dp + d0 + cx];
+#pragma unroll
+    for (int u = 0; u < MPT; ++u) {
+      const int e = threadIdx.x + u * kSimtThreads;
+      ms[e / kDC][e % kDC] = mr[u];
+      ps[e / kDC][e % kDC] = pr[u];
     }
     __syncthreads();
+    if (d0 + kDC < Dp) fetch(d0 + kDC);
 #pragma unroll 2
     for (int d = 0; d < kDC; d += 4) {
       float4 xv[4], mv[NQ], pv[NQ];
@@ -148,7 +170,7 @@ __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, i
 // (Alg. 1, step 1).  Writes log Z_i for the chunk, optionally to the caller's
 // per-point buffer, and one fp64 partial log-likelihood per tile.
 template <typename T>
-__global__ void __launch_bounds__(kSimtThreads)
+__global__ void __launch_bounds__(kSimtThreads, 2)
     lse_simt_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp, int Kp,
                     const float* __restrict__ mu, const float* __restrict__ prec,
                     const float* __restrict__ cconst, float* __restrict__ logz,
@@ -531,7 +553,7 @@ __global__ void finalize_kernel(int K, const double* __restrict__ nk, const doub
 // log-sum-exp and a running top-m of log z (ranking by log z equals ranking by r,
 // exp being monotone), ties kept in component order.  Epilogue per §4.3.
 template <typename T>
-__global__ void __launch_bounds__(kSimtThreads)
+__global__ void __launch_bounds__(kSimtThreads, 2)
     soft_assign_simt_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp, int Kp,
                             int K, const float* __restrict__ mu, const float* __restrict__ prec,
                             const float* __restrict__ cconst, int top_m, float thr,
