@@ -192,6 +192,8 @@ def parse():
     ap.add_argument("--workload", default="table1-1e8", choices=sorted(WORKLOADS))
     ap.add_argument("--prec", default="auto", choices=["auto", "fp32", "fp16x3"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-block-skip", action="store_true",
+                    help="dense statistics sweep on the tensor cores (fgmm_set_block_skip 0)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--mode", default="em", choices=["em", "kmeans", "assign"],
@@ -378,6 +380,7 @@ def main():
     except q.FgmmError:
         g.set_precision(q.PREC_FP32)
     prec_set = {q.PREC_FP32: "fp32", q.PREC_FP16X3: "fp16x3", q.PREC_AUTO: "auto"}[g.precision]
+    g.set_block_skip(not args.no_block_skip)
     wd, md, vd = g.new_params(wt, mu, var)
     if world > 1:
         for t in (wd, md, vd):
@@ -534,7 +537,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": workload_name(w), "precision": prec_used,
-                       "precision_setting": prec_set,
+                       "precision_setting": prec_set, "block_skip": g.block_skip,
                        "l2": f"inputs larger than L2 (X = {N * D * 4 / 1e9:.1f} GB per GPU)"
                        if N * D * 4 > 126e6 else "inputs smaller than L2",
                        "parallelism": (f"dp{world}: row shards of one mixture fit, one all-gather "

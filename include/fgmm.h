@@ -96,6 +96,20 @@ int fgmm_destroy(fgmm_handle h);
 int fgmm_set_precision(fgmm_handle h, int prec);
 int fgmm_get_precision(fgmm_handle h, int* prec_out);
 
+/* Block skipping in the tensor-core statistics sweep (on by default).
+ * Paper: "Flash-GMM", §3.1 and Algorithm 1.  Sweep 2 forms r_ik = exp(log z_ik - log Z_i)
+ * for all i, k and adds them into the statistics.  The tensor-core path keeps r as
+ * fp16(r 2^15), which is exactly 0 once log z_ik < log Z_i - 27.7.  With skipping on,
+ * sweep 1 marks for each point the 128-component blocks that come within 30 nats of
+ * log Z_i.  Sweep 2 then visits the points grouped by those marks, and only the
+ * (128-point tile, block) pairs that hold a mark; every pair it leaves out adds
+ * exactly 0.  Results match the dense sweep up to the order of fp32 additions and stay
+ * bitwise reproducible from run to run.  Only K of 129 ... 4096 is affected (2 to 32
+ * blocks); the CUDA-core path never is.
+ * enable: 0 off, nonzero on.  FGMM_ERR_INVALID_ARG for a NULL handle. */
+int fgmm_set_block_skip(fgmm_handle h, int enable);
+int fgmm_get_block_skip(fgmm_handle h, int* enable_out);
+
 /* Path the last fgmm_em_step of this handle ran: FGMM_PREC_FP32 (CUDA cores) or
  * FGMM_PREC_FP16X3 (tensor cores).  Under FGMM_PREC_AUTO the choice is made on the
  * device per step, so this call synchronises the device.  -1 before any step. */
@@ -331,7 +345,7 @@ int fgmm_ivf_search(int K, int D, const float* centroids, const int64_t* offsets
  * memory), so that launches which did work are counted apart ("active").
  * Disabled by default; costs two event records per launch, and one 4-byte copy
  * per gated launch, when enabled. */
-#define FGMM_PROF_KERNELS 23
+#define FGMM_PROF_KERNELS 25
 typedef struct fgmm_profile {
   int64_t launches;          /* kernels launched while enabled (all kinds) */
   int64_t sweep1_launches;   /* log-sum-exp sweep (first pass over the components) */

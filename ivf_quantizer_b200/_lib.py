@@ -23,7 +23,7 @@ STATIC_MAX_K = 1 << 14
 EMPTY_NK = 1e-6
 CHUNK_POINTS = 1 << 20
 
-PROF_KERNELS = 23
+PROF_KERNELS = 25
 
 
 class Profile(ctypes.Structure):
@@ -45,6 +45,8 @@ SIGNATURES = {
     "fgmm_destroy": (_int, [_vp]),
     "fgmm_set_precision": (_int, [_vp, _int]),
     "fgmm_get_precision": (_int, [_vp, _c.POINTER(_int)]),
+    "fgmm_set_block_skip": (_int, [_vp, _int]),
+    "fgmm_get_block_skip": (_int, [_vp, _c.POINTER(_int)]),
     "fgmm_workspace_bytes": (_int, [_vp, _c.POINTER(_c.c_size_t)]),
     "fgmm_last_step_path": (_int, [_vp, _c.POINTER(_int)]),
     "fgmm_em_step": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),

@@ -106,7 +106,7 @@ const char* const kKernelNames[fgmm::KI_COUNT] = {
     "prep_simt",   "lse_simt",  "ll_accumulate", "stats_simt",   "reduce_stats", "mstep",
     "finalize",    "soft_assign", "auto_check", "redo_reset",    "remask",
     "stiff_compact", "side_lse", "ll_partials", "side_stats",    "side_reduce",
-    "km_assign",   "km_seed_update"};
+    "km_assign",   "km_seed_update", "tc_order", "tc_gather"};
 static_assert(fgmm::KI_COUNT == FGMM_PROF_KERNELS, "kernel table and public arrays differ");
 }  // namespace
 
@@ -155,7 +155,8 @@ void free_ws(Workspace& w) {
                   w.stats,  w.nk,     w.status, w.center, w.dscale, w.wop,
                   w.tck,    w.tks,    w.xop,    w.mode, w.stiff,    w.stiff_list, w.n_stiff,
                   w.side_part, w.mode2, w.canon, w.tcraw, w.tcm, w.tcpk, w.tckf, w.lzlow,
-                  w.side_flag, w.km_word, w.grey, w.grey_pos, w.grey_stats};
+                  w.side_flag, w.km_word, w.grey, w.grey_pos, w.grey_stats,
+                  w.bmask, w.perm, w.lzp, w.ord_hist, w.tmask, w.tlist, w.tcnt};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -232,6 +233,16 @@ cudaError_t alloc_ws(Ctx& c) {
     if ((e = alloc(&w.side_flag, (size_t)kChunk, &t)) != cudaSuccess) return e;
     if ((e = cudaMemset(w.side_flag, 0, (size_t)kChunk)) != cudaSuccess) return e;
     if ((e = alloc(&w.xop, (size_t)2 * kChunk * w.K1, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.bmask, (size_t)kChunk, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.perm, (size_t)kChunk, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.lzp, (size_t)kChunk, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.ord_hist, (size_t)(kChunk / kOrdPts) * (kSkipMaxBlocks + 1), &t)) !=
+        cudaSuccess)
+      return e;
+    if ((e = alloc(&w.tmask, (size_t)(kChunk / 128), &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.tlist, (size_t)kSkipMaxBlocks * (kChunk / 128), &t)) != cudaSuccess)
+      return e;
+    if ((e = alloc(&w.tcnt, (size_t)kSkipMaxBlocks, &t)) != cudaSuccess) return e;
     // rows past the end of a short chunk are read by the tensor cores (and multiplied
     // by r = 0): keep them finite from the start
     if ((e = cudaMemset(w.xop, 0, (size_t)2 * kChunk * w.K1 * sizeof(__half))) != cudaSuccess)
@@ -320,6 +331,18 @@ int fgmm_set_precision(fgmm_handle h, int prec) {
 int fgmm_get_precision(fgmm_handle h, int* prec_out) {
   if (!h || !prec_out) return FGMM_ERR_INVALID_ARG;
   *prec_out = h->c.prec;
+  return FGMM_OK;
+}
+
+int fgmm_set_block_skip(fgmm_handle h, int enable) {
+  if (!h) return FGMM_ERR_INVALID_ARG;
+  h->c.skip = enable != 0;
+  return FGMM_OK;
+}
+
+int fgmm_get_block_skip(fgmm_handle h, int* enable_out) {
+  if (!h || !enable_out) return FGMM_ERR_INVALID_ARG;
+  *enable_out = h->c.skip ? 1 : 0;
   return FGMM_OK;
 }
 
@@ -428,12 +451,15 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       int64_t ldc;
       const int b = acquire(c0, nc, &Xc, &ldc);
       float* lzo = logz_out ? logz_out + c0 : nullptr;
-      if ((r = launch_tc_convert(c, Xc, x_dtype, nc, ldc, gate, s)) == cudaSuccess &&
+      if ((r = launch_tc_convert(c, Xc, x_dtype, nc, ldc, nullptr, gate, s)) == cudaSuccess &&
           (r = launch_tc_lse(c, nc, lzo, gate, s)) == cudaSuccess &&
           // stiff components (AUTO) join log Z here; then the chunk's log-likelihood
           (r = launch_side_lse(c, Xc, x_dtype, nc, ldc, lzo, gate, s)) == cudaSuccess &&
           (r = launch_ll_accumulate(c, nc, gate, fixed_mode, kModeTensor, s)) == cudaSuccess &&
-          want_stats && (r = launch_tc_stats(c, nc, gate, s)) == cudaSuccess)
+          want_stats &&
+          // block skipping: sweep 2 runs on phi rewritten in the order of the block masks
+          (!tc_skip(c) || (r = launch_tc_order(c, Xc, x_dtype, nc, ldc, gate, s)) == cudaSuccess) &&
+          (r = launch_tc_stats(c, nc, gate, s)) == cudaSuccess)
         r = launch_side_stats(c, Xc, x_dtype, nc, ldc, gate, s);
       release(b);
       if (r == cudaSuccess) r = copy_err;

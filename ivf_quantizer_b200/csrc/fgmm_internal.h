@@ -31,6 +31,15 @@ constexpr int kSideParts = 64;       // AUTO side path: point ranges per chunk
 constexpr float kSideCut = 40.f;
 // AUTO: a component with fewer effective points than this in the previous step is grey
 constexpr double kGreyNk = 8.0;
+// Block skipping in the tensor-core statistics sweep.  That sweep stores r as
+// fp16(r 2^15), which is exactly 0 for r <= 2^-40, i.e. for a log-density 27.7 nats or
+// more below log Z.  A (point tile, 128-component block) pair in which every point has
+// every log-density of the block more than kSkipCut nats below its log Z therefore adds
+// exactly nothing to N_k, S1, S2, and is left out.  The 2.3-nat margin covers the two
+// sweeps' rounding differences (about 1e-4 nats) many times over.
+constexpr float kSkipCut = 30.f;
+constexpr int kSkipMaxBlocks = 32;   // block masks are 32-bit words: K <= 4096
+constexpr int kOrdPts = 4096;        // points per CTA of the counting sort
 
 static inline int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
@@ -73,6 +82,14 @@ struct Workspace {
   float* lzlow = nullptr;   // [1] log Z below which a point is always flagged
   uint8_t* side_flag = nullptr;  // [kChunk] 1: the point may have a stiff component within kCut
   __half* xop = nullptr;    // [2][kChunk][K1] phi(x) hi / lo of the current chunk
+  // block skipping (sweep 2 visits only the (tile, block) pairs that can contribute)
+  uint32_t* bmask = nullptr;  // [kChunk] per point: blocks within kSkipCut of log Z
+  int* perm = nullptr;        // [kChunk] sweep-2 order: row j of phi is point perm[j]
+  float* lzp = nullptr;       // [kChunk] log Z in sweep-2 order
+  int* ord_hist = nullptr;    // [kChunk / kOrdPts][kSkipMaxBlocks + 1] counts, then offsets
+  uint32_t* tmask = nullptr;  // [kChunk / 128] per sweep-2 tile: OR of its points' masks
+  int* tlist = nullptr;       // [kSkipMaxBlocks][kChunk / 128] active tiles of each block
+  int* tcnt = nullptr;        // [kSkipMaxBlocks] their number
   int* mode = nullptr;      // [1] path of the current step: 0 tensor cores, 1 CUDA cores
   int* mode2 = nullptr;     // [1] AUTO: tensor when the hybrid redo pass must run
   int* stiff = nullptr;     // [Kt] AUTO: 1 = component handled by the CUDA-core side path
@@ -109,7 +126,7 @@ enum KernelId {
   KI_FINALIZE,
   KI_SOFT_ASSIGN, KI_AUTO_CHECK, KI_REDO_RESET, KI_REMASK,
   KI_STIFF_COMPACT, KI_SIDE_LSE, KI_LL_PARTIALS, KI_SIDE_STATS, KI_SIDE_REDUCE,
-  KI_KM_ASSIGN, KI_KM_SEED,
+  KI_KM_ASSIGN, KI_KM_SEED, KI_TC_ORDER, KI_TC_GATHER,
   KI_COUNT
 };
 
@@ -130,13 +147,13 @@ struct Ctx {
   Profiler* prof = nullptr;
   int last_path = -1;      // FGMM_PREC_FP32 / FGMM_PREC_FP16X3, or -1
   bool last_auto = false;  // last step decided its path on the device
+  bool skip = true;        // block skipping in the tensor-core statistics sweep
 };
 
 // Path codes stored in Workspace::mode.
 constexpr int kModeTensor = 0;
 constexpr int kModeSimt = 1;
 
-// Brackets one kernel launch with profiling events when profiling is enabled.
 // Brackets one launch with events when profiling is enabled.  A launch whose kernel
 // returns at once unless *gate == required passes gate (else nullptr): the profiler then
 // snapshots the word in stream order, so that it can tell launches that did work from
@@ -201,10 +218,17 @@ cudaError_t launch_side_lse(const Ctx& c, const void* X, int x_dtype, int64_t n,
                             float* logz_out, const int* mode, cudaStream_t s);
 cudaError_t launch_side_stats(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
                               const int* mode, cudaStream_t s);
+// perm: nullptr for the natural order, else row j of phi is point perm[j] of the chunk
 cudaError_t launch_tc_convert(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
-                              const int* mode, cudaStream_t s);
+                              const int* perm, const int* mode, cudaStream_t s);
+// block skipping applies to this handle's tensor-core sweeps
+bool tc_skip(const Ctx& c);
 cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* mode,
                           cudaStream_t s);
+// block skipping (fgmm_order.cu): sweep-2 order from sweep 1's block masks, phi and
+// log Z rewritten in that order, and the active tiles of every component block
+cudaError_t launch_tc_order(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                            const int* mode, cudaStream_t s);
 cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream_t s);
 cudaError_t run_bounded_wait_probe(int64_t limit_ns, int* status_host);
 // soft assignment on caller-provided scratch (allocation-free entry point)

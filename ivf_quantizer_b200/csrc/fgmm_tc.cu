@@ -238,18 +238,19 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
 
 // ------------------------------------------------------------------ X -> phi (fp16 hi / lo)
 // Thread per (point, group of 8 dims).  xop[part][i][j]: part 0 hi, 1 lo; j < Dq the
-// scaled centred coordinate, Dq + d its square.
+// scaled centred coordinate, Dq + d its square.  With perm, row i holds point perm[i].
 template <typename T>
 __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dq,
                                   int64_t ncmax, const float* __restrict__ center,
                                   const float* __restrict__ scale, __half* __restrict__ xop,
-                                  const int* mode) {
+                                  const int* __restrict__ perm, const int* mode) {
   if (mode && *mode != 0) return;
   const int groups = Dq / 8;
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= n * groups) return;
   const int64_t i = e / groups;
   const int g = (int)(e % groups);
+  const int64_t src = perm ? (int64_t)__ldg(perm + i) : i;
   const int K1 = 2 * Dq;
   __align__(16) __half xh[8], xl[8], qh[8], ql[8];
 #pragma unroll
@@ -258,8 +259,8 @@ __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ld
     float xv = 0.f;
     if (d < D) {
       float x;
-      if constexpr (sizeof(T) == 4) x = __ldg(reinterpret_cast<const float*>(X) + i * ldx + d);
-      else x = __bfloat162float(X[i * ldx + d]);
+      if constexpr (sizeof(T) == 4) x = __ldg(reinterpret_cast<const float*>(X) + src * ldx + d);
+      else x = __bfloat162float(X[src * ldx + d]);
       xv = (x - center[d]) * scale[d];
     }
     split16(xv, xh[u], xl[u]);
@@ -299,7 +300,22 @@ struct LseBars {
   float xm[2][3][BM];   // (max, sum, filter max) of column groups 1..3, per tile buffer
   float xs[2][3][BM];
   float xf[2][3][BM];
+  uint2 xk[2][3][BM];   // candidate blocks of column groups 1..3 (block skipping)
+  float xo[2][3][BM];   // their largest block maximum left out of the candidates
 };
+
+// Block skipping, sweep 1 side.  Every epilogue thread keeps, for its row and its 32
+// columns, the (at most kCand) largest block maxima that lie within the cut of its
+// running maximum; a block that falls out of range can never come back, the maximum
+// only grows.  A block pushed out of a full list leaves its maximum in `ovm`; if that
+// is within the cut of log Z in the end, the row is marked dense (every block).  At the
+// end of a tile the column groups 1..3 hand their candidates to group 0 as 16-bit codes
+// (block << 8 | q, q = floor((max - block max) / step)); decoding gives max - q step >=
+// the true block maximum, so the test against log Z - cut can only keep a block.
+constexpr int kCand = 4;
+constexpr float kCut2 = kSkipCut * kLog2e;       // the cut in log2 units
+constexpr float kQStep = kCut2 / 255.f;
+constexpr uint32_t kCodeEmpty = 0xFFFFu;
 
 template <int NKC>
 __global__ void __launch_bounds__(kLseThreads, 1)
@@ -309,7 +325,7 @@ __global__ void __launch_bounds__(kLseThreads, 1)
                   float* __restrict__ logz_out,
                   const __half* __restrict__ xop, const float* __restrict__ ckf,
                   const float* __restrict__ lzlow, uint8_t* __restrict__ side_flag,
-                  const int* mode, int* status) {
+                  uint32_t* __restrict__ bmask, const int* mode, int* status) {
   if (mode && *mode != kModeTensor) return;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -476,6 +492,11 @@ __global__ void __launch_bounds__(kLseThreads, 1)
       if (t + (int)gridDim.x < ntiles) put_xlo(t + gridDim.x, (jt + 1) & 1);
       float m = -CUDART_INF_F, s = 0.f;   // in log2 units
       float fm = -CUDART_INF_F;            // max over stiff components of estimate + E_k
+      float cbm[kCand];                    // candidate blocks: block maximum (-inf: free)
+      int cid[kCand];                      //                   block index
+      float ovm = -CUDART_INF_F;           // largest block maximum pushed out of the list
+#pragma unroll
+      for (int e = 0; e < kCand; ++e) { cbm[e] = -CUDART_INF_F; cid[e] = 0; }
       for (int kb = 0; kb < nkb; ++kb, ++its) {
         const int b = its & 1;
         if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full[b], (its >> 1) & 1, abort))) {
@@ -527,6 +548,28 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             s = s * exp2f(m - nm) + acc;
             m = nm;
           }
+          if (bmask) {
+            const float thr = m - kCut2;
+#pragma unroll
+            for (int e = 0; e < kCand; ++e)
+              if (cbm[e] <= thr) cbm[e] = -CUDART_INF_F;
+            if (bm > thr) {
+              int slot = -1, mi = 0;
+              float mn = CUDART_INF_F;
+#pragma unroll
+              for (int e = 0; e < kCand; ++e) {
+                if (slot < 0 && cbm[e] == -CUDART_INF_F) slot = e;
+                if (cbm[e] < mn) { mn = cbm[e]; mi = e; }
+              }
+              if (slot < 0) {            // full: the smaller of bm and the list's least goes
+                if (bm > mn) { ovm = fmaxf(ovm, mn); slot = mi; }
+                else ovm = fmaxf(ovm, bm);
+              }
+#pragma unroll
+              for (int e = 0; e < kCand; ++e)
+                if (e == slot) { cbm[e] = bm; cid[e] = kb; }
+            }
+          }
         }
         ptx::tc_fence_before();
         __syncwarp();
@@ -545,6 +588,20 @@ __global__ void __launch_bounds__(kLseThreads, 1)
         bars->xm[xb][g - 1][r] = m;
         bars->xs[xb][g - 1][r] = s;
         bars->xf[xb][g - 1][r] = fm;
+        if (bmask) {
+          uint32_t code[kCand];
+#pragma unroll
+          for (int e = 0; e < kCand; ++e) {
+            code[e] = kCodeEmpty;
+            const float dl = m - cbm[e];   // < cut for a live entry (else it is below the cut)
+            if (cbm[e] > -CUDART_INF_F && dl < kCut2) {
+              const int qd = min(254, (int)floorf(dl * (1.f / kQStep)));
+              code[e] = ((uint32_t)cid[e] << 8) | (uint32_t)qd;
+            }
+          }
+          bars->xk[xb][g - 1][r] = make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
+          bars->xo[xb][g - 1][r] = ovm;
+        }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&bars->xc_full[xb]);
       } else {
@@ -555,11 +612,17 @@ __global__ void __launch_bounds__(kLseThreads, 1)
         }
         float mq[4] = {m, 0.f, 0.f, 0.f}, sq[4] = {s, 0.f, 0.f, 0.f};
         float f2 = fm;
+        uint2 kq[3];
+        float ov = ovm;
 #pragma unroll
         for (int o = 0; o < 3; ++o) {
           mq[o + 1] = bars->xm[xb][o][r];
           sq[o + 1] = bars->xs[xb][o][r];
           f2 = fmaxf(f2, bars->xf[xb][o][r]);
+          if (bmask) {
+            kq[o] = bars->xk[xb][o][r];
+            ov = fmaxf(ov, bars->xo[xb][o][r]);
+          }
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&bars->xc_empty[xb]);
@@ -576,6 +639,25 @@ __global__ void __launch_bounds__(kLseThreads, 1)
           if (logz_out) logz_out[i] = lz;
           // may a stiff component come within kSideCut nats of log Z here?
           side_flag[i] = (f2 > lz2 - kSideCut * kLog2e) || !(lz >= *lzlow);
+          if (bmask) {
+            const float lim = lz2 - kCut2;
+            uint32_t mk = 0;
+            bool dense = ov > lim || !(lz2 > -CUDART_INF_F);
+#pragma unroll
+            for (int e = 0; e < kCand; ++e)
+              if (cbm[e] > lim) mk |= 1u << cid[e];
+#pragma unroll
+            for (int o = 0; o < 3; ++o) {
+              const uint32_t w2[2] = {kq[o].x, kq[o].y};
+#pragma unroll
+              for (int e = 0; e < kCand; ++e) {
+                const uint32_t cd = (w2[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                if (cd != kCodeEmpty && mq[o + 1] - (float)(cd & 255u) * kQStep > lim)
+                  mk |= 1u << (cd >> 8);
+              }
+            }
+            bmask[i] = dense ? (nkb >= 32 ? 0xFFFFFFFFu : (1u << nkb) - 1u) : mk;
+          }
         }
       }
     }
@@ -617,7 +699,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     int nc, int ncmax, int Kt, int slice_len, int flush_tiles,
                     const float* __restrict__ ck, const float* __restrict__ kscale,
                     const float* __restrict__ logz, double* __restrict__ stats, int kstride,
-                    int Dp, const __half* __restrict__ wop, const int* mode, int* status) {
+                    int Dp, const __half* __restrict__ wop, const int* __restrict__ tlist,
+                    const int* __restrict__ tcnt, int tl_stride, const int* mode, int* status) {
   if (mode && *mode != kModeTensor) return;
   constexpr int Dq = NKC * 32;            // features: phi has 2 Dq = NKC * 64 entries
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -630,10 +713,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb = blockIdx.x;
-  const int p0 = blockIdx.y * slice_len;
-  const int p1 = min(nc, p0 + slice_len);
-  const int ntl = (p1 > p0) ? (p1 - p0 + BM - 1) / BM : 0;
+  // The CTA's point tiles: a contiguous slice of the chunk, or (block skipping) an even
+  // share of the block's list of active tiles, tiles of 128 rows of the reordered phi.
+  int p0, p1, ntl, l0 = 0;
+  if (tlist) {
+    const int na = tcnt[kb];
+    const int per = (na + (int)gridDim.y - 1) / (int)gridDim.y;
+    l0 = min(na, (int)blockIdx.y * per);
+    ntl = min(na, l0 + per) - l0;
+    p0 = 0;
+    p1 = nc;
+    tlist += (size_t)kb * tl_stride + l0;
+  } else {
+    p0 = blockIdx.y * slice_len;
+    p1 = min(nc, p0 + slice_len);
+    ntl = (p1 > p0) ? (p1 - p0 + BM - 1) / BM : 0;
+  }
   if (ntl == 0) return;  // uniform over the CTA, before any barrier or TMEM use
+  // first row of the CTA's tile j
+  auto tile_row = [&](int j) -> int { return tlist ? __ldg(tlist + j) * BM : p0 + j * BM; };
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bars->w_full, 1);
@@ -684,7 +782,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           int tile;
           if (which == 0) { if (g >= ntl) continue; tile = g; }
           else { if (g == 0) continue; tile = g - 1; }
-          const int row0 = p0 + tile * BM;
+          const int row0 = tile_row(tile);
           if (which == 0) {  // log Z of the tile's points, for the epilogue
             const int lb = tile & 1;
             if (tile >= 2 &&
@@ -848,7 +946,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) ptx::mbar_arrive(&bars->wlo_ready);
     }
     for (int tile = 0; tile < ntl && !*abort; ++tile) {
-      const int row0 = p0 + tile * BM;
+      const int row0 = tile_row(tile);
       const int b = tile & 1;
       const int nvalid = p1 - row0;            // points of this tile inside the slice
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full, tile & 1, abort)))
@@ -1085,19 +1183,25 @@ cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* mean
 }
 
 cudaError_t launch_tc_convert(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
-                              const int* mode, cudaStream_t s) {
+                              const int* perm, const int* mode, cudaStream_t s) {
   const Workspace& w = c.ws;
   const int64_t total = n * (w.Dq / 8);
   const unsigned grid = (unsigned)ceil_div64(total, 256);
-  prof_begin(c, KI_TC_CONVERT, s, mode, kModeTensor);
+  const KernelId id = perm ? KI_TC_GATHER : KI_TC_CONVERT;
+  prof_begin(c, id, s, mode, kModeTensor);
   if (x_dtype == FGMM_BF16)
     tc_convert_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dq, kChunk,
-                                           w.center, w.dscale, w.xop, mode);
+                                           w.center, w.dscale, w.xop, perm, mode);
   else
     tc_convert_kernel<<<grid, 256, 0, s>>>((const float*)X, n, ldx, c.D, w.Dq, kChunk, w.center,
-                                           w.dscale, w.xop, mode);
-  prof_end(c, KI_TC_CONVERT, s);
+                                           w.dscale, w.xop, perm, mode);
+  prof_end(c, id, s);
   return cudaGetLastError();
+}
+
+bool tc_skip(const Ctx& c) {
+  const int nkb = c.ws.Kt / BKc;
+  return c.skip && c.tc.ready && c.ws.bmask && nkb >= 2 && nkb <= kSkipMaxBlocks;
 }
 
 cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* mode,
@@ -1115,8 +1219,9 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
   case N_:                                                                                    \
     tc_lse_kernel<N_><<<grid, kLseThreads, smem, s>>>(tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, \
                                                      w.tks, params ? 1 : 0, w.logz, logz_out,   \
-                                                     w.xop, w.tckf, w.lzlow,                  \
-                                                     w.side_flag, mode, w.status);            \
+                                                     w.xop, w.tckf, w.lzlow, w.side_flag,     \
+                                                     tc_skip(c) ? w.bmask : nullptr, mode,    \
+                                                     w.status);                               \
     break;
   switch (nkc) {
     LSE_CASE(1)
@@ -1146,14 +1251,17 @@ cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream
   const CUtensorMap& tx = c.tc.tmap_x;
   const CUtensorMap& tw = c.tc.tmap_w;
   const int flush_tiles = 8;  // fp32 runs of 1024 points (64 MMA steps) between fp64 flushes
+  // block skipping: phi and log Z were rewritten in sweep-2 order, tiles come from lists
+  const bool skip = tc_skip(c);
+  const float* lz = skip ? w.lzp : w.logz;
+  const int* tl = skip ? w.tlist : nullptr;
+  const int tl_stride = (int)(kChunk / BM);
   prof_begin(c, KI_TC_STATS, s, mode, kModeTensor);
 #define STATS_CASE(N_)                                                                         \
   case N_:                                                                                     \
-    tc_stats_kernel<N_><<<grid, kTcThreads, stats_smem(N_), s>>>(tx, tw, (int)n, (int)kChunk, \
-                                                                 w.Kt,                        \
-                                                          slice, flush_tiles, w.tck, w.tks,    \
-                                                          w.logz, w.stats, w.KpS, w.Dp, w.wop, \
-                                                          mode, w.status);                     \
+    tc_stats_kernel<N_><<<grid, kTcThreads, stats_smem(N_), s>>>(                              \
+        tx, tw, (int)n, (int)kChunk, w.Kt, slice, flush_tiles, w.tck, w.tks, lz, w.stats,      \
+        w.KpS, w.Dp, w.wop, tl, w.tcnt, tl_stride, mode, w.status);                            \
     break;
   switch (nkc) {
     STATS_CASE(1)

@@ -75,6 +75,17 @@ class GMM:
         check(LIB.fgmm_get_precision(self._h, ctypes.byref(v)), "fgmm_get_precision")
         return v.value
 
+    def set_block_skip(self, enable: bool):
+        """Skip (tile, block) pairs of the tensor-core statistics sweep whose
+        responsibilities are all zero at fp16 resolution (fgmm_set_block_skip)."""
+        check(LIB.fgmm_set_block_skip(self._h, 1 if enable else 0), "fgmm_set_block_skip")
+
+    @property
+    def block_skip(self) -> bool:
+        v = ctypes.c_int()
+        check(LIB.fgmm_get_block_skip(self._h, ctypes.byref(v)), "fgmm_get_block_skip")
+        return bool(v.value)
+
     def last_step_path(self) -> int:
         """PREC_FP32 or PREC_FP16X3: the path the last step ran (synchronises under AUTO)."""
         v = ctypes.c_int()
