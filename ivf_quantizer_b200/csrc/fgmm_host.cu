@@ -68,6 +68,10 @@ struct fgmm::Profiler {
   cudaEvent_t pending = nullptr;
   int64_t pending_snap = -1;
   int pending_required = 0;
+  // The gate words change only between passes over the data, so within one pass every
+  // launch behind the same gate shares one snapshot (one small copy per gate and pass
+  // instead of one per launch); prof_gates_changed() starts a new epoch.
+  std::vector<std::pair<const int*, int64_t>> gate_snap;
   cudaEvent_t get() {
     if (!pool.empty()) {
       cudaEvent_t e = pool.back();
@@ -118,16 +122,27 @@ void prof_begin(const Ctx& c, KernelId, cudaStream_t s, const int* gate, int req
   if (!p->enabled) return;
   p->pending_snap = -1;
   if (gate) {
-    const int64_t i = p->new_snap();
-    if (i >= 0 &&
-        cudaMemcpyAsync(p->snap_slot(i), gate, sizeof(int), cudaMemcpyDeviceToHost, s) ==
-            cudaSuccess) {
+    int64_t i = -1;
+    for (auto& gs : p->gate_snap)
+      if (gs.first == gate) i = gs.second;
+    if (i < 0) {
+      i = p->new_snap();
+      if (i >= 0 &&
+          cudaMemcpyAsync(p->snap_slot(i), gate, sizeof(int), cudaMemcpyDeviceToHost, s) !=
+              cudaSuccess)
+        i = -1;
+      if (i >= 0) p->gate_snap.push_back({gate, i});
+    }
+    if (i >= 0) {
       p->pending_snap = i;
       p->pending_required = required;
     }
   }
   p->pending = p->get();
   cudaEventRecord(p->pending, s);
+}
+void prof_gates_changed(const Ctx& c) {
+  if (c.prof) c.prof->gate_snap.clear();
 }
 void prof_end(const Ctx& c, KernelId k, cudaStream_t s) {
   Profiler* p = c.prof;
@@ -156,7 +171,7 @@ void free_ws(Workspace& w) {
                   w.tck,    w.tks,    w.xop,    w.mode, w.stiff,    w.stiff_list, w.n_stiff,
                   w.side_part, w.mode2, w.canon, w.tcraw, w.tcm, w.tcpk, w.tckf, w.lzlow,
                   w.side_flag, w.km_word, w.grey, w.grey_pos, w.grey_stats,
-                  w.bmask, w.perm, w.lzp, w.ord_hist, w.tmask, w.tlist, w.tcnt};
+                  w.bmask, w.perm, w.perm2, w.lzp, w.ord_hist, w.ord_tot, w.tmask, w.tlist, w.tcnt};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -235,9 +250,10 @@ cudaError_t alloc_ws(Ctx& c) {
     if ((e = alloc(&w.xop, (size_t)2 * kChunk * w.K1, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.bmask, (size_t)kChunk, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.perm, (size_t)kChunk, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.perm2, (size_t)kChunk, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.lzp, (size_t)kChunk, &t)) != cudaSuccess) return e;
-    if ((e = alloc(&w.ord_hist, (size_t)(kChunk / kOrdPts) * (kSkipMaxBlocks + 1), &t)) !=
-        cudaSuccess)
+    if ((e = alloc(&w.ord_tot, (size_t)kOrdBuckets, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.ord_hist, (size_t)(kChunk / kOrdPts) * kOrdBuckets, &t)) != cudaSuccess)
       return e;
     if ((e = alloc(&w.tmask, (size_t)(kChunk / 128), &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.tlist, (size_t)kSkipMaxBlocks * (kChunk / 128), &t)) != cudaSuccess)
@@ -390,6 +406,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
   cudaError_t e;
   const Workspace& w = c.ws;
   if (host_x && (e = ensure_staging(h)) != cudaSuccess) return map_cuda(e);
+  prof_gates_changed(c);
   // which path(s) to enqueue: FP32 -> CUDA cores; FP16X3 -> tensor cores; AUTO ->
   // both, each kernel returning at once unless the device-side mode word (set by the
   // tensor-core preparation's conditioning check) selects its path
@@ -441,7 +458,9 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
     if (b >= 0) cudaEventRecord(hs.consumed[b], s);
   };
   // one tensor-core pass over all chunks, its kernels gated on the word `gate`
+  prof_gates_changed(c);
   auto tc_pass = [&](const int* gate) -> cudaError_t {
+    prof_gates_changed(c);   // the gate words were last written before this pass
     // the grey components' side-path statistics of this pass accumulate from zero
     cudaError_t r = cudaMemsetAsync(w.grey_stats, 0,
                                     (size_t)kSideMaxStiff * (1 + 2 * (size_t)w.Dp) * sizeof(double), s);
@@ -479,6 +498,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       // the side path and the pass is redone (gated on mode2); a failure after that sends
       // the step to the CUDA-core kernels below (gated on mode)
       if ((e = launch_auto_check(c, 0, s)) != cudaSuccess) return map_cuda(e);
+      prof_gates_changed(c);
       if ((e = launch_stiff_compact(c, w.mode2, w.mode, s)) != cudaSuccess) return map_cuda(e);
       word = kModeTensor;
       if (host_x && (rc = read_word(w.mode2, &word, s))) return rc;
@@ -486,6 +506,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       if ((e = launch_auto_check(c, 1, s)) != cudaSuccess) return map_cuda(e);
     }
   }
+  prof_gates_changed(c);
   int simt_word = kModeSimt;
   if (run_simt && host_x && auto_mode && (rc = read_word(w.mode, &simt_word, s))) return rc;
   if (run_simt && simt_word == kModeSimt) {
@@ -706,6 +727,7 @@ int fgmm_profile_read(fgmm_handle h, fgmm_profile* out, int reset) {
     p->recs.clear();
     p->launches = 0;
     p->nsnap = 0;
+    p->gate_snap.clear();
   }
   return FGMM_OK;
 }

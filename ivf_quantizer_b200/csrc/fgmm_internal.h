@@ -39,7 +39,8 @@ constexpr double kGreyNk = 8.0;
 // sweeps' rounding differences (about 1e-4 nats) many times over.
 constexpr float kSkipCut = 30.f;
 constexpr int kSkipMaxBlocks = 32;   // block masks are 32-bit words: K <= 4096
-constexpr int kOrdPts = 4096;        // points per CTA of the counting sort
+constexpr int kOrdPts = 4096;        // points per CTA of the radix sort
+constexpr int kOrdBuckets = 256;     // values of one 8-bit radix digit
 
 static inline int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
@@ -85,8 +86,10 @@ struct Workspace {
   // block skipping (sweep 2 visits only the (tile, block) pairs that can contribute)
   uint32_t* bmask = nullptr;  // [kChunk] per point: blocks within kSkipCut of log Z
   int* perm = nullptr;        // [kChunk] sweep-2 order: row j of phi is point perm[j]
+  int* perm2 = nullptr;       // [kChunk] the other buffer of the radix passes
   float* lzp = nullptr;       // [kChunk] log Z in sweep-2 order
-  int* ord_hist = nullptr;    // [kChunk / kOrdPts][kSkipMaxBlocks + 1] counts, then offsets
+  int* ord_hist = nullptr;    // [kOrdBuckets][kChunk / kOrdPts] counts, then offsets
+  int* ord_tot = nullptr;     // [kOrdBuckets] points per digit value
   uint32_t* tmask = nullptr;  // [kChunk / 128] per sweep-2 tile: OR of its points' masks
   int* tlist = nullptr;       // [kSkipMaxBlocks][kChunk / 128] active tiles of each block
   int* tcnt = nullptr;        // [kSkipMaxBlocks] their number
@@ -161,6 +164,9 @@ constexpr int kModeSimt = 1;
 void prof_begin(const Ctx& c, KernelId k, cudaStream_t s, const int* gate = nullptr,
                 int required = 0);
 void prof_end(const Ctx& c, KernelId k, cudaStream_t s);
+// A kernel that may write a gate word has been enqueued: launches after it take new
+// snapshots of their gate (until then, launches behind one gate share a snapshot).
+void prof_gates_changed(const Ctx& c);
 
 // ---------------------------------------------------------------- launchers
 // `mode` arguments: nullptr runs the kernel unconditionally; otherwise the kernel

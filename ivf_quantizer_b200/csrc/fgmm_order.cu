@@ -8,8 +8,9 @@
 // exactly nothing.  Sweep 1 records, per point, the blocks that come within kSkipCut of
 // log Z (a bit mask).  The kernels here
 //   order_count / order_scan / order_scatter
-//                 a stable counting sort of the chunk's points by bucket: the single
-//                 block of a one-block point, or a last bucket for every other point;
+//                 a stable LSD radix sort of the chunk's points by their 32-bit block
+//                 mask, 8 bits per pass (one pass up to 8 blocks, four for 32), so that
+//                 points with the same set of blocks become neighbours;
 //   tile_mask     per tile of the sorted order, the OR of its points' masks, and log Z
 //                 in the sorted order;
 //   block_list    per component block, the tiles whose mask holds it, in increasing order.
@@ -24,13 +25,10 @@ namespace fgmm {
 namespace {
 
 constexpr int kOrdThreads = 256;
-constexpr int kOrdBuckets = kSkipMaxBlocks + 1;
+static_assert(kOrdThreads == kOrdBuckets, "one thread per digit value");
+static_assert(FGMM_CHUNK_POINTS / kOrdPts <= kOrdThreads, "one scan thread per counting CTA");
 constexpr int kTileRows = 128;
 constexpr int kListThreads = 1024;
-
-__device__ __forceinline__ int order_key(uint32_t m, int nkb) {
-  return __popc(m) == 1 ? __ffs(m) - 1 : nkb;
-}
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t r;
@@ -38,81 +36,89 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return r;
 }
 
-// Counts of each bucket among the kOrdPts points of this CTA.
-__global__ void order_count_kernel(const uint32_t* __restrict__ bmask, int n, int nkb,
-                                   int* __restrict__ hist, const int* mode) {
+// Counts of each digit value among the kOrdPts points of this CTA (positions
+// [c kOrdPts, (c + 1) kOrdPts) of the current order: point in[j], or j without `in`).
+__global__ void order_count_kernel(const uint32_t* __restrict__ bmask, const int* __restrict__ in,
+                                   int n, int shift, int* __restrict__ hist, const int* mode) {
   if (mode && *mode != kModeTensor) return;
   __shared__ int cnt[kOrdBuckets];
-  const int nb = nkb + 1;
-  for (int b = threadIdx.x; b < nb; b += blockDim.x) cnt[b] = 0;
+  for (int b = threadIdx.x; b < kOrdBuckets; b += blockDim.x) cnt[b] = 0;
   __syncthreads();
-  const int i0 = blockIdx.x * kOrdPts;
+  const int j0 = blockIdx.x * kOrdPts;
   for (int j = threadIdx.x; j < kOrdPts; j += blockDim.x) {
-    const int i = i0 + j;
-    if (i < n) atomicAdd(&cnt[order_key(bmask[i], nkb)], 1);
+    const int jj = j0 + j;
+    if (jj < n) atomicAdd(&cnt[(bmask[in ? in[jj] : jj] >> shift) & (kOrdBuckets - 1)], 1);
   }
   __syncthreads();
-  for (int b = threadIdx.x; b < nb; b += blockDim.x) hist[blockIdx.x * nb + b] = cnt[b];
+  for (int b = threadIdx.x; b < kOrdBuckets; b += blockDim.x)
+    hist[(size_t)b * gridDim.x + blockIdx.x] = cnt[b];   // digit-major: the scan order
 }
 
-// hist[c][b] (counts) -> exclusive prefix sums in (bucket, CTA) order: the first sorted
-// position of CTA c's points of bucket b.  One CTA of kListThreads threads.
-__global__ void order_scan_kernel(int* __restrict__ hist, int ncta, int nb, const int* mode) {
-  if (mode && *mode != kModeTensor) return;
-  __shared__ int wsum[32];
-  const int E = ncta * nb;
-  const int per = (E + blockDim.x - 1) / blockDim.x;
-  const int e0 = threadIdx.x * per;
-  // scan position e = b * ncta + c is stored at hist[c * nb + b]
-  auto at = [&](int e) -> int& { return hist[(e % ncta) * nb + e / ncta]; };
-  int local = 0;
-  for (int e = e0; e < e0 + per && e < E; ++e) local += at(e);
+// Exclusive prefix sum over the 256 threads of a CTA (kOrdThreads == kOrdBuckets);
+// `tot` receives the sum.  `ws` holds 8 ints of shared memory.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* ws, int* tot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int v = local;
+  int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += u;
+    const int u = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += u;
   }
-  if (lane == 31) wsum[warp] = v;
+  if (lane == 31) ws[warp] = x;
   __syncthreads();
-  if (warp == 0) {
-    int t = lane < (int)(blockDim.x >> 5) ? wsum[lane] : 0;
+  int before = 0, all = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += u;
-    }
-    wsum[lane] = t;   // inclusive over warps
+  for (int w2 = 0; w2 < kOrdThreads / 32; ++w2) {
+    const int t = ws[w2];
+    before += w2 < warp ? t : 0;
+    all += t;
   }
-  __syncthreads();
-  int run = v - local + (warp > 0 ? wsum[warp - 1] : 0);
-  for (int e = e0; e < e0 + per && e < E; ++e) {
-    const int cnt = at(e);
-    at(e) = run;
-    run += cnt;
-  }
+  __syncthreads();   // ws may be reused by the caller
+  *tot = all;
+  return before + x - v;
 }
 
-// Stable scatter: CTA c walks its points in index order, 256 at a time; a point's
-// position is its bucket's running offset + the points of the same bucket in earlier
-// warps of the round + those in earlier lanes of its warp.
+// CTA per digit value b: hist[b][c] (counts of CTA c, digit-major) -> exclusive prefix
+// over c, and the digit's total in dtot[b].
 __global__ void __launch_bounds__(kOrdThreads)
-    order_scatter_kernel(const uint32_t* __restrict__ bmask, int n, int nkb,
-                         const int* __restrict__ offs, int* __restrict__ perm, const int* mode) {
+    order_scan_kernel(int* __restrict__ hist, int ncta, int* __restrict__ dtot, const int* mode) {
+  if (mode && *mode != kModeTensor) return;
+  __shared__ int ws[kOrdThreads / 32];
+  const int b = blockIdx.x, c = threadIdx.x;   // ncta <= kOrdThreads
+  int* row = hist + (size_t)b * ncta;
+  const int v = c < ncta ? row[c] : 0;
+  int tot;
+  const int ex = block_exclusive_scan(v, ws, &tot);
+  if (c < ncta) row[c] = ex;
+  if (c == 0) dtot[b] = tot;
+}
+
+// Stable scatter of one radix pass: CTA c walks its positions in order, 256 at a time;
+// an element's new position is its digit's running offset + the elements with the same
+// digit in earlier warps of the round + those in earlier lanes of its warp.
+__global__ void __launch_bounds__(kOrdThreads)
+    order_scatter_kernel(const uint32_t* __restrict__ bmask, const int* __restrict__ in, int n,
+                         int shift, const int* __restrict__ offs, const int* __restrict__ dtot,
+                         int* __restrict__ out, const int* mode) {
   if (mode && *mode != kModeTensor) return;
   constexpr int kWarps = kOrdThreads / 32;
   __shared__ int run[kOrdBuckets];
   __shared__ int wc[kWarps][kOrdBuckets];
-  const int nb = nkb + 1;
+  __shared__ int ws[kWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int b = threadIdx.x; b < nb; b += blockDim.x) run[b] = offs[blockIdx.x * nb + b];
-  const int i0 = blockIdx.x * kOrdPts;
+  {  // first position of digit b: the totals of the smaller digits + earlier CTAs' counts
+    const int b = threadIdx.x;   // kOrdThreads == kOrdBuckets
+    int tot;
+    const int base = block_exclusive_scan(dtot[b], ws, &tot);
+    run[b] = base + offs[(size_t)b * gridDim.x + blockIdx.x];
+  }
+  const int j0 = blockIdx.x * kOrdPts;
   for (int r0 = 0; r0 < kOrdPts; r0 += kOrdThreads) {
     for (int e = threadIdx.x; e < kWarps * kOrdBuckets; e += blockDim.x) (&wc[0][0])[e] = 0;
     __syncthreads();
-    const int i = i0 + r0 + (int)threadIdx.x;
-    const int k = i < n ? order_key(bmask[i], nkb) : -1;
+    const int jj = j0 + r0 + (int)threadIdx.x;
+    const int p = jj < n ? (in ? in[jj] : jj) : -1;
+    const int k = p >= 0 ? (int)((bmask[p] >> shift) & (kOrdBuckets - 1)) : -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, k);
     const int rank = __popc(peers & lanemask_lt());
     if (k >= 0 && rank == 0) wc[warp][k] = __popc(peers);
@@ -120,14 +126,14 @@ __global__ void __launch_bounds__(kOrdThreads)
     if (k >= 0) {
       int pos = run[k] + rank;
       for (int w2 = 0; w2 < warp; ++w2) pos += wc[w2][k];
-      perm[pos] = i;
+      out[pos] = p;
     }
     __syncthreads();
-    if ((int)threadIdx.x < nb) {
+    for (int b = threadIdx.x; b < kOrdBuckets; b += blockDim.x) {
       int add = 0;
 #pragma unroll
-      for (int w2 = 0; w2 < kWarps; ++w2) add += wc[w2][threadIdx.x];
-      run[threadIdx.x] += add;
+      for (int w2 = 0; w2 < kWarps; ++w2) add += wc[w2][b];
+      run[b] += add;
     }
     __syncthreads();
   }
@@ -189,21 +195,30 @@ cudaError_t launch_tc_order(const Ctx& c, const void* X, int x_dtype, int64_t n,
                             const int* mode, cudaStream_t s) {
   const Workspace& w = c.ws;
   const int nkb = w.Kt / 128;
-  const int nb = nkb + 1;
   const int ni = (int)n;
   const int ncta = (int)ceil_div64(n, kOrdPts);
   const int ntiles = (int)ceil_div64(n, kTileRows);
+  const int passes = (nkb + 7) / 8;
   cudaError_t e;
-  prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
-  order_count_kernel<<<ncta, kOrdThreads, 0, s>>>(w.bmask, ni, nkb, w.ord_hist, mode);
-  prof_end(c, KI_TC_ORDER, s);
-  prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
-  order_scan_kernel<<<1, kListThreads, 0, s>>>(w.ord_hist, ncta, nb, mode);
-  prof_end(c, KI_TC_ORDER, s);
-  prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
-  order_scatter_kernel<<<ncta, kOrdThreads, 0, s>>>(w.bmask, ni, nkb, w.ord_hist, w.perm, mode);
-  prof_end(c, KI_TC_ORDER, s);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // ping-pong between perm2 and perm so that the last pass lands in perm
+  const int* in = nullptr;
+  int* out = (passes & 1) ? w.perm : w.perm2;
+  for (int ps = 0; ps < passes; ++ps) {
+    const int shift = 8 * ps;
+    prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
+    order_count_kernel<<<ncta, kOrdThreads, 0, s>>>(w.bmask, in, ni, shift, w.ord_hist, mode);
+    prof_end(c, KI_TC_ORDER, s);
+    prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
+    order_scan_kernel<<<kOrdBuckets, kOrdThreads, 0, s>>>(w.ord_hist, ncta, w.ord_tot, mode);
+    prof_end(c, KI_TC_ORDER, s);
+    prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
+    order_scatter_kernel<<<ncta, kOrdThreads, 0, s>>>(w.bmask, in, ni, shift, w.ord_hist,
+                                                       w.ord_tot, out, mode);
+    prof_end(c, KI_TC_ORDER, s);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    in = out;
+    out = (out == w.perm) ? w.perm2 : w.perm;
+  }
   if ((e = launch_tc_convert(c, X, x_dtype, n, ldx, w.perm, mode, s)) != cudaSuccess) return e;
   prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
   tile_mask_kernel<<<(unsigned)ceil_div64(ntiles, 8), 256, 0, s>>>(w.perm, w.bmask, w.logz, ni,
