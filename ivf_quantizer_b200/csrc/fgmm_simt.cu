@@ -644,6 +644,17 @@ __global__ void tc_variance_check_kernel(int K, int D, int Dp, int kstride,
   const int k = blockIdx.x;
   if (stiff[k]) return;  // the side path's statistics are centred on the mean: exact
   const size_t row = (size_t)(1 + 2 * Dp);
+  const int gp = grey_pos[k];
+  if (gp >= 0) {
+    // a grey component (few points last step): its side-path statistics, centred on the
+    // mean and free of the fp16 rounding of small responsibilities, replace the
+    // tensor-core ones in slot 0, the other slots are cleared; no pass is redone
+    for (int c = threadIdx.x; c < (int)row; c += blockDim.x)
+      for (int s = 0; s < nslots; ++s)
+        stats[stat_idx(true, s, k, c, kstride, row)] = (s == 0) ? grey_stats[(size_t)gp * row + c] : 0.0;
+    if (threadIdx.x == 0) stiff[k] = 1;
+    return;
+  }
   double nk = 0.0;  // tensor-core slot layout (this check runs after tensor-core passes only)
   for (int s = 0; s < nslots; ++s) nk += stats[stat_idx(true, s, k, 0, kstride, row)];
   // Below one effective point the new mean and variance rest on far-tail
@@ -667,15 +678,7 @@ __global__ void tc_variance_check_kernel(int K, int D, int Dp, int kstride,
   if (bad) atomicExch(&bad_any, 1);
   __syncthreads();
   if (!bad_any) return;
-  const int gp = grey_pos[k];
-  if (gp >= 0) {
-    // a grey component: its side-path statistics (centred on the mean, exact) replace
-    // the tensor-core ones in slot 0, the other slots are cleared; no pass is redone
-    for (int c = threadIdx.x; c < (int)row; c += blockDim.x)
-      for (int s = 0; s < nslots; ++s)
-        stats[stat_idx(true, s, k, c, kstride, row)] = (s == 0) ? grey_stats[(size_t)gp * row + c] : 0.0;
-    if (threadIdx.x == 0) stiff[k] = 1;
-  } else if (threadIdx.x == 0) {
+  if (threadIdx.x == 0) {
     if (stage == 0) {
       stiff[k] = 1;
       atomicExch(redo, kModeTensor);
