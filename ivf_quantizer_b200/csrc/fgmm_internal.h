@@ -24,6 +24,7 @@ constexpr int kFlushTiles = 64;  // fp32 run length (tiles) before an fp64 flush
 constexpr int64_t kChunk = FGMM_CHUNK_POINTS;  // points per chunk: bounds every N-sized buffer
 constexpr int kSideMaxStiff = 256;   // AUTO side path: most stiff components per step
 constexpr int kSideParts = 64;       // AUTO side path: point ranges per chunk
+constexpr int kSidePairs = 4;        // AUTO side path: (component, log z) pairs kept per point
 // AUTO side path: a stiff or grey component whose log-density is more than this many
 // nats below a point's log Z is skipped there: its responsibility is below
 // exp(-40) = 4e-18, far under fp32 resolution of log Z and under what the tensor-core
@@ -82,6 +83,11 @@ struct Workspace {
   float* tckf = nullptr;    // [Kt] c_k + E_k for stiff components, -inf otherwise
   float* lzlow = nullptr;   // [1] log Z below which a point is always flagged
   uint8_t* side_flag = nullptr;  // [kChunk] 1: the point may have a stiff component within kCut
+  // side-path components within kCut of a flagged point, found while merging log Z and
+  // reused by the statistics (a count above kSidePairs: the statistics re-evaluate)
+  uint8_t* pair_cnt = nullptr;   // [kChunk] number of such components
+  uint8_t* pair_j = nullptr;     // [kChunk][kSidePairs] their index in the side-path list
+  float* pair_l = nullptr;       // [kChunk][kSidePairs] their log z
   __half* xop = nullptr;    // [2][kChunk][K1] phi(x) hi / lo of the current chunk
   // block skipping (sweep 2 visits only the (tile, block) pairs that can contribute)
   uint32_t* bmask = nullptr;  // [kChunk] per point: blocks within kSkipCut of log Z

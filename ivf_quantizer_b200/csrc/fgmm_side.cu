@@ -147,32 +147,52 @@ __global__ void stiff_compact_kernel(const int* __restrict__ stiff, const int* _
   }
 }
 
-// Thread per point: merge the stiff components' log-densities into log Z.
+// Thread per point: merge the stiff components' log-densities into log Z.  Every stiff
+// or grey component that comes within kCut of the point's log Z is remembered (index in
+// the side-path list and log z, up to kSidePairs of them) for the statistics, which then
+// need no second evaluation; the grey ones are evaluated for that alone (their
+// log-densities are in the tensor-core log Z already).
 template <typename T>
 __global__ void side_lse_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp,
                                 const float* __restrict__ mu, const float* __restrict__ prec,
                                 const float* __restrict__ cconst, const int* __restrict__ list,
                                 const int* __restrict__ n_stiff, const uint8_t* __restrict__ flag,
                                 float* __restrict__ logz, float* __restrict__ logz_out,
-                                const int* mode) {
+                                uint8_t* __restrict__ pair_cnt, uint8_t* __restrict__ pair_j,
+                                float* __restrict__ pair_l, const int* mode) {
   if (mode && *mode != kModeTensor) return;
-  const int ns = *n_stiff;
-  if (ns == 0) return;
+  const int ns = n_stiff[0], nall = n_stiff[0] + n_stiff[1];
+  if (nall == 0) return;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n || !flag[i]) return;  // unflagged: no stiff component within kCut of log Z
+  if (i >= n) return;
+  if (!flag[i]) {  // unflagged: no stiff or grey component within kCut of log Z
+    pair_cnt[i] = 0;
+    return;
+  }
   const T* x = X + i * ldx;
   float lz = logz[i];
-  for (int j = 0; j < ns; ++j) {
+  int cnt = 0;
+  for (int j = 0; j < nall; ++j) {
     const int k = list[j];
     const float l = stiff_logit(x, D, mu + (size_t)k * Dp, prec + (size_t)k * Dp, cconst[k],
                                 lz - kCut);
     if (l > -CUDART_INF_F) {
-      const float m = fmaxf(lz, l);
-      lz = (lz > -CUDART_INF_F) ? m + log1pf(expf(fminf(lz, l) - m)) : l;
+      if (cnt < kSidePairs) {
+        pair_j[i * kSidePairs + cnt] = (uint8_t)j;
+        pair_l[i * kSidePairs + cnt] = l;
+      }
+      ++cnt;
+      if (j < ns) {
+        const float m = fmaxf(lz, l);
+        lz = (lz > -CUDART_INF_F) ? m + log1pf(expf(fminf(lz, l) - m)) : l;
+      }
     }
   }
-  logz[i] = lz;
-  if (logz_out) logz_out[i] = lz;
+  pair_cnt[i] = (uint8_t)min(cnt, 255);
+  if (ns > 0) {
+    logz[i] = lz;
+    if (logz_out) logz_out[i] = lz;
+  }
 }
 
 // Fixed-order per-block fp64 sums of log Z over [b * 4096, (b + 1) * 4096).
@@ -213,7 +233,8 @@ __global__ void __launch_bounds__(256)
     side_stats_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp,
                       const float* __restrict__ mu, const float* __restrict__ prec,
                       const float* __restrict__ cconst, const int* __restrict__ list,
-                      const int* __restrict__ n_stiff, const uint8_t* __restrict__ flag,
+                      const int* __restrict__ n_stiff, const uint8_t* __restrict__ pair_cnt,
+                      const uint8_t* __restrict__ pair_j, const float* __restrict__ pair_l,
                       const float* __restrict__ logz, double* __restrict__ part, const int* mode) {
   if (mode && *mode != kModeTensor) return;
   const int j = blockIdx.x;
@@ -235,9 +256,16 @@ __global__ void __launch_bounds__(256)
   for (int64_t b = w0; b < w1; b += 32) {
     const int64_t i = b + lane;
     float r = 0.f;
-    if (i < w1 && flag[i]) {
+    const int cnt = i < w1 ? pair_cnt[i] : 0;
+    if (cnt > 0) {
       const float lz = logz[i];
-      const float l = stiff_logit(X + i * ldx, D, muk, pk, ck, lz - kCut);
+      float l = -CUDART_INF_F;
+      if (cnt <= kSidePairs) {   // the log z that side_lse found, if j was within the cut
+        for (int s = 0; s < cnt; ++s)
+          if (pair_j[i * kSidePairs + s] == j) l = pair_l[i * kSidePairs + s];
+      } else {                   // more components than slots: evaluate again
+        l = stiff_logit(X + i * ldx, D, muk, pk, ck, lz - kCut);
+      }
       if (l > -CUDART_INF_F && lz > -CUDART_INF_F) r = fminf(expf(l - lz), 1.f);
     }
     unsigned live = __ballot_sync(0xffffffffu, r > 0.f);
@@ -317,13 +345,11 @@ cudaError_t launch_side_lse(const Ctx& c, const void* X, int x_dtype, int64_t n,
   if (x_dtype == FGMM_BF16)
     side_lse_kernel<<<grid, 128, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
                                          w.cconst, w.stiff_list, w.n_stiff, w.side_flag, w.logz,
-                                         logz_out,
-                                         mode);
+                                         logz_out, w.pair_cnt, w.pair_j, w.pair_l, mode);
   else
     side_lse_kernel<<<grid, 128, 0, s>>>((const float*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
                                          w.cconst, w.stiff_list, w.n_stiff, w.side_flag, w.logz,
-                                         logz_out,
-                                         mode);
+                                         logz_out, w.pair_cnt, w.pair_j, w.pair_l, mode);
   prof_end(c, KI_SIDE_LSE, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -340,12 +366,12 @@ cudaError_t launch_side_stats(const Ctx& c, const void* X, int x_dtype, int64_t 
   prof_begin(c, KI_SIDE_STATS, s, mode, kModeTensor);
   if (x_dtype == FGMM_BF16)
     side_stats_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dp, w.mu,
-                                           w.prec, w.cconst, w.stiff_list, w.n_stiff, w.side_flag,
-                                           w.logz, w.side_part, mode);
+                                           w.prec, w.cconst, w.stiff_list, w.n_stiff, w.pair_cnt,
+                                           w.pair_j, w.pair_l, w.logz, w.side_part, mode);
   else
     side_stats_kernel<<<grid, 256, 0, s>>>((const float*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
-                                           w.cconst, w.stiff_list, w.n_stiff, w.side_flag,
-                                           w.logz, w.side_part, mode);
+                                           w.cconst, w.stiff_list, w.n_stiff, w.pair_cnt,
+                                           w.pair_j, w.pair_l, w.logz, w.side_part, mode);
   prof_end(c, KI_SIDE_STATS, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
