@@ -88,6 +88,8 @@ struct Workspace {
   uint8_t* pair_cnt = nullptr;   // [kChunk] number of such components
   uint8_t* pair_j = nullptr;     // [kChunk][kSidePairs] their index in the side-path list
   float* pair_l = nullptr;       // [kChunk][kSidePairs] their log z
+  int* flagged = nullptr;        // [kChunk] the flagged points of the chunk, as a list
+  int* n_flagged = nullptr;      // [1] their number
   __half* xop = nullptr;    // [2][kChunk][K1] phi(x) hi / lo of the current chunk
   // block skipping (sweep 2 visits only the (tile, block) pairs that can contribute)
   uint32_t* bmask = nullptr;  // [kChunk] per point: blocks within kSkipCut of log Z

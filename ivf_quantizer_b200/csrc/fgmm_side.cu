@@ -147,7 +147,38 @@ __global__ void stiff_compact_kernel(const int* __restrict__ stiff, const int* _
   }
 }
 
-// Thread per point: merge the stiff components' log-densities into log Z.  Every stiff
+// The flagged points of the chunk, as a list (in no particular order: each is handled on
+// its own), so that side_lse runs on full warps; the other points get pair count 0.
+__global__ void side_flagged_kernel(const uint8_t* __restrict__ flag, int64_t n,
+                                    const int* __restrict__ n_stiff, int* __restrict__ list,
+                                    int* __restrict__ count, uint8_t* __restrict__ pair_cnt,
+                                    const int* mode) {
+  if (mode && *mode != kModeTensor) return;
+  if (n_stiff[0] + n_stiff[1] == 0) return;
+  __shared__ int wsum[8], base;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t i0 = (int64_t)blockIdx.x * 4096;
+  for (int r0 = 0; r0 < 4096; r0 += 256) {
+    const int64_t i = i0 + r0 + threadIdx.x;
+    const bool f = i < n && flag[i];
+    if (i < n && !f) pair_cnt[i] = 0;
+    const unsigned m = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) wsum[warp] = __popc(m);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int t = 0;
+      for (int w2 = 0; w2 < 8; ++w2) t += wsum[w2];
+      base = t ? atomicAdd(count, t) : 0;
+    }
+    __syncthreads();
+    int off = base;
+    for (int w2 = 0; w2 < warp; ++w2) off += wsum[w2];
+    if (f) list[off + __popc(m & ((1u << lane) - 1u))] = (int)i;
+    __syncthreads();
+  }
+}
+
+// Thread per flagged point: merge the stiff components' log-densities into log Z.  Every stiff
 // or grey component that comes within kCut of the point's log Z is remembered (index in
 // the side-path list and log z, up to kSidePairs of them) for the statistics, which then
 // need no second evaluation; the grey ones are evaluated for that alone (their
@@ -156,19 +187,17 @@ template <typename T>
 __global__ void side_lse_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp,
                                 const float* __restrict__ mu, const float* __restrict__ prec,
                                 const float* __restrict__ cconst, const int* __restrict__ list,
-                                const int* __restrict__ n_stiff, const uint8_t* __restrict__ flag,
+                                const int* __restrict__ n_stiff,
                                 float* __restrict__ logz, float* __restrict__ logz_out,
                                 uint8_t* __restrict__ pair_cnt, uint8_t* __restrict__ pair_j,
-                                float* __restrict__ pair_l, const int* mode) {
+                                float* __restrict__ pair_l, const int* __restrict__ flagged,
+                                const int* __restrict__ n_flagged, const int* mode) {
   if (mode && *mode != kModeTensor) return;
   const int ns = n_stiff[0], nall = n_stiff[0] + n_stiff[1];
   if (nall == 0) return;
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  if (!flag[i]) {  // unflagged: no stiff or grey component within kCut of log Z
-    pair_cnt[i] = 0;
-    return;
-  }
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= *n_flagged) return;
+  const int64_t i = flagged[e];
   const T* x = X + i * ldx;
   float lz = logz[i];
   int cnt = 0;
@@ -341,17 +370,25 @@ cudaError_t launch_side_lse(const Ctx& c, const void* X, int x_dtype, int64_t n,
                             float* logz_out, const int* mode, cudaStream_t s) {
   const unsigned grid = (unsigned)ceil_div64(n, 128);
   const Workspace& w = c.ws;
+  cudaError_t e = cudaMemsetAsync(w.n_flagged, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  prof_begin(c, KI_SIDE_LSE, s, mode, kModeTensor);
+  side_flagged_kernel<<<(unsigned)ceil_div64(n, 4096), 256, 0, s>>>(
+      w.side_flag, n, w.n_stiff, w.flagged, w.n_flagged, w.pair_cnt, mode);
+  prof_end(c, KI_SIDE_LSE, s);
   prof_begin(c, KI_SIDE_LSE, s, mode, kModeTensor);
   if (x_dtype == FGMM_BF16)
     side_lse_kernel<<<grid, 128, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
-                                         w.cconst, w.stiff_list, w.n_stiff, w.side_flag, w.logz,
-                                         logz_out, w.pair_cnt, w.pair_j, w.pair_l, mode);
+                                         w.cconst, w.stiff_list, w.n_stiff, w.logz,
+                                         logz_out, w.pair_cnt, w.pair_j, w.pair_l, w.flagged,
+                                         w.n_flagged, mode);
   else
     side_lse_kernel<<<grid, 128, 0, s>>>((const float*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
-                                         w.cconst, w.stiff_list, w.n_stiff, w.side_flag, w.logz,
-                                         logz_out, w.pair_cnt, w.pair_j, w.pair_l, mode);
+                                         w.cconst, w.stiff_list, w.n_stiff, w.logz,
+                                         logz_out, w.pair_cnt, w.pair_j, w.pair_l, w.flagged,
+                                         w.n_flagged, mode);
   prof_end(c, KI_SIDE_LSE, s);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   prof_begin(c, KI_LL_PARTIALS, s, mode, kModeTensor);
   ll_partials_kernel<<<(unsigned)ceil_div64(n, 4096), 256, 0, s>>>(w.logz, n, w.ll_tiles, mode);

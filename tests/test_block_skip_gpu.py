@@ -125,6 +125,14 @@ def test_two_blocks_ragged():
     compare_step(c[:3], _oracle(X, w, mu, var), X.numpy(), logz_gpu=c[4], loglik_gpu=c[3])
 
 
+def test_bf16_input():
+    X = synth.generate("table1", 7_001, seed=12).to(torch.bfloat16)
+    w, mu, var = synth.init_params(X.float(), 512, seed=12)
+    a = _step(X, w, mu, var, True)
+    b = _step(X, w, mu, var, False)
+    _agree(a, b, X.float())
+
+
 def test_two_chunks():
     import ivf_quantizer_b200 as q
     N = q.CHUNK_POINTS + 3_001
