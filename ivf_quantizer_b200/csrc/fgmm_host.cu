@@ -173,7 +173,7 @@ void free_ws(Workspace& w) {
                   w.side_flag, w.pair_cnt, w.pair_j, w.pair_l, w.flagged, w.n_flagged, w.km_word,
                   w.grey, w.grey_pos,
                   w.grey_stats,
-                  w.bmask, w.perm, w.perm2, w.lzp, w.ord_hist, w.ord_tot, w.tmask, w.tlist, w.tcnt};
+                  w.lbuf, w.bmask, w.perm, w.perm2, w.lzp, w.ord_hist, w.ord_tot, w.tmask, w.tlist, w.tcnt};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -200,13 +200,17 @@ cudaError_t alloc_ws(Ctx& c) {
   const bool tc = tc_supported(c);
   int s_tc = c.num_sms / (w.Kt / 128);
   if (s_tc < 1) s_tc = 1;
-  w.slots = tc && s_tc > kSlices ? s_tc : kSlices;
+  // the tensor-core statistics sweep writes up to 2 s_tc slots (block skipping)
+  w.slots = tc && 2 * s_tc > kSlices ? 2 * s_tc : kSlices;
   size_t t = 0;
   cudaError_t e;
   const size_t kd = (size_t)w.Kp * w.Dp;
   if ((e = alloc(&w.mu, kd, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.prec, kd, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.cconst, (size_t)w.Kp, &t)) != cudaSuccess) return e;
+  if (w.Dp > kFC && w.Kp <= kLbufMaxKp &&
+      (e = alloc(&w.lbuf, (size_t)kChunk * w.Kp, &t)) != cudaSuccess)
+    return e;
   if ((e = alloc(&w.logz, (size_t)kChunk, &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.ll_tiles, (size_t)(kChunk / 32), &t)) != cudaSuccess) return e;
   if ((e = alloc(&w.ll_total, (size_t)1, &t)) != cudaSuccess) return e;
@@ -523,7 +527,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       int64_t ldc;
       const int b = acquire(c0, nc, &Xc, &ldc);
       float* lzo = logz_out ? logz_out + c0 : nullptr;
-      if ((e = launch_lse_simt(c, Xc, x_dtype, nc, ldc, lzo, mode, s)) == cudaSuccess &&
+      if ((e = launch_lse_simt(c, Xc, x_dtype, nc, ldc, lzo, want_stats, mode, s)) == cudaSuccess &&
           (e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeSimt, s)) == cudaSuccess &&
           want_stats)
         e = launch_stats_simt(c, Xc, x_dtype, nc, ldc, mode, s);

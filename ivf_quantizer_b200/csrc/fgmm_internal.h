@@ -21,6 +21,7 @@ constexpr int kDC = 32;        // feature chunk staged in shared memory
 constexpr int kFC = 128;       // features per CTA in the statistics sweep
 constexpr int kSlices = 16;    // point slices of a chunk in the statistics sweep
 constexpr int kFlushTiles = 64;  // fp32 run length (tiles) before an fp64 flush
+constexpr int kLbufMaxKp = 1024; // largest Kp whose chunk of log-densities is kept (4 GB)
 constexpr int64_t kChunk = FGMM_CHUNK_POINTS;  // points per chunk: bounds every N-sized buffer
 constexpr int kSideMaxStiff = 256;   // AUTO side path: most stiff components per step
 constexpr int kSideParts = 64;       // AUTO side path: point ranges per chunk
@@ -116,6 +117,10 @@ struct Workspace {
   float* mu = nullptr;     // [Kp, Dp] means, zero padded
   float* prec = nullptr;   // [Kp, Dp] -1/(2 sigma^2), zero padded
   float* cconst = nullptr; // [Kp] log pi_k - 1/2 sum_d log(2 pi sigma_kd^2); -inf if absent
+  // D > kFC: the statistics sweep covers the features in several CTAs per component
+  // block, each of which would recompute the log-densities; the log-sum-exp sweep keeps
+  // them here instead (allocated for Kp <= kLbufMaxKp only)
+  float* lbuf = nullptr;   // [kChunk][Kp] log z_ik of the chunk
   // per chunk
   float* logz = nullptr;   // [kChunk] log Z_i of the chunk being processed
   double* ll_tiles = nullptr;  // [kChunk / 32] partial log-likelihoods of the chunk
@@ -181,8 +186,10 @@ void prof_gates_changed(const Ctx& c);
 // returns at once unless *mode selects its path (AUTO decides on the device).
 cudaError_t launch_prep_simt(const Ctx& c, const float* weights, const float* means,
                              const float* vars, cudaStream_t s);
+// keep_logits: also write every log z_ik of the chunk to ws.lbuf (when it exists), for the
+// statistics sweep to read instead of recomputing them once per feature block
 cudaError_t launch_lse_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
-                            float* logz_out, const int* mode, cudaStream_t s);
+                            float* logz_out, bool keep_logits, const int* mode, cudaStream_t s);
 cudaError_t launch_ll_accumulate(const Ctx& c, int64_t n, const int* mode, int fixed_mode,
                                  int required, cudaStream_t s);
 // AUTO only: variance-cancellation check after a tensor-core pass.  Stage 0: failing
@@ -224,6 +231,9 @@ cudaError_t launch_kmeans_seed(const Ctx& c, const void* X, int x_dtype, int64_t
 bool tc_supported(const Ctx& c);
 cudaError_t tc_init(Ctx& c);
 int tc_slices(const Ctx& c);
+// statistics slots the tensor-core statistics sweep may write (block skipping can give a
+// busy block more CTAs than tc_slices); the reduction sums this many
+int tc_stat_slots(const Ctx& c);
 cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* means,
                            const float* vars, bool auto_mode, cudaStream_t s);
 // AUTO side path for stiff components (fgmm_side.cu)

@@ -169,13 +169,13 @@ __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, i
 // One CTA per 64-point tile; online log-sum-exp over blocks of 64 components
 // (Alg. 1, step 1).  Writes log Z_i for the chunk, optionally to the caller's
 // per-point buffer, and one fp64 partial log-likelihood per tile.
-template <typename T>
+template <typename T, bool KEEP>
 __global__ void __launch_bounds__(kSimtThreads, 2)
     lse_simt_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp, int Kp,
                     const float* __restrict__ mu, const float* __restrict__ prec,
                     const float* __restrict__ cconst, float* __restrict__ logz,
                     float* __restrict__ logz_out, double* __restrict__ ll_tiles,
-                    const int* mode) {
+                    float* __restrict__ lbuf, const int* mode) {
   if (mode && *mode != kModeSimt) return;
   __shared__ __align__(16) float xs[kTP][kDC + 4];
   __shared__ __align__(16) float ms[kKB][kDC + 4];
@@ -199,6 +199,11 @@ __global__ void __launch_bounds__(kSimtThreads, 2)
       float bm = -CUDART_INF_F;
 #pragma unroll
       for (int q = 0; q < 4; ++q) { l[q] = acc[j][q] + cc[q]; bm = fmaxf(bm, l[q]); }
+      if (KEEP && i0 + ty + 16 * j < n) {   // kept for the statistics sweep (D > kFC)
+        float* lr = lbuf + (size_t)(i0 + ty + 16 * j) * Kp + kb + tx;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) lr[16 * q] = l[q];
+      }
 #pragma unroll
       for (int off = 8; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
       const float nm = fmaxf(run_m[j], bm);
@@ -274,7 +279,7 @@ __global__ void __launch_bounds__(kSimtThreads)
                       const float* __restrict__ mu, const float* __restrict__ prec,
                       const float* __restrict__ cconst, const float* __restrict__ logz,
                       double* __restrict__ stats, int kstride, int64_t slice_len,
-                      const int* mode) {
+                      const float* __restrict__ lbuf, const int* mode) {
   if (mode && *mode != kModeSimt) return;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   StatsSmem& sm = *reinterpret_cast<StatsSmem*>(smem_raw);
@@ -330,8 +335,24 @@ __global__ void __launch_bounds__(kSimtThreads)
       const int64_t i = i0 + threadIdx.x;
       sm.lz[threadIdx.x] = (i < p_end) ? logz[i] : -CUDART_INF_F;
     }
-    float acc[4][2];
-    logit_tile<2>(X, p_end, ldx, D, Dp, i0, kb, mu, prec, sm.xs, sm.ms, sm.ps, acc);
+    float lg[4][2];   // log z of the tile's points for the CTA's 32 components
+    if (lbuf) {       // kept by the log-sum-exp sweep: the same values, bit for bit
+      __syncthreads();   // sm.lz of this tile (no logit_tile barrier in this branch)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t i = i0 + ty + 16 * j;
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          lg[j][q] = i < p_end ? lbuf[(size_t)i * Kp + kb + tx + 16 * q] : -CUDART_INF_F;
+      }
+    } else {
+      float acc[4][2];
+      logit_tile<2>(X, p_end, ldx, D, Dp, i0, kb, mu, prec, sm.xs, sm.ms, sm.ps, acc);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) lg[j][q] = acc[j][q] + cc[q];
+    }
     // responsibilities of this tile for the CTA's 32 components
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -339,7 +360,7 @@ __global__ void __launch_bounds__(kSimtThreads)
       const float lz = sm.lz[r];
       const bool ok = lz > -CUDART_INF_F && lz < CUDART_INF_F;
 #pragma unroll
-      for (int q = 0; q < 2; ++q) sm.rs[r][tx + 16 * q] = ok ? expf(acc[j][q] + cc[q] - lz) : 0.f;
+      for (int q = 0; q < 2; ++q) sm.rs[r][tx + 16 * q] = ok ? expf(lg[j][q] - lz) : 0.f;
     }
     // the tile's features for the statistics
     for (int e = threadIdx.x; e < kTP * kFC; e += kSimtThreads) {
@@ -720,17 +741,20 @@ cudaError_t launch_prep_simt(const Ctx& c, const float* weights, const float* me
 }
 
 cudaError_t launch_lse_simt(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
-                            float* logz_out, const int* mode, cudaStream_t s) {
+                            float* logz_out, bool keep_logits, const int* mode, cudaStream_t s) {
   const unsigned grid = (unsigned)ceil_div64(n, kTP);
+  float* lb = keep_logits ? c.ws.lbuf : nullptr;
   prof_begin(c, KI_LSE_SIMT, s, mode, kModeSimt);
-  if (x_dtype == FGMM_BF16)
-    lse_simt_kernel<<<grid, kSimtThreads, 0, s>>>(
-        (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
-        c.ws.logz, logz_out, c.ws.ll_tiles, mode);
-  else
-    lse_simt_kernel<<<grid, kSimtThreads, 0, s>>>((const float*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp,
-                                                  c.ws.mu, c.ws.prec, c.ws.cconst, c.ws.logz,
-                                                  logz_out, c.ws.ll_tiles, mode);
+#define LSE_SIMT(T_, K_)                                                                        \
+  lse_simt_kernel<T_, K_><<<grid, kSimtThreads, 0, s>>>(                                        \
+      (const T_*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst, c.ws.logz,  \
+      logz_out, c.ws.ll_tiles, lb, mode)
+  if (x_dtype == FGMM_BF16) {
+    if (lb) LSE_SIMT(__nv_bfloat16, true); else LSE_SIMT(__nv_bfloat16, false);
+  } else {
+    if (lb) LSE_SIMT(float, true); else LSE_SIMT(float, false);
+  }
+#undef LSE_SIMT
   prof_end(c, KI_LSE_SIMT, s);
   return cudaGetLastError();
 }
@@ -763,11 +787,12 @@ cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t 
   if (x_dtype == FGMM_BF16)
     stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>(
         (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
-        c.ws.logz, c.ws.stats, c.ws.KpS, slice, mode);
+        c.ws.logz, c.ws.stats, c.ws.KpS, slice, c.ws.lbuf, mode);
   else
     stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>((const float*)X, n, ldx, c.D, c.ws.Dp,
                                                        c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
-                                                       c.ws.logz, c.ws.stats, c.ws.KpS, slice, mode);
+                                                       c.ws.logz, c.ws.stats, c.ws.KpS, slice,
+                                                       c.ws.lbuf, mode);
   prof_end(c, KI_STATS_SIMT, s);
   return cudaGetLastError();
 }
@@ -776,7 +801,7 @@ cudaError_t launch_reduce_stats(const Ctx& c, const float* means, double* out, c
                                 int fixed_mode, cudaStream_t s) {
   prof_begin(c, KI_REDUCE_STATS, s);
   reduce_stats_kernel<<<c.K, kSimtThreads, 0, s>>>(
-      c.K, c.D, c.ws.Dp, c.ws.KpS, c.ws.stats, kSlices, c.tc.ready ? tc_slices(c) : 1, mode,
+      c.K, c.D, c.ws.Dp, c.ws.KpS, c.ws.stats, kSlices, c.tc.ready ? tc_stat_slots(c) : 1, mode,
       fixed_mode, c.tc.ready ? c.ws.stiff : nullptr, means, c.ws.center, c.ws.dscale,
       c.ws.ll_total, out);
   prof_end(c, KI_REDUCE_STATS, s);
@@ -841,7 +866,7 @@ cudaError_t launch_auto_check(const Ctx& c, int stage, cudaStream_t s) {
   const size_t n = (size_t)w.slots * w.KpS * (1 + 2 * (size_t)w.Dp);
   prof_begin(c, KI_AUTO_CHECK, s);
   tc_variance_check_kernel<<<c.K, kSimtThreads, 0, s>>>(c.K, c.D, w.Dp, w.KpS, w.stats,
-                                                        tc_slices(c), w.stiff,
+                                                        tc_stat_slots(c), w.stiff,
                                                         stage == 0 ? w.mode : w.mode2, w.mode2,
                                                         w.mode, stage, w.grey_pos,
                                                         w.grey_stats);

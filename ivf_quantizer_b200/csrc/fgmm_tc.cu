@@ -700,7 +700,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const float* __restrict__ ck, const float* __restrict__ kscale,
                     const float* __restrict__ logz, double* __restrict__ stats, int kstride,
                     int Dp, const __half* __restrict__ wop, const int* __restrict__ tlist,
-                    const int* __restrict__ tcnt, int tl_stride, const int* mode, int* status) {
+                    const int* __restrict__ tcnt, int tl_stride, int max_cta, const int* mode,
+                    int* status) {
   if (mode && *mode != kModeTensor) return;
   constexpr int Dq = NKC * 32;            // features: phi has 2 Dq = NKC * 64 entries
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -712,14 +713,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb = blockIdx.x;
-  // The CTA's point tiles: a contiguous slice of the chunk, or (block skipping) an even
-  // share of the block's list of active tiles, tiles of 128 rows of the reordered phi.
+  // The CTA's component block kb, statistics slot, and point tiles: grid (block, slice)
+  // with a contiguous slice of the chunk each; or (block skipping, 1-D grid of G CTAs)
+  // the G CTAs shared among the blocks in proportion to their active tiles, block b
+  // taking c_b = 1 + floor(n_b (G - nkb) / sum n) CTAs (none if n_b = 0, at most
+  // max_cta), each an even share of b's list; tiles are 128 rows of the reordered phi.
+  // The shares depend on the counts alone: every CTA derives the same ones.
+  int kb = blockIdx.x, sl = blockIdx.y;
   int p0, p1, ntl, l0 = 0;
   if (tlist) {
-    const int na = tcnt[kb];
-    const int per = (na + (int)gridDim.y - 1) / (int)gridDim.y;
-    l0 = min(na, (int)blockIdx.y * per);
+    const int nkb = Kt / BKc;
+    const int G = (int)gridDim.x;
+    long long tot = 0;
+    for (int b = 0; b < nkb; ++b) tot += tcnt[b];
+    int before = 0, na = 0, cb = 0;
+    kb = -1;
+    for (int b = 0; b < nkb; ++b) {
+      const int nb = tcnt[b];
+      const int c = nb > 0 ? min(max_cta, 1 + (int)((long long)nb * (G - nkb) / tot)) : 0;
+      if (kb < 0 && (int)blockIdx.x < before + c) { kb = b; sl = blockIdx.x - before; na = nb; cb = c; }
+      before += c;
+    }
+    if (kb < 0) return;  // a spare CTA: uniform over the CTA, before any barrier
+    const int per = (na + cb - 1) / cb;
+    l0 = min(na, sl * per);
     ntl = min(na, l0 + per) - l0;
     p0 = 0;
     p1 = nc;
@@ -924,7 +941,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const size_t row = (size_t)(1 + 2 * Dp);
     // this CTA's slot, [row][kstride] layout: statistic c of component k at c * kstride + k
-    double* slot = stats + stat_idx(true, blockIdx.y, k, 0, kstride, row);
+    double* slot = stats + stat_idx(true, sl, k, 0, kstride, row);
     float nk = 0.f;
     int tiles_since_flush = 0, flushes = 0;
     // R^T row kl, points 64g .. 64g+63 = box g: 8-row atoms of 1024 B, 128 B per row,
@@ -1234,6 +1251,11 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
   return cudaGetLastError();
 }
 
+int tc_stat_slots(const Ctx& c) {
+  const int S2 = 2 * tc_slices(c);
+  return S2 < c.ws.slots ? S2 : c.ws.slots;
+}
+
 int tc_slices(const Ctx& c) {
   const int nkb = c.ws.Kt / BKc;
   int S = c.num_sms / nkb;
@@ -1247,12 +1269,13 @@ cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream
   const int nkc = w.K1 / 64;
   const int S = tc_slices(c);
   int slice = (int)ceil_div64(ceil_div64(n, S), BM) * BM;
-  dim3 grid(w.Kt / BKc, S);
+  const bool skip = tc_skip(c);
+  // block skipping: a 1-D grid of the same size, shared among the blocks by their work
+  const dim3 grid = skip ? dim3((w.Kt / BKc) * S, 1) : dim3(w.Kt / BKc, S);
   const CUtensorMap& tx = c.tc.tmap_x;
   const CUtensorMap& tw = c.tc.tmap_w;
   const int flush_tiles = 8;  // fp32 runs of 1024 points (64 MMA steps) between fp64 flushes
   // block skipping: phi and log Z were rewritten in sweep-2 order, tiles come from lists
-  const bool skip = tc_skip(c);
   const float* lz = skip ? w.lzp : w.logz;
   const int* tl = skip ? w.tlist : nullptr;
   const int tl_stride = (int)(kChunk / BM);
@@ -1261,7 +1284,7 @@ cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream
   case N_:                                                                                     \
     tc_stats_kernel<N_><<<grid, kTcThreads, stats_smem(N_), s>>>(                              \
         tx, tw, (int)n, (int)kChunk, w.Kt, slice, flush_tiles, w.tck, w.tks, lz, w.stats,      \
-        w.KpS, w.Dp, w.wop, tl, w.tcnt, tl_stride, mode, w.status);                            \
+        w.KpS, w.Dp, w.wop, tl, w.tcnt, tl_stride, tc_stat_slots(c), mode, w.status);          \
     break;
   switch (nkc) {
     STATS_CASE(1)
