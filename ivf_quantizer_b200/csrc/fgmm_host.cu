@@ -173,7 +173,7 @@ void free_ws(Workspace& w) {
                   w.side_flag, w.pair_cnt, w.pair_j, w.pair_l, w.flagged, w.n_flagged, w.km_word,
                   w.grey, w.grey_pos,
                   w.grey_stats,
-                  w.lbuf, w.bmask, w.perm, w.perm2, w.lzp, w.ord_hist, w.ord_tot, w.tmask, w.tlist, w.tcnt};
+                  w.lbuf, w.bmx, w.bmask, w.perm, w.perm2, w.lzp, w.ord_hist, w.ord_tot, w.tmask, w.tlist, w.tcnt};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -259,6 +259,16 @@ cudaError_t alloc_ws(Ctx& c) {
     if ((e = alloc(&w.flagged, (size_t)kChunk, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.n_flagged, (size_t)1, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.xop, (size_t)2 * kChunk * w.K1, &t)) != cudaSuccess) return e;
+    // rows past the end of a short chunk are read by the tensor cores (and multiplied
+    // by r = 0): keep them finite from the start
+    if ((e = cudaMemset(w.xop, 0, (size_t)2 * kChunk * w.K1 * sizeof(__half))) != cudaSuccess)
+      return e;
+  }
+  // block skipping (tensor-core statistics sweep, or the CUDA-core one for 4 to 32
+  // blocks of 128 components)
+  const int nkb_simt = (w.Kp + 127) / 128;
+  const bool simt_blocks = nkb_simt >= 4 && nkb_simt <= kSkipMaxBlocks;
+  if (tc || simt_blocks) {
     if ((e = alloc(&w.bmask, (size_t)kChunk, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.perm, (size_t)kChunk, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.perm2, (size_t)kChunk, &t)) != cudaSuccess) return e;
@@ -266,15 +276,13 @@ cudaError_t alloc_ws(Ctx& c) {
     if ((e = alloc(&w.ord_tot, (size_t)kOrdBuckets, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.ord_hist, (size_t)(kChunk / kOrdPts) * kOrdBuckets, &t)) != cudaSuccess)
       return e;
-    if ((e = alloc(&w.tmask, (size_t)(kChunk / 128), &t)) != cudaSuccess) return e;
-    if ((e = alloc(&w.tlist, (size_t)kSkipMaxBlocks * (kChunk / 128), &t)) != cudaSuccess)
+    if ((e = alloc(&w.tmask, (size_t)(kChunk / kTP), &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.tlist, (size_t)kSkipMaxBlocks * (kChunk / kTP), &t)) != cudaSuccess)
       return e;
     if ((e = alloc(&w.tcnt, (size_t)kSkipMaxBlocks, &t)) != cudaSuccess) return e;
-    // rows past the end of a short chunk are read by the tensor cores (and multiplied
-    // by r = 0): keep them finite from the start
-    if ((e = cudaMemset(w.xop, 0, (size_t)2 * kChunk * w.K1 * sizeof(__half))) != cudaSuccess)
-      return e;
   }
+  if (simt_blocks && (e = alloc(&w.bmx, (size_t)kChunk * (w.Kp / kKB), &t)) != cudaSuccess)
+    return e;
   w.bytes = t;
   if (tc && (e = tc_init(c)) != cudaSuccess) return e;
   return cudaSuccess;
@@ -529,7 +537,8 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       float* lzo = logz_out ? logz_out + c0 : nullptr;
       if ((e = launch_lse_simt(c, Xc, x_dtype, nc, ldc, lzo, want_stats, mode, s)) == cudaSuccess &&
           (e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeSimt, s)) == cudaSuccess &&
-          want_stats)
+          want_stats &&
+          (!simt_skip(c) || (e = launch_simt_order(c, nc, mode, s)) == cudaSuccess))
         e = launch_stats_simt(c, Xc, x_dtype, nc, ldc, mode, s);
       release(b);
       if (e == cudaSuccess) e = copy_err;

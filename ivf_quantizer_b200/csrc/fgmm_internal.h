@@ -41,6 +41,11 @@ constexpr double kGreyNk = 8.0;
 // sweeps' rounding differences (about 1e-4 nats) many times over.
 constexpr float kSkipCut = 30.f;
 constexpr int kSkipMaxBlocks = 32;   // block masks are 32-bit words: K <= 4096
+// The same on the CUDA-core path, whose fp32 statistics keep every responsibility down to
+// the underflow of expf (about e^-104): there a pair is left out when every log-density
+// is more than kSimtSkipCut nats below log Z, i.e. each dropped r is below e^-50 = 2e-22,
+// and all that a component can lose over 10^9 points is below 2e-13 effective points.
+constexpr float kSimtSkipCut = 50.f;
 constexpr int kOrdPts = 4096;        // points per CTA of the radix sort
 constexpr int kOrdBuckets = 256;     // values of one 8-bit radix digit
 
@@ -99,8 +104,9 @@ struct Workspace {
   float* lzp = nullptr;       // [kChunk] log Z in sweep-2 order
   int* ord_hist = nullptr;    // [kOrdBuckets][kChunk / kOrdPts] counts, then offsets
   int* ord_tot = nullptr;     // [kOrdBuckets] points per digit value
-  uint32_t* tmask = nullptr;  // [kChunk / 128] per sweep-2 tile: OR of its points' masks
-  int* tlist = nullptr;       // [kSkipMaxBlocks][kChunk / 128] active tiles of each block
+  uint32_t* tmask = nullptr;  // [kChunk / kTP] per sweep-2 tile: OR of its points' masks
+  int* tlist = nullptr;       // [kSkipMaxBlocks][kChunk / tile rows] active tiles of each block
+  float* bmx = nullptr;       // CUDA-core path: [kChunk][Kp / kKB] largest log z per 64 components
   int* tcnt = nullptr;        // [kSkipMaxBlocks] their number
   int* mode = nullptr;      // [1] path of the current step: 0 tensor cores, 1 CUDA cores
   int* mode2 = nullptr;     // [1] AUTO: tensor when the hybrid redo pass must run
@@ -254,6 +260,10 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
 cudaError_t launch_tc_order(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
                             const int* mode, cudaStream_t s);
 cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream_t s);
+// block skipping on the CUDA-core path: masks from sweep 1's block maxima (ws.bmx), the
+// sweep-2 order (ws.perm, ws.lzp) and the active 64-point tiles of each 128-component block
+bool simt_skip(const Ctx& c);
+cudaError_t launch_simt_order(const Ctx& c, int64_t n, const int* mode, cudaStream_t s);
 cudaError_t run_bounded_wait_probe(int64_t limit_ns, int* status_host);
 // soft assignment on caller-provided scratch (allocation-free entry point)
 cudaError_t launch_prep_simt_raw(int K, int D, int Kp, int Dp, int cov, const float* weights,

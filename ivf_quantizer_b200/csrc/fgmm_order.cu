@@ -18,6 +18,8 @@
 // then runs each block over its own list.  Every step is deterministic (counts, prefix
 // sums, ordered scatter), so the sums stay bitwise reproducible from run to run; they
 // differ from the natural order only by the order of fp32 additions.
+#include <math_constants.h>
+
 #include "fgmm_internal.h"
 
 namespace fgmm {
@@ -39,8 +41,9 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 // Counts of each digit value among the kOrdPts points of this CTA (positions
 // [c kOrdPts, (c + 1) kOrdPts) of the current order: point in[j], or j without `in`).
 __global__ void order_count_kernel(const uint32_t* __restrict__ bmask, const int* __restrict__ in,
-                                   int n, int shift, int* __restrict__ hist, const int* mode) {
-  if (mode && *mode != kModeTensor) return;
+                                   int n, int shift, int* __restrict__ hist, const int* mode,
+                                   int required) {
+  if (mode && *mode != required) return;
   __shared__ int cnt[kOrdBuckets];
   for (int b = threadIdx.x; b < kOrdBuckets; b += blockDim.x) cnt[b] = 0;
   __syncthreads();
@@ -81,8 +84,9 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* ws, int* tot) {
 // CTA per digit value b: hist[b][c] (counts of CTA c, digit-major) -> exclusive prefix
 // over c, and the digit's total in dtot[b].
 __global__ void __launch_bounds__(kOrdThreads)
-    order_scan_kernel(int* __restrict__ hist, int ncta, int* __restrict__ dtot, const int* mode) {
-  if (mode && *mode != kModeTensor) return;
+    order_scan_kernel(int* __restrict__ hist, int ncta, int* __restrict__ dtot, const int* mode,
+                      int required) {
+  if (mode && *mode != required) return;
   __shared__ int ws[kOrdThreads / 32];
   const int b = blockIdx.x, c = threadIdx.x;   // ncta <= kOrdThreads
   int* row = hist + (size_t)b * ncta;
@@ -99,8 +103,8 @@ __global__ void __launch_bounds__(kOrdThreads)
 __global__ void __launch_bounds__(kOrdThreads)
     order_scatter_kernel(const uint32_t* __restrict__ bmask, const int* __restrict__ in, int n,
                          int shift, const int* __restrict__ offs, const int* __restrict__ dtot,
-                         int* __restrict__ out, const int* mode) {
-  if (mode && *mode != kModeTensor) return;
+                         int* __restrict__ out, const int* mode, int required) {
+  if (mode && *mode != required) return;
   constexpr int kWarps = kOrdThreads / 32;
   __shared__ int run[kOrdBuckets];
   __shared__ int wc[kWarps][kOrdBuckets];
@@ -139,18 +143,19 @@ __global__ void __launch_bounds__(kOrdThreads)
   }
 }
 
-// One warp per tile of the sorted order: OR of the block masks, log Z gathered.
+// One warp per tile (`trows` rows, a multiple of 32) of the sorted order: OR of the
+// block masks, log Z gathered.
 __global__ void tile_mask_kernel(const int* __restrict__ perm, const uint32_t* __restrict__ bmask,
-                                 const float* __restrict__ logz, int n, float* __restrict__ lzp,
-                                 uint32_t* __restrict__ tmask, const int* mode) {
-  if (mode && *mode != kModeTensor) return;
+                                 const float* __restrict__ logz, int n, int trows,
+                                 float* __restrict__ lzp, uint32_t* __restrict__ tmask,
+                                 const int* mode, int required) {
+  if (mode && *mode != required) return;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t * kTileRows >= n) return;
+  if (t * trows >= n) return;
   uint32_t m = 0;
-#pragma unroll
-  for (int j = 0; j < kTileRows / 32; ++j) {
-    const int i = t * kTileRows + j * 32 + lane;
+  for (int j = 0; j < trows / 32; ++j) {
+    const int i = t * trows + j * 32 + lane;
     if (i < n) {
       const int p = perm[i];
       lzp[i] = logz[p];
@@ -164,8 +169,8 @@ __global__ void tile_mask_kernel(const int* __restrict__ perm, const uint32_t* _
 // CTA per component block b: the tiles whose mask holds b, in increasing order.
 __global__ void __launch_bounds__(kListThreads)
     block_list_kernel(const uint32_t* __restrict__ tmask, int ntiles, int* __restrict__ tlist,
-                      int stride, int* __restrict__ tcnt, const int* mode) {
-  if (mode && *mode != kModeTensor) return;
+                      int stride, int* __restrict__ tcnt, const int* mode, int required) {
+  if (mode && *mode != required) return;
   __shared__ int wsum[kListThreads / 32];
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -189,46 +194,100 @@ __global__ void __launch_bounds__(kListThreads)
   if (threadIdx.x == 0) tcnt[b] = base;
 }
 
-}  // namespace
+// CUDA-core path: per point, the 128-component blocks whose largest log z (from the
+// per-64-component maxima of the log-sum-exp sweep) lies within kSimtSkipCut of log Z.
+__global__ void simt_mask_kernel(const float* __restrict__ bmx, const float* __restrict__ logz,
+                                 int n, int nb64, int nkb, uint32_t* __restrict__ bmask,
+                                 const int* mode) {
+  if (mode && *mode != kModeSimt) return;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float lz = logz[i];
+  const float lim = lz - kSimtSkipCut;
+  uint32_t m = 0;
+  const float* b = bmx + (size_t)i * nb64;
+  for (int q = 0; q < nb64; ++q)
+    if (b[q] > lim) m |= 1u << (q >> 1);
+  const uint32_t full = nkb >= 32 ? 0xFFFFFFFFu : (1u << nkb) - 1u;
+  bmask[i] = (lz > -CUDART_INF_F && lz < CUDART_INF_F && m) ? m : full;
+}
 
-cudaError_t launch_tc_order(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
-                            const int* mode, cudaStream_t s) {
+// Radix passes over the block masks: the last one leaves the order in perm.
+cudaError_t order_sort(const Ctx& c, int nkb, int ni, const int* mode, int required,
+                       cudaStream_t s) {
   const Workspace& w = c.ws;
-  const int nkb = w.Kt / 128;
-  const int ni = (int)n;
-  const int ncta = (int)ceil_div64(n, kOrdPts);
-  const int ntiles = (int)ceil_div64(n, kTileRows);
+  const int ncta = (int)ceil_div64(ni, kOrdPts);
   const int passes = (nkb + 7) / 8;
-  cudaError_t e;
-  // ping-pong between perm2 and perm so that the last pass lands in perm
   const int* in = nullptr;
   int* out = (passes & 1) ? w.perm : w.perm2;
   for (int ps = 0; ps < passes; ++ps) {
     const int shift = 8 * ps;
-    prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
-    order_count_kernel<<<ncta, kOrdThreads, 0, s>>>(w.bmask, in, ni, shift, w.ord_hist, mode);
+    prof_begin(c, KI_TC_ORDER, s, mode, required);
+    order_count_kernel<<<ncta, kOrdThreads, 0, s>>>(w.bmask, in, ni, shift, w.ord_hist, mode,
+                                                    required);
     prof_end(c, KI_TC_ORDER, s);
-    prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
-    order_scan_kernel<<<kOrdBuckets, kOrdThreads, 0, s>>>(w.ord_hist, ncta, w.ord_tot, mode);
+    prof_begin(c, KI_TC_ORDER, s, mode, required);
+    order_scan_kernel<<<kOrdBuckets, kOrdThreads, 0, s>>>(w.ord_hist, ncta, w.ord_tot, mode,
+                                                          required);
     prof_end(c, KI_TC_ORDER, s);
-    prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
+    prof_begin(c, KI_TC_ORDER, s, mode, required);
     order_scatter_kernel<<<ncta, kOrdThreads, 0, s>>>(w.bmask, in, ni, shift, w.ord_hist,
-                                                       w.ord_tot, out, mode);
+                                                       w.ord_tot, out, mode, required);
     prof_end(c, KI_TC_ORDER, s);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     in = out;
     out = (out == w.perm) ? w.perm2 : w.perm;
   }
-  if ((e = launch_tc_convert(c, X, x_dtype, n, ldx, w.perm, mode, s)) != cudaSuccess) return e;
-  prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
+  return cudaSuccess;
+}
+
+// Tile masks (tiles of trows positions), log Z in sorted order, lists of active tiles.
+cudaError_t order_lists(const Ctx& c, int nkb, int ni, int trows, const int* mode, int required,
+                        cudaStream_t s) {
+  const Workspace& w = c.ws;
+  const int ntiles = (int)ceil_div64(ni, trows);
+  prof_begin(c, KI_TC_ORDER, s, mode, required);
   tile_mask_kernel<<<(unsigned)ceil_div64(ntiles, 8), 256, 0, s>>>(w.perm, w.bmask, w.logz, ni,
-                                                                   w.lzp, w.tmask, mode);
+                                                                   trows, w.lzp, w.tmask, mode,
+                                                                   required);
   prof_end(c, KI_TC_ORDER, s);
-  prof_begin(c, KI_TC_ORDER, s, mode, kModeTensor);
-  block_list_kernel<<<nkb, kListThreads, 0, s>>>(w.tmask, ntiles, w.tlist, (int)(kChunk / kTileRows),
-                                                 w.tcnt, mode);
+  prof_begin(c, KI_TC_ORDER, s, mode, required);
+  block_list_kernel<<<nkb, kListThreads, 0, s>>>(w.tmask, ntiles, w.tlist, (int)(kChunk / trows),
+                                                 w.tcnt, mode, required);
   prof_end(c, KI_TC_ORDER, s);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_order(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
+                            const int* mode, cudaStream_t s) {
+  const int nkb = c.ws.Kt / 128;
+  cudaError_t e;
+  if ((e = order_sort(c, nkb, (int)n, mode, kModeTensor, s)) != cudaSuccess) return e;
+  if ((e = launch_tc_convert(c, X, x_dtype, n, ldx, c.ws.perm, mode, s)) != cudaSuccess) return e;
+  return order_lists(c, nkb, (int)n, kTileRows, mode, kModeTensor, s);
+}
+
+bool simt_skip(const Ctx& c) {
+  // with fewer blocks there is too little to leave out (measured: 2 blocks at D = 960
+  // lose 13% to the ordering and the indirect loads)
+  const int nkb = (c.ws.Kp + 127) / 128;
+  return c.skip && c.ws.bmx && nkb >= 4 && nkb <= kSkipMaxBlocks;
+}
+
+cudaError_t launch_simt_order(const Ctx& c, int64_t n, const int* mode, cudaStream_t s) {
+  const Workspace& w = c.ws;
+  const int nkb = (w.Kp + 127) / 128;
+  prof_begin(c, KI_TC_ORDER, s, mode, kModeSimt);
+  simt_mask_kernel<<<(unsigned)ceil_div64(n, 256), 256, 0, s>>>(w.bmx, w.logz, (int)n, w.Kp / kKB,
+                                                                nkb, w.bmask, mode);
+  prof_end(c, KI_TC_ORDER, s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if ((e = order_sort(c, nkb, (int)n, mode, kModeSimt, s)) != cudaSuccess) return e;
+  return order_lists(c, nkb, (int)n, kTP, mode, kModeSimt, s);
 }
 
 }  // namespace fgmm

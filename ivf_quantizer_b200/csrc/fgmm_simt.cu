@@ -79,13 +79,15 @@ __global__ void prep_simt_kernel(int K, int D, int Kp, int Dp, int cov, const fl
 // summed in fp32 and the chunk sums in fp64, so that the rounding of the sum does not
 // grow with D (at D = 960 a plain fp32 sum of log-densities near -2700 carries ~5e-3
 // nats of error, enough to move the responsibilities of shared points by 0.5%).
+// rows: nullptr, or the point behind each position i0 + r (block-skipping order).
 template <int NQ, typename T>
 __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, int64_t ldx, int D,
                                            int Dp, int64_t i0, int kb,
                                            const float* __restrict__ mu,
                                            const float* __restrict__ prec,
                                            float (*xs)[kDC + 4], float (*ms)[kDC + 4],
-                                           float (*ps)[kDC + 4], float (&acc)[4][NQ]) {
+                                           float (*ps)[kDC + 4], float (&acc)[4][NQ],
+                                           const int* __restrict__ rows = nullptr) {
   constexpr int KBLK = 16 * NQ;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   double dacc[4][NQ];
@@ -103,7 +105,7 @@ __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, i
       const int r = e / kDC, cx = e % kDC;
       const int64_t i = i0 + r;
       const int d = d0 + cx;
-      xr[u] = (i < n && d < D) ? ld_x(X + i * ldx + d) : 0.f;
+      xr[u] = (i < n && d < D) ? ld_x(X + (rows ? (int64_t)rows[i] : i) * ldx + d) : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < MPT; ++u) {
@@ -169,13 +171,13 @@ __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, i
 // One CTA per 64-point tile; online log-sum-exp over blocks of 64 components
 // (Alg. 1, step 1).  Writes log Z_i for the chunk, optionally to the caller's
 // per-point buffer, and one fp64 partial log-likelihood per tile.
-template <typename T, bool KEEP>
+template <typename T, bool KEEP, bool BMAX>
 __global__ void __launch_bounds__(kSimtThreads, 2)
     lse_simt_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp, int Kp,
                     const float* __restrict__ mu, const float* __restrict__ prec,
                     const float* __restrict__ cconst, float* __restrict__ logz,
                     float* __restrict__ logz_out, double* __restrict__ ll_tiles,
-                    float* __restrict__ lbuf, const int* mode) {
+                    float* __restrict__ lbuf, float* __restrict__ bmx, const int* mode) {
   if (mode && *mode != kModeSimt) return;
   __shared__ __align__(16) float xs[kTP][kDC + 4];
   __shared__ __align__(16) float ms[kKB][kDC + 4];
@@ -206,6 +208,9 @@ __global__ void __launch_bounds__(kSimtThreads, 2)
       }
 #pragma unroll
       for (int off = 8; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+      // block skipping: the point's largest log z in this block of kKB components
+      if (BMAX && tx == 0 && i0 + ty + 16 * j < n)
+        bmx[(size_t)(i0 + ty + 16 * j) * (Kp / kKB) + kb / kKB] = bm;
       const float nm = fmaxf(run_m[j], bm);
       const bool live = nm > -CUDART_INF_F;
       float s = 0.f;
@@ -279,16 +284,34 @@ __global__ void __launch_bounds__(kSimtThreads)
                       const float* __restrict__ mu, const float* __restrict__ prec,
                       const float* __restrict__ cconst, const float* __restrict__ logz,
                       double* __restrict__ stats, int kstride, int64_t slice_len,
-                      const float* __restrict__ lbuf, const int* mode) {
+                      const float* __restrict__ lbuf, const int* __restrict__ rows,
+                      const int* __restrict__ tlist, const int* __restrict__ tcnt, int tl_stride,
+                      const int* mode) {
   if (mode && *mode != kModeSimt) return;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   StatsSmem& sm = *reinterpret_cast<StatsSmem*>(smem_raw);
   const int kb = blockIdx.x * kKBs;
   const int s = blockIdx.y;
   const int f0 = blockIdx.z * kFC;
-  const int64_t p_begin = (int64_t)s * slice_len;
-  const int64_t p_end = min(n, p_begin + slice_len);
-  if (p_begin >= p_end) return;  // uniform over the CTA
+  // Point tiles of the CTA: positions [p_begin, p_end) of the chunk in steps of kTP; or
+  // (block skipping, tlist) an even share of the active tiles of the 128-component block
+  // holding the CTA's components, over the chunk in sweep-2 order (position i is point
+  // rows[i], its log Z at logz[i]).
+  int64_t p_begin = 0, p_end = n;
+  int ntl = 0;
+  if (tlist) {
+    const int b = kb / 128;
+    const int na = tcnt[b];
+    const int per = (na + (int)gridDim.y - 1) / (int)gridDim.y;
+    const int l0 = min(na, s * per);
+    ntl = min(na, l0 + per) - l0;
+    tlist += (size_t)b * tl_stride + l0;
+    if (ntl == 0) return;  // uniform over the CTA
+  } else {
+    p_begin = (int64_t)s * slice_len;
+    p_end = min(n, p_begin + slice_len);
+    if (p_begin >= p_end) return;  // uniform over the CTA
+  }
 
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int fl = threadIdx.x % kFC;            // this thread's feature (local)
@@ -330,7 +353,10 @@ __global__ void __launch_bounds__(kSimtThreads)
   };
 
   int tiles = 0;
-  for (int64_t i0 = p_begin; i0 < p_end; i0 += kTP) {
+  for (int jt = 0;; ++jt) {
+    const int64_t i0 = tlist ? (jt < ntl ? (int64_t)__ldg(tlist + jt) * kTP : p_end)
+                             : p_begin + (int64_t)jt * kTP;
+    if (i0 >= p_end) break;   // uniform over the CTA
     if (threadIdx.x < kTP) {
       const int64_t i = i0 + threadIdx.x;
       sm.lz[threadIdx.x] = (i < p_end) ? logz[i] : -CUDART_INF_F;
@@ -343,11 +369,12 @@ __global__ void __launch_bounds__(kSimtThreads)
         const int64_t i = i0 + ty + 16 * j;
 #pragma unroll
         for (int q = 0; q < 2; ++q)
-          lg[j][q] = i < p_end ? lbuf[(size_t)i * Kp + kb + tx + 16 * q] : -CUDART_INF_F;
+          lg[j][q] = i < p_end ? lbuf[(size_t)(rows ? rows[i] : i) * Kp + kb + tx + 16 * q]
+                               : -CUDART_INF_F;
       }
     } else {
       float acc[4][2];
-      logit_tile<2>(X, p_end, ldx, D, Dp, i0, kb, mu, prec, sm.xs, sm.ms, sm.ps, acc);
+      logit_tile<2>(X, p_end, ldx, D, Dp, i0, kb, mu, prec, sm.xs, sm.ms, sm.ps, acc, rows);
 #pragma unroll
       for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -367,7 +394,7 @@ __global__ void __launch_bounds__(kSimtThreads)
       const int r = e / kFC, cx = e % kFC;
       const int64_t i = i0 + r;
       const int d = f0 + cx;
-      sm.xf[r][cx] = (i < p_end && d < D) ? ld_x(X + i * ldx + d) : 0.f;
+      sm.xf[r][cx] = (i < p_end && d < D) ? ld_x(X + (rows ? (int64_t)rows[i] : i) * ldx + d) : 0.f;
     }
     __syncthreads();
 #pragma unroll 2
@@ -744,15 +771,24 @@ cudaError_t launch_lse_simt(const Ctx& c, const void* X, int x_dtype, int64_t n,
                             float* logz_out, bool keep_logits, const int* mode, cudaStream_t s) {
   const unsigned grid = (unsigned)ceil_div64(n, kTP);
   float* lb = keep_logits ? c.ws.lbuf : nullptr;
+  float* bx = keep_logits && simt_skip(c) ? c.ws.bmx : nullptr;
   prof_begin(c, KI_LSE_SIMT, s, mode, kModeSimt);
-#define LSE_SIMT(T_, K_)                                                                        \
-  lse_simt_kernel<T_, K_><<<grid, kSimtThreads, 0, s>>>(                                        \
+#define LSE_SIMT(T_, K_, B_)                                                                    \
+  lse_simt_kernel<T_, K_, B_><<<grid, kSimtThreads, 0, s>>>(                                    \
       (const T_*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst, c.ws.logz,  \
-      logz_out, c.ws.ll_tiles, lb, mode)
+      logz_out, c.ws.ll_tiles, lb, bx, mode)
   if (x_dtype == FGMM_BF16) {
-    if (lb) LSE_SIMT(__nv_bfloat16, true); else LSE_SIMT(__nv_bfloat16, false);
+    if (lb) {
+      if (bx) LSE_SIMT(__nv_bfloat16, true, true); else LSE_SIMT(__nv_bfloat16, true, false);
+    } else {
+      if (bx) LSE_SIMT(__nv_bfloat16, false, true); else LSE_SIMT(__nv_bfloat16, false, false);
+    }
   } else {
-    if (lb) LSE_SIMT(float, true); else LSE_SIMT(float, false);
+    if (lb) {
+      if (bx) LSE_SIMT(float, true, true); else LSE_SIMT(float, true, false);
+    } else {
+      if (bx) LSE_SIMT(float, false, true); else LSE_SIMT(float, false, false);
+    }
   }
 #undef LSE_SIMT
   prof_end(c, KI_LSE_SIMT, s);
@@ -783,16 +819,23 @@ cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t 
   int64_t slice = ceil_div64(n, kSlices);
   slice = ceil_div64(slice, kTP) * kTP;
   dim3 grid(c.ws.Kp / kKBs, kSlices, (unsigned)ceil_div64(c.ws.Dp, kFC));
+  // block skipping: the chunk in sweep-2 order (rows, log Z), tiles from the lists
+  const bool skip = simt_skip(c);
+  const int* rows = skip ? c.ws.perm : nullptr;
+  const float* lz = skip ? c.ws.lzp : c.ws.logz;
+  const int* tl = skip ? c.ws.tlist : nullptr;
+  const int tl_stride = (int)(kChunk / kTP);
   prof_begin(c, KI_STATS_SIMT, s, mode, kModeSimt);
   if (x_dtype == FGMM_BF16)
     stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>(
         (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
-        c.ws.logz, c.ws.stats, c.ws.KpS, slice, c.ws.lbuf, mode);
+        lz, c.ws.stats, c.ws.KpS, slice, c.ws.lbuf, rows, tl, c.ws.tcnt, tl_stride, mode);
   else
     stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>((const float*)X, n, ldx, c.D, c.ws.Dp,
                                                        c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
-                                                       c.ws.logz, c.ws.stats, c.ws.KpS, slice,
-                                                       c.ws.lbuf, mode);
+                                                       lz, c.ws.stats, c.ws.KpS, slice,
+                                                       c.ws.lbuf, rows, tl, c.ws.tcnt, tl_stride,
+                                                       mode);
   prof_end(c, KI_STATS_SIMT, s);
   return cudaGetLastError();
 }

@@ -10,6 +10,11 @@ from run to run and within the parity tolerances of the oracle.
 Cases: well separated (one block per point), partly overlapping (a mix of one-block and
 several-block points), fully overlapping (every point in every block), the largest
 block count (K = 4096: 32 blocks), two blocks with a ragged tail, two chunks, AUTO.
+
+The CUDA-core path (FGMM_PREC_FP32) skips the same way with a cut of 50 nats (each
+left-out responsibility is below 2e-22): checked on the IVF shape, on D = 960 (its
+statistics read the log-densities kept by sweep 1, through the reordering) and on
+32 blocks.
 """
 import numpy as np
 import pytest
@@ -26,7 +31,7 @@ def _step(X, w, mu, var, skip, prec="fp16x3", steps=1):
     import ivf_quantizer_b200 as q
     K, D = mu.shape
     g = q.GMM(K, D)
-    g.set_precision({"fp16x3": q.PREC_FP16X3, "auto": q.PREC_AUTO}[prec])
+    g.set_precision({"fp16x3": q.PREC_FP16X3, "auto": q.PREC_AUTO, "fp32": q.PREC_FP32}[prec])
     g.set_block_skip(skip)
     assert g.block_skip == skip
     Xd = torch.as_tensor(X).cuda().contiguous()
@@ -189,3 +194,33 @@ def test_skip_shortens_the_statistics_sweep():
         g.close()
     print(ms)
     assert ms[True] < 0.6 * ms[False]
+
+
+def test_fp32_path_ivf_shape():
+    X = synth.generate("ivf", 20_000 + 11, seed=13)
+    w, mu, var = synth.init_params(X, 512, seed=13)   # 4 blocks of 128 components
+    a = _step(X, w, mu, var, True, prec="fp32")
+    b = _step(X, w, mu, var, False, prec="fp32")
+    _agree(a, b, X)
+    compare_step(a[:3], _oracle(X, w, mu, var), X.numpy(), logz_gpu=a[4], loglik_gpu=a[3])
+
+
+def test_fp32_path_high_dimension():
+    X = synth.generate("border", 4_000 + 3, seed=14)
+    w, mu, var = synth.init_params(X, 512, seed=14)   # D = 960: kept log-densities
+    a = _step(X, w, mu, var, True, prec="fp32")
+    b = _step(X, w, mu, var, False, prec="fp32")
+    _agree(a, b, X)
+    compare_step(a[:3], _oracle(X, w, mu, var), X.numpy(), logz_gpu=a[4], loglik_gpu=a[3])
+
+
+def test_fp32_path_most_blocks_two_steps():
+    X = synth.generate("table1", 6_000, seed=15)[:, :64].contiguous()
+    w, mu, var = synth.init_params(X, 4096, seed=15)  # 32 blocks
+    a = _step(X, w, mu, var, True, prec="fp32")
+    b = _step(X, w, mu, var, False, prec="fp32")
+    _agree(a, b, X)
+    a2 = _step(X, w, mu, var, True, prec="fp32", steps=2)
+    b2 = _step(X, w, mu, var, True, prec="fp32", steps=2)
+    for ta, tb in zip(a2[:3], b2[:3]):
+        assert np.array_equal(ta, tb)                  # bitwise reproducible
