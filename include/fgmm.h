@@ -104,8 +104,12 @@ int fgmm_get_precision(fgmm_handle h, int* prec_out);
  * log Z_i.  Sweep 2 then visits the points grouped by those marks, and only the
  * (128-point tile, block) pairs that hold a mark; every pair it leaves out adds
  * exactly 0.  Results match the dense sweep up to the order of fp32 additions and stay
- * bitwise reproducible from run to run.  Only K of 129 ... 4096 is affected (2 to 32
- * blocks); the CUDA-core path never is.
+ * bitwise reproducible from run to run.  Tensor-core path: K of 129 ... 4096 (2 to 32
+ * blocks).  The CUDA-core path (FGMM_PREC_FP32, or an AUTO step sent there) skips the
+ * same way for K of 385 ... 4096 (4 to 32 blocks, counted as K rounded up to 64, then
+ * to 128).  Its fp32 statistics keep responsibilities down to about e^-104, so there a
+ * pair is left out only when every log-density is 50 nats or more below log Z_i: each
+ * dropped r is below 2e-22.
  * enable: 0 off, nonzero on.  FGMM_ERR_INVALID_ARG for a NULL handle. */
 int fgmm_set_block_skip(fgmm_handle h, int enable);
 int fgmm_get_block_skip(fgmm_handle h, int* enable_out);
