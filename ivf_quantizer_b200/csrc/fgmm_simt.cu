@@ -278,7 +278,7 @@ struct StatsSmem {
   float lz[kTP];
 };
 
-template <typename T>
+template <typename T, bool LISTED>
 __global__ void __launch_bounds__(kSimtThreads)
     stats_simt_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp, int Kp,
                       const float* __restrict__ mu, const float* __restrict__ prec,
@@ -299,7 +299,11 @@ __global__ void __launch_bounds__(kSimtThreads)
   // rows[i], its log Z at logz[i]).
   int64_t p_begin = 0, p_end = n;
   int ntl = 0;
-  if (tlist) {
+  if (!LISTED) {   // compile-time: the plain path carries none of the reordering
+    rows = nullptr;
+    tlist = nullptr;
+  }
+  if (LISTED) {
     const int b = kb / 128;
     const int na = tcnt[b];
     const int per = (na + (int)gridDim.y - 1) / (int)gridDim.y;
@@ -354,8 +358,8 @@ __global__ void __launch_bounds__(kSimtThreads)
 
   int tiles = 0;
   for (int jt = 0;; ++jt) {
-    const int64_t i0 = tlist ? (jt < ntl ? (int64_t)__ldg(tlist + jt) * kTP : p_end)
-                             : p_begin + (int64_t)jt * kTP;
+    const int64_t i0 = LISTED ? (jt < ntl ? (int64_t)__ldg(tlist + jt) * kTP : p_end)
+                              : p_begin + (int64_t)jt * kTP;
     if (i0 >= p_end) break;   // uniform over the CTA
     if (threadIdx.x < kTP) {
       const int64_t i = i0 + threadIdx.x;
@@ -810,9 +814,13 @@ cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t 
   const size_t smem = sizeof(StatsSmem);
   static bool attr_set = false;
   if (!attr_set) {
-    cudaFuncSetAttribute(stats_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    cudaFuncSetAttribute(stats_simt_kernel<__nv_bfloat16>,
+    cudaFuncSetAttribute(stats_simt_kernel<float, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(stats_simt_kernel<__nv_bfloat16, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(stats_simt_kernel<float, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(stats_simt_kernel<__nv_bfloat16, true>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     attr_set = true;
   }
@@ -826,16 +834,16 @@ cudaError_t launch_stats_simt(const Ctx& c, const void* X, int x_dtype, int64_t 
   const int* tl = skip ? c.ws.tlist : nullptr;
   const int tl_stride = (int)(kChunk / kTP);
   prof_begin(c, KI_STATS_SIMT, s, mode, kModeSimt);
-  if (x_dtype == FGMM_BF16)
-    stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>(
-        (const __nv_bfloat16*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
-        lz, c.ws.stats, c.ws.KpS, slice, c.ws.lbuf, rows, tl, c.ws.tcnt, tl_stride, mode);
-  else
-    stats_simt_kernel<<<grid, kSimtThreads, smem, s>>>((const float*)X, n, ldx, c.D, c.ws.Dp,
-                                                       c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst,
-                                                       lz, c.ws.stats, c.ws.KpS, slice,
-                                                       c.ws.lbuf, rows, tl, c.ws.tcnt, tl_stride,
-                                                       mode);
+#define STATS_SIMT(T_, L_)                                                                      \
+  stats_simt_kernel<T_, L_><<<grid, kSimtThreads, smem, s>>>(                                   \
+      (const T_*)X, n, ldx, c.D, c.ws.Dp, c.ws.Kp, c.ws.mu, c.ws.prec, c.ws.cconst, lz,         \
+      c.ws.stats, c.ws.KpS, slice, c.ws.lbuf, rows, tl, c.ws.tcnt, tl_stride, mode)
+  if (x_dtype == FGMM_BF16) {
+    if (skip) STATS_SIMT(__nv_bfloat16, true); else STATS_SIMT(__nv_bfloat16, false);
+  } else {
+    if (skip) STATS_SIMT(float, true); else STATS_SIMT(float, false);
+  }
+#undef STATS_SIMT
   prof_end(c, KI_STATS_SIMT, s);
   return cudaGetLastError();
 }
