@@ -239,7 +239,9 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
 // ------------------------------------------------------------------ X -> phi (fp16 hi / lo)
 // Thread per (point, group of 8 dims).  xop[part][i][j]: part 0 hi, 1 lo; j < Dq the
 // scaled centred coordinate, Dq + d its square.  With perm, row i holds point perm[i].
-template <typename T>
+// VEC (fp32 X, 16-byte aligned rows, D a multiple of 8): each group of 8 features is
+// read as two 16-byte loads.
+template <typename T, bool VEC>
 __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dq,
                                   int64_t ncmax, const float* __restrict__ center,
                                   const float* __restrict__ scale, __half* __restrict__ xop,
@@ -253,13 +255,24 @@ __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ld
   const int64_t src = perm ? (int64_t)__ldg(perm + i) : i;
   const int K1 = 2 * Dq;
   __align__(16) __half xh[8], xl[8], qh[8], ql[8];
+  float xr[8];
+  if constexpr (VEC) {
+    if (8 * g < D) {
+      const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(X) +
+                                                        src * ldx + 8 * g);
+      const float4 a = __ldg(p), b = __ldg(p + 1);
+      xr[0] = a.x; xr[1] = a.y; xr[2] = a.z; xr[3] = a.w;
+      xr[4] = b.x; xr[5] = b.y; xr[6] = b.z; xr[7] = b.w;
+    }
+  }
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int d = 8 * g + u;
     float xv = 0.f;
     if (d < D) {
       float x;
-      if constexpr (sizeof(T) == 4) x = __ldg(reinterpret_cast<const float*>(X) + src * ldx + d);
+      if constexpr (VEC) x = xr[u];
+      else if constexpr (sizeof(T) == 4) x = __ldg(reinterpret_cast<const float*>(X) + src * ldx + d);
       else x = __bfloat162float(X[src * ldx + d]);
       xv = (x - center[d]) * scale[d];
     }
@@ -1206,12 +1219,17 @@ cudaError_t launch_tc_convert(const Ctx& c, const void* X, int x_dtype, int64_t 
   const unsigned grid = (unsigned)ceil_div64(total, 256);
   const KernelId id = perm ? KI_TC_GATHER : KI_TC_CONVERT;
   prof_begin(c, id, s, mode, kModeTensor);
+  const bool vec = x_dtype == FGMM_F32 && (uintptr_t)X % 16 == 0 && ldx % 4 == 0 && c.D % 8 == 0;
   if (x_dtype == FGMM_BF16)
-    tc_convert_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dq, kChunk,
-                                           w.center, w.dscale, w.xop, perm, mode);
+    tc_convert_kernel<__nv_bfloat16, false><<<grid, 256, 0, s>>>(
+        (const __nv_bfloat16*)X, n, ldx, c.D, w.Dq, kChunk, w.center, w.dscale, w.xop, perm, mode);
+  else if (vec)
+    tc_convert_kernel<float, true><<<grid, 256, 0, s>>>((const float*)X, n, ldx, c.D, w.Dq, kChunk,
+                                                        w.center, w.dscale, w.xop, perm, mode);
   else
-    tc_convert_kernel<<<grid, 256, 0, s>>>((const float*)X, n, ldx, c.D, w.Dq, kChunk, w.center,
-                                           w.dscale, w.xop, perm, mode);
+    tc_convert_kernel<float, false><<<grid, 256, 0, s>>>((const float*)X, n, ldx, c.D, w.Dq,
+                                                         kChunk, w.center, w.dscale, w.xop, perm,
+                                                         mode);
   prof_end(c, id, s);
   return cudaGetLastError();
 }
