@@ -170,7 +170,7 @@ void free_ws(Workspace& w) {
                   w.stats,  w.nk,     w.status, w.center, w.dscale, w.wop,
                   w.tck,    w.tks,    w.xop,    w.mode, w.stiff,    w.stiff_list, w.n_stiff,
                   w.side_part, w.mode2, w.canon, w.tcraw, w.tcm, w.tcpk, w.tckf, w.lzlow,
-                  w.side_flag, w.pair_cnt, w.pair_j, w.pair_l, w.flagged, w.n_flagged, w.km_word,
+                  w.side_flag, w.pair_cnt, w.pair_j, w.pair_l, w.flagged, w.n_flagged, w.flag_cnt, w.km_word,
                   w.grey, w.grey_pos,
                   w.grey_stats,
                   w.lbuf, w.bmx, w.bmask, w.perm, w.perm2, w.lzp, w.ord_hist, w.ord_tot, w.tmask, w.tlist, w.tcnt};
@@ -258,6 +258,7 @@ cudaError_t alloc_ws(Ctx& c) {
     if ((e = alloc(&w.pair_l, (size_t)kChunk * kSidePairs, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.flagged, (size_t)kChunk, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.n_flagged, (size_t)1, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.flag_cnt, (size_t)(kChunk / 4096), &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.xop, (size_t)2 * kChunk * w.K1, &t)) != cudaSuccess) return e;
     // rows past the end of a short chunk are read by the tensor cores (and multiplied
     // by r = 0): keep them finite from the start

@@ -96,6 +96,7 @@ struct Workspace {
   float* pair_l = nullptr;       // [kChunk][kSidePairs] their log z
   int* flagged = nullptr;        // [kChunk] the flagged points of the chunk, as a list
   int* n_flagged = nullptr;      // [1] their number
+  int* flag_cnt = nullptr;       // [kChunk / 4096] flagged points per 4096-point block
   __half* xop = nullptr;    // [2][kChunk][K1] phi(x) hi / lo of the current chunk
   // block skipping (sweep 2 visits only the (tile, block) pairs that can contribute)
   uint32_t* bmask = nullptr;  // [kChunk] per point: blocks within kSkipCut of log Z

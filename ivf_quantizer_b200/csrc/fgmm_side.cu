@@ -147,34 +147,63 @@ __global__ void stiff_compact_kernel(const int* __restrict__ stiff, const int* _
   }
 }
 
-// The flagged points of the chunk, as a list (in no particular order: each is handled on
-// its own), so that side_lse runs on full warps; the other points get pair count 0.
+// The flagged points of the chunk as a list in increasing index order, so that side_lse
+// runs on full warps and side_stats visits only them, deterministically: per 4096-point
+// CTA a count (side_flag_count), then each CTA writes its points after those of the CTAs
+// before it (side_flagged).  Unflagged points get pair count 0.
+__global__ void side_flag_count_kernel(const uint8_t* __restrict__ flag, int64_t n,
+                                       const int* __restrict__ n_stiff, int* __restrict__ cnts,
+                                       uint8_t* __restrict__ pair_cnt, const int* mode) {
+  if (mode && *mode != kModeTensor) return;
+  if (n_stiff[0] + n_stiff[1] == 0) return;
+  __shared__ int wsum[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t i0 = (int64_t)blockIdx.x * 4096;
+  int c = 0;
+  for (int r0 = 0; r0 < 4096; r0 += 256) {
+    const int64_t i = i0 + r0 + threadIdx.x;
+    const bool f = i < n && flag[i];
+    if (i < n && !f) pair_cnt[i] = 0;
+    c += __popc(__ballot_sync(0xffffffffu, f));
+  }
+  if (lane == 0) wsum[warp] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int w2 = 0; w2 < 8; ++w2) t += wsum[w2];
+    cnts[blockIdx.x] = t;
+  }
+}
+
 __global__ void side_flagged_kernel(const uint8_t* __restrict__ flag, int64_t n,
-                                    const int* __restrict__ n_stiff, int* __restrict__ list,
-                                    int* __restrict__ count, uint8_t* __restrict__ pair_cnt,
+                                    const int* __restrict__ n_stiff, const int* __restrict__ cnts,
+                                    int* __restrict__ list, int* __restrict__ count,
                                     const int* mode) {
   if (mode && *mode != kModeTensor) return;
   if (n_stiff[0] + n_stiff[1] == 0) return;
   __shared__ int wsum[8], base;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int b = 0; b < (int)blockIdx.x; ++b) t += cnts[b];
+    base = t;
+    if (blockIdx.x == gridDim.x - 1) *count = t + cnts[blockIdx.x];
+  }
   const int64_t i0 = (int64_t)blockIdx.x * 4096;
   for (int r0 = 0; r0 < 4096; r0 += 256) {
     const int64_t i = i0 + r0 + threadIdx.x;
     const bool f = i < n && flag[i];
-    if (i < n && !f) pair_cnt[i] = 0;
     const unsigned m = __ballot_sync(0xffffffffu, f);
     if (lane == 0) wsum[warp] = __popc(m);
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int t = 0;
-      for (int w2 = 0; w2 < 8; ++w2) t += wsum[w2];
-      base = t ? atomicAdd(count, t) : 0;
+    int off = base, tot = 0;
+    for (int w2 = 0; w2 < 8; ++w2) {
+      off += w2 < warp ? wsum[w2] : 0;
+      tot += wsum[w2];
     }
-    __syncthreads();
-    int off = base;
-    for (int w2 = 0; w2 < warp; ++w2) off += wsum[w2];
     if (f) list[off + __popc(m & ((1u << lane) - 1u))] = (int)i;
     __syncthreads();
+    if (threadIdx.x == 0) base += tot;
   }
 }
 
@@ -264,7 +293,9 @@ __global__ void __launch_bounds__(256)
                       const float* __restrict__ cconst, const int* __restrict__ list,
                       const int* __restrict__ n_stiff, const uint8_t* __restrict__ pair_cnt,
                       const uint8_t* __restrict__ pair_j, const float* __restrict__ pair_l,
-                      const float* __restrict__ logz, double* __restrict__ part, const int* mode) {
+                      const float* __restrict__ logz, const int* __restrict__ flagged,
+                      const int* __restrict__ n_flagged, double* __restrict__ part,
+                      const int* mode) {
   if (mode && *mode != kModeTensor) return;
   const int j = blockIdx.x;
   if (j >= n_stiff[0] + n_stiff[1]) return;   // stiff, then grey components
@@ -274,8 +305,10 @@ __global__ void __launch_bounds__(256)
   const float* muk = mu + (size_t)k * Dp;
   const float* pk = prec + (size_t)k * Dp;
   const float ck = cconst[k];
-  const int64_t range = (n + kSideParts - 1) / kSideParts;
-  const int64_t p0 = (int64_t)blockIdx.y * range, p1 = min(n, p0 + range);
+  // the p-th of kSideParts equal ranges of the flagged list (points in index order)
+  const int64_t nf = *n_flagged;
+  const int64_t range = (nf + kSideParts - 1) / kSideParts;
+  const int64_t p0 = (int64_t)blockIdx.y * range, p1 = min(nf, p0 + range);
   const int64_t wlen = (range + 7) / 8;
   const int64_t w0 = p0 + warp * wlen, w1 = min(p1, w0 + wlen);
   SideAcc& a = acc[warp];
@@ -283,9 +316,9 @@ __global__ void __launch_bounds__(256)
   float nk = 0.f;
   __syncwarp();
   for (int64_t b = w0; b < w1; b += 32) {
-    const int64_t i = b + lane;
+    const int64_t i = b + lane < w1 ? (int64_t)flagged[b + lane] : 0;
     float r = 0.f;
-    const int cnt = i < w1 ? pair_cnt[i] : 0;
+    const int cnt = b + lane < w1 ? pair_cnt[i] : 0;
     if (cnt > 0) {
       const float lz = logz[i];
       float l = -CUDART_INF_F;
@@ -302,7 +335,7 @@ __global__ void __launch_bounds__(256)
       const int src = __ffs(live) - 1;
       live &= live - 1;
       const float rr = __shfl_sync(0xffffffffu, r, src);
-      const T* x = X + (b + src) * ldx;
+      const T* x = X + __shfl_sync(0xffffffffu, i, src) * ldx;
       for (int d = lane; d < D; d += 32) {
         const float t = ldx_f(x + d) - muk[d];
         const float rt = rr * t;
@@ -370,11 +403,16 @@ cudaError_t launch_side_lse(const Ctx& c, const void* X, int x_dtype, int64_t n,
                             float* logz_out, const int* mode, cudaStream_t s) {
   const unsigned grid = (unsigned)ceil_div64(n, 128);
   const Workspace& w = c.ws;
+  const unsigned nfc = (unsigned)ceil_div64(n, 4096);
   cudaError_t e = cudaMemsetAsync(w.n_flagged, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
   prof_begin(c, KI_SIDE_LSE, s, mode, kModeTensor);
-  side_flagged_kernel<<<(unsigned)ceil_div64(n, 4096), 256, 0, s>>>(
-      w.side_flag, n, w.n_stiff, w.flagged, w.n_flagged, w.pair_cnt, mode);
+  side_flag_count_kernel<<<nfc, 256, 0, s>>>(w.side_flag, n, w.n_stiff, w.flag_cnt, w.pair_cnt,
+                                             mode);
+  prof_end(c, KI_SIDE_LSE, s);
+  prof_begin(c, KI_SIDE_LSE, s, mode, kModeTensor);
+  side_flagged_kernel<<<nfc, 256, 0, s>>>(w.side_flag, n, w.n_stiff, w.flag_cnt, w.flagged,
+                                          w.n_flagged, mode);
   prof_end(c, KI_SIDE_LSE, s);
   prof_begin(c, KI_SIDE_LSE, s, mode, kModeTensor);
   if (x_dtype == FGMM_BF16)
@@ -404,11 +442,13 @@ cudaError_t launch_side_stats(const Ctx& c, const void* X, int x_dtype, int64_t 
   if (x_dtype == FGMM_BF16)
     side_stats_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)X, n, ldx, c.D, w.Dp, w.mu,
                                            w.prec, w.cconst, w.stiff_list, w.n_stiff, w.pair_cnt,
-                                           w.pair_j, w.pair_l, w.logz, w.side_part, mode);
+                                           w.pair_j, w.pair_l, w.logz, w.flagged, w.n_flagged,
+                                           w.side_part, mode);
   else
     side_stats_kernel<<<grid, 256, 0, s>>>((const float*)X, n, ldx, c.D, w.Dp, w.mu, w.prec,
                                            w.cconst, w.stiff_list, w.n_stiff, w.pair_cnt,
-                                           w.pair_j, w.pair_l, w.logz, w.side_part, mode);
+                                           w.pair_j, w.pair_l, w.logz, w.flagged, w.n_flagged,
+                                           w.side_part, mode);
   prof_end(c, KI_SIDE_STATS, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
