@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kOrdThreads)
   __shared__ int run[kOrdBuckets];
   __shared__ int wc[kWarps][kOrdBuckets];
   __shared__ int ws[kWarps];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int warp = threadIdx.x >> 5;
   {  // first position of digit b: the totals of the smaller digits + earlier CTAs' counts
     const int b = threadIdx.x;   // kOrdThreads == kOrdBuckets
     int tot;
