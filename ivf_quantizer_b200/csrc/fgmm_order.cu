@@ -1,4 +1,4 @@
-// Block skipping in the tensor-core statistics sweep: the point order of sweep 2.
+// Block skipping in the statistics sweep: the point order of sweep 2 (both paths).
 //
 // Paper: "Flash-GMM: A Memory-Efficient Kernel for Scalable Soft Clustering", §3.1 and
 // Algorithm 1.  Sweep 2 forms r_ik = exp(log z_ik - log Z_i) for every point and every
@@ -18,6 +18,11 @@
 // then runs each block over its own list.  Every step is deterministic (counts, prefix
 // sums, ordered scatter), so the sums stay bitwise reproducible from run to run; they
 // differ from the natural order only by the order of fp32 additions.
+//
+// The CUDA-core path uses the same sort and lists with 64-point tiles: simt_mask builds
+// the masks from sweep 1's per-64-component maxima against log Z - kSimtSkipCut (its fp32
+// statistics keep r down to e^-104, so there the cut is set for r < 2e-22 instead), and
+// its statistics sweep reads X through the permutation instead of a converted copy.
 #include <math_constants.h>
 
 #include "fgmm_internal.h"
