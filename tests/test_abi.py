@@ -67,6 +67,10 @@ def test_calls_on_null_handle_are_invalid():
     assert LIB.fgmm_soft_assign(z, one, 0, 10, 4, one, one, one, 1, 0.0, one, z, z) == \
         _lib.ERR_INVALID_ARG
     assert LIB.fgmm_set_precision(z, 0) == _lib.ERR_INVALID_ARG
+    assert LIB.fgmm_set_block_skip(z, 1) == _lib.ERR_INVALID_ARG
+    v = ctypes.c_int(7)
+    assert LIB.fgmm_get_block_skip(z, ctypes.byref(v)) == _lib.ERR_INVALID_ARG
+    assert v.value == 7
     assert LIB.fgmm_get_status(z, z) == _lib.ERR_INVALID_ARG
     assert LIB.fgmm_destroy(z) == _lib.OK
 
