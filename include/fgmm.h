@@ -54,8 +54,11 @@ enum fgmm_cov { FGMM_COV_DIAG = 0, FGMM_COV_SPHERICAL = 1 };
  *            accumulation (about 22 significant bits per product).
  *   FP16   : tensor cores, one fp16 product per term (fast, ~11 bits; fails
  *            the 1e-4 log-likelihood tolerance on the Table-1 generator).
- *   AUTO   : the default; FP16X3 where every component is well conditioned for
- *            the expanded form, FP32 otherwise (decided on the device per step). */
+ *   AUTO   : the default; FP16X3 for the components that are well conditioned for
+ *            the expanded form, the others ("stiff") on a CUDA-core side path in the
+ *            direct form, decided per component and per step on the device; the whole
+ *            step goes to FP32 when more than 256 components are stiff or a variance
+ *            check still fails after one redo pass. */
 enum fgmm_prec { FGMM_PREC_FP32 = 0, FGMM_PREC_FP16X3 = 1, FGMM_PREC_FP16 = 2, FGMM_PREC_AUTO = 3 };
 
 /* Element type of X. */
