@@ -28,17 +28,21 @@
 // Kernels (one chunk of <= 2^20 points at a time):
 //   tc_center     per-dimension centre and scale from the parameters
 //   tc_prep       W' hi/lo, c_k, 2^t_k; conditioning check for AUTO mode
-//   tc_convert    X chunk -> phi hi/lo (fp16, row-major, TMA-ready)
-//   tc_lse        sweep 1: persistent, one 128-point tile per CTA at a time; phi tile
-//                 resident in smem, W streamed through a TMA ring; S = phi W^T in
-//                 TMEM (double buffered), online log-sum-exp by a 4-warp epilogue.
-//   tc_stats      sweep 2: CTA owns a 128-component block (W resident) and a slice
-//                 of points; S^T = W phi^T in TMEM, responsibilities written as the
-//                 A operand of the second GEMM acc += R^T phi (TMEM, 128 x 2Dq),
-//                 flushed to the CTA's fp64 slot.
+//   tc_convert    X chunk -> phi hi/lo (fp16, row-major, TMA-ready); with a
+//                 permutation, the chunk in sweep-2 order (block skipping)
+//   tc_lse        sweep 1: persistent, one 128-point tile per CTA at a time; phi hi
+//                 resident in smem, phi lo in TMEM, W' streamed through a TMA ring;
+//                 S = phi W'^T in TMEM (double buffered), online log-sum-exp by 16
+//                 epilogue warps (four column quarters), block masks for skipping.
+//   tc_stats      sweep 2: CTA owns a 128-component block (W' hi resident in smem, lo
+//                 in TMEM) and a slice of points, or with block skipping a share of the
+//                 block's active tiles; S^T = W' phi^T in TMEM, responsibilities
+//                 written as the A operand of the second GEMM acc += R^T phi (TMEM,
+//                 128 x 2Dq), flushed to the CTA's fp64 slot.
 //
 // Warp roles in both sweeps: warp 0 TMA producer, warp 1 MMA issuer (one thread,
-// also owns the TMEM allocation), warps 4..7 epilogue (TMEM lane quarters 0..3).
+// also owns the TMEM allocation), warps 4.. epilogue (warp w reads TMEM lane quarter
+// w % 4): 16 epilogue warps in sweep 1, 8 in sweep 2.
 // Every wait is bounded (ptx::mbar_wait); on expiry the kernel latches
 // FGMM_ERR_TIMEOUT, the other roles see the abort flag, and the CTA drains and frees
 // its TMEM before returning.
