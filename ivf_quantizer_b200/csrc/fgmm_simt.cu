@@ -11,8 +11,12 @@
 // This is the FGMM_PREC_FP32 mode: log-densities in the direct form
 // sum_d -(x_d - mu_kd)^2 / (2 sigma_kd^2), statistics centred on each
 // component's current mean (sum r (x - mu), sum r (x - mu)^2), which keeps the
-// variance update free of cancellation.  The N x K matrix of responsibilities
-// only ever exists as one 64 x 32 tile in shared memory.
+// variance update free of cancellation.  The responsibilities only ever exist as
+// one 64 x 32 tile in shared memory.  Two exceptions: for D > 128 the log-sum-exp sweep
+// keeps the chunk's log-densities (2^20 x Kp) for the statistics sweep, whose
+// feature-block CTAs would otherwise each recompute them.  With block skipping it
+// writes each point's largest log-density per 64 components, and the statistics sweep
+// visits the points in the resulting order (fgmm_order.cu).
 //
 // Data layout: prepared parameters are zero padded to [Kp, Dp] (Kp multiple of
 // 64, Dp multiple of 32); padded / dead components carry cconst = -inf so that
