@@ -6,10 +6,14 @@
 // ("Flash-GMM: A Memory-Efficient Kernel for Scalable Soft Clustering", §2 for the
 // density and Eqs. (1)-(3); the same quantities as the tensor-core sweeps, exactly).
 //
-//   stiff_compact      ordered list of the stiff components (deterministic)
-//   side_lse           per point: log Z <- logsumexp(log Z_tensor, log z_ik for stiff k)
+//   stiff_compact      ordered list of the stiff (then grey) components (deterministic)
+//   side_flag_count,   the points that sweep 1 flagged (a side component may come within
+//   side_flagged       the cut), as a list in index order
+//   side_lse           per flagged point: log Z <- logsumexp(log Z_tensor, log z_ik for
+//                      stiff k); keeps the (component, log z) pairs within the cut
 //   ll_partials        per-block fp64 sums of the chunk's log Z (fixed order)
-//   side_stats         per stiff component: N_k, sum r (x - mu), sum r (x - mu)^2
+//   side_stats         per side component, over the flagged list: N_k, sum r (x - mu),
+//                      sum r (x - mu)^2 from the kept pairs
 //
 // A stiff component's log-density is evaluated dimension by dimension and abandoned
 // as soon as its upper bound (the constant plus the partial sum, every remaining term
