@@ -122,6 +122,27 @@ int fgmm_get_block_skip(fgmm_handle h, int* enable_out);
  * device per step, so this call synchronises the device.  -1 before any step. */
 int fgmm_last_step_path(fgmm_handle h, int* path_out);
 
+/* What the last fgmm_em_step / fgmm_em_partial of this handle did, for tests and
+ * benchmarks that must show which regime they covered.  Synchronises the device.
+ *   path           : as fgmm_last_step_path (-1 before any step)
+ *   n_stiff        : FGMM_PREC_AUTO: components the last pass evaluated on the CUDA-core
+ *                    side path (ill-conditioned for the expanded form); 0 otherwise
+ *   n_grey         : FGMM_PREC_AUTO: components kept on the tensor cores whose statistics
+ *                    the side path also took (fewer than 8 effective points before)
+ *   skip_pairs     : block skipping, last chunk of the last tensor-core pass: the
+ *                    (point tile, component block) pairs the statistics sweep visited;
+ *                    -1 when that sweep ran dense or did not run
+ *   skip_pairs_all : the pairs a dense sweep of that chunk visits (tiles x blocks)
+ * FGMM_ERR_INVALID_ARG for a NULL handle or output. */
+typedef struct fgmm_step_info {
+  int path;
+  int n_stiff;
+  int n_grey;
+  int64_t skip_pairs;
+  int64_t skip_pairs_all;
+} fgmm_step_info;
+int fgmm_last_step_info(fgmm_handle h, fgmm_step_info* out);
+
 /* Bytes of device memory the handle holds (independent of N). */
 int fgmm_workspace_bytes(fgmm_handle h, size_t* bytes_out);
 

@@ -37,6 +37,11 @@ class Profile(ctypes.Structure):
                 ("kernel_active_ms", ctypes.c_double * PROF_KERNELS)]
 
 
+class StepInfo(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("n_stiff", ctypes.c_int), ("n_grey", ctypes.c_int),
+                ("skip_pairs", ctypes.c_int64), ("skip_pairs_all", ctypes.c_int64)]
+
+
 # every exported symbol of include/fgmm.h with (restype, argtypes)
 _c = ctypes
 _vp, _i64, _int, _dbl, _flt = _c.c_void_p, _c.c_int64, _c.c_int, _c.c_double, _c.c_float
@@ -49,6 +54,7 @@ SIGNATURES = {
     "fgmm_get_block_skip": (_int, [_vp, _c.POINTER(_int)]),
     "fgmm_workspace_bytes": (_int, [_vp, _c.POINTER(_c.c_size_t)]),
     "fgmm_last_step_path": (_int, [_vp, _c.POINTER(_int)]),
+    "fgmm_last_step_info": (_int, [_vp, _c.POINTER(StepInfo)]),
     "fgmm_em_step": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_fit": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _int, _dbl,
                         _c.POINTER(_dbl), _c.POINTER(_int), _vp]),

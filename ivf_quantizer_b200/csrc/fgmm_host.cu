@@ -550,6 +550,8 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
     return map_cuda(e);
   h->c.last_auto = auto_mode;
   h->c.last_path = fixed_mode == kModeTensor ? FGMM_PREC_FP16X3 : FGMM_PREC_FP32;
+  h->c.last_nc = N - (N - 1) / kChunk * kChunk;
+  h->c.last_stats = want_stats;
   return FGMM_OK;
 }
 }  // namespace
@@ -619,6 +621,38 @@ int fgmm_last_step_path(fgmm_handle h, int* path_out) {
   if (e != cudaSuccess) return map_cuda(e);
   *path_out = m == kModeTensor ? FGMM_PREC_FP16X3 : FGMM_PREC_FP32;
   return FGMM_OK;
+}
+
+int fgmm_last_step_info(fgmm_handle h, fgmm_step_info* out) {
+  if (!h || !out) return FGMM_ERR_INVALID_ARG;
+  int rc = fgmm_last_step_path(h, &out->path);
+  if (rc) return rc;
+  out->n_stiff = out->n_grey = 0;
+  out->skip_pairs = out->skip_pairs_all = -1;
+  if (out->path < 0) return FGMM_OK;
+  const Ctx& c = h->c;
+  const Workspace& w = c.ws;
+  if ((rc = set_device(c))) return rc;
+  cudaError_t e = cudaDeviceSynchronize();
+  int ns[2] = {0, 0};
+  if (e == cudaSuccess && c.last_auto && w.n_stiff)
+    e = cudaMemcpy(ns, w.n_stiff, sizeof(ns), cudaMemcpyDeviceToHost);
+  out->n_stiff = ns[0];
+  out->n_grey = ns[1];
+  // block lists of the last chunk: 128-point tiles on the tensor cores, 64 on CUDA cores
+  const bool tc = out->path == FGMM_PREC_FP16X3;
+  const bool skipped = c.last_stats && (tc ? tc_skip(c) : simt_skip(c));
+  if (e == cudaSuccess && skipped) {
+    const int nkb = tc ? w.Kt / 128 : (w.Kp + 127) / 128;
+    const int rows = tc ? 128 : kTP;
+    std::vector<int> cnt(nkb);
+    e = cudaMemcpy(cnt.data(), w.tcnt, nkb * sizeof(int), cudaMemcpyDeviceToHost);
+    int64_t tot = 0;
+    for (int v : cnt) tot += v;
+    out->skip_pairs = tot;
+    out->skip_pairs_all = (int64_t)nkb * ((c.last_nc + rows - 1) / rows);
+  }
+  return map_cuda(e);
 }
 
 int fgmm_fit(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx, float* weights,

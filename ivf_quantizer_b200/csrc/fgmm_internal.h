@@ -171,6 +171,8 @@ struct Ctx {
   int last_path = -1;      // FGMM_PREC_FP32 / FGMM_PREC_FP16X3, or -1
   bool last_auto = false;  // last step decided its path on the device
   bool skip = true;        // block skipping in the tensor-core statistics sweep
+  int64_t last_nc = 0;     // points of the last chunk of the last step (fgmm_last_step_info)
+  bool last_stats = false; // the last step ran a statistics sweep
 };
 
 // Path codes stored in Workspace::mode.

@@ -399,6 +399,12 @@ __global__ void __launch_bounds__(kLseThreads, 1)
       for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++j) {
         const int row0 = t * BM;
         x_issued = j + 1;
+        // phi lo rows that the epilogue warps read with plain loads one tile ahead: start
+        // moving them into L2 two tiles ahead (64 KB per tile at D = 128)
+        for (int ta = (j == 0 ? t + (int)gridDim.x : t + 2 * (int)gridDim.x);
+             ta <= t + 2 * (int)gridDim.x && ta < ntiles; ta += gridDim.x)
+          ptx::bulk_prefetch_l2(xop + ((size_t)ncmax + (size_t)ta * BM) * (NKC * 64),
+                                BM * NKC * 128);
         for (int c = 0; c < NKC; ++c) {
           if (j > 0 && !ptx::mbar_wait(&bars->x_empty[c], (j - 1) & 1, abort)) goto fail_p;
           ptx::mbar_arrive_expect_tx(&bars->x_full[c], BOX);
@@ -527,6 +533,11 @@ __global__ void __launch_bounds__(kLseThreads, 1)
           uint32_t u[32];
           ptx::tmem_ld32(tmem + lane_base + b * 128 + col, u);
           ptx::tmem_wait_ld();
+          // the values are in registers: hand the S buffer back to the MMA warp now, so
+          // that the products of block kb + 2 overlap this block's arithmetic
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&bars->s_empty[b]);
           float v[32];
           float bm = -CUDART_INF_F;
           const int k0 = kb * BKc + col;
@@ -588,9 +599,6 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             }
           }
         }
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->s_empty[b]);
       }
       if (*abort) break;
       // combine the four column quarters of each row

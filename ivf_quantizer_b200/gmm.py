@@ -92,6 +92,14 @@ class GMM:
         check(LIB.fgmm_last_step_path(self._h, ctypes.byref(v)), "fgmm_last_step_path")
         return v.value
 
+    def last_step_info(self) -> dict:
+        """What the last step did (fgmm_last_step_info; synchronises): path, stiff and
+        grey component counts (AUTO), and the statistics sweep's visited and dense
+        (tile, block) pair counts on the last chunk (-1 when it ran dense)."""
+        v = _lib.StepInfo()
+        check(LIB.fgmm_last_step_info(self._h, ctypes.byref(v)), "fgmm_last_step_info")
+        return {f: getattr(v, f) for f, _ in _lib.StepInfo._fields_}
+
     @property
     def workspace_bytes(self) -> int:
         v = ctypes.c_size_t()

@@ -204,7 +204,7 @@ def em_step(X, weights, means, variances, cov_type=COV_DIAG, reg_covar=1e-6):
     return StepResult(w_new, mu_new, var_new, loglik, logZ, Nk, empty)
 
 
-def shard_statistics(X, weights, means, variances, cov_type=COV_DIAG):
+def shard_statistics(X, weights, means, variances, cov_type=COV_DIAG, logz_out=None):
     """The sufficient statistics one shard of the rows contributes to an EM step.
 
     Layout (fp64, length K (1 + 2D) + 1), per component k at offset k (1 + 2D):
@@ -212,6 +212,7 @@ def shard_statistics(X, weights, means, variances, cov_type=COV_DIAG):
     about the INPUT means μ_k, then Σ_i log Z_i.  Every entry is a sum over rows, so
     the statistics of disjoint shards add up to those of their union; §2's M-step
     (Eqs. (1)-(3)) is a function of the sums alone (m_step_from_statistics).
+    logz_out: optional float64 array [N] that receives the per-point log Z_i.
     """
     X = _as_f64(X)
     N, D = X.shape
@@ -223,6 +224,8 @@ def shard_statistics(X, weights, means, variances, cov_type=COV_DIAG):
     ll = 0.0
     for s, e in _row_chunks(N, K):
         lz, R = e_step(X[s:e], weights, mu, variances, cov_type)
+        if logz_out is not None:
+            logz_out[s:e] = lz
         ll += float(np.sum(lz))
         st[:, 0] += R.sum(axis=0)
         for k in range(K):

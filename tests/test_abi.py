@@ -96,3 +96,10 @@ def test_profile_layout_and_kernel_names():
     assert b"tc_lse" in names and b"tc_stats" in names and b"stats_simt" in names
     assert _lib.LIB.fgmm_profile_kernel_name(-1) is None
     assert _lib.LIB.fgmm_profile_kernel_name(_lib.PROF_KERNELS) is None
+
+
+def test_step_info_rejects_null_arguments():
+    from ivf_quantizer_b200 import _lib
+    info = _lib.StepInfo()
+    assert _lib.LIB.fgmm_last_step_info(None, ctypes.byref(info)) == _lib.ERR_INVALID_ARG
+    assert _lib.LIB.fgmm_last_step_info(None, None) == _lib.ERR_INVALID_ARG

@@ -25,6 +25,10 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["config"]["workload"].startswith("c1 ")
+    # the oracle runs on every core of the host, and says so
+    cores = len(os.sched_getaffinity(0))
+    assert d["cpu_baseline"]["cores"] == cores
+    assert d["cpu_baseline"]["cpu_model"] and d["cpu_baseline"]["extrapolated"] is False
 
 
 def test_recorded_traffic_is_tied_to_the_sweep_sources():

@@ -7,12 +7,15 @@ that hold at any size: the step's log-likelihood equals the fp64 sum of the
 per-point values, the weights form a distribution, every parameter is finite
 and positive where it must be, and device memory beyond X does not grow.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
 
 import synth
 from oracle import gmm_oracle as O
+from tests._cmp import compare_step
 
 pytestmark = pytest.mark.gpu
 
@@ -66,6 +69,42 @@ def test_full_size_step(big_x, prec):
     wn = wd.double().cpu().numpy()
     assert abs(wn.sum() - 1.0) < 1e-5 and np.all(wn >= 0)
     assert torch.isfinite(md).all() and torch.isfinite(vd).all() and bool((vd > 0).all())
+    g.close()
+
+
+@pytest.mark.skipif(os.environ.get("FGMM_FULL_ORACLE") != "1",
+                    reason="opt-in: the oracle over all 10^8 rows takes ~8e4 core-seconds "
+                           "(set FGMM_FULL_ORACLE=1)")
+@pytest.mark.parametrize("t", [0, 29])
+def test_full_size_teacher_forced_all_rows(big_x, t):
+    """The bench's step (AUTO, block skipping) at full size, teacher-forced at iteration
+    t: the oracle runs one step from the GPU's parameters Θ_t over all 10^8 rows, X
+    streamed back to the host in shards for a pool of oracle processes; weights, means,
+    variances, every per-point log Z and the log-likelihood are compared."""
+    from tests._pool_oracle import host_cores, teacher_forced_step_stream
+    import ivf_quantizer_b200 as q
+    X = big_x
+    w, mu, var = synth.init_params(X, K, seed=0)
+    g = q.GMM(K, D, precision=q.PREC_AUTO)
+    wd, md, vd = g.new_params(w, mu, var)
+    for _ in range(t):
+        g.step(X, wd, md, vd)
+    g.check_status()
+    w_in, m_in, v_in = (a.double().cpu().numpy() for a in (wd, md, vd))
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    lz = torch.empty(N, dtype=torch.float32, device="cuda")
+    g.step(X, wd, md, vd, loglik=ll, logz=lz)
+    info = g.last_step_info()
+    g.check_status()
+    print("step", t, info, "host cores", host_cores())
+    ref = teacher_forced_step_stream(lambda a, b: X[a:b].double().cpu().numpy(), N,
+                                     w_in, m_in, v_in)
+    # the per-dimension data scale for the means' floor, from a seeded row sample
+    gen = torch.Generator().manual_seed(5)
+    sample = X[torch.randint(0, N, (200_000,), generator=gen).cuda()].cpu().numpy()
+    out = compare_step((wd.cpu().numpy(), md.cpu().numpy(), vd.cpu().numpy()), ref, sample,
+                       logz_gpu=lz.cpu().numpy(), loglik_gpu=float(ll.item()))
+    print(out)
     g.close()
 
 

@@ -183,6 +183,32 @@ def test_responsibilities_are_a_distribution():
     np.testing.assert_allclose(R.sum(axis=1), 1.0, rtol=1e-14)
 
 
+def test_fit_tolerance_rule_from_the_k1_fixed_point():
+    """§2's stopping rule (a small change of the log-likelihood between successive
+    iterations), read as |L_t - L_(t-1)| / N < tol.  With K = 1 the first step lands on
+    the maximum-likelihood parameters (closed form: sample mean, population variance)
+    and every later step returns them unchanged, so L_1 = L_2 exactly and the change
+    seen after iteration 3 is 0, while the change after iteration 2 is
+    d1 = |L(MLE) - L(Θ_0)| / N > 0.  Hence: tol = 0 runs every iteration; any tol in
+    (0, d1] stops after 3 (d1 < tol is false at d1 itself: strict); tol above d1 stops
+    after 2.  A rule without the division by N, or with <= instead of <, fails."""
+    rng = np.random.default_rng(31)
+    N, D = 400, 3
+    X = rng.normal(loc=[1.0, -1.0, 2.0], scale=[0.5, 1.5, 1.0], size=(N, D))
+    mu0, var0 = np.zeros((1, D)), np.full((1, D), 3.0)
+    _, mu_a, var_a, lls, it = O.fit(X, [1.0], mu0, var0, max_iters=6, tol=0.0)
+    assert it == 6 and len(lls) == 6
+    np.testing.assert_allclose(mu_a[0], X.mean(axis=0), rtol=1e-13)
+    np.testing.assert_allclose(var_a[0], X.var(axis=0) + 1e-6, rtol=1e-12)
+    assert lls[1] == lls[2]            # the fixed point: identical parameters, identical L
+    d1 = abs(lls[1] - lls[0]) / N
+    assert d1 > 0
+    for tol, want in ((1e-300, 3), (0.5 * d1, 3), (d1, 3), (2.0 * d1, 2)):
+        *_, lls_t, it_t = O.fit(X, [1.0], mu0, var0, max_iters=6, tol=tol)
+        assert it_t == want, (tol, d1, it_t)
+        assert lls_t == lls[:want]
+
+
 @pytest.mark.parametrize("cov", [O.COV_DIAG, O.COV_SPHERICAL])
 def test_loglik_monotone(cov):
     """EM never decreases the likelihood (Dempster et al. 1977, cited in §2)."""

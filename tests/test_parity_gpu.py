@@ -128,6 +128,58 @@ def test_table1_teacher_forced_late_iteration(prec, N, K):
     print(_check(X, wd.cpu().numpy(), md.cpu().numpy(), vd.cpu().numpy(), prec=prec))
 
 
+@pytest.mark.parametrize("prec", SAFE_PRECISIONS)
+def test_fit_tolerance_early_stop(prec):
+    """fgmm_fit with tol > 0 stops after the first iteration t whose log-likelihood
+    change |L_t - L_(t-1)| / N is below tol (§2's stopping rule), and its parameters are
+    those of the same number of single steps.  tol is placed between two successive
+    changes of the GPU's own trajectory with a clear margin on both sides; the oracle's
+    free-running trajectory (10,000 points, D = 16, K = 16, where it is compared
+    iteration by iteration) must stop at the same iteration."""
+    import ivf_quantizer_b200 as q
+    X = synth.generate("c1", 10_000, seed=4)
+    N = X.shape[0]
+    w, mu, var = synth.init_params(X, 16, seed=4)
+    g = _gmm(16, 16, prec=prec)
+    Xd = X.cuda()
+    wd, md, vd = g.new_params(w, mu, var)
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    lls, traj = [], []
+    for _ in range(30):
+        g.step(Xd, wd, md, vd, loglik=ll)
+        lls.append(ll.item())
+        traj.append((wd.clone(), md.clone(), vd.clone()))
+    g.check_status()
+    _, _, _, rlls, _ = O.fit(X.double().numpy(), w.double().numpy(), mu.double().numpy(),
+                             var.double().numpy(), 0, 1e-6, max_iters=30)
+    d = np.abs(np.diff(lls)) / N          # d[j]: change seen after iteration j + 2
+    rd = np.abs(np.diff(rlls)) / N
+    pick = None
+    for j in range(2, len(d) - 1):
+        hi = min(d[:j + 1].min(), rd[:j + 1].min())
+        lo = max(d[j + 1], rd[j + 1])
+        if hi > 2.0 * lo:
+            pick = (j, float(np.sqrt(hi * lo)))
+            break
+    assert pick is not None, d
+    j, tol = pick
+    want = j + 3
+    *_, it_o = O.fit(X.double().numpy(), w.double().numpy(), mu.double().numpy(),
+                     var.double().numpy(), 0, 1e-6, max_iters=30, tol=tol)
+    assert it_o == want
+    wd2, md2, vd2 = g.new_params(w, mu, var)
+    fll, it = g.fit(Xd, wd2, md2, vd2, max_iters=30, tol=tol)
+    assert it == want, (it, want, tol)
+    tw, tm, tv = traj[want - 1]
+    assert torch.equal(wd2, tw) and torch.equal(md2, tm) and torch.equal(vd2, tv)
+    assert fll == lls[want - 1]
+    # max_iters still bounds a tolerance that is never met
+    wd3, md3, vd3 = g.new_params(w, mu, var)
+    _, it3 = g.fit(Xd, wd3, md3, vd3, max_iters=4, tol=1e-300)
+    assert it3 == 4 and torch.equal(md3, traj[3][1])
+    g.close()
+
+
 @pytest.mark.parametrize("N,D,K", [(1, 1, 1), (5, 3, 2), (63, 7, 5), (65, 33, 65), (130, 130, 3),
                                    (200, 1, 70), (777, 100, 100), (300, 260, 9), (129, 128, 129),
                                    (1000, 64, 257)])
@@ -301,7 +353,7 @@ def test_soft_assign(top_m, thr):
     decisive, bad = ids_match_where_decisive(ids.cpu().numpy(), rid, rresp, R, thr)
     assert decisive.sum() >= 50, decisive.mean()
     assert len(bad) == 0, bad[:10]
-    gr = resp.cpu().numpy()
+    gr = resp.cpu().numpy().astype(np.float64)
     ok = decisive[:, None] & (rid >= 0)
     # log r = log z - log Z carries the per-point log-likelihood tolerance (1e-4 of |log Z|)
     lz = O.logsumexp_rows(O.log_joint(X.double().numpy(), w.double().numpy(),
