@@ -172,6 +172,15 @@ def cpu_model() -> str:
     return "unknown"
 
 
+def _oracle_worker_init():
+    # one BLAS thread per worker process: the pool already has one process per core
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        pass
+
+
 def _oracle_shard(args):
     """Worker: the oracle's statistics of one row shard (runs in a spawned process)."""
     X, w, mu, var = args
@@ -190,7 +199,7 @@ class OraclePool:
     def __init__(self, procs=None):
         import multiprocessing as mp
         self.procs = max(1, procs or host_cores())
-        self.pool = mp.get_context("spawn").Pool(self.procs)
+        self.pool = mp.get_context("spawn").Pool(self.procs, initializer=_oracle_worker_init)
         self.pool.map(_oracle_shard, [(np.zeros((1, 1)), np.ones(1), np.zeros((1, 1)),
                                        np.ones((1, 1)))] * self.procs)
 
@@ -242,7 +251,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="table1-1e8", choices=sorted(WORKLOADS))
-    ap.add_argument("--prec", default="auto", choices=["auto", "fp32", "fp16x3"])
+    ap.add_argument("--prec", default="auto", choices=["auto", "fp32", "fp16x3", "fp16"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-block-skip", action="store_true",
                     help="dense statistics sweep on the tensor cores (fgmm_set_block_skip 0)")
@@ -422,7 +431,8 @@ def main():
             dist.barrier()
 
     N, D, K = w["N"], w["D"], w["K"]
-    prec = {"auto": q.PREC_AUTO, "fp32": q.PREC_FP32, "fp16x3": q.PREC_FP16X3}[args.prec]
+    prec = {"auto": q.PREC_AUTO, "fp32": q.PREC_FP32, "fp16x3": q.PREC_FP16X3,
+            "fp16": q.PREC_FP16}[args.prec]
     X = torch.empty(N, D, device=dev, dtype=torch.float32)
     synth.generate(w["gen"], N, seed=rank, device=dev, out=X)
     # every rank starts from rank 0's initial parameters: the ranks fit ONE mixture to
@@ -433,7 +443,8 @@ def main():
         g.set_precision(prec)
     except q.FgmmError:
         g.set_precision(q.PREC_FP32)
-    prec_set = {q.PREC_FP32: "fp32", q.PREC_FP16X3: "fp16x3", q.PREC_AUTO: "auto"}[g.precision]
+    prec_set = {q.PREC_FP32: "fp32", q.PREC_FP16X3: "fp16x3", q.PREC_AUTO: "auto",
+                q.PREC_FP16: "fp16"}[g.precision]
     g.set_block_skip(not args.no_block_skip)
     wd, md, vd = g.new_params(wt, mu, var)
     if world > 1:
@@ -496,7 +507,7 @@ def main():
     pts_per_launch = N / n_chunks                       # one launch = one chunk of points
     flops_per_launch = 4.0 * D * K * pts_per_launch     # each sweep: 4*D flops per (point, comp)
     achieved = flops_per_launch / (avg_ms / 1e3) / 1e12 if launches else 0.0
-    prec_used = "fp16x3" if dom.startswith("tc_") else "fp32"
+    prec_used = ("fp16" if prec_set == "fp16" else "fp16x3") if dom.startswith("tc_") else "fp32"
     if prec_used == "fp32":
         clk = float(peaks.get("sm_max_mhz", 1965.0))
         peak = 148 * 128 * 2 * clk * 1e6 / 1e12
@@ -506,8 +517,9 @@ def main():
         peak = float(peaks["bf16_tflops_sustained"])
         roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_note":
                 f"fp16 dense peak = bf16 dense, {peak_src}, sustained; algorithmic flops "
-                f"(4*D per point-component per sweep), the three-product split and the "
-                f"recompute are not counted"}
+                f"(4*D per point-component per sweep); the split products "
+                f"({3 if prec_used == 'fp16x3' else 1} per term) and the recompute are not "
+                f"counted"}
     traffic = recorded_traffic(dom, prec_used)
     roof.update({"kernel": dom, "achieved": achieved, "peak": peak,
                  "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,

@@ -52,8 +52,12 @@ enum fgmm_cov { FGMM_COV_DIAG = 0, FGMM_COV_SPHERICAL = 1 };
  *   FP16X3 : tensor cores (tcgen05), expanded form [x, x^2] . W with every
  *            operand split into two fp16 halves and three products, fp32
  *            accumulation (about 22 significant bits per product).
- *   FP16   : tensor cores, one fp16 product per term (fast, ~11 bits; fails
- *            the 1e-4 log-likelihood tolerance on the Table-1 generator).
+ *   FP16   : tensor cores, one fp16 product per term in both sweeps (about 11
+ *            significant bits per term; no W' lo or phi lo operands).  A speed mode for
+ *            callers that can accept its error: it does not hold the 1e-4 per-point
+ *            log-likelihood accuracy of the other modes where the expanded-form terms
+ *            are large next to the log-density (high D, tight components far from
+ *            the data's centre); AUTO never selects it.
  *   AUTO   : the default; FP16X3 for the components that are well conditioned for
  *            the expanded form, the others ("stiff") on a CUDA-core side path in the
  *            direct form, decided per component and per step on the device; the whole
@@ -95,7 +99,8 @@ int fgmm_create(int K, int D, int cov_type, double reg_covar, fgmm_handle* out);
 int fgmm_destroy(fgmm_handle h);
 
 /* Select the precision mode (enum fgmm_prec).  FGMM_ERR_INVALID_ARG for an
- * unknown value. */
+ * unknown value; FGMM_ERR_UNSUPPORTED for a tensor-core mode (FP16X3, FP16) when the
+ * handle's D has no tensor-core path (D > 128). */
 int fgmm_set_precision(fgmm_handle h, int prec);
 int fgmm_get_precision(fgmm_handle h, int* prec_out);
 
@@ -117,8 +122,9 @@ int fgmm_get_precision(fgmm_handle h, int* prec_out);
 int fgmm_set_block_skip(fgmm_handle h, int enable);
 int fgmm_get_block_skip(fgmm_handle h, int* enable_out);
 
-/* Path the last fgmm_em_step of this handle ran: FGMM_PREC_FP32 (CUDA cores) or
- * FGMM_PREC_FP16X3 (tensor cores).  Under FGMM_PREC_AUTO the choice is made on the
+/* Path the last fgmm_em_step of this handle ran: FGMM_PREC_FP32 (CUDA cores),
+ * FGMM_PREC_FP16X3 (tensor cores, split products) or FGMM_PREC_FP16 (tensor cores, one
+ * product, when selected explicitly).  Under FGMM_PREC_AUTO the choice is made on the
  * device per step, so this call synchronises the device.  -1 before any step. */
 int fgmm_last_step_path(fgmm_handle h, int* path_out);
 
@@ -255,8 +261,8 @@ int fgmm_soft_assign(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64
  * device synchronisation is not acceptable.  fgmm_create allocates a workspace, so
  * those callers cannot use a handle.
  *
- * Same result as fgmm_soft_assign (§4.2-4.3) with the same arguments, but without a
- * handle: K, D and cov_type are passed directly.  Its scratch (padded means,
+ * Same result as fgmm_soft_assign with the same arguments, but without a handle: K, D
+ * and cov_type are passed directly.  Its scratch (padded means,
  * precisions and per-component constants) lives in one fixed array inside the
  * library's own device memory, which every GPU that loads the library holds until
  * the process exits (about 2.1 MB).  Limits: padded K x padded D <= FGMM_STATIC_MAX_KD
@@ -265,7 +271,10 @@ int fgmm_soft_assign(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64
  *
  * The first call on a device looks up that array's device address (once per device,
  * with that device current), and the CUDA runtime may allocate the array then if it
- * loads modules lazily; make this first call before any stream capture.  Every
+ * loads modules lazily; make this first call before any stream capture.  The address
+ * is kept for the life of the process: after cudaDeviceReset (or anything else that
+ * destroys and re-creates the device's primary context) it is stale, and this call
+ * must not be used on that device again.  Every
  * call shares the array and overwrites what the previous call left there; calls that
  * overlap on the GPU (two streams, two host threads) race on it and must be
  * serialised by the caller.  The call synchronises the stream and returns the device

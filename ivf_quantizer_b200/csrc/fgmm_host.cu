@@ -358,8 +358,8 @@ int fgmm_set_precision(fgmm_handle h, int prec) {
   if (prec != FGMM_PREC_FP32 && prec != FGMM_PREC_FP16X3 && prec != FGMM_PREC_FP16 &&
       prec != FGMM_PREC_AUTO)
     return FGMM_ERR_INVALID_ARG;
-  if (prec == FGMM_PREC_FP16) return FGMM_ERR_UNSUPPORTED;
-  if (prec == FGMM_PREC_FP16X3 && !h->c.tc.ready) return FGMM_ERR_UNSUPPORTED;
+  if ((prec == FGMM_PREC_FP16X3 || prec == FGMM_PREC_FP16) && !h->c.tc.ready)
+    return FGMM_ERR_UNSUPPORTED;
   h->c.prec = prec;
   return FGMM_OK;
 }
@@ -431,7 +431,8 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
   // both, each kernel returning at once unless the device-side mode word (set by the
   // tensor-core preparation's conditioning check) selects its path
   const bool auto_mode = c.prec == FGMM_PREC_AUTO && c.tc.ready;
-  const bool run_tc = (c.prec == FGMM_PREC_FP16X3 || auto_mode) && c.tc.ready;
+  const bool run_tc =
+      (c.prec == FGMM_PREC_FP16X3 || c.prec == FGMM_PREC_FP16 || auto_mode) && c.tc.ready;
   const bool run_simt = c.prec == FGMM_PREC_FP32 || !c.tc.ready || auto_mode;
   const int fixed_mode = run_tc && !run_simt ? kModeTensor : kModeSimt;
   const int* mode = auto_mode ? w.mode : nullptr;
@@ -549,7 +550,9 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
   if (want_stats && (e = launch_reduce_stats(c, means, st, mode, fixed_mode, s)) != cudaSuccess)
     return map_cuda(e);
   h->c.last_auto = auto_mode;
-  h->c.last_path = fixed_mode == kModeTensor ? FGMM_PREC_FP16X3 : FGMM_PREC_FP32;
+  h->c.last_path = fixed_mode != kModeTensor ? FGMM_PREC_FP32
+                   : c.prec == FGMM_PREC_FP16   ? FGMM_PREC_FP16
+                                                : FGMM_PREC_FP16X3;
   h->c.last_nc = N - (N - 1) / kChunk * kChunk;
   h->c.last_stats = want_stats;
   return FGMM_OK;
@@ -640,7 +643,7 @@ int fgmm_last_step_info(fgmm_handle h, fgmm_step_info* out) {
   out->n_stiff = ns[0];
   out->n_grey = ns[1];
   // block lists of the last chunk: 128-point tiles on the tensor cores, 64 on CUDA cores
-  const bool tc = out->path == FGMM_PREC_FP16X3;
+  const bool tc = out->path == FGMM_PREC_FP16X3 || out->path == FGMM_PREC_FP16;
   const bool skipped = c.last_stats && (tc ? tc_skip(c) : simt_skip(c));
   if (e == cudaSuccess && skipped) {
     const int nkb = tc ? w.Kt / 128 : (w.Kp + 127) / 128;

@@ -46,6 +46,22 @@ constexpr int kSkipMaxBlocks = 32;   // block masks are 32-bit words: K <= 4096
 // is more than kSimtSkipCut nats below log Z, i.e. each dropped r is below e^-50 = 2e-22,
 // and all that a component can lose over 10^9 points is below 2e-13 effective points.
 constexpr float kSimtSkipCut = 50.f;
+// Tensor-core statistics: the products accumulate in fp32 in TMEM for a run of tiles
+// before each fp64 flush, and each MMA step loses up to about half an fp32 unit of the
+// running sum (measured on B200: the error of the raw moments grows linearly with the
+// run length, i.e. it is biased, not a random walk).  The variance update
+// S2/N_k - (S1/N_k)^2 multiplies that relative error by A = (S2/N_k) / variance =
+// 1 + (mu - c)^2 / sigma^2.  Measured at K = 1024, D = 128 in the steady state with
+// block skipping (whose sorted tiles put a component's points into fewer, denser runs):
+// largest relative variance error over 1.3e5 (component, dimension) pairs = 2.3e-3 with
+// 8-tile runs, 6.9e-4 with 2-tile runs, 3.1e-4 with 1-tile runs, at A up to ~510; the
+// dense sweep's runs hold few non-zero responsibilities per component and stay below
+// 2e-4 with 8-tile runs.  Hence 2-tile runs with block skipping, 8 without, and
+// components whose A exceeds kMaxAmplification go to the direct-form CUDA-core side path:
+// with 2-tile runs the error is ~1.35e-6 A, at most 6e-4 below the bound.
+constexpr int kFlushTilesDense = 8;
+constexpr int kFlushTilesSkip = 2;
+constexpr float kMaxAmplification = 450.f;
 constexpr int kOrdPts = 4096;        // points per CTA of the radix sort
 constexpr int kOrdBuckets = 256;     // values of one 8-bit radix digit
 

@@ -30,10 +30,11 @@
 //   tc_prep       W' hi/lo, c_k, 2^t_k; conditioning check for AUTO mode
 //   tc_convert    X chunk -> phi hi/lo (fp16, row-major, TMA-ready); with a
 //                 permutation, the chunk in sweep-2 order (block skipping)
-//   tc_lse        sweep 1: persistent, one 128-point tile per CTA at a time; phi hi
-//                 resident in smem, phi lo in TMEM, W' streamed through a TMA ring;
-//                 S = phi W'^T in TMEM (double buffered), online log-sum-exp by 16
-//                 epilogue warps (four column quarters), block masks for skipping.
+//   tc_lse        sweep 1: persistent, one pair of 128-point tiles per CTA at a time
+//                 (each W' box feeds the products of both tiles); phi hi resident in
+//                 smem, phi lo in TMEM, W' streamed through a TMA ring; S = phi W'^T in
+//                 TMEM (one buffer per tile), online log-sum-exp by 16 epilogue warps
+//                 (four column quarters, one row of each tile), block masks for skipping.
 //   tc_stats      sweep 2: CTA owns a 128-component block (W' hi resident in smem, lo
 //                 in TMEM) and a slice of points, or with block skipping a share of the
 //                 block's active tiles; S^T = W' phi^T in TMEM, responsibilities
@@ -62,7 +63,6 @@ constexpr int BM = 128;          // points per tile
 constexpr int BKc = 128;         // components per block
 constexpr int KC = 64;           // K elements per swizzle row / TMA box
 constexpr int BOX = 128 * 64 * 2;  // bytes of one [128 rows][64 fp16] box
-constexpr int SW = 8;            // W ring stages (sweep 1)
 constexpr int SX = 8;            // X ring stages (sweep 2)
 constexpr float kRScale = 32768.f;  // r is stored as fp16(r * 2^15)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -133,7 +133,8 @@ __global__ void tc_center_kernel(int K, int D, int cov, const float* __restrict_
 //   * its expanded-form logit error, ~2^-20 sqrt(sum_d t_d^2) with
 //     t_d = 1.5 (|mu~| + sigma)^2 / sigma^2 (the size of the cancelling terms near
 //     its mean), exceeds 1e-3 nats (a collapsed or very tight component);
-//   * its variance update would cancel: A_d = 1 + mu~_d^2 / sigma_d^2 > 900 for some d;
+//   * its variance update would cancel: A_d = 1 + mu~_d^2 / sigma_d^2 > kMaxAmplification
+//     for some d;
 //   * it had fewer than 4 effective points in the previous step (about to collapse).
 __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
                                const float* __restrict__ w, const float* __restrict__ means,
@@ -199,7 +200,7 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
       const float mx = rmax[0];
       if (mx > 0.f && isfinite(mx)) pw = exp2f(ceilf(log2f(mx)) - 14.f);
       if (stiff && wk > 0.f)
-        is_stiff = !(ldexp(sqrt(rt[0]), -20) <= 1e-3) || !(amax[0] <= 900.f) ||
+        is_stiff = !(ldexp(sqrt(rt[0]), -20) <= 1e-3) || !(amax[0] <= kMaxAmplification) ||
                    (nk_prev[k] < 4.0);
       // few points last step: the variance check may fail, so its side-path statistics
       // are taken as well (AUTO; swapped in instead of redoing the pass)
@@ -292,34 +293,45 @@ __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ld
 }
 
 // ------------------------------------------------------------------ sweep 1 (log Z)
-// 640 threads: warp 0 TMA producer, warp 1 MMA issuer, warps 4..19 epilogue.  The four
-// epilogue warpgroups split each 128-column S tile in quarters (columns 32g .. 32g+31;
-// four warps per scheduler hide the TMEM-load and exp latencies) and keep a running
-// (max, sum) per row; at the end of a tile groups 1..3 hand their pairs to group 0
+// 640 threads: warp 0 TMA producer, warp 1 MMA issuer, warps 4..19 epilogue.  A CTA works
+// on pairs of 128-point tiles (A = 2p, B = 2p + 1): every W' box that the TMA brings in
+// feeds the products of both tiles, so each byte streamed from L2 serves 256 points (the
+// W' stream of a 128-point tile would need about as many L2 bytes per clock as the
+// products it feeds can take).  The four epilogue warpgroups split each 128-column S
+// tile in quarters (columns 32g .. 32g+31; four warps per scheduler hide the TMEM-load
+// and exp latencies), one row of A and the same row of B per thread, and keep a running
+// (max, sum) per row; at the end of the pair groups 1..3 hand their pairs to group 0
 // through shared memory, which writes log Z.
-// phi hi of the point tile sits in shared memory (A operand of two products); phi lo
-// sits in tensor memory (A operand of the third), written there by the epilogue warps
-// one tile ahead, so that shared memory holds an 8-stage ring of W' boxes.
+// phi hi of both tiles sits in shared memory (A operand of two products); phi lo sits in
+// tensor memory (A operand of the third), written there by the epilogue warps as soon as
+// the previous pair's last products on that tile have completed.  TMEM: S_A, S_B (one
+// 128-column buffer each; the MMA warp refills S_A while the epilogue drains S_B and the
+// other way round), phi lo of A and B.
 constexpr int kEpiWarps = 8;                        // statistics sweep
 constexpr int kTcThreads = 128 + 32 * kEpiWarps;
 constexpr int kLseEpiWarps = 16;                    // log-sum-exp sweep
 constexpr int kLseThreads = 128 + 32 * kLseEpiWarps;
+constexpr int kLseRingMax = 8;
+// W' ring stages of sweep 1: as many boxes as fit beside the pair's phi hi (an even
+// number: the hi and lo box of a chunk are used together)
+__host__ __device__ constexpr int lse_ring(int nkc) { return nkc >= 4 ? 4 : (nkc == 3 ? 6 : 8); }
 
 struct LseBars {
-  uint64_t x_full[4], x_empty[4];
+  uint64_t x_full[2][4], x_empty[2][4];   // [tile of the pair][chunk]
   uint64_t xlo_ready[2];
-  uint64_t w_full[SW], w_empty[SW];
+  uint64_t w_full[kLseRingMax], w_empty[kLseRingMax];
   uint64_t s_full[2], s_empty[2];
   uint64_t xc_full[2], xc_empty[2];
   uint64_t drain;
   uint32_t tmem;
   int abort;
-  float xm[2][3][BM];   // (max, sum, filter max) of column groups 1..3, per tile buffer
+  float xm[2][3][BM];   // (max, sum, filter max) of column groups 1..3, per tile of the pair
   float xs[2][3][BM];
   float xf[2][3][BM];
   uint2 xk[2][3][BM];   // candidate blocks of column groups 1..3 (block skipping)
   float xo[2][3][BM];   // their largest block maximum left out of the candidates
 };
+static_assert(sizeof(LseBars) % 16 == 0, "the staged parameters after LseBars are read as float4");
 
 // Block skipping, sweep 1 side.  Every epilogue thread keeps, for its row and its 32
 // columns, the (at most kCand) largest block maxima that lie within the cut of its
@@ -334,7 +346,26 @@ constexpr float kCut2 = kSkipCut * kLog2e;       // the cut in log2 units
 constexpr float kQStep = kCut2 / 255.f;
 constexpr uint32_t kCodeEmpty = 0xFFFFu;
 
-template <int NKC>
+// Running state of one row in sweep 1 (log2 units).
+struct RowState {
+  float m, s;          // running max and sum
+  float fm;            // max over stiff components of estimate + error bound
+  float ovm;           // largest block maximum pushed out of the candidate list
+  float cbm[kCand];    // candidate blocks: block maximum (-inf: free)
+  uint32_t cid;        //                   block index of entry e in bits 8e .. 8e+7
+  __device__ __forceinline__ void reset() {
+    m = fm = ovm = -CUDART_INF_F;
+    s = 0.f;
+    cid = 0;
+#pragma unroll
+    for (int e = 0; e < kCand; ++e) cbm[e] = -CUDART_INF_F;
+  }
+  __device__ __forceinline__ uint32_t block(int e) const { return (cid >> (8 * e)) & 255u; }
+};
+
+// SPLIT: the three-product fp16 hi/lo split (FGMM_PREC_FP16X3 and AUTO); false: one fp16
+// product per term (FGMM_PREC_FP16: no W' lo boxes, no phi lo)
+template <int NKC, bool SPLIT>
 __global__ void __launch_bounds__(kLseThreads, 1)
     tc_lse_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                   int nc, int ncmax, int Kt, const float* __restrict__ ck,
@@ -344,11 +375,13 @@ __global__ void __launch_bounds__(kLseThreads, 1)
                   const float* __restrict__ lzlow, uint8_t* __restrict__ side_flag,
                   uint32_t* __restrict__ bmask, const int* mode, int* status) {
   if (mode && *mode != kModeTensor) return;
+  constexpr int SWL = lse_ring(NKC);
+  constexpr int NP = SPLIT ? 2 : 1;                   // W' boxes per chunk (hi, lo)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  unsigned char* xbuf = base;                         // [NKC][BOX]: phi hi of the tile
-  unsigned char* wring = base + NKC * BOX;            // [SW][BOX]
-  LseBars* bars = reinterpret_cast<LseBars*>(wring + SW * BOX);
+  unsigned char* xbuf = base;                         // [2][NKC][BOX]: phi hi of the pair
+  unsigned char* wring = base + 2 * NKC * BOX;        // [SWL][BOX]
+  LseBars* bars = reinterpret_cast<LseBars*>(wring + SWL * BOX);
   float* ckl = reinterpret_cast<float*>(bars + 1);    // [Kt] c_k log2(e)   (if staged)
   float* ksl = ckl + Kt;                              // [Kt] 2^t_k log2(e) (if staged)
   float* cfl = ksl + Kt;                              // [Kt] (c_k + E_k) log2(e) (if staged)
@@ -356,11 +389,17 @@ __global__ void __launch_bounds__(kLseThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = (nc + BM - 1) / BM;
+  const int npairs = (ntiles + 1) / 2;
   const int nkb = Kt / BKc;
+  const int G = (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int c = 0; c < 4; ++c) { ptx::mbar_init(&bars->x_full[c], 1); ptx::mbar_init(&bars->x_empty[c], 1); }
-    for (int s = 0; s < SW; ++s) { ptx::mbar_init(&bars->w_full[s], 1); ptx::mbar_init(&bars->w_empty[s], 1); }
+    for (int t = 0; t < 2; ++t)
+      for (int c = 0; c < 4; ++c) {
+        ptx::mbar_init(&bars->x_full[t][c], 1);
+        ptx::mbar_init(&bars->x_empty[t][c], 1);
+      }
+    for (int s = 0; s < SWL; ++s) { ptx::mbar_init(&bars->w_full[s], 1); ptx::mbar_init(&bars->w_empty[s], 1); }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&bars->s_full[b], 1);
       ptx::mbar_init(&bars->s_empty[b], kLseEpiWarps);
@@ -385,8 +424,8 @@ __global__ void __launch_bounds__(kLseThreads, 1)
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  // TMEM columns: [0, 256) S double-buffered, [256 + 128 b, ...) phi lo of tile buffer b
-  // (two fp16 per column, 2 Dq / 2 = NKC * 32 columns)
+  // TMEM columns: [128 t, 128 t + 128) S of tile t of the pair; [256 + 128 t, ...) phi lo
+  // of tile t (two fp16 per column, 2 Dq / 2 = NKC * 32 columns)
   const uint32_t tmem = bars->tmem;
   const uint32_t xlo_tmem = tmem + 256;
 
@@ -396,25 +435,32 @@ __global__ void __launch_bounds__(kLseThreads, 1)
       ptx::prefetch_tmap(&tmw);
       uint32_t itw = 0;
       int j = 0, x_issued = 0;
-      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++j) {
-        const int row0 = t * BM;
-        x_issued = j + 1;
-        // phi lo rows that the epilogue warps read with plain loads one tile ahead: start
-        // moving them into L2 two tiles ahead (64 KB per tile at D = 128)
-        for (int ta = (j == 0 ? t + (int)gridDim.x : t + 2 * (int)gridDim.x);
-             ta <= t + 2 * (int)gridDim.x && ta < ntiles; ta += gridDim.x)
-          ptx::bulk_prefetch_l2(xop + ((size_t)ncmax + (size_t)ta * BM) * (NKC * 64),
-                                BM * NKC * 128);
-        for (int c = 0; c < NKC; ++c) {
-          if (j > 0 && !ptx::mbar_wait(&bars->x_empty[c], (j - 1) & 1, abort)) goto fail_p;
-          ptx::mbar_arrive_expect_tx(&bars->x_full[c], BOX);
-          ptx::tma_load_2d(xbuf + c * BOX, &tmx, &bars->x_full[c], c * KC, row0);
+      bool last_b = false;
+      for (int p = blockIdx.x; p < npairs && !*abort; p += G, ++j) {
+        const int tA = 2 * p;
+        const bool hasB = tA + 1 < ntiles;
+        // phi lo rows that the epilogue warps read with plain loads at the end of this
+        // pair (those of the next pair): start moving them into L2 now
+        const int pn = p + G;
+        if (SPLIT && pn < npairs) {
+          const int ntl = min(2, ntiles - 2 * pn);
+          ptx::bulk_prefetch_l2(xop + ((size_t)ncmax + (size_t)2 * pn * BM) * (NKC * 64),
+                                (uint32_t)ntl * BM * NKC * 128);
         }
+        x_issued = j + 1;
+        last_b = hasB;
+        for (int t = 0; t < (hasB ? 2 : 1); ++t)
+          for (int c = 0; c < NKC; ++c) {
+            if (j > 0 && !ptx::mbar_wait(&bars->x_empty[t][c], (j - 1) & 1, abort)) goto fail_p;
+            ptx::mbar_arrive_expect_tx(&bars->x_full[t][c], BOX);
+            ptx::tma_load_2d(xbuf + (t * NKC + c) * BOX, &tmx, &bars->x_full[t][c], c * KC,
+                             (tA + t) * BM);
+          }
         for (int kb = 0; kb < nkb; ++kb)
           for (int c = 0; c < NKC; ++c)
-            for (int part = 0; part < 2; ++part, ++itw) {
-              const int s = itw % SW;
-              if (itw >= SW && !ptx::mbar_wait(&bars->w_empty[s], ((itw / SW) - 1) & 1, abort))
+            for (int part = 0; part < NP; ++part, ++itw) {
+              const int s = itw % SWL;
+              if (itw >= SWL && !ptx::mbar_wait(&bars->w_empty[s], ((itw / SWL) - 1) & 1, abort))
                 goto fail_p;
               ptx::mbar_arrive_expect_tx(&bars->w_full[s], BOX);
               ptx::tma_load_2d(wring + s * BOX, &tmw, &bars->w_full[s], c * KC,
@@ -427,52 +473,63 @@ __global__ void __launch_bounds__(kLseThreads, 1)
       bars->abort = 1;
     done_p:
       if (*abort) {  // let every copy this thread started land before the CTA exits
-        for (int c = 0; c < NKC && x_issued > 0; ++c) ptx::mbar_drain(&bars->x_full[c], (x_issued - 1) & 1);
-        for (uint32_t k = (itw > SW ? itw - SW : 0); k < itw; ++k)
-          ptx::mbar_drain(&bars->w_full[k % SW], (k / SW) & 1);
+        for (int t = 0; t < (last_b ? 2 : 1) && x_issued > 0; ++t)
+          for (int c = 0; c < NKC; ++c) ptx::mbar_drain(&bars->x_full[t][c], (x_issued - 1) & 1);
+        for (uint32_t k = (itw > SWL ? itw - SWL : 0); k < itw; ++k)
+          ptx::mbar_drain(&bars->w_full[k % SWL], (k / SWL) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = ptx::idesc_f16(128, 128, false, false);
-      uint32_t itw = 0, its = 0;
+      uint32_t itw = 0;
       int j = 0;
-      for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++j) {
-        for (int kb = 0; kb < nkb; ++kb, ++its) {
-          const int b = its & 1;
-          if (its >= 2 && !ptx::mbar_wait(&bars->s_empty[b], ((its >> 1) - 1) & 1, abort)) goto fail_m;
-          ptx::tc_fence_after();
-          const uint32_t d_tmem = tmem + b * 128;
-          if (kb == 0 && !ptx::mbar_wait(&bars->xlo_ready[j & 1], (j >> 1) & 1, abort)) goto fail_m;
-          const uint32_t xl_tmem = xlo_tmem + (j & 1) * 128;
+      for (int p = blockIdx.x; p < npairs && !*abort; p += G, ++j) {
+        const int nt = (2 * p + 1 < ntiles) ? 2 : 1;
+        for (int kb = 0; kb < nkb; ++kb) {
+          const uint32_t u = (uint32_t)(j * nkb + kb);   // use of each S buffer
           for (int c = 0; c < NKC; ++c) {
-            if (kb == 0 && !ptx::mbar_wait(&bars->x_full[c], j & 1, abort)) goto fail_m;
-            const int sh = itw % SW;
-            if (!ptx::mbar_wait(&bars->w_full[sh], (itw / SW) & 1, abort)) goto fail_m;
+            const int sh = itw % SWL;
+            if (!ptx::mbar_wait(&bars->w_full[sh], (itw / SWL) & 1, abort)) goto fail_m;
             ++itw;
-            const int sl = itw % SW;
-            if (!ptx::mbar_wait(&bars->w_full[sl], (itw / SW) & 1, abort)) goto fail_m;
-            ++itw;
-            ptx::tc_fence_after();
-            const uint32_t xa_hi = ptx::smem_u32(xbuf + c * BOX);
-            const uint32_t wb_hi = ptx::smem_u32(wring + sh * BOX);
-            const uint32_t wb_lo = ptx::smem_u32(wring + sl * BOX);
-#pragma unroll
-            for (int ks = 0; ks < KC / 16; ++ks) {
-              const uint32_t o = ks * 32;
-              const uint64_t ah = ptx::smem_desc_sw128(xa_hi + o, 16, 1024);
-              const uint64_t bh = ptx::smem_desc_sw128(wb_hi + o, 16, 1024);
-              const uint64_t bl = ptx::smem_desc_sw128(wb_lo + o, 16, 1024);
-              ptx::mma_f16_ss(d_tmem, ah, bh, idesc, (c > 0 || ks > 0) ? 1u : 0u);
-              ptx::mma_f16_ss(d_tmem, ah, bl, idesc, 1u);
+            int sl = sh;
+            if constexpr (SPLIT) {
+              sl = itw % SWL;
+              if (!ptx::mbar_wait(&bars->w_full[sl], (itw / SWL) & 1, abort)) goto fail_m;
+              ++itw;
+            }
+            // K-major 128 B-swizzled boxes: one descriptor per box, + 2 (32 bytes) per K-step
+            constexpr uint64_t kHiK = ptx::sw128_hi(16, 1024);
+            const uint64_t bh0 = ptx::sw128_desc(ptx::smem_u32(wring + sh * BOX), kHiK);
+            const uint64_t bl0 = ptx::sw128_desc(ptx::smem_u32(wring + sl * BOX), kHiK);
+            for (int t = 0; t < nt; ++t) {
+              if (c == 0) {
+                // S_t free (its previous block read out), phi lo of this pair in place
+                if (u >= 1 && !ptx::mbar_wait(&bars->s_empty[t], (u - 1) & 1, abort)) goto fail_m;
+                if (SPLIT && kb == 0 && !ptx::mbar_wait(&bars->xlo_ready[t], j & 1, abort))
+                  goto fail_m;
+              }
+              if (kb == 0 && !ptx::mbar_wait(&bars->x_full[t][c], j & 1, abort)) goto fail_m;
+              ptx::tc_fence_after();
+              const uint32_t d_tmem = tmem + t * 128;
               // phi lo from TMEM: K elements c*64 + ks*16 .. +15 = columns c*32 + ks*8 .. +7
-              ptx::mma_f16_ts(d_tmem, xl_tmem + c * 32 + ks * 8, bh, idesc, 1u);
+              const uint32_t xl_tmem = xlo_tmem + t * 128 + c * 32;
+              const uint64_t ah0 = ptx::sw128_desc(ptx::smem_u32(xbuf + (t * NKC + c) * BOX), kHiK);
+#pragma unroll
+              for (int ks = 0; ks < KC / 16; ++ks) {
+                const uint64_t dk = (uint64_t)(2 * ks);
+                ptx::mma_f16_ss(d_tmem, ah0 + dk, bh0 + dk, idesc, (c > 0 || ks > 0) ? 1u : 0u);
+                if constexpr (SPLIT) {
+                  ptx::mma_f16_ss(d_tmem, ah0 + dk, bl0 + dk, idesc, 1u);
+                  ptx::mma_f16_ts(d_tmem, xl_tmem + ks * 8, bh0 + dk, idesc, 1u);
+                }
+              }
+              if (kb == nkb - 1) ptx::mma_commit(&bars->x_empty[t][c]);
+              if (c == NKC - 1) ptx::mma_commit(&bars->s_full[t]);
             }
             ptx::mma_commit(&bars->w_empty[sh]);
-            ptx::mma_commit(&bars->w_empty[sl]);
-            if (kb == nkb - 1) ptx::mma_commit(&bars->x_empty[c]);
+            if constexpr (SPLIT) ptx::mma_commit(&bars->w_empty[sl]);
           }
-          ptx::mma_commit(&bars->s_full[b]);
         }
       }
       goto done_m;
@@ -490,55 +547,55 @@ __global__ void __launch_bounds__(kLseThreads, 1)
     const int q = warp & 3;                // TMEM lane quarter
     const int r = q * 32 + lane;           // row of the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    // phi lo of tile t into TMEM buffer b: this thread's row, K elements
-    // g*NKC*32 .. +NKC*32-1 = columns g*NKC*16 .. +NKC*16-1 (row t*BM + r < ncmax)
-    auto put_xlo = [&](int t, int b) {
+    // phi lo of `tile` into TMEM buffer t: this thread's row, K elements
+    // g*NKC*32 .. +NKC*32-1 = columns g*NKC*16 .. +NKC*16-1 (row tile*BM + r < ncmax)
+    auto put_xlo = [&](int tile, int t) {
       const uint4* src = reinterpret_cast<const uint4*>(
-          xop + ((size_t)ncmax + (size_t)t * BM + r) * (NKC * 64) + g * (NKC * 16));
+          xop + ((size_t)ncmax + (size_t)tile * BM + r) * (NKC * 64) + g * (NKC * 16));
 #pragma unroll
       for (int c8 = 0; c8 < NKC; ++c8) {   // 8 columns = 16 fp16 per store
         const uint4 v0 = __ldg(src + 2 * c8), v1 = __ldg(src + 2 * c8 + 1);
         const uint32_t r8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        ptx::tmem_st8(xlo_tmem + b * 128 + lane_base + g * (NKC * 8) + c8 * 8, r8);
+        ptx::tmem_st8(xlo_tmem + t * 128 + lane_base + g * (NKC * 8) + c8 * 8, r8);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&bars->xlo_ready[b]);
+      if (lane == 0) ptx::mbar_arrive(&bars->xlo_ready[t]);
     };
-    if (blockIdx.x < ntiles) put_xlo(blockIdx.x, 0);
-    uint32_t its = 0;
-    int jt = 0;
-    for (int t = blockIdx.x; t < ntiles && !*abort; t += gridDim.x, ++jt) {
-      // the next tile's phi lo goes into the buffer of tile jt - 1, whose MMAs have all
-      // completed: this thread has consumed every S block they produced
-      if (t + (int)gridDim.x < ntiles) put_xlo(t + gridDim.x, (jt + 1) & 1);
-      float m = -CUDART_INF_F, s = 0.f;   // in log2 units
-      float fm = -CUDART_INF_F;            // max over stiff components of estimate + E_k
-      float cbm[kCand];                    // candidate blocks: block maximum (-inf: free)
-      int cid[kCand];                      //                   block index
-      float ovm = -CUDART_INF_F;           // largest block maximum pushed out of the list
+    if (SPLIT && (int)blockIdx.x < npairs) {
+      put_xlo(2 * blockIdx.x, 0);
+      if (2 * (int)blockIdx.x + 1 < ntiles) put_xlo(2 * blockIdx.x + 1, 1);
+    }
+    int j = 0;
+    for (int p = blockIdx.x; p < npairs && !*abort; p += G, ++j) {
+      const int nt = (2 * p + 1 < ntiles) ? 2 : 1;
+      const int pn = p + G;
+      RowState st[2];
+      st[0].reset();
+      st[1].reset();
+      for (int kb = 0; kb < nkb && !*abort; ++kb) {
+        const uint32_t u = (uint32_t)(j * nkb + kb);
 #pragma unroll
-      for (int e = 0; e < kCand; ++e) { cbm[e] = -CUDART_INF_F; cid[e] = 0; }
-      for (int kb = 0; kb < nkb; ++kb, ++its) {
-        const int b = its & 1;
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full[b], (its >> 1) & 1, abort))) {
-          set_status(status, FGMM_ERR_TIMEOUT);
-          bars->abort = 1;
-          break;
-        }
-        ptx::tc_fence_after();
-        {
+        for (int t = 0; t < 2; ++t) {
+          if (t >= nt) break;
+          RowState& S = st[t];
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full[t], u & 1, abort))) {
+            set_status(status, FGMM_ERR_TIMEOUT);
+            bars->abort = 1;
+            break;
+          }
+          ptx::tc_fence_after();
           const int col = 32 * g;            // column within the 128-component block
-          uint32_t u[32];
-          ptx::tmem_ld32(tmem + lane_base + b * 128 + col, u);
+          uint32_t uu[32];
+          ptx::tmem_ld32(tmem + lane_base + t * 128 + col, uu);
           ptx::tmem_wait_ld();
-          // the values are in registers: hand the S buffer back to the MMA warp now, so
-          // that the products of block kb + 2 overlap this block's arithmetic
+          // the values are in registers: hand S_t back to the MMA warp now
           ptx::tc_fence_before();
           __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&bars->s_empty[b]);
-          float v[32];
+          if (lane == 0) ptx::mbar_arrive(&bars->s_empty[t]);
+          // log2-scaled log-densities of the 32 columns, two per packed fp32x2 operation
+          uint64_t v2[16];
           float bm = -CUDART_INF_F;
           const int k0 = kb * BKc + col;
 #pragma unroll
@@ -556,132 +613,154 @@ __global__ void __launch_bounds__(kLseThreads, 1)
               kk.x *= kLog2e; kk.y *= kLog2e; kk.z *= kLog2e; kk.w *= kLog2e;
               cf.x *= kLog2e; cf.y *= kLog2e; cf.z *= kLog2e; cf.w *= kLog2e;
             }
-            const float uu[4] = {__uint_as_float(u[4 * e4 + 0]), __uint_as_float(u[4 * e4 + 1]),
-                                 __uint_as_float(u[4 * e4 + 2]), __uint_as_float(u[4 * e4 + 3])};
-            v[4 * e4 + 0] = fmaf(uu[0], kk.x, cc.x);
-            v[4 * e4 + 1] = fmaf(uu[1], kk.y, cc.y);
-            v[4 * e4 + 2] = fmaf(uu[2], kk.z, cc.z);
-            v[4 * e4 + 3] = fmaf(uu[3], kk.w, cc.w);
+            const uint64_t f01 = ptx::f2_pack(__uint_as_float(uu[4 * e4 + 0]), __uint_as_float(uu[4 * e4 + 1]));
+            const uint64_t f23 = ptx::f2_pack(__uint_as_float(uu[4 * e4 + 2]), __uint_as_float(uu[4 * e4 + 3]));
+            const uint64_t k01 = ptx::f2_pack(kk.x, kk.y), k23 = ptx::f2_pack(kk.z, kk.w);
+            v2[2 * e4 + 0] = ptx::f2_fma(f01, k01, ptx::f2_pack(cc.x, cc.y));
+            v2[2 * e4 + 1] = ptx::f2_fma(f23, k23, ptx::f2_pack(cc.z, cc.w));
             // stiff components (c_k = -inf above): estimate + error bound, for the filter
-            fm = fmaxf(fm, fmaxf(fmaxf(fmaf(uu[0], kk.x, cf.x), fmaf(uu[1], kk.y, cf.y)),
-                                 fmaxf(fmaf(uu[2], kk.z, cf.z), fmaf(uu[3], kk.w, cf.w))));
-#pragma unroll
-            for (int z = 0; z < 4; ++z) bm = fmaxf(bm, v[4 * e4 + z]);
+            float g[4], v[4];
+            ptx::f2_unpack(ptx::f2_fma(f01, k01, ptx::f2_pack(cf.x, cf.y)), g[0], g[1]);
+            ptx::f2_unpack(ptx::f2_fma(f23, k23, ptx::f2_pack(cf.z, cf.w)), g[2], g[3]);
+            ptx::f2_unpack(v2[2 * e4 + 0], v[0], v[1]);
+            ptx::f2_unpack(v2[2 * e4 + 1], v[2], v[3]);
+            S.fm = fmaxf(S.fm, fmaxf(fmaxf(g[0], g[1]), fmaxf(g[2], g[3])));
+            bm = fmaxf(bm, fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
           }
-          const float nm = fmaxf(m, bm);
+          const float nm = fmaxf(S.m, bm);
           if (nm > -CUDART_INF_F) {
-            float acc = 0.f;
+            // every argument is <= 0 after the shift, so 2^x in (0, 1]; the SFU's exp2
+            // (flushing results below 2^-126, far under fp32 resolution of the sum)
+            const uint64_t shift = ptx::f2_pack(-nm, -nm);
+            uint64_t acc2 = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) acc += exp2f(v[e] - nm);
-            s = s * exp2f(m - nm) + acc;
-            m = nm;
+            for (int e2 = 0; e2 < 16; ++e2) {
+              float t0, t1;
+              ptx::f2_unpack(ptx::f2_add(v2[e2], shift), t0, t1);
+              acc2 = ptx::f2_add(acc2, ptx::f2_pack(ptx::ex2(t0), ptx::ex2(t1)));
+            }
+            float a0, a1;
+            ptx::f2_unpack(acc2, a0, a1);
+            S.s = S.s * ptx::ex2(S.m - nm) + (a0 + a1);
+            S.m = nm;
           }
           if (bmask) {
-            const float thr = m - kCut2;
+            const float thr = S.m - kCut2;
 #pragma unroll
             for (int e = 0; e < kCand; ++e)
-              if (cbm[e] <= thr) cbm[e] = -CUDART_INF_F;
+              if (S.cbm[e] <= thr) S.cbm[e] = -CUDART_INF_F;
             if (bm > thr) {
               int slot = -1, mi = 0;
               float mn = CUDART_INF_F;
 #pragma unroll
               for (int e = 0; e < kCand; ++e) {
-                if (slot < 0 && cbm[e] == -CUDART_INF_F) slot = e;
-                if (cbm[e] < mn) { mn = cbm[e]; mi = e; }
+                if (slot < 0 && S.cbm[e] == -CUDART_INF_F) slot = e;
+                if (S.cbm[e] < mn) { mn = S.cbm[e]; mi = e; }
               }
               if (slot < 0) {            // full: the smaller of bm and the list's least goes
-                if (bm > mn) { ovm = fmaxf(ovm, mn); slot = mi; }
-                else ovm = fmaxf(ovm, bm);
+                if (bm > mn) { S.ovm = fmaxf(S.ovm, mn); slot = mi; }
+                else S.ovm = fmaxf(S.ovm, bm);
               }
 #pragma unroll
               for (int e = 0; e < kCand; ++e)
-                if (e == slot) { cbm[e] = bm; cid[e] = kb; }
+                if (e == slot) {
+                  S.cbm[e] = bm;
+                  S.cid = (S.cid & ~(255u << (8 * e))) | ((uint32_t)kb << (8 * e));
+                }
             }
           }
+          // after the pair's last block on tile t every product reading phi lo of t has
+          // completed (S_t's last commit covers them): the next pair's phi lo of that tile
+          // goes in while the tensor cores finish the other tile
+          if (SPLIT && kb == nkb - 1 && pn < npairs && 2 * pn + t < ntiles) put_xlo(2 * pn + t, t);
         }
       }
       if (*abort) break;
-      // combine the four column quarters of each row
-      const int xb = jt & 1, use = jt >> 1;
-      if (g >= 1) {
-        if (use >= 1 &&
-            !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->xc_empty[xb], (use - 1) & 1, abort))) {
-          set_status(status, FGMM_ERR_TIMEOUT);
-          bars->abort = 1;
-          break;
-        }
-        bars->xm[xb][g - 1][r] = m;
-        bars->xs[xb][g - 1][r] = s;
-        bars->xf[xb][g - 1][r] = fm;
-        if (bmask) {
-          uint32_t code[kCand];
+      // combine the four column quarters of each row, per tile of the pair
 #pragma unroll
-          for (int e = 0; e < kCand; ++e) {
-            code[e] = kCodeEmpty;
-            const float dl = m - cbm[e];   // < cut for a live entry (else it is below the cut)
-            if (cbm[e] > -CUDART_INF_F && dl < kCut2) {
-              const int qd = min(254, (int)floorf(dl * (1.f / kQStep)));
-              code[e] = ((uint32_t)cid[e] << 8) | (uint32_t)qd;
-            }
+      for (int t = 0; t < 2; ++t) {
+        if (t >= nt) break;
+        const RowState& S = st[t];
+        if (g >= 1) {
+          if (j >= 1 &&
+              !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->xc_empty[t], (j - 1) & 1, abort))) {
+            set_status(status, FGMM_ERR_TIMEOUT);
+            bars->abort = 1;
+            break;
           }
-          bars->xk[xb][g - 1][r] = make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
-          bars->xo[xb][g - 1][r] = ovm;
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->xc_full[xb]);
-      } else {
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->xc_full[xb], use & 1, abort))) {
-          set_status(status, FGMM_ERR_TIMEOUT);
-          bars->abort = 1;
-          break;
-        }
-        float mq[4] = {m, 0.f, 0.f, 0.f}, sq[4] = {s, 0.f, 0.f, 0.f};
-        float f2 = fm;
-        uint2 kq[3];
-        float ov = ovm;
-#pragma unroll
-        for (int o = 0; o < 3; ++o) {
-          mq[o + 1] = bars->xm[xb][o][r];
-          sq[o + 1] = bars->xs[xb][o][r];
-          f2 = fmaxf(f2, bars->xf[xb][o][r]);
+          bars->xm[t][g - 1][r] = S.m;
+          bars->xs[t][g - 1][r] = S.s;
+          bars->xf[t][g - 1][r] = S.fm;
           if (bmask) {
-            kq[o] = bars->xk[xb][o][r];
-            ov = fmaxf(ov, bars->xo[xb][o][r]);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->xc_empty[xb]);
-        const float M = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-        float S = 0.f;
-        if (M > -CUDART_INF_F)
+            uint32_t code[kCand];
 #pragma unroll
-          for (int o = 0; o < 4; ++o) S += sq[o] * exp2f(mq[o] - M);
-        const int i = t * BM + r;
-        const float lz2 = M + log2f(S);
-        const float lz = lz2 / kLog2e;
-        if (i < nc) {
-          logz[i] = lz;
-          if (logz_out) logz_out[i] = lz;
-          // may a stiff component come within kSideCut nats of log Z here?
-          side_flag[i] = (f2 > lz2 - kSideCut * kLog2e) || !(lz >= *lzlow);
-          if (bmask) {
-            const float lim = lz2 - kCut2;
-            uint32_t mk = 0;
-            bool dense = ov > lim || !(lz2 > -CUDART_INF_F);
-#pragma unroll
-            for (int e = 0; e < kCand; ++e)
-              if (cbm[e] > lim) mk |= 1u << cid[e];
-#pragma unroll
-            for (int o = 0; o < 3; ++o) {
-              const uint32_t w2[2] = {kq[o].x, kq[o].y};
-#pragma unroll
-              for (int e = 0; e < kCand; ++e) {
-                const uint32_t cd = (w2[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-                if (cd != kCodeEmpty && mq[o + 1] - (float)(cd & 255u) * kQStep > lim)
-                  mk |= 1u << (cd >> 8);
+            for (int e = 0; e < kCand; ++e) {
+              code[e] = kCodeEmpty;
+              const float dl = S.m - S.cbm[e];   // < cut for a live entry (else below the cut)
+              if (S.cbm[e] > -CUDART_INF_F && dl < kCut2) {
+                const int qd = min(254, (int)floorf(dl * (1.f / kQStep)));
+                code[e] = (S.block(e) << 8) | (uint32_t)qd;
               }
             }
-            bmask[i] = dense ? (nkb >= 32 ? 0xFFFFFFFFu : (1u << nkb) - 1u) : mk;
+            bars->xk[t][g - 1][r] = make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
+            bars->xo[t][g - 1][r] = S.ovm;
+          }
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&bars->xc_full[t]);
+        } else {
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->xc_full[t], j & 1, abort))) {
+            set_status(status, FGMM_ERR_TIMEOUT);
+            bars->abort = 1;
+            break;
+          }
+          float mq[4] = {S.m, 0.f, 0.f, 0.f}, sq[4] = {S.s, 0.f, 0.f, 0.f};
+          float f2 = S.fm;
+          uint2 kq[3];
+          float ov = S.ovm;
+#pragma unroll
+          for (int o = 0; o < 3; ++o) {
+            mq[o + 1] = bars->xm[t][o][r];
+            sq[o + 1] = bars->xs[t][o][r];
+            f2 = fmaxf(f2, bars->xf[t][o][r]);
+            if (bmask) {
+              kq[o] = bars->xk[t][o][r];
+              ov = fmaxf(ov, bars->xo[t][o][r]);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&bars->xc_empty[t]);
+          const float M = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+          float Ssum = 0.f;
+          if (M > -CUDART_INF_F)
+#pragma unroll
+            for (int o = 0; o < 4; ++o) Ssum += sq[o] * exp2f(mq[o] - M);
+          const int i = (2 * p + t) * BM + r;
+          const float lz2 = M + log2f(Ssum);
+          const float lz = lz2 / kLog2e;
+          if (i < nc) {
+            logz[i] = lz;
+            if (logz_out) logz_out[i] = lz;
+            // may a stiff component come within kSideCut nats of log Z here?
+            side_flag[i] = (f2 > lz2 - kSideCut * kLog2e) || !(lz >= *lzlow);
+            if (bmask) {
+              const float lim = lz2 - kCut2;
+              uint32_t mk = 0;
+              bool dense = ov > lim || !(lz2 > -CUDART_INF_F);
+#pragma unroll
+              for (int e = 0; e < kCand; ++e)
+                if (S.cbm[e] > lim) mk |= 1u << S.block(e);
+#pragma unroll
+              for (int o = 0; o < 3; ++o) {
+                const uint32_t w2[2] = {kq[o].x, kq[o].y};
+#pragma unroll
+                for (int e = 0; e < kCand; ++e) {
+                  const uint32_t cd = (w2[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                  if (cd != kCodeEmpty && mq[o + 1] - (float)(cd & 255u) * kQStep > lim)
+                    mk |= 1u << (cd >> 8);
+                }
+              }
+              bmask[i] = dense ? (nkb >= 32 ? 0xFFFFFFFFu : (1u << nkb) - 1u) : mk;
+            }
           }
         }
       }
@@ -718,7 +797,7 @@ struct StatBars {
 };
 static_assert(offsetof(StatBars, lz) % 16 == 0, "log Z tiles must be 16-byte aligned");
 
-template <int NKC>
+template <int NKC, bool SPLIT>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_stats_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                     int nc, int ncmax, int Kt, int slice_len, int flush_tiles,
@@ -729,6 +808,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     int* status) {
   if (mode && *mode != kModeTensor) return;
   constexpr int Dq = NKC * 32;            // features: phi has 2 Dq = NKC * 64 entries
+  constexpr int NP = SPLIT ? 2 : 1;       // phi boxes per chunk (hi, lo)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   unsigned char* wbuf = base;                          // [NKC][BOX]: W' hi of the block
@@ -838,7 +918,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             lz_issued = tile + 1;
           }
           for (int c = 0; c < NKC; ++c)
-            for (int part = 0; part < 2; ++part, ++itx) {
+            for (int part = 0; part < NP; ++part, ++itx) {
               const int s = itx % SX;
               if (itx >= SX && !ptx::mbar_wait(&bars->x_empty[s], ((itx / SX) - 1) & 1, abort)) {
                 set_status(status, FGMM_ERR_TIMEOUT);
@@ -868,7 +948,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool fresh = true;   // next G2 starts a new accumulation period
       int flushes = 0;
       if (!ptx::mbar_wait(&bars->w_full, 0, abort)) goto fail_m;
-      if (!ptx::mbar_wait(&bars->wlo_ready, 0, abort)) goto fail_m;
+      if (SPLIT && !ptx::mbar_wait(&bars->wlo_ready, 0, abort)) goto fail_m;
       for (int g = 0; g <= ntl && !*abort; ++g) {
         if (g < ntl) {  // ---- G1(g): S^T is single-buffered, released once loaded
           if (g >= 1 && !ptx::mbar_wait(&bars->s_empty, (g - 1) & 1, abort)) goto fail_m;
@@ -878,26 +958,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int sh = itx % SX;
             if (!ptx::mbar_wait(&bars->x_full[sh], (itx / SX) & 1, abort)) goto fail_m;
             ++itx;
-            const int sl = itx % SX;
-            if (!ptx::mbar_wait(&bars->x_full[sl], (itx / SX) & 1, abort)) goto fail_m;
-            ++itx;
+            int sl = sh;
+            if constexpr (SPLIT) {
+              sl = itx % SX;
+              if (!ptx::mbar_wait(&bars->x_full[sl], (itx / SX) & 1, abort)) goto fail_m;
+              ++itx;
+            }
             ptx::tc_fence_after();
-            const uint32_t wa_hi = ptx::smem_u32(wbuf + c * BOX);
-            const uint32_t xb_hi = ptx::smem_u32(xring + sh * BOX);
-            const uint32_t xb_lo = ptx::smem_u32(xring + sl * BOX);
+            // K-major boxes: one descriptor per box, + 2 (32 bytes) per K-step
+            constexpr uint64_t kHiK = ptx::sw128_hi(16, 1024);
+            const uint64_t ah0 = ptx::sw128_desc(ptx::smem_u32(wbuf + c * BOX), kHiK);
+            const uint64_t bh0 = ptx::sw128_desc(ptx::smem_u32(xring + sh * BOX), kHiK);
+            const uint64_t bl0 = ptx::sw128_desc(ptx::smem_u32(xring + sl * BOX), kHiK);
+            // W' lo from TMEM: K elements c*64 + ks*16 .. +15 = columns c*32 + ks*8 .. +7
+            const uint32_t wl_tmem = wlo_tmem + c * 32;
 #pragma unroll
             for (int ks = 0; ks < KC / 16; ++ks) {
-              const uint32_t o = ks * 32;
-              const uint64_t ah = ptx::smem_desc_sw128(wa_hi + o, 16, 1024);
-              const uint64_t bh = ptx::smem_desc_sw128(xb_hi + o, 16, 1024);
-              const uint64_t bl = ptx::smem_desc_sw128(xb_lo + o, 16, 1024);
-              ptx::mma_f16_ss(d_tmem, ah, bh, idesc1, (c > 0 || ks > 0) ? 1u : 0u);
-              ptx::mma_f16_ss(d_tmem, ah, bl, idesc1, 1u);
-              // W' lo from TMEM: K elements c*64 + ks*16 .. +15 = columns c*32 + ks*8 .. +7
-              ptx::mma_f16_ts(d_tmem, wlo_tmem + c * 32 + ks * 8, bh, idesc1, 1u);
+              const uint64_t dk = (uint64_t)(2 * ks);
+              ptx::mma_f16_ss(d_tmem, ah0 + dk, bh0 + dk, idesc1, (c > 0 || ks > 0) ? 1u : 0u);
+              if constexpr (SPLIT) {
+                ptx::mma_f16_ss(d_tmem, ah0 + dk, bl0 + dk, idesc1, 1u);
+                ptx::mma_f16_ts(d_tmem, wl_tmem + ks * 8, bh0 + dk, idesc1, 1u);
+              }
             }
             ptx::mma_commit(&bars->x_empty[sh]);
-            ptx::mma_commit(&bars->x_empty[sl]);
+            if constexpr (SPLIT) ptx::mma_commit(&bars->x_empty[sl]);
           }
           ptx::mma_commit(&bars->s_full);
         }
@@ -908,30 +993,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             goto fail_m;
           ptx::tc_fence_after();
           const uint32_t r0 = ptx::smem_u32(rbuf);
-          // A phase's phi boxes sit in ring slots hi(0), lo(0), hi(1), lo(1), ...; when the
-          // ring holds a whole number of phases, every phase starts at a multiple of its
-          // size, its hi boxes are two slots apart without wrapping, and one MMA with
-          // N = 64 NKC features (leading byte offset 2 BOX between the 64-feature atoms)
-          // covers all chunks.
-          constexpr int CP = (SX % (2 * NKC) == 0) ? NKC : 1;
+          // A phase's phi boxes sit in ring slots hi(0), lo(0), hi(1), lo(1), ... (hi(0),
+          // hi(1), ... with one product); when the ring holds a whole number of phases,
+          // every phase starts at a multiple of its size, its hi boxes are NP slots apart
+          // without wrapping, and one MMA with N = 64 NKC features (leading byte offset
+          // NP BOX between the 64-feature atoms) covers all chunks.
+          constexpr int CP = (SX % (NP * NKC) == 0) ? NKC : 1;
           constexpr uint32_t idesc2 = ptx::idesc_f16(128, 64 * CP, false, true);
           for (int c = 0; c < NKC; c += CP) {
             const uint32_t it0 = itx;
-            for (int i = 0; i < 2 * CP; ++i, ++itx)
+            for (int i = 0; i < NP * CP; ++i, ++itx)
               if (!ptx::mbar_wait(&bars->x_full[itx % SX], (itx / SX) & 1, abort)) goto fail_m;
             ptx::tc_fence_after();
-            const uint32_t xb_hi = ptx::smem_u32(xring + (it0 % SX) * BOX);
-            const uint32_t xb_lo = ptx::smem_u32(xring + ((it0 + 1) % SX) * BOX);
             const uint32_t d_tmem = acc_tmem + c * 64;
+            constexpr uint64_t kHiA = ptx::sw128_hi(16, 1024);
+            constexpr uint64_t kHiB = ptx::sw128_hi(NP * BOX, 1024);
+            const uint64_t a0 = ptx::sw128_desc(r0, kHiA);
+            const uint64_t bh0 = ptx::sw128_desc(ptx::smem_u32(xring + (it0 % SX) * BOX), kHiB);
+            const uint64_t bl0 = ptx::sw128_desc(ptx::smem_u32(xring + ((it0 + 1) % SX) * BOX), kHiB);
 #pragma unroll
             for (int ks = 0; ks < BM / 16; ++ks) {
               // A = R^T (K-major, K = points): box ks/4, 32 B per 16 points inside it
-              const uint64_t a = ptx::smem_desc_sw128(r0 + (ks >> 2) * BOX + (ks & 3) * 32, 16, 1024);
+              const uint64_t a = a0 + (uint64_t)((((ks >> 2) * BOX) + (ks & 3) * 32) >> 4);
               // B = phi (MN-major, K = points = rows): 16 rows = 2 atoms of 1024 B
-              const uint64_t bh = ptx::smem_desc_sw128(xb_hi + ks * 2048, 2 * BOX, 1024);
-              const uint64_t bl = ptx::smem_desc_sw128(xb_lo + ks * 2048, 2 * BOX, 1024);
-              ptx::mma_f16_ss(d_tmem, a, bh, idesc2, (fresh && ks == 0) ? 0u : 1u);
-              ptx::mma_f16_ss(d_tmem, a, bl, idesc2, 1u);
+              const uint64_t db = (uint64_t)(ks * (2048 >> 4));
+              ptx::mma_f16_ss(d_tmem, a, bh0 + db, idesc2, (fresh && ks == 0) ? 0u : 1u);
+              if constexpr (SPLIT) ptx::mma_f16_ss(d_tmem, a, bl0 + db, idesc2, 1u);
             }
             for (uint32_t i = it0; i < itx; ++i) ptx::mma_commit(&bars->x_empty[i % SX]);
           }
@@ -974,7 +1061,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     unsigned char* rrow = rbuf + g * BOX + (kl >> 3) * 1024 + (kl & 7) * 128;
     // W' lo of this component into TMEM (the third product's A operand): this
     // warpgroup writes K elements g*Dq .. g*Dq+Dq-1 = columns g*Dq/2 .. +Dq/2-1
-    {
+    if constexpr (SPLIT) {
       const uint4* src = reinterpret_cast<const uint4*>(wop + ((size_t)Kt + k) * (2 * Dq) + g * Dq);
 #pragma unroll 1
       for (int c8 = 0; c8 < Dq / 16; ++c8) {   // 8 columns = 16 fp16 per store
@@ -1006,28 +1093,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) ptx::mbar_arrive(&bars->s_empty);
       const float* lzt = bars->lz[b];
       uint32_t pk[2][16];
+      // t = log2(r 2^15) = S ksl + (ckl - log Z log2(e)), two points per packed operation;
+      // r <= 1 up to rounding, and the clamp keeps fp16(r 2^15) finite even where the two
+      // sweeps' roundings disagree.  Rows past the tile's points get r = 0.
+      const uint64_t ksl2 = ptx::f2_pack(ksl, ksl), ckl2 = ptx::f2_pack(ckl, ckl);
+      const uint64_t nl2e = ptx::f2_pack(-kLog2e, -kLog2e);
+      const bool full = nvalid >= BM;
+      uint64_t nk2 = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int pb = 64 * g + 32 * h;        // first point of this 32-column group
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float4 lz4 = *reinterpret_cast<const float4*>(lzt + pb + e);
-          const float lzv[4] = {lz4.x, lz4.y, lz4.z, lz4.w};
+          float t[4];
+          ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(u[h][e]), __uint_as_float(u[h][e + 1])),
+                                     ksl2, ptx::f2_fma(ptx::f2_pack(lz4.x, lz4.y), nl2e, ckl2)),
+                         t[0], t[1]);
+          ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(u[h][e + 2]), __uint_as_float(u[h][e + 3])),
+                                     ksl2, ptx::f2_fma(ptx::f2_pack(lz4.z, lz4.w), nl2e, ckl2)),
+                         t[2], t[3]);
           float rr[4];
 #pragma unroll
-          for (int z = 0; z < 4; ++z) {
-            // t = log2(r 2^15); r <= 1 up to rounding, and the clamp keeps fp16(r 2^15)
-            // finite even where the two sweeps' roundings disagree
-            const float t = fminf(fmaf(__uint_as_float(u[h][e + z]), ksl, fmaf(-lzv[z], kLog2e, ckl)), 15.f);
-            rr[z] = exp2f(pb + e + z < nvalid ? t : -CUDART_INF_F);
-          }
+          for (int z = 0; z < 4; ++z)
+            rr[z] = ptx::ex2((full || pb + e + z < nvalid) ? fminf(t[z], 15.f) : -CUDART_INF_F);
           const __half2 h01 = __floats2half2_rn(rr[0], rr[1]);
           const __half2 h23 = __floats2half2_rn(rr[2], rr[3]);
           const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-          nk += (f01.x + f01.y) + (f23.x + f23.y);
+          nk2 = ptx::f2_add(nk2, ptx::f2_add(ptx::f2_pack(f01.x, f01.y), ptx::f2_pack(f23.x, f23.y)));
           pk[h][e >> 1] = *reinterpret_cast<const uint32_t*>(&h01);
           pk[h][(e >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&h23);
         }
+      }
+      {
+        float n0, n1;
+        ptx::f2_unpack(nk2, n0, n1);
+        nk += n0 + n1;
       }
       // R^T of the previous tile must have been consumed by G2 before it is overwritten
       if (tile >= 1 &&
@@ -1162,19 +1263,24 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows) {
 }
 
 size_t lse_smem(int nkc, int Kt, bool params) {
-  return 1024 + (size_t)(nkc + SW) * BOX + sizeof(LseBars) +
+  return 1024 + (size_t)(2 * nkc + lse_ring(nkc)) * BOX + sizeof(LseBars) +
          (params ? 3 * (size_t)Kt * sizeof(float) : 0);
 }
 constexpr size_t kMaxDynSmem = 232448;  // 227 KB per block on sm_100
 size_t stats_smem(int nkc) { return 1024 + (size_t)(nkc + SX + 2) * BOX + sizeof(StatBars); }
 
+template <int NKC, bool SPLIT>
+cudaError_t set_attrs_split() {
+  cudaError_t e = cudaFuncSetAttribute(tc_lse_kernel<NKC, SPLIT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxDynSmem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(tc_stats_kernel<NKC, SPLIT>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)stats_smem(NKC));
+}
 template <int NKC>
 cudaError_t set_attrs() {
-  cudaError_t e = cudaFuncSetAttribute(tc_lse_kernel<NKC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kMaxDynSmem);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(tc_stats_kernel<NKC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)stats_smem(NKC));
+  cudaError_t e = set_attrs_split<NKC, true>();
+  return e != cudaSuccess ? e : set_attrs_split<NKC, false>();
 }
 
 }  // namespace
@@ -1255,20 +1361,24 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
                           cudaStream_t s) {
   const Workspace& w = c.ws;
   const int nkc = w.K1 / 64;
-  const int ntiles = (int)ceil_div64(n, BM);
-  const int grid = ntiles < c.num_sms ? ntiles : c.num_sms;
+  const int npairs = (int)ceil_div64(ceil_div64(n, BM), 2);   // sweep 1 works on tile pairs
+  const int grid = npairs < c.num_sms ? npairs : c.num_sms;
   const CUtensorMap& tx = c.tc.tmap_x;
   const CUtensorMap& tw = c.tc.tmap_w;
   const bool params = lse_smem(nkc, w.Kt, true) <= kMaxDynSmem;
   const size_t smem = lse_smem(nkc, w.Kt, params);
+  const bool split = c.prec != FGMM_PREC_FP16;
   prof_begin(c, KI_TC_LSE, s, mode, kModeTensor);
 #define LSE_CASE(N_)                                                                          \
   case N_:                                                                                    \
-    tc_lse_kernel<N_><<<grid, kLseThreads, smem, s>>>(tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, \
-                                                     w.tks, params ? 1 : 0, w.logz, logz_out,   \
-                                                     w.xop, w.tckf, w.lzlow, w.side_flag,     \
-                                                     tc_skip(c) ? w.bmask : nullptr, mode,    \
-                                                     w.status);                               \
+    if (split)                                                                                \
+      tc_lse_kernel<N_, true><<<grid, kLseThreads, smem, s>>>(                                \
+          tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, w.tks, params ? 1 : 0, w.logz, logz_out,   \
+          w.xop, w.tckf, w.lzlow, w.side_flag, tc_skip(c) ? w.bmask : nullptr, mode, w.status); \
+    else                                                                                      \
+      tc_lse_kernel<N_, false><<<grid, kLseThreads, smem, s>>>(                               \
+          tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, w.tks, params ? 1 : 0, w.logz, logz_out,   \
+          w.xop, w.tckf, w.lzlow, w.side_flag, tc_skip(c) ? w.bmask : nullptr, mode, w.status); \
     break;
   switch (nkc) {
     LSE_CASE(1)
@@ -1304,17 +1414,24 @@ cudaError_t launch_tc_stats(const Ctx& c, int64_t n, const int* mode, cudaStream
   const dim3 grid = skip ? dim3((w.Kt / BKc) * S, 1) : dim3(w.Kt / BKc, S);
   const CUtensorMap& tx = c.tc.tmap_x;
   const CUtensorMap& tw = c.tc.tmap_w;
-  const int flush_tiles = 8;  // fp32 runs of 1024 points (64 MMA steps) between fp64 flushes
+  // fp32 runs (in tiles of 128 points) between fp64 flushes of the statistics
+  const int flush_tiles = skip ? kFlushTilesSkip : kFlushTilesDense;
   // block skipping: phi and log Z were rewritten in sweep-2 order, tiles come from lists
   const float* lz = skip ? w.lzp : w.logz;
   const int* tl = skip ? w.tlist : nullptr;
   const int tl_stride = (int)(kChunk / BM);
+  const bool split = c.prec != FGMM_PREC_FP16;
   prof_begin(c, KI_TC_STATS, s, mode, kModeTensor);
 #define STATS_CASE(N_)                                                                         \
   case N_:                                                                                     \
-    tc_stats_kernel<N_><<<grid, kTcThreads, stats_smem(N_), s>>>(                              \
-        tx, tw, (int)n, (int)kChunk, w.Kt, slice, flush_tiles, w.tck, w.tks, lz, w.stats,      \
-        w.KpS, w.Dp, w.wop, tl, w.tcnt, tl_stride, tc_stat_slots(c), mode, w.status);          \
+    if (split)                                                                                 \
+      tc_stats_kernel<N_, true><<<grid, kTcThreads, stats_smem(N_), s>>>(                      \
+          tx, tw, (int)n, (int)kChunk, w.Kt, slice, flush_tiles, w.tck, w.tks, lz, w.stats,    \
+          w.KpS, w.Dp, w.wop, tl, w.tcnt, tl_stride, tc_stat_slots(c), mode, w.status);        \
+    else                                                                                       \
+      tc_stats_kernel<N_, false><<<grid, kTcThreads, stats_smem(N_), s>>>(                     \
+          tx, tw, (int)n, (int)kChunk, w.Kt, slice, flush_tiles, w.tck, w.tks, lz, w.stats,    \
+          w.KpS, w.Dp, w.wop, tl, w.tcnt, tl_stride, tc_stat_slots(c), mode, w.status);        \
     break;
   switch (nkc) {
     STATS_CASE(1)

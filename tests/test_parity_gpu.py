@@ -23,7 +23,8 @@ SAFE_PRECISIONS = ["fp32", "auto"]
 def _gmm(K, D, cov=0, reg=1e-6, prec="fp32"):
     import ivf_quantizer_b200 as q
     g = q.GMM(K, D, cov, reg)
-    g.set_precision({"fp32": q.PREC_FP32, "fp16x3": q.PREC_FP16X3, "auto": q.PREC_AUTO}[prec])
+    g.set_precision({"fp32": q.PREC_FP32, "fp16x3": q.PREC_FP16X3, "auto": q.PREC_AUTO,
+                     "fp16": q.PREC_FP16}[prec])
     return g
 
 
@@ -481,3 +482,33 @@ def test_high_dim_border_shape(dtype):
                     var.double().numpy())
     print(compare_step((wd.cpu().numpy(), md.cpu().numpy(), vd.cpu().numpy()), ref,
                        X.float().numpy(), logz_gpu=lz.cpu().numpy()))
+
+
+@pytest.mark.parametrize("gen,N,K,seed", [("c1", 10_000, 16, 30), ("table1", 20_000, 64, 31),
+                                          ("table1", 3000 + 77, 256, 32)])
+def test_fp16_one_product_mode_against_the_oracle(gen, N, K, seed):
+    """FGMM_PREC_FP16 (one fp16 product per term in both sweeps) runs on the tensor cores
+    and its error against the oracle is measured, not assumed: per-point log Z to within
+    the mode's class (relative 1e-2: one fp16 rounding, 2^-11, of terms that sum to a few
+    times |log z|), parameters valid, and the same step with the split products (FP16X3)
+    inside the fp32-class tolerance on the same input."""
+    import ivf_quantizer_b200 as q
+    X = synth.generate(gen, N, seed=seed)
+    w, mu, var = synth.init_params(X, K, seed=seed)
+    ref = O.em_step(X.double().numpy(), w.double().numpy(), mu.double().numpy(),
+                    var.double().numpy())
+    errs = {}
+    for prec in ("fp16", "fp16x3"):
+        g = _gmm(K, X.shape[1], prec=prec)
+        wd, md, vd = g.new_params(w, mu, var)
+        lz = torch.empty(N, device="cuda")
+        g.step(X.cuda(), wd, md, vd, logz=lz)
+        assert g.status() == 0
+        assert g.last_step_path() == {"fp16": q.PREC_FP16, "fp16x3": q.PREC_FP16X3}[prec]
+        errs[prec] = float((np.abs(lz.cpu().numpy() - ref.logZ) / np.abs(ref.logZ)).max())
+        assert torch.isfinite(md).all() and bool((vd > 0).all())
+        assert abs(float(wd.double().sum()) - 1.0) < 1e-5
+        g.close()
+    print(gen, N, K, errs)
+    assert errs["fp16"] <= 1e-2
+    assert errs["fp16x3"] <= 1e-4
