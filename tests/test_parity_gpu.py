@@ -394,9 +394,18 @@ def _step_with(X, w, mu, var, prec):
 
 
 def test_auto_takes_tensor_cores_when_well_conditioned():
+    """The Table-1 shape with per-dimension sigma in [1, 3]: every component stays well
+    inside the expanded form's conditioning bounds (no component is stiff before or
+    after the pass), so AUTO runs exactly the FP16X3 step, bit for bit."""
     import ivf_quantizer_b200 as q
-    X = synth.generate("table1", 20000, seed=16)
+    X = synth.generate(synth.spec("table1", sigma_lo=1.0), 20000, seed=16)
     w, mu, var = synth.init_params(X, 64, seed=16)
+    g = _gmm(64, 128, prec="auto")
+    wd, md, vd = g.new_params(w, mu, var)
+    g.step(X.cuda(), wd, md, vd)
+    info = g.last_step_info()
+    g.close()
+    assert info["n_stiff"] == 0 and info["n_grey"] == 0, info
     pa, *ra = _step_with(X, w, mu, var, "auto")
     pt, *rt = _step_with(X, w, mu, var, "fp16x3")
     assert pa == q.PREC_FP16X3 and pt == q.PREC_FP16X3
