@@ -302,15 +302,16 @@ __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ld
 }
 
 // ------------------------------------------------------------------ sweep 1 (log Z)
-// 640 threads: warp 0 TMA producer, warp 1 MMA issuer, warps 4..19 epilogue.  A CTA works
+// 384 threads: warp 0 TMA producer, warp 1 MMA issuer, warps 4..11 epilogue.  A CTA works
 // on pairs of 128-point tiles (A = 2p, B = 2p + 1): every W' box that the TMA brings in
 // feeds the products of both tiles, so each byte streamed from L2 serves 256 points (the
 // W' stream of a 128-point tile would need about as many L2 bytes per clock as the
-// products it feeds can take).  The four epilogue warpgroups split each 128-column S
-// tile in quarters (columns 32g .. 32g+31; four warps per scheduler hide the TMEM-load
-// and exp latencies), one row of A and the same row of B per thread, and keep a running
-// (max, sum) per row; at the end of the pair groups 1..3 hand their pairs to group 0
-// through shared memory, which writes log Z.
+// products it feeds can take).  The two epilogue warpgroups split each 128-column S tile
+// in halves (columns 64h .. 64h+63), one row of A and the same row of B per thread, and
+// keep a running (max, sum) per row, the 64 columns' maxima and sums as four independent
+// partial chains; at the end of the pair half 1 hands its values to half 0 through shared
+// memory, which writes log Z.  Two epilogue warps per scheduler (not four) leave the
+// single MMA-issuing thread the issue slots it needs to keep the tensor pipe fed.
 // phi hi of both tiles sits in shared memory (A operand of two products); phi lo sits in
 // tensor memory (A operand of the third), written there by the epilogue warps as soon as
 // the previous pair's last products on that tile have completed.  TMEM: S_A, S_B (one
@@ -318,7 +319,7 @@ __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ld
 // other way round), phi lo of A and B.
 constexpr int kEpiWarps = 8;                        // statistics sweep
 constexpr int kTcThreads = 128 + 32 * kEpiWarps;
-constexpr int kLseEpiWarps = 16;                    // log-sum-exp sweep
+constexpr int kLseEpiWarps = 8;                     // log-sum-exp sweep
 constexpr int kLseThreads = 128 + 32 * kLseEpiWarps;
 constexpr int kLseRingMax = 8;
 // W' ring stages of sweep 1: as many boxes as fit beside the pair's phi hi (an even
@@ -334,20 +335,20 @@ struct LseBars {
   uint64_t drain;
   uint32_t tmem;
   int abort;
-  float xm[2][3][BM];   // (max, sum, filter max) of column groups 1..3, per tile of the pair
-  float xs[2][3][BM];
-  float xf[2][3][BM];
-  uint2 xk[2][3][BM];   // candidate blocks of column groups 1..3 (block skipping)
-  float xo[2][3][BM];   // their largest block maximum left out of the candidates
+  float xm[2][BM];      // (max, sum, filter max) of column half 1, per tile of the pair
+  float xs[2][BM];
+  float xf[2][BM];
+  uint2 xk[2][BM];      // candidate blocks of column half 1 (block skipping)
+  float xo[2][BM];      // their largest block maximum left out of the candidates
 };
 static_assert(sizeof(LseBars) % 16 == 0, "the staged parameters after LseBars are read as float4");
 
-// Block skipping, sweep 1 side.  Every epilogue thread keeps, for its row and its 32
+// Block skipping, sweep 1 side.  Every epilogue thread keeps, for its row and its 64
 // columns, the (at most kCand) largest block maxima that lie within the cut of its
 // running maximum; a block that falls out of range can never come back, the maximum
 // only grows.  A block pushed out of a full list leaves its maximum in `ovm`; if that
 // is within the cut of log Z in the end, the row is marked dense (every block).  At the
-// end of a tile the column groups 1..3 hand their candidates to group 0 as 16-bit codes
+// end of a tile column half 1 hands its candidates to half 0 as 16-bit codes
 // (block << 8 | q, q = floor((max - block max) / step)); decoding gives max - q step >=
 // the true block maximum, so the test against log Z - cut can only keep a block.
 constexpr int kCand = 4;
@@ -413,8 +414,8 @@ __global__ void __launch_bounds__(kLseThreads, 1)
       ptx::mbar_init(&bars->s_full[b], 1);
       ptx::mbar_init(&bars->s_empty[b], kLseEpiWarps);
       ptx::mbar_init(&bars->xlo_ready[b], kLseEpiWarps);
-      ptx::mbar_init(&bars->xc_full[b], 3 * kLseEpiWarps / 4);
-      ptx::mbar_init(&bars->xc_empty[b], kLseEpiWarps / 4);
+      ptx::mbar_init(&bars->xc_full[b], kLseEpiWarps / 2);
+      ptx::mbar_init(&bars->xc_empty[b], kLseEpiWarps / 2);
     }
     ptx::mbar_init(&bars->drain, 1);
     bars->abort = 0;
@@ -515,13 +516,16 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             const uint64_t bl0 = ptx::sw128_desc(ptx::smem_u32(wring + sl * BOX), kHiK);
             for (int t = 0; t < nt; ++t) {
               if (ci == 0) {
-                // S_t free (its previous block read out), phi lo of this pair in place
+                // S_t free (its previous block read out), phi lo of this pair in place; the
+                // epilogue warps' TMEM accesses before their arrivals are ordered ahead of
+                // these products by the fence (TMA arrivals need none: the async proxy
+                // completes its writes before the barrier phase does)
                 if (u >= 1 && !ptx::mbar_wait(&bars->s_empty[t], (u - 1) & 1, abort)) goto fail_m;
                 if (SPLIT && kb == 0 && !ptx::mbar_wait(&bars->xlo_ready[t], j & 1, abort))
                   goto fail_m;
+                ptx::tc_fence_after();
               }
               if (kb == 0 && !ptx::mbar_wait(&bars->x_full[t][c], j & 1, abort)) goto fail_m;
-              ptx::tc_fence_after();
               const uint32_t d_tmem = tmem + t * 128;
               // phi lo from TMEM: K elements c*64 + ks*16 .. +15 = columns c*32 + ks*8 .. +7
               const uint32_t xl_tmem = xlo_tmem + t * 128 + c * 32;
@@ -554,20 +558,20 @@ __global__ void __launch_bounds__(kLseThreads, 1)
       }
     }
   } else if (warp >= 4) {
-    const int g = (warp - 4) >> 2;         // column quarter of the S tile
+    const int h = (warp - 4) >> 2;         // column half of the S tile (64 columns)
     const int q = warp & 3;                // TMEM lane quarter
     const int r = q * 32 + lane;           // row of the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     // phi lo of `tile` into TMEM buffer t: this thread's row, K elements
-    // g*NKC*32 .. +NKC*32-1 = columns g*NKC*16 .. +NKC*16-1 (row tile*BM + r < ncmax)
+    // h*NKC*32 .. +NKC*32-1 = columns h*NKC*16 .. +NKC*16-1 (row tile*BM + r < ncmax)
     auto put_xlo = [&](int tile, int t) {
       const uint4* src = reinterpret_cast<const uint4*>(
-          xop + ((size_t)ncmax + (size_t)tile * BM + r) * (NKC * 64) + g * (NKC * 16));
+          xop + ((size_t)ncmax + (size_t)tile * BM + r) * (NKC * 64) + h * (NKC * 32));
 #pragma unroll
-      for (int c8 = 0; c8 < NKC; ++c8) {   // 8 columns = 16 fp16 per store
+      for (int c8 = 0; c8 < 2 * NKC; ++c8) {   // 8 columns = 16 fp16 per store
         const uint4 v0 = __ldg(src + 2 * c8), v1 = __ldg(src + 2 * c8 + 1);
         const uint32_t r8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        ptx::tmem_st8(xlo_tmem + t * 128 + lane_base + g * (NKC * 8) + c8 * 8, r8);
+        ptx::tmem_st8(xlo_tmem + t * 128 + lane_base + h * (NKC * 16) + c8 * 8, r8);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -591,26 +595,30 @@ __global__ void __launch_bounds__(kLseThreads, 1)
         for (int t = 0; t < 2; ++t) {
           if (t >= nt) break;
           RowState& S = st[t];
-          if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full[t], u & 1, abort))) {
+          if (!ptx::mbar_wait_warp(&bars->s_full[t], u & 1, abort)) {
             set_status(status, FGMM_ERR_TIMEOUT);
             bars->abort = 1;
             break;
           }
           ptx::tc_fence_after();
-          const int col = 32 * g;            // column within the 128-component block
-          uint32_t uu[32];
-          ptx::tmem_ld32(tmem + lane_base + t * 128 + col, uu);
+          const int col = 64 * h;            // first column within the 128-component block
+          uint32_t ua[32], ub[32];
+          ptx::tmem_ld32(tmem + lane_base + t * 128 + col, ua);
+          ptx::tmem_ld32(tmem + lane_base + t * 128 + col + 32, ub);
           ptx::tmem_wait_ld();
           // the values are in registers: hand S_t back to the MMA warp now
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&bars->s_empty[t]);
-          // log2-scaled log-densities of the 32 columns, two per packed fp32x2 operation
-          uint64_t v2[16];
-          float bm = -CUDART_INF_F;
+          // log2-scaled log-densities of the 64 columns, two per packed fp32x2 operation;
+          // the maxima and sums run as four independent partial chains
+          uint64_t v2[32];
+          float bmx[4], fmx[4];
+#pragma unroll
+          for (int z = 0; z < 4; ++z) bmx[z] = fmx[z] = -CUDART_INF_F;
           const int k0 = kb * BKc + col;
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
+          for (int e4 = 0; e4 < 16; ++e4) {
             float4 cc, kk, cf;
             if (params_in_smem) {
               cc = *reinterpret_cast<const float4*>(ckl + k0 + 4 * e4);
@@ -624,8 +632,10 @@ __global__ void __launch_bounds__(kLseThreads, 1)
               kk.x *= kLog2e; kk.y *= kLog2e; kk.z *= kLog2e; kk.w *= kLog2e;
               cf.x *= kLog2e; cf.y *= kLog2e; cf.z *= kLog2e; cf.w *= kLog2e;
             }
-            const uint64_t f01 = ptx::f2_pack(__uint_as_float(uu[4 * e4 + 0]), __uint_as_float(uu[4 * e4 + 1]));
-            const uint64_t f23 = ptx::f2_pack(__uint_as_float(uu[4 * e4 + 2]), __uint_as_float(uu[4 * e4 + 3]));
+            const uint32_t* uv = e4 < 8 ? ua : ub;
+            const int o4 = 4 * (e4 & 7);
+            const uint64_t f01 = ptx::f2_pack(__uint_as_float(uv[o4 + 0]), __uint_as_float(uv[o4 + 1]));
+            const uint64_t f23 = ptx::f2_pack(__uint_as_float(uv[o4 + 2]), __uint_as_float(uv[o4 + 3]));
             const uint64_t k01 = ptx::f2_pack(kk.x, kk.y), k23 = ptx::f2_pack(kk.z, kk.w);
             v2[2 * e4 + 0] = ptx::f2_fma(f01, k01, ptx::f2_pack(cc.x, cc.y));
             v2[2 * e4 + 1] = ptx::f2_fma(f23, k23, ptx::f2_pack(cc.z, cc.w));
@@ -635,23 +645,27 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             ptx::f2_unpack(ptx::f2_fma(f23, k23, ptx::f2_pack(cf.z, cf.w)), g[2], g[3]);
             ptx::f2_unpack(v2[2 * e4 + 0], v[0], v[1]);
             ptx::f2_unpack(v2[2 * e4 + 1], v[2], v[3]);
-            S.fm = fmaxf(S.fm, fmaxf(fmaxf(g[0], g[1]), fmaxf(g[2], g[3])));
-            bm = fmaxf(bm, fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
+            fmx[e4 & 3] = fmaxf(fmx[e4 & 3], fmaxf(fmaxf(g[0], g[1]), fmaxf(g[2], g[3])));
+            bmx[e4 & 3] = fmaxf(bmx[e4 & 3], fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
           }
+          S.fm = fmaxf(S.fm, fmaxf(fmaxf(fmx[0], fmx[1]), fmaxf(fmx[2], fmx[3])));
+          const float bm = fmaxf(fmaxf(bmx[0], bmx[1]), fmaxf(bmx[2], bmx[3]));
           const float nm = fmaxf(S.m, bm);
           if (nm > -CUDART_INF_F) {
             // every argument is <= 0 after the shift, so 2^x in (0, 1]; the SFU's exp2
             // (flushing results below 2^-126, far under fp32 resolution of the sum)
             const uint64_t shift = ptx::f2_pack(-nm, -nm);
-            uint64_t acc2 = ptx::f2_pack(0.f, 0.f);
+            uint64_t acc[4];
 #pragma unroll
-            for (int e2 = 0; e2 < 16; ++e2) {
+            for (int z = 0; z < 4; ++z) acc[z] = ptx::f2_pack(0.f, 0.f);
+#pragma unroll
+            for (int e2 = 0; e2 < 32; ++e2) {
               float t0, t1;
               ptx::f2_unpack(ptx::f2_add(v2[e2], shift), t0, t1);
-              acc2 = ptx::f2_add(acc2, ptx::f2_pack(ptx::ex2(t0), ptx::ex2(t1)));
+              acc[e2 & 3] = ptx::f2_add(acc[e2 & 3], ptx::f2_pack(ptx::ex2(t0), ptx::ex2(t1)));
             }
             float a0, a1;
-            ptx::f2_unpack(acc2, a0, a1);
+            ptx::f2_unpack(ptx::f2_add(ptx::f2_add(acc[0], acc[1]), ptx::f2_add(acc[2], acc[3])), a0, a1);
             S.s = S.s * ptx::ex2(S.m - nm) + (a0 + a1);
             S.m = nm;
           }
@@ -687,21 +701,21 @@ __global__ void __launch_bounds__(kLseThreads, 1)
         }
       }
       if (*abort) break;
-      // combine the four column quarters of each row, per tile of the pair
+      // combine the two column halves of each row, per tile of the pair
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (t >= nt) break;
         const RowState& S = st[t];
-        if (g >= 1) {
+        if (h == 1) {
           if (j >= 1 &&
-              !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->xc_empty[t], (j - 1) & 1, abort))) {
+              !ptx::mbar_wait_warp(&bars->xc_empty[t], (j - 1) & 1, abort)) {
             set_status(status, FGMM_ERR_TIMEOUT);
             bars->abort = 1;
             break;
           }
-          bars->xm[t][g - 1][r] = S.m;
-          bars->xs[t][g - 1][r] = S.s;
-          bars->xf[t][g - 1][r] = S.fm;
+          bars->xm[t][r] = S.m;
+          bars->xs[t][r] = S.s;
+          bars->xf[t][r] = S.fm;
           if (bmask) {
             uint32_t code[kCand];
 #pragma unroll
@@ -713,38 +727,30 @@ __global__ void __launch_bounds__(kLseThreads, 1)
                 code[e] = (S.block(e) << 8) | (uint32_t)qd;
               }
             }
-            bars->xk[t][g - 1][r] = make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
-            bars->xo[t][g - 1][r] = S.ovm;
+            bars->xk[t][r] = make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
+            bars->xo[t][r] = S.ovm;
           }
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&bars->xc_full[t]);
         } else {
-          if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->xc_full[t], j & 1, abort))) {
+          if (!ptx::mbar_wait_warp(&bars->xc_full[t], j & 1, abort)) {
             set_status(status, FGMM_ERR_TIMEOUT);
             bars->abort = 1;
             break;
           }
-          float mq[4] = {S.m, 0.f, 0.f, 0.f}, sq[4] = {S.s, 0.f, 0.f, 0.f};
-          float f2 = S.fm;
-          uint2 kq[3];
+          const float m1 = bars->xm[t][r], s1 = bars->xs[t][r];
+          const float f2 = fmaxf(S.fm, bars->xf[t][r]);
+          uint2 kq = make_uint2(0u, 0u);
           float ov = S.ovm;
-#pragma unroll
-          for (int o = 0; o < 3; ++o) {
-            mq[o + 1] = bars->xm[t][o][r];
-            sq[o + 1] = bars->xs[t][o][r];
-            f2 = fmaxf(f2, bars->xf[t][o][r]);
-            if (bmask) {
-              kq[o] = bars->xk[t][o][r];
-              ov = fmaxf(ov, bars->xo[t][o][r]);
-            }
+          if (bmask) {
+            kq = bars->xk[t][r];
+            ov = fmaxf(ov, bars->xo[t][r]);
           }
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&bars->xc_empty[t]);
-          const float M = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+          const float M = fmaxf(S.m, m1);
           float Ssum = 0.f;
-          if (M > -CUDART_INF_F)
-#pragma unroll
-            for (int o = 0; o < 4; ++o) Ssum += sq[o] * exp2f(mq[o] - M);
+          if (M > -CUDART_INF_F) Ssum = S.s * exp2f(S.m - M) + s1 * exp2f(m1 - M);
           const int i = (2 * p + t) * BM + r;
           const float lz2 = M + log2f(Ssum);
           const float lz = lz2 / kLog2e;
@@ -760,15 +766,12 @@ __global__ void __launch_bounds__(kLseThreads, 1)
 #pragma unroll
               for (int e = 0; e < kCand; ++e)
                 if (S.cbm[e] > lim) mk |= 1u << S.block(e);
+              const uint32_t w2[2] = {kq.x, kq.y};
 #pragma unroll
-              for (int o = 0; o < 3; ++o) {
-                const uint32_t w2[2] = {kq[o].x, kq[o].y};
-#pragma unroll
-                for (int e = 0; e < kCand; ++e) {
-                  const uint32_t cd = (w2[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-                  if (cd != kCodeEmpty && mq[o + 1] - (float)(cd & 255u) * kQStep > lim)
-                    mk |= 1u << (cd >> 8);
-                }
+              for (int e = 0; e < kCand; ++e) {
+                const uint32_t cd = (w2[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                if (cd != kCodeEmpty && m1 - (float)(cd & 255u) * kQStep > lim)
+                  mk |= 1u << (cd >> 8);
               }
               bmask[i] = dense ? (nkb >= 32 ? 0xFFFFFFFFu : (1u << nkb) - 1u) : mk;
             }
@@ -978,7 +981,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               if (!ptx::mbar_wait(&bars->x_full[sl], (itx / SX) & 1, abort)) goto fail_m;
               ++itx;
             }
-            ptx::tc_fence_after();
+            // (TMA arrivals: no tcgen05 fence needed; the one after s_empty orders the
+            // epilogue's reads of S^T ahead of these products)
             // K-major boxes: one descriptor per box, + 2 (32 bytes) per K-step
             constexpr uint64_t kHiK = ptx::sw128_hi(16, 1024);
             const uint64_t ah0 = ptx::sw128_desc(ptx::smem_u32(wbuf + c * BOX), kHiK);
@@ -1018,7 +1022,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t it0 = itx;
             for (int i = 0; i < NP * CP; ++i, ++itx)
               if (!ptx::mbar_wait(&bars->x_full[itx % SX], (itx / SX) & 1, abort)) goto fail_m;
-            ptx::tc_fence_after();
             const uint32_t d_tmem = acc_tmem + c * 64;
             constexpr uint64_t kHiA = ptx::sw128_hi(16, 1024);
             constexpr uint64_t kHiB = ptx::sw128_hi(NP * BOX, 1024);
@@ -1092,9 +1095,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int row0 = tile_row(tile);
       const int b = tile & 1;
       const int nvalid = p1 - row0;            // points of this tile inside the slice
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->s_full, tile & 1, abort)))
+      if (!ptx::mbar_wait_warp(&bars->s_full, tile & 1, abort))
         goto fail_e;
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->lz_full[b], (tile >> 1) & 1, abort)))
+      if (!ptx::mbar_wait_warp(&bars->lz_full[b], (tile >> 1) & 1, abort))
         goto fail_e;
       ptx::tc_fence_after();
       // load this warpgroup's 64 columns of S^T, then free the buffer for G1(tile + 1)
@@ -1146,7 +1149,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       // R^T of the previous tile must have been consumed by G2 before it is overwritten
       if (tile >= 1 &&
-          !__all_sync(0xffffffffu, ptx::mbar_wait(&bars->r_empty, (tile - 1) & 1, abort)))
+          !ptx::mbar_wait_warp(&bars->r_empty, (tile - 1) & 1, abort))
         goto fail_e;
 #pragma unroll
       for (int h = 0; h < 2; ++h)
@@ -1163,7 +1166,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::mbar_arrive(&bars->r_full);
       }
       if (++tiles_since_flush == flush_tiles || tile == ntl - 1) {
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->acc_full, flushes & 1, abort)))
+        if (!ptx::mbar_wait_warp(&bars->acc_full, flushes & 1, abort))
           goto fail_e;
         ptx::tc_fence_after();
         const double inv = 1.0 / (double)kRScale;
@@ -1185,7 +1188,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&bars->nk_full);
         } else {
-          if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bars->nk_full, flushes & 1, abort)))
+          if (!ptx::mbar_wait_warp(&bars->nk_full, flushes & 1, abort))
             goto fail_e;
           atomicAdd(slot, ((double)nk + (double)bars->nkx[kl]) * inv);
         }

@@ -81,6 +81,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait of a whole warp: lane 0 alone polls the mbarrier (barrier operations of
+// 32 lanes on one word are serialised by the shared-memory pipe, which the tensor cores'
+// operand reads and the TMA share), then the warp synchronises with it; the warp's other
+// lanes are ordered after lane 0's acquire by the warp barrier.  Returns lane 0's result
+// on every lane.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  int ok = 1;
+  if ((threadIdx.x & 31u) == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
 // Bounded wait that ignores the abort flag: used while draining after an abort, so
 // that no copy or MMA is still writing when the CTA frees its resources.
 __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
