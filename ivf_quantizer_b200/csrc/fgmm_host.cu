@@ -169,6 +169,7 @@ void free_ws(Workspace& w) {
   void* ptrs[] = {w.mu,     w.prec,   w.cconst, w.logz, w.ll_tiles, w.ll_total,
                   w.stats,  w.nk,     w.status, w.center, w.dscale, w.wop,
                   w.tck,    w.tks,    w.xop,    w.mode, w.stiff,    w.stiff_list, w.n_stiff,
+                  w.tce,    w.acut,   w.alist,  w.nalist,
                   w.side_part, w.mode2, w.canon, w.tcraw, w.tcm, w.tcpk, w.tckf, w.lzlow,
                   w.side_flag, w.pair_cnt, w.pair_j, w.pair_l, w.flagged, w.n_flagged, w.flag_cnt, w.km_word,
                   w.grey, w.grey_pos,
@@ -251,6 +252,10 @@ cudaError_t alloc_ws(Ctx& c) {
     if ((e = alloc(&w.tcpk, (size_t)w.Kt, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.tckf, (size_t)w.Kt, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.lzlow, (size_t)1, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.tce, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.acut, (size_t)1, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.alist, (size_t)w.Kt, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.nalist, (size_t)1, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.side_flag, (size_t)kChunk, &t)) != cudaSuccess) return e;
     if ((e = cudaMemset(w.side_flag, 0, (size_t)kChunk)) != cudaSuccess) return e;
     if ((e = alloc(&w.pair_cnt, (size_t)kChunk, &t)) != cudaSuccess) return e;
@@ -717,13 +722,38 @@ int fgmm_soft_assign(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64
   cudaError_t e;
   if ((e = launch_prep_simt(c, weights, means, vars, s)) != cudaSuccess) return map_cuda(e);
   const size_t eb = dtype_bytes(x_dtype);
+  // Tensor-core filtered path (split-product modes, 2 to 32 component blocks): sweep 1 on
+  // the tensor cores with every component marks, per point, the 128-component blocks
+  // whose log-densities come within the cut of log Z; the cut is what the exact result
+  // needs (30 nats for log Z and the ranks; -ln(tau) when the threshold reaches further;
+  // fp32's exp underflow, 104 nats, when tau = 0) widened by the expanded form's error
+  // bounds.  The CUDA-core kernel then evaluates exactly, in the direct form, only those
+  // blocks, over the points regrouped by mask.
+  const int nkb = c.ws.Kt / 128;
+  const bool tc = c.tc.ready && c.ws.bmask && nkb >= 2 && nkb <= kSkipMaxBlocks &&
+                  (c.prec == FGMM_PREC_FP16X3 || c.prec == FGMM_PREC_AUTO);
+  if (tc) {
+    const float base = r_threshold > 0.f ? fmaxf(kSkipCut, -logf(r_threshold) + 1.f) : 104.f;
+    if ((e = launch_tc_prep(c, weights, means, vars, false, s, true)) != cudaSuccess ||
+        (e = launch_assign_cut(c, base, s)) != cudaSuccess)
+      return map_cuda(e);
+  }
   for (int64_t c0 = 0; c0 < N; c0 += kChunk) {
     const int64_t nc = (N - c0 < kChunk) ? N - c0 : kChunk;
     const void* Xc = (const char*)X + (size_t)c0 * ldx * eb;
-    if ((e = launch_soft_assign_simt(c, Xc, x_dtype, nc, ldx, top_m, r_threshold,
-                                     ids + c0 * top_m, resp ? resp + c0 * top_m : nullptr, s)) !=
-        cudaSuccess)
+    int32_t* idc = ids + c0 * top_m;
+    float* rc_ = resp ? resp + c0 * top_m : nullptr;
+    if (tc) {
+      if ((e = launch_tc_convert(c, Xc, x_dtype, nc, ldx, nullptr, nullptr, s)) != cudaSuccess ||
+          (e = launch_tc_lse(c, nc, nullptr, nullptr, s, true)) != cudaSuccess ||
+          (e = launch_assign_order(c, nc, s)) != cudaSuccess ||
+          (e = launch_soft_assign_skip(c, Xc, x_dtype, nc, ldx, top_m, r_threshold, idc, rc_, s)) !=
+              cudaSuccess)
+        return map_cuda(e);
+    } else if ((e = launch_soft_assign_simt(c, Xc, x_dtype, nc, ldx, top_m, r_threshold, idc, rc_,
+                                            s)) != cudaSuccess) {
       return map_cuda(e);
+    }
   }
   return FGMM_OK;
 }

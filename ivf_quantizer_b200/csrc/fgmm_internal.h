@@ -62,6 +62,11 @@ constexpr float kSimtSkipCut = 50.f;
 constexpr int kFlushTilesDense = 8;
 constexpr int kFlushTilesSkip = 2;
 constexpr float kMaxAmplification = 450.f;
+// Tensor-core filtered assignment: a component whose expanded-form logit-error bound
+// exceeds this many nats (a collapsed or very tight component far from the centre)
+// leaves the filter and is evaluated exactly for every point instead, so that one such
+// component cannot widen the block-mask cut for all the others.
+constexpr float kAssignMaxE = 0.5f;
 constexpr int kOrdPts = 4096;        // points per CTA of the radix sort
 constexpr int kOrdBuckets = 256;     // values of one 8-bit radix digit
 
@@ -104,6 +109,14 @@ struct Workspace {
   float* tcpk = nullptr;    // [Kt] P_k = log pi_k + log N(mu_k | mu_k, Sigma_k), the peak
   float* tckf = nullptr;    // [Kt] c_k + E_k for stiff components, -inf otherwise
   float* lzlow = nullptr;   // [1] log Z below which a point is always flagged
+  // tensor-core assignment: per-component bound on the expanded-form logit error, and the
+  // block-mask cut it widens (log2 units)
+  float* tce = nullptr;     // [Kt] E_k
+  float* acut = nullptr;    // [1]
+  // components whose bound exceeds kAssignMaxE: left out of the tensor-core filter and
+  // evaluated exactly for every point (ordered, padded to a multiple of 64 with 0)
+  int* alist = nullptr;     // [Kt]
+  int* nalist = nullptr;    // [1]
   uint8_t* side_flag = nullptr;  // [kChunk] 1: the point may have a stiff component within kCut
   // side-path components within kCut of a flagged point, found while merging log Z and
   // reused by the statistics (a count above kSidePairs: the statistics re-evaluate)
@@ -259,8 +272,11 @@ int tc_slices(const Ctx& c);
 // statistics slots the tensor-core statistics sweep may write (block skipping can give a
 // busy block more CTAs than tc_slices); the reduction sums this many
 int tc_stat_slots(const Ctx& c);
+// assign: the assignment's preparation (components whose logit-error bound exceeds
+// kAssignMaxE are marked and listed in ws.alist instead of AUTO's stiffness rules)
 cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* means,
-                           const float* vars, bool auto_mode, cudaStream_t s);
+                           const float* vars, bool auto_mode, cudaStream_t s,
+                           bool assign = false);
 // AUTO side path for stiff components (fgmm_side.cu)
 cudaError_t launch_stiff_compact(const Ctx& c, int* gate, int* mode, cudaStream_t s);
 cudaError_t launch_side_lse(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,
@@ -272,8 +288,19 @@ cudaError_t launch_tc_convert(const Ctx& c, const void* X, int x_dtype, int64_t 
                               const int* perm, const int* mode, cudaStream_t s);
 // block skipping applies to this handle's tensor-core sweeps
 bool tc_skip(const Ctx& c);
+// assign: block masks for the assignment (always kept, with the cut in ws.acut)
 cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* mode,
-                          cudaStream_t s);
+                          cudaStream_t s, bool assign = false);
+// the assignment's block-mask cut from the components' logit-error bounds: base_nats
+// (what the exact evaluation needs within the cut) + 8 max_k E_k + 0.5 nats
+cudaError_t launch_assign_cut(const Ctx& c, float base_nats, cudaStream_t s);
+// block order and 64-row tile masks from ws.bmask (assignment)
+cudaError_t launch_assign_order(const Ctx& c, int64_t n, cudaStream_t s);
+// CUDA-core assignment over the sorted 64-point tiles, visiting only the 128-component
+// blocks of each tile's mask; results written for the original point indices
+cudaError_t launch_soft_assign_skip(const Ctx& c, const void* X, int x_dtype, int64_t n,
+                                    int64_t ldx, int top_m, float r_threshold, int32_t* ids,
+                                    float* resp, cudaStream_t s);
 // block skipping (fgmm_order.cu): sweep-2 order from sweep 1's block masks, phi and
 // log Z rewritten in that order, and the active tiles of every component block
 cudaError_t launch_tc_order(const Ctx& c, const void* X, int x_dtype, int64_t n, int64_t ldx,

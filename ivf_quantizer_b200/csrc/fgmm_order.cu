@@ -275,6 +275,13 @@ cudaError_t launch_tc_order(const Ctx& c, const void* X, int x_dtype, int64_t n,
   return order_lists(c, nkb, (int)n, kTileRows, mode, kModeTensor, s);
 }
 
+cudaError_t launch_assign_order(const Ctx& c, int64_t n, cudaStream_t s) {
+  const int nkb = c.ws.Kt / 128;
+  cudaError_t e;
+  if ((e = order_sort(c, nkb, (int)n, nullptr, 0, s)) != cudaSuccess) return e;
+  return order_lists(c, nkb, (int)n, kTP, nullptr, 0, s);
+}
+
 bool simt_skip(const Ctx& c) {
   // with fewer blocks there is too little to leave out (measured: 2 blocks at D = 960
   // lose 13% to the ordering and the indirect loads)

@@ -84,6 +84,8 @@ __global__ void prep_simt_kernel(int K, int D, int Kp, int Dp, int cov, const fl
 // grow with D (at D = 960 a plain fp32 sum of log-densities near -2700 carries ~5e-3
 // nats of error, enough to move the responsibilities of shared points by 0.5%).
 // rows: nullptr, or the point behind each position i0 + r (block-skipping order).
+// kidx: nullptr, or the components of the tile's columns (column r is component kidx[r];
+// kb is then unused).
 template <int NQ, typename T>
 __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, int64_t ldx, int D,
                                            int Dp, int64_t i0, int kb,
@@ -91,7 +93,8 @@ __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, i
                                            const float* __restrict__ prec,
                                            float (*xs)[kDC + 4], float (*ms)[kDC + 4],
                                            float (*ps)[kDC + 4], float (&acc)[4][NQ],
-                                           const int* __restrict__ rows = nullptr) {
+                                           const int* __restrict__ rows = nullptr,
+                                           const int* __restrict__ kidx = nullptr) {
   constexpr int KBLK = 16 * NQ;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   double dacc[4][NQ];
@@ -115,8 +118,9 @@ __device__ __forceinline__ void logit_tile(const T* __restrict__ X, int64_t n, i
     for (int u = 0; u < MPT; ++u) {
       const int e = threadIdx.x + u * kSimtThreads;
       const int r = e / kDC, cx = e % kDC;
-      mr[u] = mu[(size_t)(kb + r) * Dp + d0 + cx];
-      pr[u] = prec[(size_t)(kb + r) * Dp + d0 + cx];
+      const int kr = kidx ? kidx[r] : kb + r;
+      mr[u] = mu[(size_t)kr * Dp + d0 + cx];
+      pr[u] = prec[(size_t)kr * Dp + d0 + cx];
     }
   };
   fetch(0);
@@ -673,6 +677,110 @@ __global__ void __launch_bounds__(kSimtThreads, 2)
   }
 }
 
+// Assignment over the points regrouped by block mask (tensor-core filtered): one CTA per
+// 64-position tile of the sorted chunk, visiting in increasing order only the
+// 128-component blocks in the tile's mask (the OR of its points' masks, each a superset
+// of the blocks whose log-densities can matter to the point), then the listed
+// components (those left out of the filter, flagged in `listed`; skipped in their
+// blocks).  Same arithmetic as soft_assign_simt_kernel on those components; the results
+// go to the original point index.  The ranking breaks exact ties between a listed and an
+// unlisted component by evaluation order rather than component index.
+template <typename T>
+__global__ void __launch_bounds__(kSimtThreads, 2)
+    soft_assign_skip_kernel(const T* __restrict__ X, int64_t n, int64_t ldx, int D, int Dp,
+                            int Kp, int K, const float* __restrict__ mu,
+                            const float* __restrict__ prec, const float* __restrict__ cconst,
+                            const int* __restrict__ perm, const uint32_t* __restrict__ tmask,
+                            const int* __restrict__ xlist, const int* __restrict__ nxlist,
+                            const int* __restrict__ listed, int top_m, float thr,
+                            int32_t* __restrict__ ids,
+                            float* __restrict__ resp) {
+  __shared__ __align__(16) float xs[kTP][kDC + 4];
+  __shared__ __align__(16) float ms[kKB][kDC + 4];
+  __shared__ __align__(16) float ps[kKB][kDC + 4];
+  __shared__ float ls[kTP][kKB + 1];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int64_t i0 = (int64_t)blockIdx.x * kTP;
+  const uint32_t mask = tmask[blockIdx.x];
+  float tv[FGMM_MAX_TOP_M];
+  int ti[FGMM_MAX_TOP_M];
+  int cnt = 0;
+  float m = -CUDART_INF_F, ssum = 0.f;
+  // the blocks of the mask in increasing order, then the listed components (those the
+  // tensor-core filter leaves out) in 64-column groups
+  const int nx = *nxlist;
+  const int nmask = __popc(mask);
+  const int ngroups = 2 * nmask + (nx + kKB - 1) / kKB;
+  uint32_t rest = mask;
+  int sub = 0;                               // 64-component half of the current block
+  for (int gi = 0; gi < ngroups; ++gi) {
+    int kb, kend;
+    const int* kidx = nullptr;
+    if (gi < 2 * nmask) {
+      const int b = __ffs(rest) - 1;          // next block of the mask, increasing
+      kb = 128 * b + kKB * sub;
+      if (sub) rest &= rest - 1u;
+      sub ^= 1;
+      if (kb >= Kp) continue;                 // uniform: K ends in this block's first half
+      kend = min(kKB, K - kb);
+    } else {
+      kb = kKB * (gi - 2 * nmask);
+      kidx = xlist + kb;
+      kend = min(kKB, nx - kb);
+    }
+    {
+      float acc[4][4];
+      logit_tile<4>(X, n, ldx, D, Dp, i0, kb, mu, prec, xs, ms, ps, acc, perm, kidx);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int cq = tx + 16 * q;
+        // a listed component is evaluated with the list, not again with its block
+        const float cc = kidx ? (cq < kend ? cconst[kidx[cq]] : -CUDART_INF_F)
+                              : (listed[kb + cq] ? -CUDART_INF_F : cconst[kb + cq]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ls[ty + 16 * j][cq] = acc[j][q] + cc;
+      }
+      __syncthreads();
+      if (threadIdx.x < kTP) {
+        const int r = threadIdx.x;
+        for (int c = 0; c < kend; ++c) {
+          const float l = ls[r][c];
+          const float nm = fmaxf(m, l);
+          if (nm > -CUDART_INF_F) {
+            ssum = ssum * expf(m - nm) + expf(l - nm);
+            m = nm;
+          }
+          if (cnt < top_m || l > tv[top_m - 1]) {
+            int p = (cnt < top_m) ? cnt : top_m - 1;
+            while (p > 0 && tv[p - 1] < l) { tv[p] = tv[p - 1]; ti[p] = ti[p - 1]; --p; }
+            tv[p] = l;
+            ti[p] = kidx ? kidx[c] : kb + c;
+            if (cnt < top_m) ++cnt;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  if (threadIdx.x < kTP) {
+    const int64_t i = i0 + threadIdx.x;
+    if (i < n) {
+      const int64_t o = perm[i];
+      const float lz = m + logf(ssum);
+      for (int rnk = 0; rnk < top_m; ++rnk) {
+        int id = -1;
+        float rv = 0.f;
+        if (rnk < cnt) {
+          const float rr = expf(tv[rnk] - lz);
+          if (rnk == 0 || rr > thr) { id = ti[rnk]; rv = rr; }
+        }
+        ids[o * top_m + rnk] = id;
+        if (resp) resp[o * top_m + rnk] = rv;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ AUTO: variance check
 // After the tensor-core sweeps, AUTO checks how much cancellation the variance update
 // S2/N_k - (S1/N_k)^2 suffers.  The statistics are raw moments about the global centre,
@@ -892,6 +1000,24 @@ cudaError_t launch_stats_sum(const double* parts, int n_parts, int64_t len, doub
   const int64_t blocks = (len + 255) / 256;
   stats_sum_kernel<<<(unsigned)(blocks < 1024 ? blocks : 1024), 256, 0, s>>>(parts, n_parts, len,
                                                                              out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_soft_assign_skip(const Ctx& c, const void* X, int x_dtype, int64_t n,
+                                    int64_t ldx, int top_m, float r_threshold, int32_t* ids,
+                                    float* resp, cudaStream_t s) {
+  const Workspace& w = c.ws;
+  const unsigned grid = (unsigned)ceil_div64(n, kTP);
+  prof_begin(c, KI_SOFT_ASSIGN, s);
+  if (x_dtype == FGMM_BF16)
+    soft_assign_skip_kernel<<<grid, kSimtThreads, 0, s>>>(
+        (const __nv_bfloat16*)X, n, ldx, c.D, w.Dp, w.Kp, c.K, w.mu, w.prec, w.cconst, w.perm,
+        w.tmask, w.alist, w.nalist, w.stiff, top_m, r_threshold, ids, resp);
+  else
+    soft_assign_skip_kernel<<<grid, kSimtThreads, 0, s>>>(
+        (const float*)X, n, ldx, c.D, w.Dp, w.Kp, c.K, w.mu, w.prec, w.cconst, w.perm, w.tmask,
+        w.alist, w.nalist, w.stiff, top_m, r_threshold, ids, resp);
+  prof_end(c, KI_SOFT_ASSIGN, s);
   return cudaGetLastError();
 }
 

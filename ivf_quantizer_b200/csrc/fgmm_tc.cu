@@ -152,7 +152,8 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
                                __half* __restrict__ wop, float* __restrict__ ck,
                                float* __restrict__ kscale, int* __restrict__ stiff,
                                float* __restrict__ craw, float* __restrict__ mq,
-                               float* __restrict__ peak, int* __restrict__ grey, int* status) {
+                               float* __restrict__ peak, int* __restrict__ grey,
+                               float* __restrict__ ek, float assign_e, int* status) {
   __shared__ double rs[kSimtThreads], rq[kSimtThreads], rt[kSimtThreads];
   __shared__ float rmax[kSimtThreads], amax[kSimtThreads];
   __shared__ float s_pow;
@@ -208,14 +209,19 @@ __global__ void tc_prep_kernel(int K, int D, int Dq, int Kt, int cov,
       if (wk > 0.f) c = (float)(log((double)wk) - 0.5 * rs[0] - 0.5 * rq[0]);
       const float mx = rmax[0];
       if (mx > 0.f && isfinite(mx)) pw = exp2f(ceilf(log2f(mx)) - 14.f);
+      const float E = (float)ldexp(sqrt(rt[0]), -20);   // bound on the logit error
       if (stiff && wk > 0.f)
-        is_stiff = !(ldexp(sqrt(rt[0]), -20) <= 1e-3) || !(amax[0] <= kMaxAmplification) ||
-                   (nk_prev[k] < 4.0);
+        is_stiff = assign_e > 0.f
+                       ? !(E <= assign_e)   // the assignment: the bound alone decides
+                       : !(E <= 1e-3f) || !(amax[0] <= kMaxAmplification) ||
+                             (nk_prev[k] < 4.0);
       // few points last step: the variance check may fail, so its side-path statistics
       // are taken as well (AUTO; swapped in instead of redoing the pass)
-      if (stiff && wk > 0.f && !is_stiff) is_grey = nk_prev[k] < kGreyNk;
+      if (stiff && wk > 0.f && !is_stiff && !(assign_e > 0.f)) is_grey = nk_prev[k] < kGreyNk;
     }
     craw[k] = c;
+    // the logit-error bound of the components left on the tensor cores (assignment cut)
+    ek[k] = (live_k && w[k] > 0.f && !is_stiff) ? (float)ldexp(sqrt(rt[0]), -20) : 0.f;
     mq[k] = live_k ? (float)rq[0] : 0.f;
     peak[k] = (live_k && w[k] > 0.f) ? (float)(log((double)w[k]) - 0.5 * rs[0]) : -CUDART_INF_F;
     if (stiff) {
@@ -340,6 +346,7 @@ struct LseBars {
   float xf[2][BM];
   uint2 xk[2][BM];      // candidate blocks of column half 1 (block skipping)
   float xo[2][BM];      // their largest block maximum left out of the candidates
+  uint32_t xr[2][BM];   // half 1's running-maximum block mask
 };
 static_assert(sizeof(LseBars) % 16 == 0, "the staged parameters after LseBars are read as float4");
 
@@ -353,7 +360,6 @@ static_assert(sizeof(LseBars) % 16 == 0, "the staged parameters after LseBars ar
 // the true block maximum, so the test against log Z - cut can only keep a block.
 constexpr int kCand = 4;
 constexpr float kCut2 = kSkipCut * kLog2e;       // the cut in log2 units
-constexpr float kQStep = kCut2 / 255.f;
 constexpr uint32_t kCodeEmpty = 0xFFFFu;
 
 // Running state of one row in sweep 1 (log2 units).
@@ -363,10 +369,15 @@ struct RowState {
   float ovm;           // largest block maximum pushed out of the candidate list
   float cbm[kCand];    // candidate blocks: block maximum (-inf: free)
   uint32_t cid;        //                   block index of entry e in bits 8e .. 8e+7
+  // blocks whose maximum was within the cut of the running maximum when seen: the
+  // running maximum only grows, so this holds every block the final test can keep (the
+  // mask of a row whose candidate list overflowed)
+  uint32_t mrun;
   __device__ __forceinline__ void reset() {
     m = fm = ovm = -CUDART_INF_F;
     s = 0.f;
     cid = 0;
+    mrun = 0;
 #pragma unroll
     for (int e = 0; e < kCand; ++e) cbm[e] = -CUDART_INF_F;
   }
@@ -383,9 +394,14 @@ __global__ void __launch_bounds__(kLseThreads, 1)
                   float* __restrict__ logz_out,
                   const __half* __restrict__ xop, const float* __restrict__ ckf,
                   const float* __restrict__ lzlow, uint8_t* __restrict__ side_flag,
-                  uint32_t* __restrict__ bmask, const int* mode, int* status) {
+                  uint32_t* __restrict__ bmask, const float* __restrict__ cutp, const int* mode,
+                  int* status) {
   if (mode && *mode != kModeTensor) return;
   constexpr int SWL = lse_ring(NKC);
+  // block-mask cut (log2 units) and the step of its 8-bit codes: the EM sweep's, or the
+  // assignment's, widened by the logit-error bounds
+  const float cut2 = cutp ? *cutp : kCut2;
+  const float qstep = cut2 * (1.f / 255.f);
   constexpr int NP = SPLIT ? 2 : 1;                   // W' boxes per chunk (hi, lo)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -670,11 +686,12 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             S.m = nm;
           }
           if (bmask) {
-            const float thr = S.m - kCut2;
+            const float thr = S.m - cut2;
 #pragma unroll
             for (int e = 0; e < kCand; ++e)
               if (S.cbm[e] <= thr) S.cbm[e] = -CUDART_INF_F;
             if (bm > thr) {
+              S.mrun |= 1u << kb;
               int slot = -1, mi = 0;
               float mn = CUDART_INF_F;
 #pragma unroll
@@ -722,13 +739,14 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             for (int e = 0; e < kCand; ++e) {
               code[e] = kCodeEmpty;
               const float dl = S.m - S.cbm[e];   // < cut for a live entry (else below the cut)
-              if (S.cbm[e] > -CUDART_INF_F && dl < kCut2) {
-                const int qd = min(254, (int)floorf(dl * (1.f / kQStep)));
+              if (S.cbm[e] > -CUDART_INF_F && dl < cut2) {
+                const int qd = min(254, (int)floorf(dl / qstep));
                 code[e] = (S.block(e) << 8) | (uint32_t)qd;
               }
             }
             bars->xk[t][r] = make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
             bars->xo[t][r] = S.ovm;
+            bars->xr[t][r] = S.mrun;
           }
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&bars->xc_full[t]);
@@ -742,9 +760,11 @@ __global__ void __launch_bounds__(kLseThreads, 1)
           const float f2 = fmaxf(S.fm, bars->xf[t][r]);
           uint2 kq = make_uint2(0u, 0u);
           float ov = S.ovm;
+          uint32_t mr = S.mrun;
           if (bmask) {
             kq = bars->xk[t][r];
             ov = fmaxf(ov, bars->xo[t][r]);
+            mr |= bars->xr[t][r];
           }
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&bars->xc_empty[t]);
@@ -760,9 +780,9 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             // may a stiff component come within kSideCut nats of log Z here?
             side_flag[i] = (f2 > lz2 - kSideCut * kLog2e) || !(lz >= *lzlow);
             if (bmask) {
-              const float lim = lz2 - kCut2;
+              const float lim = lz2 - cut2;
               uint32_t mk = 0;
-              bool dense = ov > lim || !(lz2 > -CUDART_INF_F);
+              const bool dense = ov > lim;
 #pragma unroll
               for (int e = 0; e < kCand; ++e)
                 if (S.cbm[e] > lim) mk |= 1u << S.block(e);
@@ -770,10 +790,12 @@ __global__ void __launch_bounds__(kLseThreads, 1)
 #pragma unroll
               for (int e = 0; e < kCand; ++e) {
                 const uint32_t cd = (w2[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-                if (cd != kCodeEmpty && m1 - (float)(cd & 255u) * kQStep > lim)
+                if (cd != kCodeEmpty && m1 - (float)(cd & 255u) * qstep > lim)
                   mk |= 1u << (cd >> 8);
               }
-              bmask[i] = dense ? (nkb >= 32 ? 0xFFFFFFFFu : (1u << nkb) - 1u) : mk;
+              // a candidate list overflowed: the running-maximum mask (a superset)
+              const uint32_t all = nkb >= 32 ? 0xFFFFFFFFu : (1u << nkb) - 1u;
+              bmask[i] = !(lz2 > -CUDART_INF_F) ? all : (dense ? (mr | mk) : mk);
             }
           }
         }
@@ -1324,8 +1346,38 @@ cudaError_t tc_init(Ctx& c) {
   return cudaSuccess;
 }
 
+// One CTA: the marked components in increasing order, padded with component 0 to a
+// multiple of 64 (the exact assignment reads 64 list entries at a time).
+__global__ void assign_list_kernel(const int* __restrict__ stiff, int K, int* __restrict__ list,
+                                   int* __restrict__ nlist) {
+  __shared__ int wsum[32];
+  __shared__ int base;
+  if (threadIdx.x == 0) base = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int k0 = 0; k0 < K; k0 += blockDim.x) {
+    const int k = k0 + (int)threadIdx.x;
+    const bool f = k < K && stiff[k];
+    const unsigned ball = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) wsum[warp] = __popc(ball);
+    __syncthreads();
+    int before = 0, tot = 0;
+    for (int w2 = 0; w2 < nw; ++w2) {
+      before += w2 < warp ? wsum[w2] : 0;
+      tot += wsum[w2];
+    }
+    if (f) list[base + before + __popc(ball & ((1u << lane) - 1u))] = k;
+    __syncthreads();
+    if (threadIdx.x == 0) base += tot;
+    __syncthreads();
+  }
+  const int n = base;
+  for (int j = n + (int)threadIdx.x; j < (n + 63) / 64 * 64; j += blockDim.x) list[j] = 0;
+  if (threadIdx.x == 0) *nlist = n;
+}
+
 cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* means,
-                           const float* vars, bool auto_mode, cudaStream_t s) {
+                           const float* vars, bool auto_mode, cudaStream_t s, bool assign) {
   const Workspace& w = c.ws;
   prof_begin(c, KI_TC_CENTER, s);
   tc_center_kernel<<<c.D, kSimtThreads, 0, s>>>(c.K, c.D, c.cov, weights, means, vars, w.center,
@@ -1334,16 +1386,21 @@ cudaError_t launch_tc_prep(const Ctx& c, const float* weights, const float* mean
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (w.Dq > c.D) cudaMemsetAsync(w.center + c.D, 0, (w.Dq - c.D) * sizeof(float), s);
-  if (!auto_mode) {
+  const bool mark = auto_mode || assign;
+  if (!mark) {
     cudaMemsetAsync(w.stiff, 0, w.Kt * sizeof(int), s);
     cudaMemsetAsync(w.grey, 0, w.Kt * sizeof(int), s);
   }
   prof_begin(c, KI_TC_PREP, s);
   tc_prep_kernel<<<w.Kt, kSimtThreads, 0, s>>>(c.K, c.D, w.Dq, w.Kt, c.cov, weights, means, vars,
                                                w.center, w.dscale, w.nk, w.wop, w.tck, w.tks,
-                                               auto_mode ? w.stiff : nullptr, w.tcraw, w.tcm,
-                                               w.tcpk, w.grey, w.status);
+                                               mark ? w.stiff : nullptr, w.tcraw, w.tcm,
+                                               w.tcpk, w.grey, w.tce,
+                                               assign ? kAssignMaxE : -1.f, w.status);
   prof_end(c, KI_TC_PREP, s);
+  if (assign) {
+    assign_list_kernel<<<1, 1024, 0, s>>>(w.stiff, c.K, w.alist, w.nalist);
+  }
   return cudaGetLastError();
 }
 
@@ -1369,13 +1426,37 @@ cudaError_t launch_tc_convert(const Ctx& c, const void* X, int x_dtype, int64_t 
   return cudaGetLastError();
 }
 
+// One CTA: cut2 = (base + 8 max_k E_k + 0.5) log2(e); a non-finite bound gives an
+// unbounded cut (every block marked: the exact evaluation then visits all of them).
+__global__ void assign_cut_kernel(const float* __restrict__ ek, int Kt, float base,
+                                  float* __restrict__ cut2) {
+  __shared__ float red[kSimtThreads];
+  float m = 0.f;
+  for (int k = threadIdx.x; k < Kt; k += blockDim.x) m = fmaxf(m, isfinite(ek[k]) ? ek[k] : CUDART_INF_F);
+  red[threadIdx.x] = m;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] = fmaxf(red[threadIdx.x], red[threadIdx.x + w]);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const float c = (base + 8.f * red[0] + 0.5f) * kLog2e;
+    *cut2 = isfinite(c) ? c : 1e30f;
+  }
+}
+
+cudaError_t launch_assign_cut(const Ctx& c, float base_nats, cudaStream_t s) {
+  assign_cut_kernel<<<1, kSimtThreads, 0, s>>>(c.ws.tce, c.ws.Kt, base_nats, c.ws.acut);
+  return cudaGetLastError();
+}
+
 bool tc_skip(const Ctx& c) {
   const int nkb = c.ws.Kt / BKc;
   return c.skip && c.tc.ready && c.ws.bmask && nkb >= 2 && nkb <= kSkipMaxBlocks;
 }
 
 cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* mode,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool assign) {
   const Workspace& w = c.ws;
   const int nkc = w.K1 / 64;
   const int npairs = (int)ceil_div64(ceil_div64(n, BM), 2);   // sweep 1 works on tile pairs
@@ -1385,17 +1466,19 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
   const bool params = lse_smem(nkc, w.Kt, true) <= kMaxDynSmem;
   const size_t smem = lse_smem(nkc, w.Kt, params);
   const bool split = c.prec != FGMM_PREC_FP16;
+  uint32_t* bm = (assign || tc_skip(c)) ? w.bmask : nullptr;
+  const float* cutp = assign ? w.acut : nullptr;
   prof_begin(c, KI_TC_LSE, s, mode, kModeTensor);
 #define LSE_CASE(N_)                                                                          \
   case N_:                                                                                    \
     if (split)                                                                                \
       tc_lse_kernel<N_, true><<<grid, kLseThreads, smem, s>>>(                                \
           tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, w.tks, params ? 1 : 0, w.logz, logz_out,   \
-          w.xop, w.tckf, w.lzlow, w.side_flag, tc_skip(c) ? w.bmask : nullptr, mode, w.status); \
+          w.xop, w.tckf, w.lzlow, w.side_flag, bm, cutp, mode, w.status);                      \
     else                                                                                      \
       tc_lse_kernel<N_, false><<<grid, kLseThreads, smem, s>>>(                               \
           tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, w.tks, params ? 1 : 0, w.logz, logz_out,   \
-          w.xop, w.tckf, w.lzlow, w.side_flag, tc_skip(c) ? w.bmask : nullptr, mode, w.status); \
+          w.xop, w.tckf, w.lzlow, w.side_flag, bm, cutp, mode, w.status);                      \
     break;
   switch (nkc) {
     LSE_CASE(1)
