@@ -403,6 +403,7 @@ __global__ void __launch_bounds__(kLseThreads, 1)
   const float cut2 = cutp ? *cutp : kCut2;
   const float qstep = cut2 * (1.f / 255.f);
   constexpr int NP = SPLIT ? 2 : 1;                   // W' boxes per chunk (hi, lo)
+  constexpr int NSL = SWL / NP;                       // W' ring slots (one K-chunk each)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   unsigned char* xbuf = base;                         // [2][NKC][BOX]: phi hi of the pair
@@ -483,16 +484,17 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             ptx::tma_load_2d(xbuf + (t * NKC + c) * BOX, &tmx, &bars->x_full[t][c], c * KC,
                              (tA + t) * BM);
           }
+        // one ring slot = the NP boxes (hi, lo) of one K-chunk under one barrier
         for (int kb = 0; kb < nkb; ++kb)
-          for (int ci = 0; ci < NKC; ++ci)
-            for (int part = 0; part < NP; ++part, ++itw) {
-              const int s = itw % SWL;
-              if (itw >= SWL && !ptx::mbar_wait(&bars->w_empty[s], ((itw / SWL) - 1) & 1, abort))
-                goto fail_p;
-              ptx::mbar_arrive_expect_tx(&bars->w_full[s], BOX);
-              ptx::tma_load_2d(wring + s * BOX, &tmw, &bars->w_full[s], lg_chunk<NKC>(ci) * KC,
-                               part * Kt + kb * BKc);
-            }
+          for (int ci = 0; ci < NKC; ++ci, ++itw) {
+            const int s = itw % NSL;
+            if (itw >= NSL && !ptx::mbar_wait(&bars->w_empty[s], ((itw / NSL) - 1) & 1, abort))
+              goto fail_p;
+            ptx::mbar_arrive_expect_tx(&bars->w_full[s], NP * BOX);
+            for (int part = 0; part < NP; ++part)
+              ptx::tma_load_2d(wring + (s * NP + part) * BOX, &tmw, &bars->w_full[s],
+                               lg_chunk<NKC>(ci) * KC, part * Kt + kb * BKc);
+          }
       }
       goto done_p;
     fail_p:
@@ -502,8 +504,8 @@ __global__ void __launch_bounds__(kLseThreads, 1)
       if (*abort) {  // let every copy this thread started land before the CTA exits
         for (int t = 0; t < (last_b ? 2 : 1) && x_issued > 0; ++t)
           for (int c = 0; c < NKC; ++c) ptx::mbar_drain(&bars->x_full[t][c], (x_issued - 1) & 1);
-        for (uint32_t k = (itw > SWL ? itw - SWL : 0); k < itw; ++k)
-          ptx::mbar_drain(&bars->w_full[k % SWL], (k / SWL) & 1);
+        for (uint32_t k = (itw > NSL ? itw - NSL : 0); k < itw; ++k)
+          ptx::mbar_drain(&bars->w_full[k % NSL], (k / NSL) & 1);
       }
     }
   } else if (warp == 1) {
@@ -517,29 +519,25 @@ __global__ void __launch_bounds__(kLseThreads, 1)
           const uint32_t u = (uint32_t)(j * nkb + kb);   // use of each S buffer
           for (int ci = 0; ci < NKC; ++ci) {
             const int c = lg_chunk<NKC>(ci);
-            const int sh = itw % SWL;
-            if (!ptx::mbar_wait(&bars->w_full[sh], (itw / SWL) & 1, abort)) goto fail_m;
+            const int sw = itw % NSL;
+            if (!ptx::mbar_wait(&bars->w_full[sw], (itw / NSL) & 1, abort)) goto fail_m;
             ++itw;
-            int sl = sh;
-            if constexpr (SPLIT) {
-              sl = itw % SWL;
-              if (!ptx::mbar_wait(&bars->w_full[sl], (itw / SWL) & 1, abort)) goto fail_m;
-              ++itw;
-            }
+            const int sh = sw * NP, sl = sw * NP + NP - 1;
             // K-major 128 B-swizzled boxes: one descriptor per box, + 2 (32 bytes) per K-step
             constexpr uint64_t kHiK = ptx::sw128_hi(16, 1024);
             const uint64_t bh0 = ptx::sw128_desc(ptx::smem_u32(wring + sh * BOX), kHiK);
             const uint64_t bl0 = ptx::sw128_desc(ptx::smem_u32(wring + sl * BOX), kHiK);
             for (int t = 0; t < nt; ++t) {
               if (ci == 0) {
-                // S_t free (its previous block read out), phi lo of this pair in place; the
-                // epilogue warps' TMEM accesses before their arrivals are ordered ahead of
-                // these products by the fence (TMA arrivals need none: the async proxy
-                // completes its writes before the barrier phase does)
+                // S_t free (its previous block read out), phi lo of this pair in place.  The
+                // epilogue warps arrive only after tcgen05.wait::ld / wait::st returned, i.e.
+                // once their TMEM reads and writes are complete, and these products are
+                // issued only after the arrival is observed.  No tcgen05 fence here: in the
+                // issuing thread an after_thread_sync fence idles the tensor pipe for several
+                // hundred cycles (the queue of issued products is short), measured on B200
                 if (u >= 1 && !ptx::mbar_wait(&bars->s_empty[t], (u - 1) & 1, abort)) goto fail_m;
                 if (SPLIT && kb == 0 && !ptx::mbar_wait(&bars->xlo_ready[t], j & 1, abort))
                   goto fail_m;
-                ptx::tc_fence_after();
               }
               if (kb == 0 && !ptx::mbar_wait(&bars->x_full[t][c], j & 1, abort)) goto fail_m;
               const uint32_t d_tmem = tmem + t * 128;
@@ -558,8 +556,7 @@ __global__ void __launch_bounds__(kLseThreads, 1)
               if (kb == nkb - 1) ptx::mma_commit(&bars->x_empty[t][c]);
               if (ci == NKC - 1) ptx::mma_commit(&bars->s_full[t]);
             }
-            ptx::mma_commit(&bars->w_empty[sh]);
-            if constexpr (SPLIT) ptx::mma_commit(&bars->w_empty[sl]);
+            ptx::mma_commit(&bars->w_empty[sw]);
           }
         }
       }
