@@ -144,6 +144,10 @@ void prof_begin(const Ctx& c, KernelId, cudaStream_t s, const int* gate, int req
 void prof_gates_changed(const Ctx& c) {
   if (c.prof) c.prof->gate_snap.clear();
 }
+void prof_extra_launch(const Ctx& c) {
+  if (c.prof) ++c.prof->launches;
+}
+
 void prof_end(const Ctx& c, KernelId k, cudaStream_t s) {
   Profiler* p = c.prof;
   if (!p || !p->enabled || !p->pending) return;
@@ -170,7 +174,7 @@ void free_ws(Workspace& w) {
                   w.stats,  w.nk,     w.status, w.center, w.dscale, w.wop,
                   w.tck,    w.tks,    w.xop,    w.mode, w.stiff,    w.stiff_list, w.n_stiff,
                   w.tce,    w.acut,   w.alist,  w.nalist,
-                  w.side_part, w.mode2, w.canon, w.tcraw, w.tcm, w.tcpk, w.tckf, w.lzlow,
+                  w.side_part, w.mode2, w.canon, w.tcraw, w.tcm, w.tcpk, w.tckf, w.lzlow, w.lpart, w.lpartf,
                   w.side_flag, w.pair_cnt, w.pair_j, w.pair_l, w.flagged, w.n_flagged, w.flag_cnt, w.km_word,
                   w.grey, w.grey_pos,
                   w.grey_stats,
@@ -252,6 +256,8 @@ cudaError_t alloc_ws(Ctx& c) {
     if ((e = alloc(&w.tcpk, (size_t)w.Kt, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.tckf, (size_t)w.Kt, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.lzlow, (size_t)1, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.lpart, (size_t)(w.Kt / 128) * kChunk, &t)) != cudaSuccess) return e;
+    if ((e = alloc(&w.lpartf, (size_t)(w.Kt / 128) * kChunk, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.tce, (size_t)w.Kt, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.acut, (size_t)1, &t)) != cudaSuccess) return e;
     if ((e = alloc(&w.alist, (size_t)w.Kt, &t)) != cudaSuccess) return e;

@@ -109,6 +109,10 @@ struct Workspace {
   float* tcpk = nullptr;    // [Kt] P_k = log pi_k + log N(mu_k | mu_k, Sigma_k), the peak
   float* tckf = nullptr;    // [Kt] c_k + E_k for stiff components, -inf otherwise
   float* lzlow = nullptr;   // [1] log Z below which a point is always flagged
+  // sweep 1: per (component block, point) the block's (max, sum of 2^(l - max)) of the
+  // log2-scaled log-densities and the stiff filter's maximum, merged into log Z after it
+  float2* lpart = nullptr;  // [Kt / 128][kChunk]
+  float* lpartf = nullptr;  // [Kt / 128][kChunk]
   // tensor-core assignment: per-component bound on the expanded-form logit error, and the
   // block-mask cut it widens (log2 units)
   float* tce = nullptr;     // [Kt] E_k
@@ -215,6 +219,8 @@ constexpr int kModeSimt = 1;
 void prof_begin(const Ctx& c, KernelId k, cudaStream_t s, const int* gate = nullptr,
                 int required = 0);
 void prof_end(const Ctx& c, KernelId k, cudaStream_t s);
+// A further kernel launched inside the current profiled region (counted, timed with it).
+void prof_extra_launch(const Ctx& c);
 // A kernel that may write a gate word has been enqueued: launches after it take new
 // snapshots of their gate (until then, launches behind one gate share a snapshot).
 void prof_gates_changed(const Ctx& c);

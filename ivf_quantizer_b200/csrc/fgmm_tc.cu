@@ -308,192 +308,143 @@ __global__ void tc_convert_kernel(const T* __restrict__ X, int64_t n, int64_t ld
 }
 
 // ------------------------------------------------------------------ sweep 1 (log Z)
-// 384 threads: warp 0 TMA producer, warp 1 MMA issuer, warps 4..11 epilogue.  A CTA works
-// on pairs of 128-point tiles (A = 2p, B = 2p + 1): every W' box that the TMA brings in
-// feeds the products of both tiles, so each byte streamed from L2 serves 256 points (the
-// W' stream of a 128-point tile would need about as many L2 bytes per clock as the
-// products it feeds can take).  The two epilogue warpgroups split each 128-column S tile
-// in halves (columns 64h .. 64h+63), one row of A and the same row of B per thread, and
-// keep a running (max, sum) per row, the 64 columns' maxima and sums as four independent
-// partial chains; at the end of the pair half 1 hands its values to half 0 through shared
-// memory, which writes log Z.  Two epilogue warps per scheduler (not four) leave the
-// single MMA-issuing thread the issue slots it needs to keep the tensor pipe fed.
-// phi hi of both tiles sits in shared memory (A operand of two products); phi lo sits in
-// tensor memory (A operand of the third), written there by the epilogue warps as soon as
-// the previous pair's last products on that tile have completed.  TMEM: S_A, S_B (one
-// 128-column buffer each; the MMA warp refills S_A while the epilogue drains S_B and the
-// other way round), phi lo of A and B.
+// Grid (component block b, point slice).  CTA (b, slice) keeps the W' rows of its 128
+// components resident in shared memory (the hi box of every K-chunk and, with the split,
+// the lo boxes) and streams the phi boxes of its slice's 128-point tiles through a TMA
+// ring; S = phi W'^T of tile j goes to TMEM buffer j mod 3, so the epilogue of a tile
+// overlaps the products of the next two and no tile waits for another's epilogue.  The
+// nkb CTAs of one slice read the same tiles in the same order: after the first, the phi
+// boxes come from L2.  With the split, three products per K-step (phi hi W' hi + phi hi
+// W' lo + phi lo W' hi), each with both operands in shared memory.
+// 640 threads: warp 0 TMA producer, warp 1 MMA issuer, warps 4..19 epilogue.  Epilogue
+// warpgroup g reads columns 32g .. 32g+31 of a tile, one row (point) per thread, and
+// reduces them to (max, sum of 2^(l - max)) in log2 units, plus the maximum of the stiff
+// components' estimate + error bound; warpgroups 1..3 hand theirs to warpgroup 0 through
+// tensor memory (the warps of one lane quarter share its lanes; shared memory is left to
+// the phi ring), and warpgroup 0 writes the block's partial of each point.  lse_merge_kernel then
+// combines the nkb partials of a point into log Z, the side-path flag and the block mask
+// (exactly the blocks whose largest log-density lies within the cut of log Z).
 constexpr int kEpiWarps = 8;                        // statistics sweep
 constexpr int kTcThreads = 128 + 32 * kEpiWarps;
-constexpr int kLseEpiWarps = 8;                     // log-sum-exp sweep
+constexpr int kLseEpiWarps = 16;                    // log-sum-exp sweep
 constexpr int kLseThreads = 128 + 32 * kLseEpiWarps;
-constexpr int kLseRingMax = 8;
-// W' ring stages of sweep 1: as many boxes as fit beside the pair's phi hi (an even
-// number: the hi and lo box of a chunk are used together)
-__host__ __device__ constexpr int lse_ring(int nkc) { return nkc >= 4 ? 4 : (nkc == 3 ? 6 : 8); }
+constexpr int kLseSBuf = 3;                         // S buffers in TMEM (3 x 128 columns)
+constexpr int kLseXcCol = 128 * kLseSBuf;           // TMEM columns of the quarters' hand-over
+constexpr int kLseRingMax = 16;
+constexpr int kLsePrefetch = 4;                     // tiles of L2 prefetch ahead (block 0)
+constexpr int kSmemMax = 232448;                    // 227 KB of dynamic shared memory
+constexpr float kCut2 = kSkipCut * kLog2e;          // the block-skipping cut in log2 units
 
 struct LseBars {
-  uint64_t x_full[2][4], x_empty[2][4];   // [tile of the pair][chunk]
-  uint64_t xlo_ready[2];
-  uint64_t w_full[kLseRingMax], w_empty[kLseRingMax];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t w_full;
+  uint64_t x_full[kLseRingMax], x_empty[kLseRingMax];
+  uint64_t s_full[kLseSBuf], s_empty[kLseSBuf];
   uint64_t xc_full[2], xc_empty[2];
   uint64_t drain;
   uint32_t tmem;
   int abort;
-  float xm[2][BM];      // (max, sum, filter max) of column half 1, per tile of the pair
-  float xs[2][BM];
-  float xf[2][BM];
-  uint2 xk[2][BM];      // candidate blocks of column half 1 (block skipping)
-  float xo[2][BM];      // their largest block maximum left out of the candidates
-  uint32_t xr[2][BM];   // half 1's running-maximum block mask
+  alignas(16) float ckl[BKc];   // the block's c_k log2(e)
+  float ksl[BKc];               //             2^t_k log2(e)
+  float cfl[BKc];               //             (c_k + E_k) log2(e) if stiff, else -inf
 };
-static_assert(sizeof(LseBars) % 16 == 0, "the staged parameters after LseBars are read as float4");
+static_assert(offsetof(LseBars, ckl) % 16 == 0, "the staged parameters are read as float4");
 
-// Block skipping, sweep 1 side.  Every epilogue thread keeps, for its row and its 64
-// columns, the (at most kCand) largest block maxima that lie within the cut of its
-// running maximum; a block that falls out of range can never come back, the maximum
-// only grows.  A block pushed out of a full list leaves its maximum in `ovm`; if that
-// is within the cut of log Z in the end, the row is marked dense (every block).  At the
-// end of a tile column half 1 hands its candidates to half 0 as 16-bit codes
-// (block << 8 | q, q = floor((max - block max) / step)); decoding gives max - q step >=
-// the true block maximum, so the test against log Z - cut can only keep a block.
-constexpr int kCand = 4;
-constexpr float kCut2 = kSkipCut * kLog2e;       // the cut in log2 units
-constexpr uint32_t kCodeEmpty = 0xFFFFu;
-
-// Running state of one row in sweep 1 (log2 units).
-struct RowState {
-  float m, s;          // running max and sum
-  float fm;            // max over stiff components of estimate + error bound
-  float ovm;           // largest block maximum pushed out of the candidate list
-  float cbm[kCand];    // candidate blocks: block maximum (-inf: free)
-  uint32_t cid;        //                   block index of entry e in bits 8e .. 8e+7
-  // blocks whose maximum was within the cut of the running maximum when seen: the
-  // running maximum only grows, so this holds every block the final test can keep (the
-  // mask of a row whose candidate list overflowed)
-  uint32_t mrun;
-  __device__ __forceinline__ void reset() {
-    m = fm = ovm = -CUDART_INF_F;
-    s = 0.f;
-    cid = 0;
-    mrun = 0;
-#pragma unroll
-    for (int e = 0; e < kCand; ++e) cbm[e] = -CUDART_INF_F;
-  }
-  __device__ __forceinline__ uint32_t block(int e) const { return (cid >> (8 * e)) & 255u; }
-};
+// phi boxes in the ring: what shared memory the resident W' block leaves
+__host__ __device__ constexpr int lse_ring(int nkc, bool split) {
+  return ((kSmemMax - 1024 - (int)sizeof(LseBars)) / BOX - (split ? 2 : 1) * nkc) < kLseRingMax
+             ? ((kSmemMax - 1024 - (int)sizeof(LseBars)) / BOX - (split ? 2 : 1) * nkc)
+             : kLseRingMax;
+}
 
 // SPLIT: the three-product fp16 hi/lo split (FGMM_PREC_FP16X3 and AUTO); false: one fp16
-// product per term (FGMM_PREC_FP16: no W' lo boxes, no phi lo)
+// product per term (FGMM_PREC_FP16: no W' lo, no phi lo)
 template <int NKC, bool SPLIT>
 __global__ void __launch_bounds__(kLseThreads, 1)
     tc_lse_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
-                  int nc, int ncmax, int Kt, const float* __restrict__ ck,
-                  const float* __restrict__ kscale, int params_in_smem, float* __restrict__ logz,
-                  float* __restrict__ logz_out,
-                  const __half* __restrict__ xop, const float* __restrict__ ckf,
-                  const float* __restrict__ lzlow, uint8_t* __restrict__ side_flag,
-                  uint32_t* __restrict__ bmask, const float* __restrict__ cutp, const int* mode,
-                  int* status) {
+                  int nc, int ncmax, int Kt, int slice_len, const float* __restrict__ ck,
+                  const float* __restrict__ kscale, const float* __restrict__ ckf,
+                  const __half* __restrict__ xop, float2* __restrict__ part,
+                  float* __restrict__ partf, const int* mode, int* status) {
   if (mode && *mode != kModeTensor) return;
-  constexpr int SWL = lse_ring(NKC);
-  // block-mask cut (log2 units) and the step of its 8-bit codes: the EM sweep's, or the
-  // assignment's, widened by the logit-error bounds
-  const float cut2 = cutp ? *cutp : kCut2;
-  const float qstep = cut2 * (1.f / 255.f);
-  constexpr int NP = SPLIT ? 2 : 1;                   // W' boxes per chunk (hi, lo)
-  constexpr int NSL = SWL / NP;                       // W' ring slots (one K-chunk each)
+  constexpr int NP = SPLIT ? 2 : 1;                   // boxes per K-chunk (hi, lo)
+  constexpr int RING = lse_ring(NKC, SPLIT);
+  static_assert(RING >= 2 * NP, "the phi ring must hold two K-chunks");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  unsigned char* xbuf = base;                         // [2][NKC][BOX]: phi hi of the pair
-  unsigned char* wring = base + 2 * NKC * BOX;        // [SWL][BOX]
-  LseBars* bars = reinterpret_cast<LseBars*>(wring + SWL * BOX);
-  float* ckl = reinterpret_cast<float*>(bars + 1);    // [Kt] c_k log2(e)   (if staged)
-  float* ksl = ckl + Kt;                              // [Kt] 2^t_k log2(e) (if staged)
-  float* cfl = ksl + Kt;                              // [Kt] (c_k + E_k) log2(e) (if staged)
+  unsigned char* wbuf = base;                         // [NP][NKC][BOX]: W' hi boxes, lo boxes
+  unsigned char* xring = base + NP * NKC * BOX;       // [RING][BOX]
+  LseBars* bars = reinterpret_cast<LseBars*>(xring + RING * BOX);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntiles = (nc + BM - 1) / BM;
-  const int npairs = (ntiles + 1) / 2;
-  const int nkb = Kt / BKc;
-  const int G = (int)gridDim.x;
+  const int kb = blockIdx.x;
+  const int p0 = blockIdx.y * slice_len;
+  const int p1 = min(nc, p0 + slice_len);
+  const int ntl = p1 > p0 ? (p1 - p0 + BM - 1) / BM : 0;
+  if (ntl == 0) return;  // uniform over the CTA, before any barrier or TMEM use
 
   if (threadIdx.x == 0) {
-    for (int t = 0; t < 2; ++t)
-      for (int c = 0; c < 4; ++c) {
-        ptx::mbar_init(&bars->x_full[t][c], 1);
-        ptx::mbar_init(&bars->x_empty[t][c], 1);
-      }
-    for (int s = 0; s < SWL; ++s) { ptx::mbar_init(&bars->w_full[s], 1); ptx::mbar_init(&bars->w_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) {
+    ptx::mbar_init(&bars->w_full, 1);
+    for (int s = 0; s < RING; ++s) { ptx::mbar_init(&bars->x_full[s], 1); ptx::mbar_init(&bars->x_empty[s], 1); }
+    for (int b = 0; b < kLseSBuf; ++b) {
       ptx::mbar_init(&bars->s_full[b], 1);
       ptx::mbar_init(&bars->s_empty[b], kLseEpiWarps);
-      ptx::mbar_init(&bars->xlo_ready[b], kLseEpiWarps);
-      ptx::mbar_init(&bars->xc_full[b], kLseEpiWarps / 2);
-      ptx::mbar_init(&bars->xc_empty[b], kLseEpiWarps / 2);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&bars->xc_full[b], 3 * kLseEpiWarps / 4);
+      ptx::mbar_init(&bars->xc_empty[b], kLseEpiWarps / 4);
     }
     ptx::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
-  if (params_in_smem)
-    for (int k = threadIdx.x; k < Kt; k += blockDim.x) {
-      ckl[k] = ck[k] * kLog2e;
-      ksl[k] = kscale[k] * kLog2e;
-      cfl[k] = ckf[k] * kLog2e;
-    }
+  int any_f = 0;
+  for (int k = threadIdx.x; k < BKc; k += blockDim.x) {
+    const int kk = kb * BKc + k;
+    bars->ckl[k] = ck[kk] * kLog2e;
+    bars->ksl[k] = kscale[kk] * kLog2e;
+    const float f = ckf ? ckf[kk] * kLog2e : -CUDART_INF_F;
+    bars->cfl[k] = f;
+    any_f |= f > -CUDART_INF_F;
+  }
   if (warp == 1) {
     ptx::tmem_alloc(&bars->tmem, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  // a block without stiff components needs no filter maximum (uniform over the CTA)
+  const bool has_f = __syncthreads_or(any_f) != 0;
   ptx::tc_fence_after();
-  // TMEM columns: [128 t, 128 t + 128) S of tile t of the pair; [256 + 128 t, ...) phi lo
-  // of tile t (two fp16 per column, 2 Dq / 2 = NKC * 32 columns)
-  const uint32_t tmem = bars->tmem;
-  const uint32_t xlo_tmem = tmem + 256;
+  const uint32_t tmem = bars->tmem;                   // S buffer b: columns 128 b .. 128 b + 127
 
   if (warp == 0) {
     if (lane == 0) {
       ptx::prefetch_tmap(&tmx);
       ptx::prefetch_tmap(&tmw);
-      uint32_t itw = 0;
-      int j = 0, x_issued = 0;
-      bool last_b = false;
-      for (int p = blockIdx.x; p < npairs && !*abort; p += G, ++j) {
-        const int tA = 2 * p;
-        const bool hasB = tA + 1 < ntiles;
-        // phi lo rows that the epilogue warps read with plain loads at the end of this
-        // pair (those of the next pair): start moving them into L2 now
-        const int pn = p + G;
-        if (SPLIT && pn < npairs) {
-          const int ntl = min(2, ntiles - 2 * pn);
-          ptx::bulk_prefetch_l2(xop + ((size_t)ncmax + (size_t)2 * pn * BM) * (NKC * 64),
-                                (uint32_t)ntl * BM * NKC * 128);
+      ptx::mbar_arrive_expect_tx(&bars->w_full, NP * NKC * BOX);
+      for (int part_ = 0; part_ < NP; ++part_)
+        for (int c = 0; c < NKC; ++c)
+          ptx::tma_load_2d(wbuf + (part_ * NKC + c) * BOX, &tmw, &bars->w_full, c * KC,
+                           part_ * Kt + kb * BKc);
+      uint32_t itx = 0;
+      for (int j = 0; j < ntl && !*abort; ++j) {
+        const int row0 = p0 + j * BM;
+        // the block-0 CTA of the slice moves the phi rows of tile j + kLsePrefetch from
+        // DRAM into L2, so that the slice's nkb CTAs find them there
+        if (kb == 0 && j + kLsePrefetch < ntl) {
+          const size_t r = (size_t)(row0 + kLsePrefetch * BM);
+          for (int part_ = 0; part_ < NP; ++part_)
+            ptx::bulk_prefetch_l2(xop + ((size_t)part_ * ncmax + r) * (NKC * 64),
+                                  (uint32_t)BM * NKC * 128);
         }
-        x_issued = j + 1;
-        last_b = hasB;
-        for (int t = 0; t < (hasB ? 2 : 1); ++t)
-          for (int ci = 0; ci < NKC; ++ci) {
-            const int c = lg_chunk<NKC>(ci);
-            if (j > 0 && !ptx::mbar_wait(&bars->x_empty[t][c], (j - 1) & 1, abort)) goto fail_p;
-            ptx::mbar_arrive_expect_tx(&bars->x_full[t][c], BOX);
-            ptx::tma_load_2d(xbuf + (t * NKC + c) * BOX, &tmx, &bars->x_full[t][c], c * KC,
-                             (tA + t) * BM);
-          }
-        // one ring slot = the NP boxes (hi, lo) of one K-chunk under one barrier
-        for (int kb = 0; kb < nkb; ++kb)
-          for (int ci = 0; ci < NKC; ++ci, ++itw) {
-            const int s = itw % NSL;
-            if (itw >= NSL && !ptx::mbar_wait(&bars->w_empty[s], ((itw / NSL) - 1) & 1, abort))
+        for (int ci = 0; ci < NKC; ++ci)
+          for (int part_ = 0; part_ < NP; ++part_, ++itx) {
+            const int s = itx % RING;
+            if (itx >= RING && !ptx::mbar_wait(&bars->x_empty[s], ((itx / RING) - 1) & 1, abort))
               goto fail_p;
-            ptx::mbar_arrive_expect_tx(&bars->w_full[s], NP * BOX);
-            for (int part = 0; part < NP; ++part)
-              ptx::tma_load_2d(wring + (s * NP + part) * BOX, &tmw, &bars->w_full[s],
-                               lg_chunk<NKC>(ci) * KC, part * Kt + kb * BKc);
+            ptx::mbar_arrive_expect_tx(&bars->x_full[s], BOX);
+            ptx::tma_load_2d(xring + s * BOX, &tmx, &bars->x_full[s], lg_chunk<NKC>(ci) * KC,
+                             part_ * ncmax + row0);
           }
       }
       goto done_p;
@@ -502,63 +453,56 @@ __global__ void __launch_bounds__(kLseThreads, 1)
       bars->abort = 1;
     done_p:
       if (*abort) {  // let every copy this thread started land before the CTA exits
-        for (int t = 0; t < (last_b ? 2 : 1) && x_issued > 0; ++t)
-          for (int c = 0; c < NKC; ++c) ptx::mbar_drain(&bars->x_full[t][c], (x_issued - 1) & 1);
-        for (uint32_t k = (itw > NSL ? itw - NSL : 0); k < itw; ++k)
-          ptx::mbar_drain(&bars->w_full[k % NSL], (k / NSL) & 1);
+        ptx::mbar_drain(&bars->w_full, 0);
+        for (uint32_t k = (itx > RING ? itx - RING : 0); k < itx; ++k)
+          ptx::mbar_drain(&bars->x_full[k % RING], (k / RING) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = ptx::idesc_f16(128, 128, false, false);
-      uint32_t itw = 0;
-      int j = 0;
-      for (int p = blockIdx.x; p < npairs && !*abort; p += G, ++j) {
-        const int nt = (2 * p + 1 < ntiles) ? 2 : 1;
-        for (int kb = 0; kb < nkb; ++kb) {
-          const uint32_t u = (uint32_t)(j * nkb + kb);   // use of each S buffer
-          for (int ci = 0; ci < NKC; ++ci) {
-            const int c = lg_chunk<NKC>(ci);
-            const int sw = itw % NSL;
-            if (!ptx::mbar_wait(&bars->w_full[sw], (itw / NSL) & 1, abort)) goto fail_m;
-            ++itw;
-            const int sh = sw * NP, sl = sw * NP + NP - 1;
-            // K-major 128 B-swizzled boxes: one descriptor per box, + 2 (32 bytes) per K-step
-            constexpr uint64_t kHiK = ptx::sw128_hi(16, 1024);
-            const uint64_t bh0 = ptx::sw128_desc(ptx::smem_u32(wring + sh * BOX), kHiK);
-            const uint64_t bl0 = ptx::sw128_desc(ptx::smem_u32(wring + sl * BOX), kHiK);
-            for (int t = 0; t < nt; ++t) {
-              if (ci == 0) {
-                // S_t free (its previous block read out), phi lo of this pair in place.  The
-                // epilogue warps arrive only after tcgen05.wait::ld / wait::st returned, i.e.
-                // once their TMEM reads and writes are complete, and these products are
-                // issued only after the arrival is observed.  No tcgen05 fence here: in the
-                // issuing thread an after_thread_sync fence idles the tensor pipe for several
-                // hundred cycles (the queue of issued products is short), measured on B200
-                if (u >= 1 && !ptx::mbar_wait(&bars->s_empty[t], (u - 1) & 1, abort)) goto fail_m;
-                if (SPLIT && kb == 0 && !ptx::mbar_wait(&bars->xlo_ready[t], j & 1, abort))
-                  goto fail_m;
-              }
-              if (kb == 0 && !ptx::mbar_wait(&bars->x_full[t][c], j & 1, abort)) goto fail_m;
-              const uint32_t d_tmem = tmem + t * 128;
-              // phi lo from TMEM: K elements c*64 + ks*16 .. +15 = columns c*32 + ks*8 .. +7
-              const uint32_t xl_tmem = xlo_tmem + t * 128 + c * 32;
-              const uint64_t ah0 = ptx::sw128_desc(ptx::smem_u32(xbuf + (t * NKC + c) * BOX), kHiK);
-#pragma unroll
-              for (int ks = 0; ks < KC / 16; ++ks) {
-                const uint64_t dk = (uint64_t)(2 * ks);
-                ptx::mma_f16_ss(d_tmem, ah0 + dk, bh0 + dk, idesc, (ci > 0 || ks > 0) ? 1u : 0u);
-                if constexpr (SPLIT) {
-                  ptx::mma_f16_ss(d_tmem, ah0 + dk, bl0 + dk, idesc, 1u);
-                  ptx::mma_f16_ts(d_tmem, xl_tmem + ks * 8, bh0 + dk, idesc, 1u);
-                }
-              }
-              if (kb == nkb - 1) ptx::mma_commit(&bars->x_empty[t][c]);
-              if (ci == NKC - 1) ptx::mma_commit(&bars->s_full[t]);
-            }
-            ptx::mma_commit(&bars->w_empty[sw]);
+      constexpr uint64_t kHiK = ptx::sw128_hi(16, 1024);
+      uint32_t itx = 0;
+      if (!ptx::mbar_wait(&bars->w_full, 0, abort)) goto fail_m;
+      for (int j = 0; j < ntl && !*abort; ++j) {
+        const int b = j % kLseSBuf;
+        const uint32_t use = (uint32_t)(j / kLseSBuf);
+        // S_b free: the epilogue arrives only after tcgen05.wait::ld returned, i.e. once
+        // its reads of S_b are complete, and these products are issued after the arrival
+        // is observed.  No tcgen05 fence here: in the issuing thread an after_thread_sync
+        // fence idles the tensor pipe for several hundred cycles (the queue of issued
+        // products is short), measured on B200
+        if (use >= 1 && !ptx::mbar_wait(&bars->s_empty[b], (use - 1) & 1, abort)) goto fail_m;
+        const uint32_t d_tmem = tmem + b * 128;
+        for (int ci = 0; ci < NKC; ++ci) {
+          const int c = lg_chunk<NKC>(ci);
+          const int sh = itx % RING;
+          if (!ptx::mbar_wait(&bars->x_full[sh], (itx / RING) & 1, abort)) goto fail_m;
+          ++itx;
+          int sl = sh;
+          if constexpr (SPLIT) {
+            sl = itx % RING;
+            if (!ptx::mbar_wait(&bars->x_full[sl], (itx / RING) & 1, abort)) goto fail_m;
+            ++itx;
           }
+          // K-major 128 B-swizzled boxes: one descriptor per box, + 2 (32 bytes) per K-step
+          const uint64_t ah0 = ptx::sw128_desc(ptx::smem_u32(xring + sh * BOX), kHiK);
+          const uint64_t al0 = ptx::sw128_desc(ptx::smem_u32(xring + sl * BOX), kHiK);
+          const uint64_t bh0 = ptx::sw128_desc(ptx::smem_u32(wbuf + c * BOX), kHiK);
+          const uint64_t bl0 = ptx::sw128_desc(ptx::smem_u32(wbuf + (NKC + c) * BOX), kHiK);
+#pragma unroll
+          for (int ks = 0; ks < KC / 16; ++ks) {
+            const uint64_t dk = (uint64_t)(2 * ks);
+            ptx::mma_f16_ss(d_tmem, ah0 + dk, bh0 + dk, idesc, (ci > 0 || ks > 0) ? 1u : 0u);
+            if constexpr (SPLIT) {
+              ptx::mma_f16_ss(d_tmem, ah0 + dk, bl0 + dk, idesc, 1u);
+              ptx::mma_f16_ss(d_tmem, al0 + dk, bh0 + dk, idesc, 1u);
+            }
+          }
+          ptx::mma_commit(&bars->x_empty[sh]);
+          if constexpr (SPLIT) ptx::mma_commit(&bars->x_empty[sl]);
         }
+        ptx::mma_commit(&bars->s_full[b]);
       }
       goto done_m;
     fail_m:
@@ -571,230 +515,121 @@ __global__ void __launch_bounds__(kLseThreads, 1)
       }
     }
   } else if (warp >= 4) {
-    const int h = (warp - 4) >> 2;         // column half of the S tile (64 columns)
+    const int g = (warp - 4) >> 2;         // column quarter of the S tile
     const int q = warp & 3;                // TMEM lane quarter
     const int r = q * 32 + lane;           // row of the tile = TMEM lane
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    // phi lo of `tile` into TMEM buffer t: this thread's row, K elements
-    // h*NKC*32 .. +NKC*32-1 = columns h*NKC*16 .. +NKC*16-1 (row tile*BM + r < ncmax)
-    auto put_xlo = [&](int tile, int t) {
-      const uint4* src = reinterpret_cast<const uint4*>(
-          xop + ((size_t)ncmax + (size_t)tile * BM + r) * (NKC * 64) + h * (NKC * 32));
-#pragma unroll
-      for (int c8 = 0; c8 < 2 * NKC; ++c8) {   // 8 columns = 16 fp16 per store
-        const uint4 v0 = __ldg(src + 2 * c8), v1 = __ldg(src + 2 * c8 + 1);
-        const uint32_t r8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        ptx::tmem_st8(xlo_tmem + t * 128 + lane_base + h * (NKC * 16) + c8 * 8, r8);
+    const float* ckg = bars->ckl + 32 * g;
+    const float* ksg = bars->ksl + 32 * g;
+    const float* cfg = bars->cfl + 32 * g;
+    for (int j = 0; j < ntl && !*abort; ++j) {
+      const int b = j % kLseSBuf;
+      const uint32_t use = (uint32_t)(j / kLseSBuf);
+      if (!ptx::mbar_wait_warp(&bars->s_full[b], use & 1, abort)) {
+        set_status(status, FGMM_ERR_TIMEOUT);
+        bars->abort = 1;
+        break;
       }
-      ptx::tmem_wait_st();
+      ptx::tc_fence_after();
+      uint32_t u[32];
+      ptx::tmem_ld32(tmem + lane_base + b * 128 + 32 * g, u);
+      ptx::tmem_wait_ld();
+      // the values are in registers: hand S_b back to the MMA warp now
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&bars->xlo_ready[t]);
-    };
-    if (SPLIT && (int)blockIdx.x < npairs) {
-      put_xlo(2 * blockIdx.x, 0);
-      if (2 * (int)blockIdx.x + 1 < ntiles) put_xlo(2 * blockIdx.x + 1, 1);
-    }
-    int j = 0;
-    for (int p = blockIdx.x; p < npairs && !*abort; p += G, ++j) {
-      const int nt = (2 * p + 1 < ntiles) ? 2 : 1;
-      const int pn = p + G;
-      RowState st[2];
-      st[0].reset();
-      st[1].reset();
-      for (int kb = 0; kb < nkb && !*abort; ++kb) {
-        const uint32_t u = (uint32_t)(j * nkb + kb);
+      if (lane == 0) ptx::mbar_arrive(&bars->s_empty[b]);
+      // log2-scaled log-densities of the 32 columns, two per packed fp32x2 operation;
+      // the maxima and sums run as four independent partial chains
+      uint64_t v2[16];
+      float mx[4], fx[4];
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (t >= nt) break;
-          RowState& S = st[t];
-          if (!ptx::mbar_wait_warp(&bars->s_full[t], u & 1, abort)) {
-            set_status(status, FGMM_ERR_TIMEOUT);
-            bars->abort = 1;
-            break;
-          }
-          ptx::tc_fence_after();
-          const int col = 64 * h;            // first column within the 128-component block
-          uint32_t ua[32], ub[32];
-          ptx::tmem_ld32(tmem + lane_base + t * 128 + col, ua);
-          ptx::tmem_ld32(tmem + lane_base + t * 128 + col + 32, ub);
-          ptx::tmem_wait_ld();
-          // the values are in registers: hand S_t back to the MMA warp now
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&bars->s_empty[t]);
-          // log2-scaled log-densities of the 64 columns, two per packed fp32x2 operation;
-          // the maxima and sums run as four independent partial chains
-          uint64_t v2[32];
-          float bmx[4], fmx[4];
+      for (int z = 0; z < 4; ++z) mx[z] = fx[z] = -CUDART_INF_F;
 #pragma unroll
-          for (int z = 0; z < 4; ++z) bmx[z] = fmx[z] = -CUDART_INF_F;
-          const int k0 = kb * BKc + col;
-#pragma unroll
-          for (int e4 = 0; e4 < 16; ++e4) {
-            float4 cc, kk, cf;
-            if (params_in_smem) {
-              cc = *reinterpret_cast<const float4*>(ckl + k0 + 4 * e4);
-              kk = *reinterpret_cast<const float4*>(ksl + k0 + 4 * e4);
-              cf = *reinterpret_cast<const float4*>(cfl + k0 + 4 * e4);
-            } else {
-              cc = __ldg(reinterpret_cast<const float4*>(ck + k0) + e4);
-              kk = __ldg(reinterpret_cast<const float4*>(kscale + k0) + e4);
-              cf = __ldg(reinterpret_cast<const float4*>(ckf + k0) + e4);
-              cc.x *= kLog2e; cc.y *= kLog2e; cc.z *= kLog2e; cc.w *= kLog2e;
-              kk.x *= kLog2e; kk.y *= kLog2e; kk.z *= kLog2e; kk.w *= kLog2e;
-              cf.x *= kLog2e; cf.y *= kLog2e; cf.z *= kLog2e; cf.w *= kLog2e;
-            }
-            const uint32_t* uv = e4 < 8 ? ua : ub;
-            const int o4 = 4 * (e4 & 7);
-            const uint64_t f01 = ptx::f2_pack(__uint_as_float(uv[o4 + 0]), __uint_as_float(uv[o4 + 1]));
-            const uint64_t f23 = ptx::f2_pack(__uint_as_float(uv[o4 + 2]), __uint_as_float(uv[o4 + 3]));
-            const uint64_t k01 = ptx::f2_pack(kk.x, kk.y), k23 = ptx::f2_pack(kk.z, kk.w);
-            v2[2 * e4 + 0] = ptx::f2_fma(f01, k01, ptx::f2_pack(cc.x, cc.y));
-            v2[2 * e4 + 1] = ptx::f2_fma(f23, k23, ptx::f2_pack(cc.z, cc.w));
-            // stiff components (c_k = -inf above): estimate + error bound, for the filter
-            float g[4], v[4];
-            ptx::f2_unpack(ptx::f2_fma(f01, k01, ptx::f2_pack(cf.x, cf.y)), g[0], g[1]);
-            ptx::f2_unpack(ptx::f2_fma(f23, k23, ptx::f2_pack(cf.z, cf.w)), g[2], g[3]);
-            ptx::f2_unpack(v2[2 * e4 + 0], v[0], v[1]);
-            ptx::f2_unpack(v2[2 * e4 + 1], v[2], v[3]);
-            fmx[e4 & 3] = fmaxf(fmx[e4 & 3], fmaxf(fmaxf(g[0], g[1]), fmaxf(g[2], g[3])));
-            bmx[e4 & 3] = fmaxf(bmx[e4 & 3], fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
-          }
-          S.fm = fmaxf(S.fm, fmaxf(fmaxf(fmx[0], fmx[1]), fmaxf(fmx[2], fmx[3])));
-          const float bm = fmaxf(fmaxf(bmx[0], bmx[1]), fmaxf(bmx[2], bmx[3]));
-          const float nm = fmaxf(S.m, bm);
-          if (nm > -CUDART_INF_F) {
-            // every argument is <= 0 after the shift, so 2^x in (0, 1]; the SFU's exp2
-            // (flushing results below 2^-126, far under fp32 resolution of the sum)
-            const uint64_t shift = ptx::f2_pack(-nm, -nm);
-            uint64_t acc[4];
-#pragma unroll
-            for (int z = 0; z < 4; ++z) acc[z] = ptx::f2_pack(0.f, 0.f);
-#pragma unroll
-            for (int e2 = 0; e2 < 32; ++e2) {
-              float t0, t1;
-              ptx::f2_unpack(ptx::f2_add(v2[e2], shift), t0, t1);
-              acc[e2 & 3] = ptx::f2_add(acc[e2 & 3], ptx::f2_pack(ptx::ex2(t0), ptx::ex2(t1)));
-            }
-            float a0, a1;
-            ptx::f2_unpack(ptx::f2_add(ptx::f2_add(acc[0], acc[1]), ptx::f2_add(acc[2], acc[3])), a0, a1);
-            S.s = S.s * ptx::ex2(S.m - nm) + (a0 + a1);
-            S.m = nm;
-          }
-          if (bmask) {
-            const float thr = S.m - cut2;
-#pragma unroll
-            for (int e = 0; e < kCand; ++e)
-              if (S.cbm[e] <= thr) S.cbm[e] = -CUDART_INF_F;
-            if (bm > thr) {
-              S.mrun |= 1u << kb;
-              int slot = -1, mi = 0;
-              float mn = CUDART_INF_F;
-#pragma unroll
-              for (int e = 0; e < kCand; ++e) {
-                if (slot < 0 && S.cbm[e] == -CUDART_INF_F) slot = e;
-                if (S.cbm[e] < mn) { mn = S.cbm[e]; mi = e; }
-              }
-              if (slot < 0) {            // full: the smaller of bm and the list's least goes
-                if (bm > mn) { S.ovm = fmaxf(S.ovm, mn); slot = mi; }
-                else S.ovm = fmaxf(S.ovm, bm);
-              }
-#pragma unroll
-              for (int e = 0; e < kCand; ++e)
-                if (e == slot) {
-                  S.cbm[e] = bm;
-                  S.cid = (S.cid & ~(255u << (8 * e))) | ((uint32_t)kb << (8 * e));
-                }
-            }
-          }
-          // after the pair's last block on tile t every product reading phi lo of t has
-          // completed (S_t's last commit covers them): the next pair's phi lo of that tile
-          // goes in while the tensor cores finish the other tile
-          if (SPLIT && kb == nkb - 1 && pn < npairs && 2 * pn + t < ntiles) put_xlo(2 * pn + t, t);
+      for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 cc = *reinterpret_cast<const float4*>(ckg + 4 * e4);
+        const float4 kk = *reinterpret_cast<const float4*>(ksg + 4 * e4);
+        const uint64_t f01 = ptx::f2_pack(__uint_as_float(u[4 * e4 + 0]), __uint_as_float(u[4 * e4 + 1]));
+        const uint64_t f23 = ptx::f2_pack(__uint_as_float(u[4 * e4 + 2]), __uint_as_float(u[4 * e4 + 3]));
+        const uint64_t k01 = ptx::f2_pack(kk.x, kk.y), k23 = ptx::f2_pack(kk.z, kk.w);
+        v2[2 * e4 + 0] = ptx::f2_fma(f01, k01, ptx::f2_pack(cc.x, cc.y));
+        v2[2 * e4 + 1] = ptx::f2_fma(f23, k23, ptx::f2_pack(cc.z, cc.w));
+        float v[4];
+        ptx::f2_unpack(v2[2 * e4 + 0], v[0], v[1]);
+        ptx::f2_unpack(v2[2 * e4 + 1], v[2], v[3]);
+        mx[e4 & 3] = fmaxf(mx[e4 & 3], fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
+        if (has_f) {
+          // stiff components (c_k = -inf above): estimate + error bound, for the filter
+          const float4 cf = *reinterpret_cast<const float4*>(cfg + 4 * e4);
+          float h[4];
+          ptx::f2_unpack(ptx::f2_fma(f01, k01, ptx::f2_pack(cf.x, cf.y)), h[0], h[1]);
+          ptx::f2_unpack(ptx::f2_fma(f23, k23, ptx::f2_pack(cf.z, cf.w)), h[2], h[3]);
+          fx[e4 & 3] = fmaxf(fx[e4 & 3], fmaxf(fmaxf(h[0], h[1]), fmaxf(h[2], h[3])));
         }
       }
-      if (*abort) break;
-      // combine the two column halves of each row, per tile of the pair
+      const float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float fm = fmaxf(fmaxf(fx[0], fx[1]), fmaxf(fx[2], fx[3]));
+      float s = 0.f;
+      if (m > -CUDART_INF_F) {
+        // every argument is <= 0 after the shift, so 2^x in (0, 1]; the SFU's exp2
+        // (flushing results below 2^-126, far under fp32 resolution of the sum)
+        const uint64_t shift = ptx::f2_pack(-m, -m);
+        uint64_t acc[4];
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (t >= nt) break;
-        const RowState& S = st[t];
-        if (h == 1) {
-          if (j >= 1 &&
-              !ptx::mbar_wait_warp(&bars->xc_empty[t], (j - 1) & 1, abort)) {
-            set_status(status, FGMM_ERR_TIMEOUT);
-            bars->abort = 1;
-            break;
-          }
-          bars->xm[t][r] = S.m;
-          bars->xs[t][r] = S.s;
-          bars->xf[t][r] = S.fm;
-          if (bmask) {
-            uint32_t code[kCand];
+        for (int z = 0; z < 4; ++z) acc[z] = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < kCand; ++e) {
-              code[e] = kCodeEmpty;
-              const float dl = S.m - S.cbm[e];   // < cut for a live entry (else below the cut)
-              if (S.cbm[e] > -CUDART_INF_F && dl < cut2) {
-                const int qd = min(254, (int)floorf(dl / qstep));
-                code[e] = (S.block(e) << 8) | (uint32_t)qd;
-              }
-            }
-            bars->xk[t][r] = make_uint2(code[0] | (code[1] << 16), code[2] | (code[3] << 16));
-            bars->xo[t][r] = S.ovm;
-            bars->xr[t][r] = S.mrun;
-          }
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&bars->xc_full[t]);
-        } else {
-          if (!ptx::mbar_wait_warp(&bars->xc_full[t], j & 1, abort)) {
-            set_status(status, FGMM_ERR_TIMEOUT);
-            bars->abort = 1;
-            break;
-          }
-          const float m1 = bars->xm[t][r], s1 = bars->xs[t][r];
-          const float f2 = fmaxf(S.fm, bars->xf[t][r]);
-          uint2 kq = make_uint2(0u, 0u);
-          float ov = S.ovm;
-          uint32_t mr = S.mrun;
-          if (bmask) {
-            kq = bars->xk[t][r];
-            ov = fmaxf(ov, bars->xo[t][r]);
-            mr |= bars->xr[t][r];
-          }
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&bars->xc_empty[t]);
-          const float M = fmaxf(S.m, m1);
-          float Ssum = 0.f;
-          if (M > -CUDART_INF_F) Ssum = S.s * exp2f(S.m - M) + s1 * exp2f(m1 - M);
-          const int i = (2 * p + t) * BM + r;
-          const float lz2 = M + log2f(Ssum);
-          const float lz = lz2 / kLog2e;
-          if (i < nc) {
-            logz[i] = lz;
-            if (logz_out) logz_out[i] = lz;
-            // may a stiff component come within kSideCut nats of log Z here?
-            side_flag[i] = (f2 > lz2 - kSideCut * kLog2e) || !(lz >= *lzlow);
-            if (bmask) {
-              const float lim = lz2 - cut2;
-              uint32_t mk = 0;
-              const bool dense = ov > lim;
+        for (int e2 = 0; e2 < 16; ++e2) {
+          float t0, t1;
+          ptx::f2_unpack(ptx::f2_add(v2[e2], shift), t0, t1);
+          acc[e2 & 3] = ptx::f2_add(acc[e2 & 3], ptx::f2_pack(ptx::ex2(t0), ptx::ex2(t1)));
+        }
+        float a0, a1;
+        ptx::f2_unpack(ptx::f2_add(ptx::f2_add(acc[0], acc[1]), ptx::f2_add(acc[2], acc[3])), a0, a1);
+        s = a0 + a1;
+      }
+      // the four column quarters of the row: quarters 1..3 hand theirs to quarter 0, in
+      // TMEM columns kLseXcCol + 16 xb + 4 (g - 1) .. +2 of the row's lane
+      const int xb = j & 1;
+      const uint32_t xc_tmem = tmem + lane_base + kLseXcCol + 16 * xb;
+      if (g != 0) {
+        if (j >= 2 && !ptx::mbar_wait_warp(&bars->xc_empty[xb], ((j >> 1) - 1) & 1, abort)) {
+          set_status(status, FGMM_ERR_TIMEOUT);
+          bars->abort = 1;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t w4[4] = {__float_as_uint(m), __float_as_uint(s), __float_as_uint(fm), 0u};
+        ptx::tmem_st4(xc_tmem + 4 * (g - 1), w4);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->xc_full[xb]);
+      } else {
+        if (!ptx::mbar_wait_warp(&bars->xc_full[xb], (j >> 1) & 1, abort)) {
+          set_status(status, FGMM_ERR_TIMEOUT);
+          bars->abort = 1;
+          break;
+        }
+        ptx::tc_fence_after();
+        uint32_t x16[16];
+        ptx::tmem_ld16(xc_tmem, x16);
+        ptx::tmem_wait_ld();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->xc_empty[xb]);
+        const float mq[4] = {m, __uint_as_float(x16[0]), __uint_as_float(x16[4]), __uint_as_float(x16[8])};
+        const float sq[4] = {s, __uint_as_float(x16[1]), __uint_as_float(x16[5]), __uint_as_float(x16[9])};
+        const float F = fmaxf(fmaxf(fm, __uint_as_float(x16[2])),
+                              fmaxf(__uint_as_float(x16[6]), __uint_as_float(x16[10])));
+        const float M = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        float S = 0.f;
+        if (M > -CUDART_INF_F) {
 #pragma unroll
-              for (int e = 0; e < kCand; ++e)
-                if (S.cbm[e] > lim) mk |= 1u << S.block(e);
-              const uint32_t w2[2] = {kq.x, kq.y};
-#pragma unroll
-              for (int e = 0; e < kCand; ++e) {
-                const uint32_t cd = (w2[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-                if (cd != kCodeEmpty && m1 - (float)(cd & 255u) * qstep > lim)
-                  mk |= 1u << (cd >> 8);
-              }
-              // a candidate list overflowed: the running-maximum mask (a superset)
-              const uint32_t all = nkb >= 32 ? 0xFFFFFFFFu : (1u << nkb) - 1u;
-              bmask[i] = !(lz2 > -CUDART_INF_F) ? all : (dense ? (mr | mk) : mk);
-            }
-          }
+          for (int z = 0; z < 4; ++z) S += sq[z] * ptx::ex2(mq[z] - M);
+        }
+        const int i = p0 + j * BM + r;
+        if (i < p1) {
+          part[(size_t)kb * ncmax + i] = make_float2(M, S);
+          partf[(size_t)kb * ncmax + i] = F;
         }
       }
     }
@@ -804,6 +639,45 @@ __global__ void __launch_bounds__(kLseThreads, 1)
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+// One thread per point: log Z from the nkb partials (m_b, s_b) of sweep 1 (log2 units),
+// log2 Z = M + log2 sum_b s_b 2^(m_b - M) with M = max_b m_b; the side-path flag (a stiff
+// component's estimate plus error bound within kSideCut nats of log Z, or log Z below
+// the bound the side path relies on); and the block mask: the blocks whose largest
+// log-density lies within the cut of log Z (every block when log Z is -inf).
+__global__ void __launch_bounds__(256)
+    lse_merge_kernel(const float2* __restrict__ part, const float* __restrict__ partf, int nc,
+                     int ncmax, int nkb, float* __restrict__ logz, float* __restrict__ logz_out,
+                     const float* __restrict__ lzlow, uint8_t* __restrict__ side_flag,
+                     uint32_t* __restrict__ bmask, const float* __restrict__ cutp, const int* mode) {
+  if (mode && *mode != kModeTensor) return;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= nc) return;
+  float M = -CUDART_INF_F, F = -CUDART_INF_F;
+  for (int b = 0; b < nkb; ++b) {
+    M = fmaxf(M, part[(size_t)b * ncmax + i].x);
+    F = fmaxf(F, partf[(size_t)b * ncmax + i]);
+  }
+  float S = 0.f;
+  if (M > -CUDART_INF_F)
+    for (int b = 0; b < nkb; ++b) {
+      const float2 v = part[(size_t)b * ncmax + i];
+      if (v.x > -CUDART_INF_F) S += v.y * exp2f(v.x - M);
+    }
+  const float lz2 = M + log2f(S);
+  const float lz = lz2 / kLog2e;
+  logz[i] = lz;
+  if (logz_out) logz_out[i] = lz;
+  side_flag[i] = (F > lz2 - kSideCut * kLog2e) || !(lz >= *lzlow);
+  if (bmask) {
+    const float lim = lz2 - (cutp ? *cutp : kCut2);
+    uint32_t mk = 0;
+    for (int b = 0; b < nkb; ++b)
+      if (part[(size_t)b * ncmax + i].x > lim) mk |= 1u << b;
+    const uint32_t all = nkb >= 32 ? 0xFFFFFFFFu : (1u << nkb) - 1u;
+    bmask[i] = !(lz2 > -CUDART_INF_F) ? all : mk;
   }
 }
 
@@ -1298,17 +1172,19 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows) {
   return r == CUDA_SUCCESS;
 }
 
-size_t lse_smem(int nkc, int Kt, bool params) {
-  return 1024 + (size_t)(2 * nkc + lse_ring(nkc)) * BOX + sizeof(LseBars) +
-         (params ? 3 * (size_t)Kt * sizeof(float) : 0);
+size_t lse_smem(int nkc, bool split) {
+  return 1024 + (size_t)((split ? 2 : 1) * nkc + lse_ring(nkc, split)) * BOX + sizeof(LseBars);
 }
-constexpr size_t kMaxDynSmem = 232448;  // 227 KB per block on sm_100
+constexpr size_t kMaxDynSmem = kSmemMax;
 size_t stats_smem(int nkc) { return 1024 + (size_t)(nkc + SX + 2) * BOX + sizeof(StatBars); }
 
 template <int NKC, bool SPLIT>
 cudaError_t set_attrs_split() {
+  static_assert(1024 + ((SPLIT ? 2 : 1) * NKC + lse_ring(NKC, SPLIT)) * BOX + sizeof(LseBars) <=
+                    (size_t)kSmemMax, "sweep 1 exceeds the shared memory of a block");
   cudaError_t e = cudaFuncSetAttribute(tc_lse_kernel<NKC, SPLIT>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxDynSmem);
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)lse_smem(NKC, SPLIT));
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(tc_stats_kernel<NKC, SPLIT>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)stats_smem(NKC));
@@ -1456,26 +1332,30 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
                           cudaStream_t s, bool assign) {
   const Workspace& w = c.ws;
   const int nkc = w.K1 / 64;
-  const int npairs = (int)ceil_div64(ceil_div64(n, BM), 2);   // sweep 1 works on tile pairs
-  const int grid = npairs < c.num_sms ? npairs : c.num_sms;
+  const int nkb = w.Kt / BKc;
+  // grid (component block, point slice), as many slices as fill the SMs once
+  int S = c.num_sms / nkb;
+  if (S < 1) S = 1;
+  const int slice = (int)ceil_div64(ceil_div64(n, S), BM) * BM;
+  const dim3 grid(nkb, S);
   const CUtensorMap& tx = c.tc.tmap_x;
   const CUtensorMap& tw = c.tc.tmap_w;
-  const bool params = lse_smem(nkc, w.Kt, true) <= kMaxDynSmem;
-  const size_t smem = lse_smem(nkc, w.Kt, params);
   const bool split = c.prec != FGMM_PREC_FP16;
+  const size_t smem = lse_smem(nkc, split);
   uint32_t* bm = (assign || tc_skip(c)) ? w.bmask : nullptr;
   const float* cutp = assign ? w.acut : nullptr;
+  const float* ckf = assign ? nullptr : w.tckf;   // the assignment has no side path
   prof_begin(c, KI_TC_LSE, s, mode, kModeTensor);
 #define LSE_CASE(N_)                                                                          \
   case N_:                                                                                    \
     if (split)                                                                                \
       tc_lse_kernel<N_, true><<<grid, kLseThreads, smem, s>>>(                                \
-          tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, w.tks, params ? 1 : 0, w.logz, logz_out,   \
-          w.xop, w.tckf, w.lzlow, w.side_flag, bm, cutp, mode, w.status);                      \
+          tx, tw, (int)n, (int)kChunk, w.Kt, slice, w.tck, w.tks, ckf, w.xop, w.lpart,       \
+          w.lpartf, mode, w.status);                                                          \
     else                                                                                      \
       tc_lse_kernel<N_, false><<<grid, kLseThreads, smem, s>>>(                               \
-          tx, tw, (int)n, (int)kChunk, w.Kt, w.tck, w.tks, params ? 1 : 0, w.logz, logz_out,   \
-          w.xop, w.tckf, w.lzlow, w.side_flag, bm, cutp, mode, w.status);                      \
+          tx, tw, (int)n, (int)kChunk, w.Kt, slice, w.tck, w.tks, ckf, w.xop, w.lpart,       \
+          w.lpartf, mode, w.status);                                                          \
     break;
   switch (nkc) {
     LSE_CASE(1)
@@ -1484,6 +1364,11 @@ cudaError_t launch_tc_lse(const Ctx& c, int64_t n, float* logz_out, const int* m
     LSE_CASE(4)
   }
 #undef LSE_CASE
+  // the merge of the blocks' partials: a second launch inside the same profiled region
+  prof_extra_launch(c);
+  lse_merge_kernel<<<(unsigned)ceil_div64(n, 256), 256, 0, s>>>(
+      w.lpart, w.lpartf, (int)n, (int)kChunk, nkb, w.logz, logz_out, w.lzlow, w.side_flag, bm,
+      cutp, mode);
   prof_end(c, KI_TC_LSE, s);
   return cudaGetLastError();
 }
