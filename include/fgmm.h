@@ -75,7 +75,8 @@ enum fgmm_status {
   FGMM_ERR_CUDA = 3,        /* a CUDA runtime call failed */
   FGMM_ERR_OOM = 4,         /* workspace allocation failed */
   FGMM_ERR_NUMERIC = 5,     /* non-finite log-likelihood, or every component empty */
-  FGMM_ERR_TIMEOUT = 6      /* a bounded device-side wait expired */
+  FGMM_ERR_TIMEOUT = 6,     /* a bounded device-side wait expired */
+  FGMM_ERR_IO = 7           /* a reader of X (file or callback) failed */
 };
 
 /* Largest top_m accepted by fgmm_soft_assign. */
@@ -182,6 +183,37 @@ int fgmm_em_step_host(fgmm_handle h, const void* X_host, int x_dtype, int64_t N,
                       float* weights, float* means, float* vars, double* loglik_out,
                       float* logz_out, fgmm_stream_t stream);
 
+/* Reader of X for the streamed steps below: fill dst (pinned host memory owned by the
+ * handle) with rows row0 .. row0 + nrows - 1 of X, row-major and contiguous (D
+ * elements of the step's x_dtype per row; nrows <= FGMM_CHUNK_POINTS).  Return 0 on
+ * success, anything else on failure.  Called on the calling thread, one chunk at a
+ * time, in increasing row order within each pass over X (a step makes one pass per
+ * sweep pair that runs: two or three under FGMM_PREC_AUTO when its device-side
+ * decision asks for the redo or the CUDA-core pass). */
+typedef int (*fgmm_read_fn)(void* ctx, int64_t row0, int64_t nrows, void* dst);
+
+/* fgmm_em_step with X produced chunk by chunk by a reader: for X on storage, the
+ * paper's path for N beyond host memory (§6, streaming from SSD into the same
+ * O(K D) buffers).  Each chunk is read into one of two pinned host buffers
+ * (2 x FGMM_CHUNK_POINTS x D x 4 bytes, allocated by the first call and kept by the
+ * handle; a buffer is refilled only after its previous copy to the device completed),
+ * copied to a device staging buffer on the copy stream of fgmm_em_step_host, and
+ * processed there, so that reading chunk i + 1 overlaps the sweeps of chunk i.
+ * Results are bit-identical to fgmm_em_step on the same rows.  Returns FGMM_ERR_IO
+ * (with the step's outputs undefined and the parameters unchanged) when the reader
+ * fails; other arguments and errors as fgmm_em_step_host.  The call returns when the
+ * last chunk has been read and its copy enqueued. */
+int fgmm_em_step_reader(fgmm_handle h, fgmm_read_fn read, void* ctx, int x_dtype, int64_t N,
+                        float* weights, float* means, float* vars, double* loglik_out,
+                        float* logz_out, fgmm_stream_t stream);
+
+/* fgmm_em_step_reader for X stored in a file: N rows of D elements of x_dtype,
+ * row-major and contiguous, starting at byte `offset` of the file at `path` (read with
+ * pread; a short read or an unopenable file gives FGMM_ERR_IO). */
+int fgmm_em_step_file(fgmm_handle h, const char* path, int64_t offset, int x_dtype, int64_t N,
+                      float* weights, float* means, float* vars, double* loglik_out,
+                      float* logz_out, fgmm_stream_t stream);
+
 /* Data-parallel EM over row shards of X (one exchange per iteration).  Each entry
  * of the M-step's input is a sum over rows (§2, Eqs. (1)-(3)), so an iteration over
  * shards held by several handles, devices or processes is: fgmm_em_partial on every
@@ -208,6 +240,19 @@ int fgmm_em_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_
 /* fgmm_em_partial with X in host memory, streamed as in fgmm_em_step_host. */
 int fgmm_em_partial_host(fgmm_handle h, const void* X_host, int x_dtype, int64_t N,
                          int64_t ldx, const float* weights, const float* means,
+                         const float* vars, double* stats_out, float* logz_out,
+                         fgmm_stream_t stream);
+
+/* fgmm_em_partial with X produced by a reader, as in fgmm_em_step_reader (a shard on
+ * storage: each rank reads its own rows). */
+int fgmm_em_partial_reader(fgmm_handle h, fgmm_read_fn read, void* ctx, int x_dtype,
+                           int64_t N, const float* weights, const float* means,
+                           const float* vars, double* stats_out, float* logz_out,
+                           fgmm_stream_t stream);
+
+/* fgmm_em_partial_reader for a shard stored in a file, as in fgmm_em_step_file. */
+int fgmm_em_partial_file(fgmm_handle h, const char* path, int64_t offset, int x_dtype,
+                         int64_t N, const float* weights, const float* means,
                          const float* vars, double* stats_out, float* logz_out,
                          fgmm_stream_t stream);
 
@@ -271,7 +316,7 @@ int fgmm_soft_assign(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64
  *
  * The first call on a device looks up that array's device address (once per device,
  * with that device current), and the CUDA runtime may allocate the array then if it
- * loads modules lazily; make this first call before any stream capture.  The address
+ * loads modules lazily.  The address
  * is kept for the life of the process: after cudaDeviceReset (or anything else that
  * destroys and re-creates the device's primary context) it is stale, and this call
  * must not be used on that device again.  Every

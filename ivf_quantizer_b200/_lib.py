@@ -15,7 +15,10 @@ LIB_PATH = os.path.join(HERE, "_fgmm.so")
 COV_DIAG, COV_SPHERICAL = 0, 1
 PREC_FP32, PREC_FP16X3, PREC_FP16, PREC_AUTO = 0, 1, 2, 3
 F32, BF16 = 0, 1
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_OOM, ERR_NUMERIC, ERR_TIMEOUT = range(7)
+# fgmm_read_fn: (ctx, row0, nrows, dst) -> 0 on success
+READ_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                           ctypes.c_void_p)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_OOM, ERR_NUMERIC, ERR_TIMEOUT, ERR_IO = range(8)
 MAX_TOP_M = 16
 IVF_MAX_TOPK = 32
 STATIC_MAX_KD = 1 << 18
@@ -82,6 +85,11 @@ SIGNATURES = {
     "fgmm_kmeans_seed_scratch_bytes": (_c.c_size_t, [_i64]),
     "fgmm_em_step_host": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fgmm_em_partial_host": (_int, [_vp, _vp, _int, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_em_step_reader": (_int, [_vp, _vp, _vp, _int, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_em_partial_reader": (_int, [_vp, _vp, _vp, _int, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_em_step_file": (_int, [_vp, _c.c_char_p, _i64, _int, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fgmm_em_partial_file": (_int, [_vp, _c.c_char_p, _i64, _int, _i64, _vp, _vp, _vp, _vp, _vp,
+                                    _vp]),
 }
 
 

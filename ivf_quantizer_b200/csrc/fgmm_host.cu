@@ -14,6 +14,9 @@
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
+#include <errno.h>
+#include <fcntl.h>
+#include <unistd.h>
 
 #include <new>
 
@@ -25,8 +28,11 @@ using namespace fgmm;
 
 // Streaming of X from host memory (fgmm_em_step_host): two device staging buffers of
 // one chunk each, filled on a copy stream while the compute stream works on the other.
+// Streaming from a reader (fgmm_em_step_reader, _file) adds two pinned host buffers
+// that the reader fills, each refilled only after its previous copy has completed.
 struct HostStaging {
   void* buf[2] = {nullptr, nullptr};
+  void* pin[2] = {nullptr, nullptr};
   cudaStream_t cs = nullptr;
   cudaEvent_t copied[2] = {nullptr, nullptr};
   cudaEvent_t consumed[2] = {nullptr, nullptr};
@@ -34,14 +40,21 @@ struct HostStaging {
   void release() {
     for (int b = 0; b < 2; ++b) {
       if (buf[b]) cudaFree(buf[b]);
+      if (pin[b]) cudaFreeHost(pin[b]);
       if (copied[b]) cudaEventDestroy(copied[b]);
       if (consumed[b]) cudaEventDestroy(consumed[b]);
-      buf[b] = nullptr;
+      buf[b] = pin[b] = nullptr;
       copied[b] = consumed[b] = nullptr;
     }
     if (cs) cudaStreamDestroy(cs);
     cs = nullptr;
   }
+};
+
+// A reader of X (fgmm_read_fn and its context), for the streamed steps.
+struct ReaderSrc {
+  fgmm_read_fn fn;
+  void* ctx;
 };
 
 struct fgmm_ctx {
@@ -418,6 +431,16 @@ cudaError_t ensure_staging(fgmm_ctx* h) {
   return e;
 }
 
+// Pinned host buffers for a reader, made on first use (after ensure_staging).
+cudaError_t ensure_pinned(fgmm_ctx* h) {
+  HostStaging& hs = h->hs;
+  const size_t bytes = (size_t)kChunk * h->c.D * sizeof(float);
+  cudaError_t e = cudaSuccess;
+  for (int b = 0; b < 2 && e == cudaSuccess; ++b)
+    if (!hs.pin[b]) e = cudaHostAlloc(&hs.pin[b], bytes, cudaHostAllocDefault);
+  return e;
+}
+
 int read_word(const int* dev, int* out, cudaStream_t s) {
   cudaError_t e = cudaMemcpyAsync(out, dev, sizeof(int), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -427,9 +450,14 @@ int read_word(const int* dev, int* out, cudaStream_t s) {
 int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ldx,
                 const float* weights, const float* means, const float* vars, double* st,
                 float* logz_out, fgmm_stream_t stream, bool host_x = false,
-                bool want_stats = true) {
-  int rc = check_x(h, X, x_dtype, N, ldx);
+                bool want_stats = true, const ReaderSrc* rd = nullptr) {
+  // a reader stands in for X: the checks see a dummy non-null pointer, rows of D
+  int rc = check_x(h, rd ? (const void*)rd : X, x_dtype, N, rd ? (h ? h->c.D : 0) : ldx);
   if (rc) return rc;
+  if (rd) {
+    host_x = true;
+    ldx = h->c.D;
+  }
   if (!weights || !means || !vars) return FGMM_ERR_INVALID_ARG;
   Ctx& c = h->c;
   if ((rc = set_device(c))) return rc;
@@ -437,6 +465,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
   cudaError_t e;
   const Workspace& w = c.ws;
   if (host_x && (e = ensure_staging(h)) != cudaSuccess) return map_cuda(e);
+  if (rd && (e = ensure_pinned(h)) != cudaSuccess) return map_cuda(e);
   prof_gates_changed(c);
   // which path(s) to enqueue: FP32 -> CUDA cores; FP16X3 -> tensor cores; AUTO ->
   // both, each kernel returning at once unless the device-side mode word (set by the
@@ -467,6 +496,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
   // copy of the next chunk overlaps the kernels of this one.
   HostStaging& hs = h->hs;
   cudaError_t copy_err = cudaSuccess;
+  bool read_failed = false;
   auto acquire = [&](int64_t c0, int64_t nc, const void** Xc, int64_t* ldc) -> int {
     if (!host_x) {
       *Xc = (const char*)X + (size_t)c0 * ldx * eb;
@@ -474,11 +504,26 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       return -1;
     }
     const int b = (int)(hs.seq++ & 1);
-    cudaError_t r = cudaStreamWaitEvent(hs.cs, hs.consumed[b], 0);
+    const void* src = rd ? nullptr : (const void*)((const char*)X + (size_t)c0 * ldx * eb);
+    cudaError_t r = cudaSuccess;
+    if (rd) {
+      // the pinned buffer's previous copy to the device (recorded as copied[b]) must be
+      // complete before the reader overwrites it
+      r = cudaEventSynchronize(hs.copied[b]);
+      if (r == cudaSuccess && !read_failed && rd->fn(rd->ctx, c0, nc, hs.pin[b]) != 0)
+        read_failed = true;
+      if (read_failed) {   // no copy: the caller enqueues nothing for this chunk
+        *Xc = hs.buf[b];
+        *ldc = c.D;
+        if (r != cudaSuccess && copy_err == cudaSuccess) copy_err = r;
+        return b;
+      }
+      src = hs.pin[b];
+    }
+    if (r == cudaSuccess) r = cudaStreamWaitEvent(hs.cs, hs.consumed[b], 0);
     if (r == cudaSuccess)
-      r = cudaMemcpy2DAsync(hs.buf[b], (size_t)c.D * eb, (const char*)X + (size_t)c0 * ldx * eb,
-                            (size_t)ldx * eb, (size_t)c.D * eb, (size_t)nc,
-                            cudaMemcpyHostToDevice, hs.cs);
+      r = cudaMemcpy2DAsync(hs.buf[b], (size_t)c.D * eb, src, (size_t)ldx * eb,
+                            (size_t)c.D * eb, (size_t)nc, cudaMemcpyHostToDevice, hs.cs);
     if (r == cudaSuccess) r = cudaEventRecord(hs.copied[b], hs.cs);
     if (r == cudaSuccess) r = cudaStreamWaitEvent(s, hs.copied[b], 0);
     if (r != cudaSuccess && copy_err == cudaSuccess) copy_err = r;
@@ -501,6 +546,10 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       const void* Xc;
       int64_t ldc;
       const int b = acquire(c0, nc, &Xc, &ldc);
+      if (read_failed) {   // nothing more of this pass is enqueued
+        release(b);
+        break;
+      }
       float* lzo = logz_out ? logz_out + c0 : nullptr;
       if ((r = launch_tc_convert(c, Xc, x_dtype, nc, ldc, nullptr, gate, s)) == cudaSuccess &&
           (r = launch_tc_lse(c, nc, lzo, gate, s)) == cudaSuccess &&
@@ -525,6 +574,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
     int word = kModeTensor;
     if (host_x && auto_mode && (rc = read_word(w.mode, &word, s))) return rc;
     if (word == kModeTensor && (e = tc_pass(mode)) != cudaSuccess) return map_cuda(e);
+    if (read_failed) return FGMM_ERR_IO;
     if (auto_mode && want_stats) {
       // AUTO: components whose new variance would lose accuracy to cancellation move to
       // the side path and the pass is redone (gated on mode2); a failure after that sends
@@ -547,6 +597,10 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       const void* Xc;
       int64_t ldc;
       const int b = acquire(c0, nc, &Xc, &ldc);
+      if (read_failed) {
+        release(b);
+        break;
+      }
       float* lzo = logz_out ? logz_out + c0 : nullptr;
       if ((e = launch_lse_simt(c, Xc, x_dtype, nc, ldc, lzo, want_stats, mode, s)) == cudaSuccess &&
           (e = launch_ll_accumulate(c, nc, mode, fixed_mode, kModeSimt, s)) == cudaSuccess &&
@@ -558,6 +612,7 @@ int run_partial(fgmm_handle h, const void* X, int x_dtype, int64_t N, int64_t ld
       if (e != cudaSuccess) return map_cuda(e);
     }
   }
+  if (read_failed) return FGMM_ERR_IO;
   if (want_stats && (e = launch_reduce_stats(c, means, st, mode, fixed_mode, s)) != cudaSuccess)
     return map_cuda(e);
   h->c.last_auto = auto_mode;
@@ -604,6 +659,89 @@ int fgmm_em_partial_host(fgmm_handle h, const void* X_host, int x_dtype, int64_t
   if (!stats_out) return FGMM_ERR_INVALID_ARG;
   return run_partial(h, X_host, x_dtype, N, ldx, weights, means, vars, stats_out, logz_out,
                      stream, true);
+}
+
+}  // extern "C"
+
+namespace {
+// X in a file: rows of row_bytes bytes from byte `offset`, read with pread.
+struct FileSrc {
+  int fd;
+  int64_t offset;
+  int64_t row_bytes;
+};
+
+int file_read(void* ctx, int64_t row0, int64_t nrows, void* dst) {
+  const FileSrc* f = static_cast<const FileSrc*>(ctx);
+  char* p = static_cast<char*>(dst);
+  int64_t left = nrows * f->row_bytes;
+  off_t at = (off_t)(f->offset + row0 * f->row_bytes);
+  while (left > 0) {
+    const ssize_t got = pread(f->fd, p, (size_t)left, at);
+    if (got < 0 && errno == EINTR) continue;
+    if (got <= 0) return 1;   // an error, or the file ends before the rows do
+    p += got;
+    at += got;
+    left -= got;
+  }
+  return 0;
+}
+
+// Open the file and run `body` with a reader of it; FGMM_ERR_IO if it cannot be opened.
+template <typename Body>
+int with_file(fgmm_handle h, const char* path, int64_t offset, int x_dtype, Body body) {
+  if (!h || !path || offset < 0 || !valid_dtype(x_dtype)) return FGMM_ERR_INVALID_ARG;
+  const int fd = open(path, O_RDONLY);
+  if (fd < 0) return FGMM_ERR_IO;
+  FileSrc f{fd, offset, (int64_t)h->c.D * (int64_t)dtype_bytes(x_dtype)};
+  const ReaderSrc rd{file_read, &f};
+  const int rc = body(&rd);
+  close(fd);
+  return rc;
+}
+}  // namespace
+
+extern "C" {
+
+int fgmm_em_step_reader(fgmm_handle h, fgmm_read_fn read, void* ctx, int x_dtype, int64_t N,
+                        float* weights, float* means, float* vars, double* loglik_out,
+                        float* logz_out, fgmm_stream_t stream) {
+  if (!h || !read) return FGMM_ERR_INVALID_ARG;
+  const ReaderSrc rd{read, ctx};
+  int rc = run_partial(h, nullptr, x_dtype, N, 0, weights, means, vars, h->c.ws.canon, logz_out,
+                       stream, true, true, &rd);
+  if (rc) return rc;
+  return map_cuda(launch_finish(h->c, h->c.ws.canon, weights, means, vars, loglik_out,
+                                (cudaStream_t)stream));
+}
+
+int fgmm_em_partial_reader(fgmm_handle h, fgmm_read_fn read, void* ctx, int x_dtype,
+                           int64_t N, const float* weights, const float* means,
+                           const float* vars, double* stats_out, float* logz_out,
+                           fgmm_stream_t stream) {
+  if (!h || !read || !stats_out) return FGMM_ERR_INVALID_ARG;
+  const ReaderSrc rd{read, ctx};
+  return run_partial(h, nullptr, x_dtype, N, 0, weights, means, vars, stats_out, logz_out,
+                     stream, true, true, &rd);
+}
+
+int fgmm_em_step_file(fgmm_handle h, const char* path, int64_t offset, int x_dtype, int64_t N,
+                      float* weights, float* means, float* vars, double* loglik_out,
+                      float* logz_out, fgmm_stream_t stream) {
+  return with_file(h, path, offset, x_dtype, [&](const ReaderSrc* rd) {
+    return fgmm_em_step_reader(h, rd->fn, rd->ctx, x_dtype, N, weights, means, vars,
+                               loglik_out, logz_out, stream);
+  });
+}
+
+int fgmm_em_partial_file(fgmm_handle h, const char* path, int64_t offset, int x_dtype,
+                         int64_t N, const float* weights, const float* means,
+                         const float* vars, double* stats_out, float* logz_out,
+                         fgmm_stream_t stream) {
+  return with_file(h, path, offset, x_dtype, [&](const ReaderSrc* rd) {
+    return fgmm_em_partial_reader(h, rd->fn, rd->ctx, x_dtype, N, weights, means, vars,
+                                  stats_out, logz_out, stream);
+  });
 }
 
 int fgmm_em_finish(fgmm_handle h, const double* stats, float* weights, float* means,
@@ -925,6 +1063,7 @@ const char* fgmm_status_string(int status) {
     case FGMM_ERR_OOM: return "out of device memory";
     case FGMM_ERR_NUMERIC: return "non-finite log-likelihood or every component empty";
     case FGMM_ERR_TIMEOUT: return "bounded device wait expired";
+    case FGMM_ERR_IO: return "reading X failed";
     default: return "unknown status";
   }
 }

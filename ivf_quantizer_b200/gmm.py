@@ -8,7 +8,9 @@ and ``fit``.
 from __future__ import annotations
 
 import ctypes
+import os
 
+import numpy as np
 import torch
 
 from . import _lib
@@ -143,6 +145,63 @@ class GMM:
         fn = LIB.fgmm_em_step if X.is_cuda else LIB.fgmm_em_step_host
         check(fn(self._h, xp, dt, n, ldx, _ptr(weights), _ptr(means), _ptr(variances),
                  _ptr(loglik), _ptr(logz), _stream()), "fgmm_em_step")
+
+    def _stream_args(self, weights, means, variances, dtype, loglik=None, logz=None, n=0):
+        self._check_params(weights, means, variances)
+        if dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError("dtype must be torch.float32 or torch.bfloat16")
+        if loglik is not None and not (loglik.is_cuda and loglik.dtype == torch.float64):
+            raise ValueError("loglik must be a CUDA float64 tensor")
+        if logz is not None and not (logz.is_cuda and logz.dtype == torch.float32
+                                     and logz.numel() >= n):
+            raise ValueError("logz must be a CUDA float32 tensor with N elements")
+        return _lib.F32 if dtype == torch.float32 else _lib.BF16
+
+    def step_file(self, path, N, weights, means, variances, dtype=torch.float32, offset=0,
+                  loglik=None, logz=None):
+        """One EM iteration with X read from a file (fgmm_em_step_file): N rows of D
+        elements of `dtype`, row-major, from byte `offset`; chunks are read into pinned
+        buffers while the previous chunk is processed.  Bit-identical to step() on the
+        same rows."""
+        dt = self._stream_args(weights, means, variances, dtype, loglik, logz, N)
+        check(LIB.fgmm_em_step_file(self._h, os.fsencode(path), int(offset), dt, int(N),
+                                    _ptr(weights), _ptr(means), _ptr(variances),
+                                    _ptr(loglik), _ptr(logz), _stream()), "fgmm_em_step_file")
+
+    def partial_file(self, path, N, weights, means, variances, dtype=torch.float32, offset=0,
+                     stats=None, logz=None):
+        """partial() with this shard's rows read from a file (fgmm_em_partial_file)."""
+        dt = self._stream_args(weights, means, variances, dtype, None, logz, N)
+        if stats is None:
+            stats = torch.empty(self.stats_len, dtype=torch.float64, device=weights.device)
+        check(LIB.fgmm_em_partial_file(self._h, os.fsencode(path), int(offset), dt, int(N),
+                                       _ptr(weights), _ptr(means), _ptr(variances),
+                                       _ptr(stats), _ptr(logz), _stream()),
+              "fgmm_em_partial_file")
+        return stats
+
+    def step_reader(self, read, N, weights, means, variances, dtype=torch.float32,
+                    loglik=None, logz=None):
+        """One EM iteration with X produced by `read(row0, out)`, which fills the numpy
+        array `out` (nrows x D of `dtype`, bf16 as uint16) with rows row0 .. and returns
+        True on success (fgmm_em_step_reader)."""
+        dt = self._stream_args(weights, means, variances, dtype, loglik, logz, N)
+        D = self.D
+        npdt = np.float32 if dtype == torch.float32 else np.uint16
+
+        def _cb(ctx, row0, nrows, dst):
+            try:
+                buf = (ctypes.c_char * (int(nrows) * D * np.dtype(npdt).itemsize)).from_address(dst)
+                out = np.frombuffer(buf, dtype=npdt).reshape(int(nrows), D)
+                return 0 if read(int(row0), out) else 1
+            except Exception:  # a failing reader ends the step with ERR_IO
+                return 1
+
+        cb = _lib.READ_FN(_cb)
+        check(LIB.fgmm_em_step_reader(self._h, ctypes.cast(cb, ctypes.c_void_p), None, dt,
+                                      int(N), _ptr(weights), _ptr(means), _ptr(variances),
+                                      _ptr(loglik), _ptr(logz), _stream()),
+              "fgmm_em_step_reader")
 
     # ---------------------------------------------------------------- sharded EM
     @property

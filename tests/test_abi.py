@@ -72,6 +72,16 @@ def test_calls_on_null_handle_are_invalid():
     assert LIB.fgmm_get_block_skip(z, ctypes.byref(v)) == _lib.ERR_INVALID_ARG
     assert v.value == 7
     assert LIB.fgmm_get_status(z, z) == _lib.ERR_INVALID_ARG
+    # X from a file or a reader: a null handle, path or reader is an argument error
+    assert LIB.fgmm_em_step_file(z, b"/nonexistent", 0, 0, 10, one, one, one, z, z, z) == \
+        _lib.ERR_INVALID_ARG
+    assert LIB.fgmm_em_partial_file(z, b"/nonexistent", 0, 0, 10, one, one, one, one, z, z) == \
+        _lib.ERR_INVALID_ARG
+    assert LIB.fgmm_em_step_reader(z, one, z, 0, 10, one, one, one, z, z, z) == \
+        _lib.ERR_INVALID_ARG
+    assert LIB.fgmm_em_partial_reader(z, one, z, 0, 10, one, one, one, one, z, z) == \
+        _lib.ERR_INVALID_ARG
+    assert LIB.fgmm_status_string(_lib.ERR_IO) == b"reading X failed"
     assert LIB.fgmm_destroy(z) == _lib.OK
 
 
