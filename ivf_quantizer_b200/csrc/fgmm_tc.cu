@@ -1175,7 +1175,6 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows) {
 size_t lse_smem(int nkc, bool split) {
   return 1024 + (size_t)((split ? 2 : 1) * nkc + lse_ring(nkc, split)) * BOX + sizeof(LseBars);
 }
-constexpr size_t kMaxDynSmem = kSmemMax;
 size_t stats_smem(int nkc) { return 1024 + (size_t)(nkc + SX + 2) * BOX + sizeof(StatBars); }
 
 template <int NKC, bool SPLIT>
